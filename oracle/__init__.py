@@ -1,0 +1,174 @@
+"""numpy bindings of the scalar CPU oracle (mxfp4_oracle.c).
+
+TEST INFRASTRUCTURE: only tests/, __graft_entry__.smoke() and bench.py's CPU
+baseline leg import this package. The CUDA library and its binding never do.
+
+bf16 data is passed as numpy uint16 arrays holding the raw bf16 bit patterns;
+fp32 data as numpy float32 arrays. All arrays are 2-D [rows, cols] row-major.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from .build import LIB, build
+
+F32, BF16 = 0, 1
+SCALE_PAGE, SCALE_FLOOR = 0, 1
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(LIB)
+        P = ctypes.c_void_p
+        i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        L.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.oracle_bf16_to_f32.restype = f32
+        L.oracle_f32_to_bf16.argtypes = [f32]
+        L.oracle_f32_to_bf16.restype = ctypes.c_uint16
+        L.oracle_scale_page.argtypes = [f32, f32]
+        L.oracle_scale_page.restype = f32
+        L.oracle_scale_floor.argtypes = [f32]
+        L.oracle_scale_floor.restype = f32
+        L.oracle_qdq_block.argtypes = [P, i32, f32, i32, P, P, P, P]
+        L.oracle_qdq_block.restype = None
+        L.oracle_group_ends.argtypes = [P, i64, i32, i64, P]
+        L.oracle_group_ends.restype = i32
+        L.oracle_colwise_scale_rows.argtypes = [P, i64, i64]
+        L.oracle_colwise_scale_rows.restype = i64
+        L.oracle_qdq_rowwise.argtypes = [P, i32, i64, i64, i64, i32, f32, i32, P, P, P, P]
+        L.oracle_qdq_rowwise.restype = i32
+        L.oracle_qdq_colwise.argtypes = [P, i32, i64, i64, i64, i32, f32, i32, P, i64, P, P, P, P]
+        L.oracle_qdq_colwise.restype = i32
+        L.oracle_ste_bwd.argtypes = [P, i32, i64, i64, P, i32, P]
+        L.oracle_ste_bwd.restype = None
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(x: np.ndarray) -> int:
+    if x.dtype == np.uint16:
+        return BF16
+    if x.dtype == np.float32:
+        return F32
+    raise TypeError(f"oracle takes uint16 (bf16 bits) or float32, got {x.dtype}")
+
+
+def bf16_to_f32(b: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to fp32 values."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16(f: float) -> int:
+    return int(lib().oracle_f32_to_bf16(float(f)))
+
+
+def scale_page(amax: float, scale_factor: float = 6.0) -> float:
+    return float(lib().oracle_scale_page(amax, scale_factor))
+
+
+def scale_floor(amax: float) -> float:
+    return float(lib().oracle_scale_floor(amax))
+
+
+def qdq_block(v, scale_factor: float = 6.0, mode: int = SCALE_PAGE):
+    """One block of fp32 values -> (out f32[n], nibble u8[n], sat u8[n], e8m0 byte)."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    n = v.size
+    out = np.empty(n, np.float32)
+    nib = np.empty(n, np.uint8)
+    sat = np.empty(n, np.uint8)
+    e8 = np.zeros(1, np.uint8)
+    lib().oracle_qdq_block(_ptr(v), n, scale_factor, mode, _ptr(out), _ptr(nib), _ptr(sat), _ptr(e8))
+    return out, nib, sat, int(e8[0])
+
+
+def group_ends(group_list, group_list_type: int, rows: int) -> np.ndarray | None:
+    """Cumulative end offsets of a group_list, or None when it is not a valid partition."""
+    gl = np.ascontiguousarray(group_list, dtype=np.int64)
+    ends = np.empty(max(gl.size, 1), np.int64)
+    rc = lib().oracle_group_ends(_ptr(gl), gl.size, group_list_type, rows, _ptr(ends))
+    return None if rc != 0 else ends[: gl.size]
+
+
+def colwise_scale_rows(ends, block: int) -> int:
+    e = np.ascontiguousarray(ends, dtype=np.int64)
+    return int(lib().oracle_colwise_scale_rows(_ptr(e), e.size, block))
+
+
+def qdq_rowwise(x: np.ndarray, block: int = 32, scale_factor: float = 6.0, mode: int = SCALE_PAGE):
+    """Row-wise QDQ of a 2-D array; returns dict(y, codes, scales, mask)."""
+    x = np.ascontiguousarray(x)
+    dt = _dtype_code(x)
+    rows, cols = x.shape
+    y = np.empty_like(x)
+    codes = np.zeros((rows, (cols + 1) // 2), np.uint8)
+    scales = np.zeros((rows, (cols + block - 1) // block), np.uint8)
+    mask = np.zeros((rows, (cols + 7) // 8), np.uint8)
+    rc = lib().oracle_qdq_rowwise(_ptr(x), dt, rows, cols, cols, block, scale_factor, mode,
+                                  _ptr(y), _ptr(codes), _ptr(scales), _ptr(mask))
+    if rc != 0:
+        raise MemoryError("oracle_qdq_rowwise failed")
+    return dict(y=y, codes=codes, scales=scales, mask=mask)
+
+
+def qdq_colwise(x: np.ndarray, block: int = 32, scale_factor: float = 6.0, mode: int = SCALE_PAGE,
+                ends=None):
+    """Column-wise QDQ (blocks down columns, restarting at group ends)."""
+    x = np.ascontiguousarray(x)
+    dt = _dtype_code(x)
+    rows, cols = x.shape
+    e = None if ends is None else np.ascontiguousarray(ends, dtype=np.int64)
+    s = colwise_scale_rows(e if e is not None else np.array([rows], np.int64), block)
+    y = np.empty_like(x)
+    codes = np.zeros((rows, (cols + 1) // 2), np.uint8)
+    scales = np.zeros((s, cols), np.uint8)
+    mask = np.zeros((rows, (cols + 7) // 8), np.uint8)
+    rc = lib().oracle_qdq_colwise(_ptr(x), dt, rows, cols, cols, block, scale_factor, mode,
+                                  _ptr(e), 0 if e is None else e.size,
+                                  _ptr(y), _ptr(codes), _ptr(scales), _ptr(mask))
+    if rc != 0:
+        raise MemoryError("oracle_qdq_colwise failed")
+    return dict(y=y, codes=codes, scales=scales, mask=mask)
+
+
+def ste_bwd(grad_out: np.ndarray, mask: np.ndarray, clip_grad: bool = True) -> np.ndarray:
+    g = np.ascontiguousarray(grad_out)
+    dt = _dtype_code(g)
+    rows, cols = g.shape
+    m = np.ascontiguousarray(mask, dtype=np.uint8)
+    assert m.shape == (rows, (cols + 7) // 8)
+    out = np.empty_like(g)
+    lib().oracle_ste_bwd(_ptr(g), dt, rows, cols, _ptr(m), int(bool(clip_grad)), _ptr(out))
+    return out
+
+
+def unpack_bits(mask: np.ndarray, cols: int) -> np.ndarray:
+    """Bit-packed [rows, ceil(cols/8)] mask -> bool [rows, cols] (bit b of byte j = col 8j+b)."""
+    return np.unpackbits(mask, axis=1, bitorder="little")[:, :cols].astype(bool)
+
+
+def unpack_nibbles(codes: np.ndarray, cols: int) -> np.ndarray:
+    """Packed [rows, ceil(cols/2)] codes -> uint8 [rows, cols] nibbles (low nibble first)."""
+    lo = codes & 0x0F
+    hi = codes >> 4
+    out = np.empty((codes.shape[0], codes.shape[1] * 2), np.uint8)
+    out[:, 0::2] = lo
+    out[:, 1::2] = hi
+    return out[:, :cols]
+
+
+__all__ = [
+    "F32", "BF16", "SCALE_PAGE", "SCALE_FLOOR", "lib", "build", "bf16_to_f32", "f32_to_bf16",
+    "scale_page", "scale_floor", "qdq_block", "group_ends", "colwise_scale_rows", "qdq_rowwise",
+    "qdq_colwise", "ste_bwd", "unpack_bits", "unpack_nibbles",
+]
