@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""MXFP4 block fake-quant benchmark: effective HBM GB/s of one training step of
+the quantiser (QDQ forward + clipped-STE backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of the MoE grouped
+activation workload (bf16 [65536, 7168], 256 multinomial groups with empty
+ones):
+  1. mxfp4_qdq_fwd, both directions from one read of x: row-wise blocks of 32
+     and column-wise blocks of 32 restarting at every group offset; writes
+     y_row, y_col, packed E2M1 codes and E8M0 scales for both directions and
+     the row and column saturation bitmasks;
+  2. mxfp4_ste_bwd, clipped STE: grad_in = grad_out with +0 where the saved
+     row-wise bitmask is set.
+value = algorithmic bytes of all ranks' steps / max-over-ranks device time.
+Inputs (x and grad_out, 940 MB each) are larger than the 126 MB L2, so no
+flush is needed between steps.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch
+(weak scaling, no data-path collective); NCCL only carries the barrier and
+the max-reduction of the timings.
+
+--impl reference times the CPU oracle (tests' reference implementation) on a
+bounded sample of the same workload on the host cores; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MXFP4 QDQ fwd+STE-bwd effective HBM GB/s and % of B200 peak, 1 GPU"
+SPEC_PEAK_GBS = 8000.0  # nominal B200 HBM3e figure quoted with the metric
+CPU_SAMPLE_ROWS = 16384
+REF_SAMPLE_ROWS = 4096
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--scale-mode", choices=["page", "floor"], default="page")
+    p.add_argument("--rows", type=int, default=65536)
+    p.add_argument("--cols", type=int, default=7168)
+    p.add_argument("--groups", type=int, default=256)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes
+# ---------------------------------------------------------------------------
+
+def step_bytes(rows: int, cols: int, s_col: int, esz: int = 2, block: int = 32) -> dict:
+    n = rows * cols
+    fwd = (n * esz                      # read x
+           + 2 * n * esz                # write y_row, y_col
+           + 2 * (rows * ((cols + 1) // 2))  # codes row + col
+           + rows * ((cols + block - 1) // block) + s_col * cols  # E8M0 scales
+           + 2 * rows * ((cols + 7) // 8))   # masks row + col
+    bwd = rows * ((cols + 7) // 8) + 2 * n * esz  # read mask + grad_out, write grad_in
+    return {"fwd": fwd, "bwd": bwd, "step": fwd + bwd}
+
+
+def workload_desc(a, s_col: int) -> dict:
+    return {
+        "workload": "moe_grouped_dual_qdq_fwd_ste_bwd",
+        "shape": [a.rows, a.cols], "dtype": "bf16", "block": 32, "groups": a.groups,
+        "group_list": "type 0 cumulative offsets, multinomial sizes p~u^4, 3 forced empty",
+        "colwise_scale_rows": s_col, "scale_mode": a.scale_mode,
+        "fwd": "row+col QDQ in one pass: y, e2m1 codes, e8m0 scales, saturation bitmasks",
+        "bwd": "clipped STE from the saved row-wise bitmask",
+        "l2": "inputs larger than L2 (x and grad_out 940 MB each at the default size); no flush",
+    }
+
+
+# ---------------------------------------------------------------------------
+# clocks (NVML read-only sampling during the timed region)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_dev: int):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_dev)
+            try:
+                pci = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(pci)
+            except Exception:  # noqa: BLE001 - fall back to the visible index
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(torch_dev)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001 - clocks are reported as unavailable
+            self.err = repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append(mhz)
+                self.reasons |= int(r)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        self._stop = threading.Event()
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.ok:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "note": getattr(self, "err", "no samples")}
+        reasons = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return 6650.0, "fallback"
+
+
+def traffic_for(kernel_src: str, launch_bytes: int):
+    """DRAM traffic per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+        if t.get("source_sha256") != sha:
+            return None
+        scale = launch_bytes / t["algorithmic_bytes_per_launch"] if t.get("algorithmic_bytes_per_launch") else 1.0
+        return int(t["dram_bytes_per_launch"] * scale)
+    except Exception:  # noqa: BLE001
+        return None
+
+
+def run_ours(a, rank: int, world: int):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from mxfp4_block_fake_b200 import _abi, ops, workloads as W
+
+    dev = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+
+    x_h, counts, offsets = W.moe_grouped(a.rows, a.cols, a.groups, seed=4 + 1000 * rank)
+    g_h = W.train_step_grad(a.rows, a.cols, seed=5 + 1000 * rank)
+    s_col = ops.mxfp4_colwise_scale_rows(offsets.tolist(), 0, a.rows, 32)
+    xd, gd, gl = x_h.cuda(), g_h.cuda(), offsets.cuda()
+
+    res = ops.alloc_outputs(xd, block=32, rowwise=True, colwise=True, num_groups=a.groups, emit_codes=True,
+                            emit_mask=True, with_status=True)
+    gi = torch.empty_like(gd)
+    fargs = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode=a.scale_mode,
+                          dirs=_abi.ROWWISE | _abi.COLWISE, group_list=gl, group_list_type=0, status=res.status)
+    ops._fill_outputs(fargs, res)
+    bargs = ops.make_args(gd, block=32, scale_factor=6.0, scale_mode=a.scale_mode, dirs=_abi.ROWWISE)
+    bargs.x = None
+    sp = stream.cuda_stream
+    mask_ptr, g_ptr, gi_ptr = res.mask_row.data_ptr(), gd.data_ptr(), gi.data_ptr()
+
+    def fwd():
+        st = _abi.mxfp4_qdq_fwd(fargs, sp)
+        if st:
+            _abi.check(st, "mxfp4_qdq_fwd")
+
+    def bwd():
+        st = _abi.mxfp4_ste_bwd(bargs, g_ptr, gi_ptr, a.cols, mask_ptr, 1, sp)
+        if st:
+            _abi.check(st, "mxfp4_ste_bwd")
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[dev])
+
+    for _ in range(a.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    _abi.check(int(res.status.item()), "group_list")
+    # soak so the clocks settle before the timed steps
+    t0 = time.time()
+    while time.time() - t0 < 0.5:
+        fwd()
+        bwd()
+        torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        start.record(stream)
+        for i in range(a.steps):
+            ev[i][0].record(stream)
+            fwd()
+            ev[i][1].record(stream)
+            bwd()
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = start.elapsed_time(end)
+    fwd_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    t = torch.tensor([ms, fwd_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, fwd_ms = float(t[0]), float(t[1])
+
+    # e2e: same step through the public entry points with host buffers
+    e2e = None
+    if not a.no_e2e:
+        xh_p, gh_p = x_h.pin_memory(), g_h.pin_memory()
+        outs = [res.y_row, res.y_col, res.codes_row, res.scales_row, res.mask_row, res.codes_col,
+                res.scales_col[:s_col], res.mask_col, gi]
+        outs_h = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        h2d = xh_p.numel() * 2 + gh_p.numel() * 2
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+
+        def e2e_step():
+            xd.copy_(xh_p, non_blocking=True)
+            gd.copy_(gh_p, non_blocking=True)
+            ops.mxfp4_qdq_fwd(xd, scale_mode=a.scale_mode, rowwise=True, colwise=True, group_list=gl,
+                              emit_codes=True, emit_mask=True, out=res)
+            ops.mxfp4_ste_bwd(gd, saved_mask=res.mask_row, clip_grad=True, out=gi)
+            for o, oh in zip(outs, outs_h):
+                oh.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(a.steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        te = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = (float(te[0]), h2d, d2h)
+
+    return dict(ms=ms, fwd_ms=fwd_ms, s_col=s_col, clocks=sampler.summary(), e2e=e2e,
+                x_h=x_h, g_h=g_h, offsets=offsets, np=np)
+
+
+def cpu_baseline(a, x_h, g_h, offsets, rows: int):
+    """The oracle, as it stands, on the first `rows` rows of the same batch."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+
+    rows = min(rows, a.rows)
+    xs = x_h[:rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+    gs = g_h[:rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+    ends = np.minimum(offsets.numpy(), rows)
+    ends = ends[: int(np.searchsorted(ends, rows)) + 1]
+    ends[-1] = rows
+    mode = O.SCALE_PAGE if a.scale_mode == "page" else O.SCALE_FLOOR
+    s_col = O.colwise_scale_rows(ends, 32)
+    t0 = time.perf_counter()
+    r = O.qdq_rowwise(xs, 32, 6.0, mode)
+    O.qdq_colwise(xs, 32, 6.0, mode, ends=ends)
+    O.ste_bwd(gs, r["mask"], True)
+    dt = time.perf_counter() - t0
+    b = step_bytes(rows, a.cols, s_col)["step"]
+    return dict(value=b / dt / 1e9, seconds=dt, rows=rows, s_col=s_col)
+
+
+def main():
+    a = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+
+    if a.impl == "reference":
+        if rank != 0:
+            return
+        run_reference(a)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        r = run_ours(a, rank, world)
+        if rank == 0:
+            peak, peak_kind = measured_peaks()
+            b = step_bytes(a.rows, a.cols, r["s_col"])
+            value = b["step"] * world * a.steps / (r["ms"] / 1e3) / 1e9
+            achieved = b["fwd"] / (r["fwd_ms"] / 1e3) / 1e9
+            src = os.path.join(ROOT, "mxfp4_block_fake_b200", "csrc", "mxfp4.cu")
+            line = {
+                "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+                "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(r["ms"] / a.steps, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded N(0,1) bf16, multinomial groups)",
+                "config": workload_desc(a, r["s_col"]),
+                "pct_of_peak": {"measured_copy_6458": round(100 * value / world / peak, 1),
+                                "spec_8000": round(100 * value / world / SPEC_PEAK_GBS, 1)},
+                "elements_per_s": round(a.rows * a.cols * world * a.steps / (r["ms"] / 1e3), 1),
+                "parts_ms": {"qdq_fwd_dual": round(r["fwd_ms"], 4),
+                             "ste_bwd": round(r["ms"] / a.steps - r["fwd_ms"], 4)},
+                "roofline": {"bound": "hbm", "kernel": "qdq_tile_kernel (dual, grouped, bf16, block 32)",
+                             "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                             "unit": "GB/s", "frac": round(achieved / peak, 4),
+                             "traffic": traffic_for(src, b["fwd"]),
+                             "algorithmic_bytes_per_launch": b["fwd"]},
+                "gpu_launches": 2 * a.steps,
+                "clocks": r["clocks"],
+            }
+            if r["e2e"] is not None:
+                ms_e, h2d, d2h = r["e2e"]
+                line["e2e"] = {"value": round(b["step"] * world * a.steps / (ms_e / 1e3) / 1e9, 2),
+                               "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                               "ms_per_step": round(ms_e / a.steps, 3)}
+            if world == 1 and not a.no_cpu_baseline:
+                cb = cpu_baseline(a, r["x_h"], r["g_h"], r["offsets"], CPU_SAMPLE_ROWS)
+                line["cpu_baseline"] = {
+                    "value": round(cb["value"], 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                    "sample": f"first {cb['rows']} of {a.rows} rows x {a.cols} cols of the same batch "
+                              f"(groups cut at the sample end), one full step, {cb['seconds']:.1f} s"}
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+def run_reference(a):
+    import numpy as np
+
+    from mxfp4_block_fake_b200 import workloads as W
+
+    x_h, counts, offsets = W.moe_grouped(a.rows, a.cols, a.groups, seed=4)
+    g_h = W.train_step_grad(a.rows, a.cols, seed=5)
+    for _ in range(a.warmup):
+        cpu_baseline(a, x_h, g_h, offsets, REF_SAMPLE_ROWS)
+    tot_b, tot_s = 0, 0.0
+    for _ in range(a.steps):
+        cb = cpu_baseline(a, x_h, g_h, offsets, REF_SAMPLE_ROWS)
+        tot_b += step_bytes(cb["rows"], a.cols, cb["s_col"])["step"]
+        tot_s += cb["seconds"]
+    value = tot_b / tot_s / 1e9
+    s_col = int(np.sum((np.diff(np.concatenate([[0], offsets.numpy()])) + 31) // 32))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(1e3 * tot_s / a.steps, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, multinomial groups)", "config": workload_desc(a, s_col),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: first {REF_SAMPLE_ROWS} rows x {a.cols} cols of the batch"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * mxfp4.h -- C ABI of libmxfp4.so: MXFP4 block fake quantisation
+ * (quantise-dequantise, "QDQ") and its straight-through-estimator backward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed (web pages cited by title and section):
+ *   amct pull request 264, "feat: MXFP4 QAT fake-quant Linear (with STE)",
+ *   mxfp4_qat/fake_quant.py:
+ *     - _block_view / _block_scale: blocks of `block` consecutive elements
+ *       share a power-of-two scale 2^k,
+ *         PAGE  mode: k = round(log2(max(amax / scale_factor, 2^-30)))
+ *       (fp32 division; round() is the exact nearest integer of log2);
+ *         FLOOR mode: k = max(floor(log2 amax) - 2, -127) (the OCP-MX rule;
+ *       scale_factor is not used).
+ *     - _round_to_e2m1 / _quant_dequant_torch: y = x / 2^k in fp32, |y| is
+ *       rounded to the E2M1 codebook {0, .5, 1, 1.5, 2, 3, 4, 6} by counting
+ *       the midpoints {.25, .75, 1.25, 1.75, 2.5, 3.5, 5} that are <= |y|
+ *       (ties go to the larger code, |y| >= 5 gives 6), the output is
+ *       sign(y) * code * 2^k in fp32, cast to the input dtype.
+ *     - mxfp4_saturation_mask: an element saturates when |x| > 6 * 2^k.
+ *     - _MXFP4FakeQuantSTE.backward: grad_in = grad_out (plain STE) or
+ *       grad_out with saturated positions set to +0.0 (clipped STE).
+ *   MindSpore hyper-parallel, fake_w4a8_gmm_func.py, FakeW4A8GroupedLinear:
+ *     - quantize_input(rowwise=, colwise=, group_list=, group_list_type=):
+ *       "row-wise" blocks run along a row, "column-wise" blocks run down a
+ *       column; with a group_list the column-wise blocks restart at every
+ *       group start so that no block straddles two MoE groups.
+ *     - normalize_group_list: type 1 = per-group counts (turned into
+ *       cumulative offsets by a running sum), type 0 = cumulative end offsets.
+ *   sglang mxfp4_npu.py: two E2M1 values packed per byte.
+ *
+ * Data layout (all row-major, element strides in elements):
+ *   x, y_row, y_col, grads      [rows][cols], leading dimensions ld / ld_y /
+ *                               ld_grad (>= cols); dtype fp32 or bf16.
+ *   codes_row, codes_col        [rows][ceil(cols/2)] bytes, contiguous; the
+ *                               nibble of element c is the low nibble of byte
+ *                               c/2 when c is even, the high one when odd;
+ *                               nibble = sign << 3 | code index (E2M1 bits).
+ *   scales_row                  [rows][ceil(cols/block)] E8M0 bytes (k + 127).
+ *   scales_col                  [S][cols] E8M0 bytes, S = sum over groups of
+ *                               ceil(group rows / block), groups in order.
+ *                               mxfp4_colwise_scale_rows() gives S from a host
+ *                               copy of the group_list; allocating
+ *                               mxfp4_colwise_scale_rows_bound() rows needs no
+ *                               host copy (rows past S are left untouched).
+ *   mask_row, mask_col          [rows][ceil(cols/8)] bytes; bit b of byte j is
+ *                               the saturation flag of element 8j+b.
+ * Non-finite blocks (a NaN or +-inf element, or a scale that overflows fp32)
+ * write the quiet NaN 0x7FC0 / 0x7FC00000 to every output element, code 0,
+ * E8M0 byte 0xFF and no saturation bits.
+ *
+ * Ownership: every pointer is a device pointer owned by the caller, except
+ * where a parameter says "host". The library allocates no memory and keeps no
+ * state between calls. Calls are asynchronous on `stream`; inputs must stay
+ * valid and outputs unread until the stream reaches the call.
+ *
+ * Errors: argument errors are found on the host before any launch and
+ * returned as a status (nothing is written). A group_list lives in device
+ * memory, so its validity (non-negative counts, non-decreasing offsets, last
+ * offset == rows) is checked by the kernels: an invalid list makes every
+ * kernel of the call write nothing and, when `status` is non-NULL, store
+ * MXFP4_EINVAL there (MXFP4_OK otherwise). No kernel traps or asserts.
+ */
+#ifndef MXFP4_H
+#define MXFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* mxfp4_stream_t;
+
+typedef enum {
+    MXFP4_OK = 0,
+    MXFP4_EINVAL = 1,       /* invalid argument (also an invalid group_list) */
+    MXFP4_EUNSUPPORTED = 2, /* valid but not supported (block other than 32/128, too many groups) */
+    MXFP4_ECUDA = 3         /* a CUDA runtime call or launch failed */
+} mxfp4_status;
+
+typedef enum { MXFP4_F32 = 0, MXFP4_BF16 = 1 } mxfp4_dtype;
+
+typedef enum {
+    MXFP4_SCALE_PAGE = 0,  /* 2^round(log2(max(amax / scale_factor, 2^-30))) */
+    MXFP4_SCALE_FLOOR = 1  /* 2^max(floor(log2 amax) - 2, -127) */
+} mxfp4_scale_mode;
+
+/* Direction bits for mxfp4_qdq_args.dirs and grad_dir. */
+#define MXFP4_ROWWISE 1u
+#define MXFP4_COLWISE 2u
+
+/* Largest num_groups a call accepts. */
+#define MXFP4_MAX_GROUPS 4096
+
+#define MXFP4_ABI_VERSION 1
+
+/*
+ * Arguments of one QDQ call. Zero-initialise and fill what is used; every
+ * NULL output is skipped.
+ *   x              input [rows][cols], leading dimension ld; may be NULL only
+ *                  when mxfp4_ste_bwd reads a saved mask.
+ *   dtype          MXFP4_F32 or MXFP4_BF16 (x, y_* and grads share it).
+ *   block          32 or 128 elements per scale.
+ *   rows, cols     >= 0; a call with rows*cols == 0 does nothing.
+ *   scale_factor   PAGE mode divisor (default 6.0); must be finite and > 0
+ *                  in every mode (the page's check).
+ *   scale_mode     mxfp4_scale_mode.
+ *   dirs           MXFP4_ROWWISE, MXFP4_COLWISE or both: both directions are
+ *                  computed from one read of x.
+ *   group_list     optional device int64[num_groups]; applies to column-wise
+ *                  blocks only; NULL means one group of all rows.
+ *   group_list_type 0 = cumulative end offsets, 1 = counts.
+ *   status         optional device int32 that receives the group_list check.
+ *   y_row, y_col   dequantised outputs, x's dtype, leading dimension ld_y.
+ */
+typedef struct mxfp4_qdq_args {
+    const void* x;
+    int32_t dtype;
+    int32_t block;
+    int64_t rows;
+    int64_t cols;
+    int64_t ld;
+    float scale_factor;
+    int32_t scale_mode;
+    uint32_t dirs;
+    int32_t group_list_type;
+    const int64_t* group_list;
+    int64_t num_groups;
+    int32_t* status;
+    void* y_row;
+    void* y_col;
+    int64_t ld_y;
+    uint8_t* codes_row;
+    uint8_t* scales_row;
+    uint8_t* mask_row;
+    uint8_t* codes_col;
+    uint8_t* scales_col;
+    uint8_t* mask_col;
+} mxfp4_qdq_args;
+
+/*
+ * QDQ forward (fake_quant.py: mxfp4_quant_dequant, mxfp4_saturation_mask;
+ * fake_w4a8_gmm_func.py: quantize_input with rowwise/colwise/group_list).
+ * One pass over x writes every requested output of every requested direction:
+ * dequantised values, packed E2M1 codes, E8M0 scales and saturation bitmasks
+ * (the bitmask is what the clipped STE backward later reads, so a forward
+ * with mask_row set is the fused "forward + saved mask" step).
+ * Returns MXFP4_OK once the work is queued.
+ */
+mxfp4_status mxfp4_qdq_fwd(const mxfp4_qdq_args* args, mxfp4_stream_t stream);
+
+/*
+ * Clipped/plain STE backward (fake_quant.py: _MXFP4FakeQuantSTE.backward).
+ *   geom        shape, dtype, block, scale mode/factor, and exactly one
+ *               direction bit in dirs (the direction whose saturation masks
+ *               the gradient), plus x and group_list when the mask is
+ *               recomputed; its output pointers are ignored.
+ *   grad_out    [rows][cols], leading dimension ld_grad, geom->dtype.
+ *   grad_in     [rows][cols], leading dimension ld_grad; may equal grad_out.
+ *   saved_mask  bit-packed mask from a forward call, or NULL to recompute the
+ *               mask from x ("saved-free": one extra read of x).
+ *   clip_grad   0: grad_in = grad_out. 1: grad_in = grad_out with +0.0 where
+ *               the element saturated.
+ */
+mxfp4_status mxfp4_ste_bwd(const mxfp4_qdq_args* geom, const void* grad_out, void* grad_in,
+                           int64_t ld_grad, const uint8_t* saved_mask, int32_t clip_grad,
+                           mxfp4_stream_t stream);
+
+/*
+ * Fused forward + clipped-STE backward in one pass: everything mxfp4_qdq_fwd
+ * writes for `args`, plus grad_in = grad_out masked by the saturation of the
+ * direction grad_dir (which must be one of args->dirs). Used when the
+ * incoming gradient is already known at quantisation time (recomputation in
+ * the backward pass, or a measured training step).
+ */
+mxfp4_status mxfp4_qdq_fwd_bwd(const mxfp4_qdq_args* args, const void* grad_out, void* grad_in,
+                               int64_t ld_grad, uint32_t grad_dir, mxfp4_stream_t stream);
+
+/*
+ * Number of column-wise scale rows S for a group_list held in HOST memory
+ * (fake_w4a8_gmm_func.py: normalize_group_list, then sum of ceil(n_g/block)).
+ * Returns -1 when the list is not a valid partition of [0, rows).
+ */
+int64_t mxfp4_colwise_scale_rows(const int64_t* host_group_list, int64_t num_groups,
+                                 int32_t group_list_type, int64_t rows, int32_t block);
+
+/* Upper bound on S that needs no group sizes: floor(rows/block) + num_groups
+ * (ceil(rows/block) without groups). */
+int64_t mxfp4_colwise_scale_rows_bound(int64_t rows, int64_t num_groups, int32_t block);
+
+/* Static English text of a status; never NULL. */
+const char* mxfp4_status_string(mxfp4_status status);
+
+/* MXFP4_ABI_VERSION of the loaded library. */
+int32_t mxfp4_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXFP4_H */

@@ -1,0 +1,1123 @@
+// mxfp4.cu -- sm_100a kernels and the C ABI of libmxfp4.so: MXFP4 block fake
+// quantisation (quantise-dequantise) and its straight-through-estimator
+// backward. The arithmetic follows amct pull request 264, "feat: MXFP4 QAT
+// fake-quant Linear (with STE)", mxfp4_qat/fake_quant.py (_block_scale,
+// _round_to_e2m1, _quant_dequant_torch, mxfp4_saturation_mask,
+// _MXFP4FakeQuantSTE) and the grouped column-wise blocking of MindSpore's
+// fake_w4a8_gmm_func.py (quantize_input, normalize_group_list).
+//
+// The work is a memory-bound block reduction plus an elementwise map, so no
+// tensor cores are used. Design:
+//  * tile kernel: a warp (block 32) or a CTA (block 128) owns a tile of
+//    `block` rows x 64..128 columns held in registers as 16-byte vectors. The
+//    row-wise block amax is a shuffle across the 4..32 lanes that share a
+//    row block, the column-wise amax a register max over the thread's rows,
+//    then a shuffle (and for block 128 a shared-memory step) across rows. One
+//    read of x therefore serves both directions. Loads are 128-bit read-only
+//    streaming loads, stores 128-bit streaming stores; grids are persistent
+//    (SM count x resident CTAs).
+//  * the block scale exponent comes from exponent/mantissa bits, with one fp32
+//    divide per block in PAGE mode (round(log2 r) = e + (mantissa >= that of
+//    sqrt 2), exact because no fp32 r lies on the rounding boundary);
+//  * an element's code index is the count of codebook midpoints <= |x/2^k|
+//    (a ladder of compares, ties up), the output sign(y)*code*2^k is formed
+//    as one exact fp32 multiply and narrowed to bf16 by dropping zero bits.
+//  * generic kernels (one thread per block, scalar accesses) serve shapes and
+//    pointers the vector path cannot (cols or ld not a multiple of 16 bytes,
+//    unaligned buffers).
+#include <cuda_runtime.h>
+
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "mxfp4.h"
+
+namespace mxfp4 {
+
+constexpr unsigned FULL = 0xFFFFFFFFu;
+constexpr uint32_t QNAN32 = 0x7FC00000u;
+constexpr int NTHREADS = 256;
+
+struct KArgs {
+    const void* x;
+    int64_t rows, cols, ld;
+    float sf;
+    int32_t mode;
+    int32_t grad_dir;  // 0, MXFP4_ROWWISE or MXFP4_COLWISE
+    void* y_row;
+    void* y_col;
+    int64_t ld_y;
+    uint8_t* codes_row;
+    uint8_t* scales_row;
+    uint8_t* mask_row;
+    uint8_t* codes_col;
+    uint8_t* scales_col;
+    uint8_t* mask_col;
+    const void* g_out;
+    void* g_in;
+    int64_t ld_g;
+    const int64_t* group_list;
+    int32_t num_groups;
+    int32_t gl_type;
+    int32_t* status;
+    uint32_t n_ct;  // column tiles of the tile kernel
+};
+
+// ---------------------------------------------------------------------------
+// Per-block parameters
+// ---------------------------------------------------------------------------
+
+struct BP {
+    float inv;      // 2^-k
+    float scale;    // 2^k
+    uint32_t lim;   // fp32 bits of fl(6 * 2^k); +inf bits once it overflows
+    uint32_t nanm;  // all ones for a non-finite block
+    uint32_t e8;    // E8M0 byte
+};
+
+// fp32 bits of 2^k for k in [-127, 127] (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ uint32_t pow2_bits(int k)
+{
+    return k >= -126 ? (uint32_t)(k + 127) << 23 : 0x00400000u;
+}
+
+// A = fp32 bits of the block's max |x| (integer max of sign-cleared bits, so a
+// NaN anywhere gives A > 0x7F800000 and an inf gives A == 0x7F800000).
+__device__ __forceinline__ BP block_params(uint32_t A, int mode, float sf)
+{
+    int k;
+    bool special = A >= 0x7F800000u;
+    if (mode == MXFP4_SCALE_FLOOR) {
+        // floor(log2 amax) - 2 from the biased exponent; subnormal and zero
+        // amax have a biased exponent of 0 and saturate at -127.
+        k = max((int)(A >> 23) - 129, -127);
+    } else {
+        // r = max(fl(amax / sf), 2^-30) is a normal fp32 number; round(log2 r)
+        // is its exponent plus one when its significand is at or above the
+        // first fp32 significand above sqrt(2) (1.0110101000001001111001100..b;
+        // fraction field 0x3504F3 < frac(sqrt 2) < 0x3504F4).
+        float r = fmaxf(__fdiv_rn(__uint_as_float(A), sf), 0x1p-30f);
+        uint32_t rb = __float_as_uint(r);
+        k = (int)(rb >> 23) - 127 + ((rb & 0x7FFFFFu) >= 0x3504F4u ? 1 : 0);
+        special = special || k > 127;  // 2^128 overflows fp32: scale = inf
+    }
+    if (special)
+        k = 0;
+    BP p;
+    p.inv = __uint_as_float(pow2_bits(-k));
+    p.scale = __uint_as_float(pow2_bits(k));
+    p.lim = k >= 126 ? 0x7F800000u : (((uint32_t)(k + 129) << 23) | 0x00400000u);
+    p.nanm = special ? 0xFFFFFFFFu : 0u;
+    p.e8 = special ? 0xFFu : (uint32_t)(k + 127);
+    return p;
+}
+
+// One element: returns the fp32 bits of sign(y) * code * 2^k with y = x * 2^-k
+// (== fl(x / 2^k)), and the E2M1 nibble and saturation flag.
+__device__ __forceinline__ uint32_t qdq_elem(uint32_t xb, const BP& p, uint32_t& nib, uint32_t& sat)
+{
+    const float y = __fmul_rn(__uint_as_float(xb), p.inv);
+    const float a = fabsf(y);
+    const uint32_t i = (uint32_t)(a >= 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a >= 1.25f) +
+                       (uint32_t)(a >= 1.75f) + (uint32_t)(a >= 2.5f) + (uint32_t)(a >= 3.5f) +
+                       (uint32_t)(a >= 5.0f);
+    // code magnitude as fp32 bits: 0, 0.5, then (i << 22) + 0x3F000000 gives
+    // 1, 1.5, 2, 3, 4, 6 for i = 2..7 (two significant bits per binade)
+    const uint32_t cb = i >= 2u ? (i << 22) + 0x3F000000u : (i == 1u ? 0x3F000000u : 0u);
+    const uint32_t neg = y < 0.0f ? 0x80000000u : 0u;  // sign(-0) and sign(+0) are 0
+    const float o = __fmul_rn(__uint_as_float(cb | neg), p.scale);
+    nib = (neg >> 28) | i;
+    sat = (xb & 0x7FFFFFFFu) > p.lim ? 1u : 0u;
+    return __float_as_uint(o);
+}
+
+// ---------------------------------------------------------------------------
+// 16-byte vectors
+// ---------------------------------------------------------------------------
+
+template <int VEC>
+struct Vec;
+
+template <>
+struct Vec<8> {  // bf16 x 8
+    static __device__ __forceinline__ void unpack(const uint4& v, uint32_t (&xb)[8])
+    {
+        xb[0] = v.x << 16; xb[1] = v.x & 0xFFFF0000u;
+        xb[2] = v.y << 16; xb[3] = v.y & 0xFFFF0000u;
+        xb[4] = v.z << 16; xb[5] = v.z & 0xFFFF0000u;
+        xb[6] = v.w << 16; xb[7] = v.w & 0xFFFF0000u;
+    }
+    // The dequantised values have at most two significant bits and are >= 2^-128
+    // in magnitude, so their bf16 narrowing is exact: keep the top halves.
+    static __device__ __forceinline__ uint4 pack(const uint32_t (&ob)[8])
+    {
+        uint4 r;
+        r.x = __byte_perm(ob[0], ob[1], 0x7632);
+        r.y = __byte_perm(ob[2], ob[3], 0x7632);
+        r.z = __byte_perm(ob[4], ob[5], 0x7632);
+        r.w = __byte_perm(ob[6], ob[7], 0x7632);
+        return r;
+    }
+    // zero the elements whose bit is set in m (8 bits)
+    static __device__ __forceinline__ uint4 mask_out(const uint4& g, uint32_t m)
+    {
+        auto half = [](uint32_t w, uint32_t two) {
+            uint32_t z = ((two & 1u) ? 0x0000FFFFu : 0u) | ((two & 2u) ? 0xFFFF0000u : 0u);
+            return w & ~z;
+        };
+        uint4 r;
+        r.x = half(g.x, m);
+        r.y = half(g.y, m >> 2);
+        r.z = half(g.z, m >> 4);
+        r.w = half(g.w, m >> 6);
+        return r;
+    }
+};
+
+template <>
+struct Vec<4> {  // fp32 x 4
+    static __device__ __forceinline__ void unpack(const uint4& v, uint32_t (&xb)[4])
+    {
+        xb[0] = v.x; xb[1] = v.y; xb[2] = v.z; xb[3] = v.w;
+    }
+    static __device__ __forceinline__ uint4 pack(const uint32_t (&ob)[4])
+    {
+        return make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    }
+    static __device__ __forceinline__ uint4 mask_out(const uint4& g, uint32_t m)
+    {
+        return make_uint4((m & 1u) ? 0u : g.x, (m & 2u) ? 0u : g.y, (m & 4u) ? 0u : g.z,
+                          (m & 8u) ? 0u : g.w);
+    }
+};
+
+__device__ __forceinline__ uint4 ld_stream(const void* p)
+{
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_stream(void* p, const uint4& v)
+{
+    __stcs(reinterpret_cast<uint4*>(p), v);
+}
+
+// ---------------------------------------------------------------------------
+// group_list plan, built by every CTA in shared memory
+// ---------------------------------------------------------------------------
+
+// Writes s_rst[g] = sum_{j<g} n_j and s_bpre[g] = sum_{j<g} ceil(n_j / BS) for
+// g = 0..G and returns S = s_bpre[G], or -1 when the list is not a partition
+// of [0, rows): a negative count, a decreasing offset, or a wrong total.
+// Every thread of the CTA must call it.
+template <int BS>
+__device__ int64_t build_plan(const KArgs& a, int32_t* s_bpre, int32_t* s_rst)
+{
+    __shared__ long long s_wr[NTHREADS / 32], s_wb[NTHREADS / 32];
+    __shared__ int s_bad;
+    const int G = a.num_groups;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = (G + NTHREADS - 1) / NTHREADS;
+    const int g0 = min(G, tid * per), g1 = min(G, g0 + per);
+    if (tid == 0)
+        s_bad = 0;
+    __syncthreads();
+
+    long long lr = 0, lb = 0;
+    bool bad = false;
+    long long prev = (a.gl_type == 0 && g0 > 0) ? (long long)a.group_list[g0 - 1] : 0;
+    for (int g = g0; g < g1; ++g) {
+        long long v = a.group_list[g];
+        long long n = a.gl_type == 1 ? v : v - prev;
+        prev = v;
+        if (n < 0 || n > a.rows) {
+            bad = true;
+            n = 0;
+        }
+        lr += n;
+        lb += (n + BS - 1) / BS;
+    }
+    long long ir = lr, ib = lb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        long long tr = __shfl_up_sync(FULL, ir, o);
+        long long tb = __shfl_up_sync(FULL, ib, o);
+        if (lane >= o) {
+            ir += tr;
+            ib += tb;
+        }
+    }
+    if (lane == 31) {
+        s_wr[warp] = ir;
+        s_wb[warp] = ib;
+    }
+    if (bad)
+        atomicOr(&s_bad, 1);
+    __syncthreads();
+    long long er = ir - lr, eb = ib - lb, tot_r = 0, tot_b = 0;
+    for (int w = 0; w < NTHREADS / 32; ++w) {
+        if (w < warp) {
+            er += s_wr[w];
+            eb += s_wb[w];
+        }
+        tot_r += s_wr[w];
+        tot_b += s_wb[w];
+    }
+    prev = (a.gl_type == 0 && g0 > 0) ? (long long)a.group_list[g0 - 1] : 0;
+    for (int g = g0; g < g1; ++g) {
+        long long v = a.group_list[g];
+        long long n = a.gl_type == 1 ? v : v - prev;
+        prev = v;
+        if (n < 0 || n > a.rows)
+            n = 0;
+        s_rst[g] = (int32_t)er;
+        s_bpre[g] = (int32_t)eb;
+        er += n;
+        eb += (n + BS - 1) / BS;
+    }
+    if (tid == 0) {
+        s_rst[G] = (int32_t)tot_r;
+        s_bpre[G] = (int32_t)tot_b;
+    }
+    __syncthreads();
+    const bool ok = !s_bad && tot_r == a.rows;
+    return ok ? (int64_t)tot_b : -1;
+}
+
+// Row-block rb -> first row and row count, for a plan built by build_plan.
+__device__ __forceinline__ void plan_lookup(const int32_t* s_bpre, const int32_t* s_rst, int G,
+                                            uint32_t rb, int bs, int64_t& row0, int& nrows)
+{
+    int lo = 0, hi = G - 1;  // largest g with s_bpre[g] <= rb
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if ((uint32_t)s_bpre[mid] <= rb)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    row0 = (int64_t)s_rst[lo] + (int64_t)(rb - (uint32_t)s_bpre[lo]) * bs;
+    nrows = (int)min((int64_t)bs, (int64_t)s_rst[lo + 1] - row0);
+}
+
+// ---------------------------------------------------------------------------
+// Tile kernel (vector path)
+// ---------------------------------------------------------------------------
+
+// T-size: 2 (bf16) or 4 (fp32) bytes. LC lanes across columns (16 bytes each),
+// LR = 32/LC lanes across rows, RPT rows per thread, WR warps down the tile.
+// A tile is BS rows (one column-wise block; a group tail may be shorter) by
+// LC*VEC columns.
+template <int ESZ, int BS, int LC, int RPT, int WR, bool ROW, bool COL, bool GROUPS, bool GRAD>
+__global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
+{
+    constexpr int VEC = 16 / ESZ;
+    constexpr int LR = 32 / LC;
+    constexpr int TC = LC * VEC;
+    constexpr int NWG = (NTHREADS / 32) / WR;
+    constexpr int BL = BS / VEC;  // lanes sharing one row-wise block
+    static_assert(LR * RPT * WR == BS, "tile rows must equal the block");
+    static_assert(!ROW || (LC % BL == 0), "a row-wise block must sit in one warp row");
+    static_assert(WR == 1 || WR == NTHREADS / 32, "a multi-warp tile takes the whole CTA");
+    using V = Vec<VEC>;
+
+    extern __shared__ int32_t s_plan[];
+    __shared__ uint32_t s_am[(COL && WR > 1) ? WR * TC : 1];
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int wg = warp / WR, wr = warp - wg * WR;
+    const int lc = lane % LC, lr = lane / LC;
+
+    uint32_t S;
+    int32_t* s_bpre = s_plan;
+    int32_t* s_rst = s_plan + (GROUPS ? a.num_groups + 1 : 0);
+    if constexpr (GROUPS) {
+        const int64_t s = build_plan<BS>(a, s_bpre, s_rst);
+        if (blockIdx.x == 0 && threadIdx.x == 0 && a.status)
+            *a.status = s < 0 ? MXFP4_EINVAL : MXFP4_OK;
+        if (s < 0)
+            return;
+        S = (uint32_t)s;
+    } else {
+        S = (uint32_t)((a.rows + BS - 1) / BS);
+    }
+
+    const char* xp = static_cast<const char*>(a.x);
+    const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8, nblk = (a.cols + BS - 1) / BS;
+    const uint32_t ntiles = S * a.n_ct;
+    const uint32_t tstride = gridDim.x * NWG;
+
+    for (uint32_t t = blockIdx.x * NWG + wg; t < ntiles; t += tstride) {
+        const uint32_t rb = t / a.n_ct, ct = t - rb * a.n_ct;
+        int64_t row0;
+        int nrows;
+        if constexpr (GROUPS) {
+            plan_lookup(s_bpre, s_rst, a.num_groups, rb, BS, row0, nrows);
+        } else {
+            row0 = (int64_t)rb * BS;
+            nrows = (int)min((int64_t)BS, a.rows - row0);
+        }
+        const int64_t col = (int64_t)ct * TC + lc * VEC;
+        const bool colok = col < a.cols;
+
+        uint4 d[RPT];
+        uint4 gv[GRAD ? RPT : 1];
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const int r = i * (LR * WR) + wr * LR + lr;
+            d[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (colok && r < nrows)
+                d[i] = ld_stream(xp + ((row0 + r) * a.ld + col) * ESZ);
+            if constexpr (GRAD) {
+                gv[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (colok && r < nrows)
+                    gv[i] = ld_stream(static_cast<const char*>(a.g_out) + ((row0 + r) * a.ld_g + col) * ESZ);
+            }
+        }
+
+        uint32_t satr[ROW ? RPT : 1];
+        uint32_t satc[COL ? RPT : 1];
+
+        if constexpr (ROW) {
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const int r = i * (LR * WR) + wr * LR + lr;
+                const bool ok = colok && r < nrows;
+                const int64_t row = row0 + r;
+                uint32_t xb[VEC];
+                V::unpack(d[i], xb);
+                uint32_t am = 0;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    am = max(am, xb[e] & 0x7FFFFFFFu);
+#pragma unroll
+                for (int o = 1; o < BL; o <<= 1)
+                    am = max(am, __shfl_xor_sync(FULL, am, o));
+                const BP p = block_params(am, a.mode, a.sf);
+                uint32_t ob[VEC];
+                uint32_t nibs = 0, sats = 0;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    uint32_t nb, st;
+                    ob[e] = qdq_elem(xb[e], p, nb, st);
+                    ob[e] = p.nanm ? QNAN32 : ob[e];
+                    nibs |= nb << (4 * e);
+                    sats |= st << e;
+                }
+                nibs &= ~p.nanm;
+                sats &= ~p.nanm;
+                satr[i] = sats;
+                if constexpr (VEC == 4) {  // two lanes form one mask byte
+                    const uint32_t other = __shfl_xor_sync(FULL, sats, 1);
+                    sats = (lc & 1) ? 0u : (sats | (other << 4));
+                }
+                if (ok) {
+                    if (a.y_row)
+                        st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * ESZ, V::pack(ob));
+                    if (a.codes_row) {
+                        if constexpr (VEC == 8)
+                            *reinterpret_cast<uint32_t*>(a.codes_row + row * cstride + col / 2) = nibs;
+                        else
+                            *reinterpret_cast<uint16_t*>(a.codes_row + row * cstride + col / 2) = (uint16_t)nibs;
+                    }
+                    if (a.mask_row && (VEC == 8 || !(lc & 1)))
+                        a.mask_row[row * mstride + col / 8] = (uint8_t)sats;
+                    if (a.scales_row && (lc % BL) == 0)
+                        a.scales_row[row * nblk + col / BS] = (uint8_t)p.e8;
+                }
+            }
+        }
+
+        if constexpr (COL) {
+            uint32_t amc[VEC];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+                amc[e] = 0;
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                uint32_t xb[VEC];
+                V::unpack(d[i], xb);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    amc[e] = max(amc[e], xb[e] & 0x7FFFFFFFu);
+            }
+#pragma unroll
+            for (int o = LC; o < 32; o <<= 1) {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    amc[e] = max(amc[e], __shfl_xor_sync(FULL, amc[e], o));
+            }
+            if constexpr (WR > 1) {
+                if (lr == 0) {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e)
+                        s_am[wr * TC + lc * VEC + e] = amc[e];
+                }
+                __syncthreads();
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    uint32_t m = 0;
+#pragma unroll
+                    for (int w = 0; w < WR; ++w)
+                        m = max(m, s_am[w * TC + lc * VEC + e]);
+                    amc[e] = m;
+                }
+            }
+            BP pc[VEC];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+                pc[e] = block_params(amc[e], a.mode, a.sf);
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const int r = i * (LR * WR) + wr * LR + lr;
+                const bool ok = colok && r < nrows;
+                const int64_t row = row0 + r;
+                uint32_t xb[VEC];
+                V::unpack(d[i], xb);
+                uint32_t ob[VEC];
+                uint32_t nibs = 0, sats = 0;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    uint32_t nb, st;
+                    ob[e] = qdq_elem(xb[e], pc[e], nb, st);
+                    ob[e] = pc[e].nanm ? QNAN32 : ob[e];
+                    nibs |= (nb & ~pc[e].nanm) << (4 * e);
+                    sats |= (st & ~pc[e].nanm) << e;
+                }
+                satc[i] = sats;
+                if constexpr (VEC == 4) {
+                    const uint32_t other = __shfl_xor_sync(FULL, sats, 1);
+                    sats = (lc & 1) ? 0u : (sats | (other << 4));
+                }
+                if (ok) {
+                    if (a.y_col)
+                        st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * ESZ, V::pack(ob));
+                    if (a.codes_col) {
+                        if constexpr (VEC == 8)
+                            *reinterpret_cast<uint32_t*>(a.codes_col + row * cstride + col / 2) = nibs;
+                        else
+                            *reinterpret_cast<uint16_t*>(a.codes_col + row * cstride + col / 2) = (uint16_t)nibs;
+                    }
+                    if (a.mask_col && (VEC == 8 || !(lc & 1)))
+                        a.mask_col[row * mstride + col / 8] = (uint8_t)sats;
+                }
+            }
+            if (a.scales_col && lr == 0 && wr == 0 && colok) {
+                uint8_t* sp = a.scales_col + (int64_t)rb * a.cols + col;
+                if constexpr (VEC == 8) {
+                    uint2 v;
+                    v.x = pc[0].e8 | (pc[1].e8 << 8) | (pc[2].e8 << 16) | (pc[3].e8 << 24);
+                    v.y = pc[4].e8 | (pc[5].e8 << 8) | (pc[6].e8 << 16) | (pc[7].e8 << 24);
+                    *reinterpret_cast<uint2*>(sp) = v;
+                } else {
+                    *reinterpret_cast<uint32_t*>(sp) =
+                        pc[0].e8 | (pc[1].e8 << 8) | (pc[2].e8 << 16) | (pc[3].e8 << 24);
+                }
+            }
+            if constexpr (WR > 1)
+                __syncthreads();  // s_am is rewritten by the next tile
+        }
+
+        if constexpr (GRAD) {
+#pragma unroll
+            for (int i = 0; i < RPT; ++i) {
+                const int r = i * (LR * WR) + wr * LR + lr;
+                if (!(colok && r < nrows))
+                    continue;
+                uint32_t m = 0;
+                if constexpr (ROW)
+                    if (a.grad_dir == MXFP4_ROWWISE)
+                        m = satr[i];
+                if constexpr (COL)
+                    if (a.grad_dir == MXFP4_COLWISE)
+                        m = satc[i];
+                st_stream(static_cast<char*>(a.g_in) + ((row0 + r) * a.ld_g + col) * ESZ, V::mask_out(gv[i], m));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Generic kernels (scalar path for any alignment / leading dimension)
+// ---------------------------------------------------------------------------
+
+template <int ESZ>
+__device__ __forceinline__ uint32_t load_bits(const void* base, int64_t i)
+{
+    if (ESZ == 2)
+        return (uint32_t)static_cast<const uint16_t*>(base)[i] << 16;
+    return static_cast<const uint32_t*>(base)[i];
+}
+
+template <int ESZ>
+__device__ __forceinline__ void store_bits(void* base, int64_t i, uint32_t v)
+{
+    if (ESZ == 2)
+        static_cast<uint16_t*>(base)[i] = (uint16_t)(v >> 16);
+    else
+        static_cast<uint32_t*>(base)[i] = v;
+}
+
+// One thread per (row, row-wise block).
+template <int ESZ, int BS, bool GRAD>
+__global__ void __launch_bounds__(NTHREADS) generic_row_kernel(const KArgs a)
+{
+    const int64_t nblk = (a.cols + BS - 1) / BS;
+    const int64_t total = a.rows * nblk;
+    const int64_t cstride = (a.cols + 1) / 2, mstride = (a.cols + 7) / 8;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = idx / nblk, b = idx - row * nblk;
+        const int64_t c0 = b * BS;
+        const int n = (int)min((int64_t)BS, a.cols - c0);
+        const int64_t xo = row * a.ld + c0;
+        uint32_t am = 0;
+        for (int j = 0; j < n; ++j)
+            am = max(am, load_bits<ESZ>(a.x, xo + j) & 0x7FFFFFFFu);
+        const BP p = block_params(am, a.mode, a.sf);
+        uint32_t nacc = 0, sacc = 0;
+        for (int j = 0; j < n; ++j) {
+            uint32_t nb, st;
+            uint32_t ob = qdq_elem(load_bits<ESZ>(a.x, xo + j), p, nb, st);
+            if (p.nanm) {
+                ob = QNAN32;
+                nb = 0;
+                st = 0;
+            }
+            if (a.y_row)
+                store_bits<ESZ>(a.y_row, row * a.ld_y + c0 + j, ob);
+            nacc |= nb << (4 * (j & 1));
+            sacc |= st << (j & 7);
+            if (a.codes_row && ((j & 1) || j == n - 1))
+                a.codes_row[row * cstride + (c0 + j) / 2] = (uint8_t)nacc;
+            if ((j & 1) || j == n - 1)
+                nacc = 0;
+            if (a.mask_row && ((j & 7) == 7 || j == n - 1))
+                a.mask_row[row * mstride + (c0 + j) / 8] = (uint8_t)sacc;
+            if ((j & 7) == 7 || j == n - 1)
+                sacc = 0;
+            if (GRAD && a.grad_dir == MXFP4_ROWWISE) {
+                const int64_t gi = row * a.ld_g + c0 + j;
+                store_bits<ESZ>(a.g_in, gi, st ? 0u : load_bits<ESZ>(a.g_out, gi));
+            }
+        }
+        if (a.scales_row)
+            a.scales_row[row * nblk + b] = (uint8_t)p.e8;
+    }
+}
+
+// One thread per (column-wise block, 8 adjacent columns): whole code and mask
+// bytes are owned by one thread.
+template <int ESZ, int BS, bool GROUPS, bool GRAD>
+__global__ void __launch_bounds__(NTHREADS) generic_col_kernel(const KArgs a)
+{
+    extern __shared__ int32_t s_plan[];
+    int32_t* s_bpre = s_plan;
+    int32_t* s_rst = s_plan + (GROUPS ? a.num_groups + 1 : 0);
+    int64_t S;
+    if (GROUPS) {
+        S = build_plan<BS>(a, s_bpre, s_rst);
+        if (blockIdx.x == 0 && threadIdx.x == 0 && a.status)
+            *a.status = S < 0 ? MXFP4_EINVAL : MXFP4_OK;
+        if (S < 0)
+            return;
+    } else {
+        S = (a.rows + BS - 1) / BS;
+    }
+    const int64_t noct = (a.cols + 7) / 8;
+    const int64_t total = S * noct;
+    const int64_t cstride = (a.cols + 1) / 2, mstride = (a.cols + 7) / 8;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t rb = idx / noct, oc = idx - rb * noct;
+        int64_t row0;
+        int nrows;
+        if (GROUPS) {
+            plan_lookup(s_bpre, s_rst, a.num_groups, (uint32_t)rb, BS, row0, nrows);
+        } else {
+            row0 = rb * BS;
+            nrows = (int)min((int64_t)BS, a.rows - row0);
+        }
+        const int64_t c0 = oc * 8;
+        const int nc = (int)min((int64_t)8, a.cols - c0);
+        uint32_t am[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            am[c] = 0;
+        for (int r = 0; r < nrows; ++r) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c < nc)
+                    am[c] = max(am[c], load_bits<ESZ>(a.x, (row0 + r) * a.ld + c0 + c) & 0x7FFFFFFFu);
+        }
+        BP p[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            p[c] = block_params(am[c], a.mode, a.sf);
+        for (int r = 0; r < nrows; ++r) {
+            const int64_t row = row0 + r;
+            uint32_t nibs = 0, sats = 0;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                if (c >= nc)
+                    continue;
+                uint32_t nb, st;
+                uint32_t ob = qdq_elem(load_bits<ESZ>(a.x, row * a.ld + c0 + c), p[c], nb, st);
+                if (p[c].nanm) {
+                    ob = QNAN32;
+                    nb = 0;
+                    st = 0;
+                }
+                if (a.y_col)
+                    store_bits<ESZ>(a.y_col, row * a.ld_y + c0 + c, ob);
+                nibs |= nb << (4 * c);
+                sats |= st << c;
+                if (GRAD && a.grad_dir == MXFP4_COLWISE) {
+                    const int64_t gi = row * a.ld_g + c0 + c;
+                    store_bits<ESZ>(a.g_in, gi, st ? 0u : load_bits<ESZ>(a.g_out, gi));
+                }
+            }
+            if (a.codes_col) {
+                for (int j = 0; j < (nc + 1) / 2; ++j)
+                    a.codes_col[row * cstride + c0 / 2 + j] = (uint8_t)(nibs >> (8 * j));
+            }
+            if (a.mask_col)
+                a.mask_col[row * mstride + oc] = (uint8_t)sats;
+        }
+        if (a.scales_col) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c < nc)
+                    a.scales_col[rb * a.cols + c0 + c] = (uint8_t)p[c].e8;
+        }
+    }
+}
+
+// grad_in = grad_out with +0 where the saved bit is set (mask may be NULL for
+// the plain STE copy). One thread per (row, 8 columns).
+template <int ESZ>
+__global__ void __launch_bounds__(NTHREADS)
+    ste_mask_kernel(int64_t rows, int64_t cols, const void* g_out, void* g_in, int64_t ld_g,
+                    const uint8_t* mask, int vec)
+{
+    const int64_t noct = (cols + 7) / 8, mstride = noct;
+    const int64_t total = rows * noct;
+    for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = idx / noct, oc = idx - row * noct;
+        const uint32_t m = mask ? (uint32_t)mask[row * mstride + oc] : 0u;
+        const int64_t base = row * ld_g + oc * 8;
+        if (vec) {
+            const char* src = static_cast<const char*>(g_out) + base * ESZ;
+            char* dst = static_cast<char*>(g_in) + base * ESZ;
+            if (ESZ == 2) {
+                st_stream(dst, Vec<8>::mask_out(ld_stream(src), m));
+            } else {
+                st_stream(dst, Vec<4>::mask_out(ld_stream(src), m));
+                st_stream(dst + 16, Vec<4>::mask_out(ld_stream(src + 16), m >> 4));
+            }
+        } else {
+            const int nc = (int)min((int64_t)8, cols - oc * 8);
+            for (int c = 0; c < nc; ++c)
+                store_bits<ESZ>(g_in, base + c, ((m >> c) & 1u) ? 0u : load_bits<ESZ>(g_out, base + c));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+struct DevInfo {
+    int sms = 0;
+};
+
+static std::mutex g_mu;
+
+static int device_sms()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return -1;
+    static DevInfo info[64];
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev < 0 || dev >= 64)
+        return -1;
+    if (info[dev].sms == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return -1;
+        info[dev].sms = n;
+    }
+    return info[dev].sms;
+}
+
+// Resident CTAs per SM of `fn`, cached per (device, kernel).
+static int occupancy(const void* fn, size_t smem)
+{
+    struct Entry {
+        const void* fn;
+        int dev;
+        size_t smem;
+        int occ;
+    };
+    static Entry cache[512];
+    static int n = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return -1;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        for (int i = 0; i < n; ++i)
+            if (cache[i].fn == fn && cache[i].dev == dev && cache[i].smem == smem)
+                return cache[i].occ;
+    }
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NTHREADS, smem) != cudaSuccess)
+        return -1;
+    if (occ < 1)
+        occ = 1;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (n < 512)
+        cache[n++] = Entry{fn, dev, smem, occ};
+    return occ;
+}
+
+static inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+typedef void (*KernelFn)(const KArgs);
+
+template <int ESZ, int BS, int LC, int RPT, int WR, bool GRAD>
+static KernelFn pick_tile(bool row, bool col, bool groups)
+{
+    if (row && col)
+        return groups ? qdq_tile_kernel<ESZ, BS, LC, RPT, WR, true, true, true, GRAD>
+                      : qdq_tile_kernel<ESZ, BS, LC, RPT, WR, true, true, false, GRAD>;
+    if (col)
+        return groups ? qdq_tile_kernel<ESZ, BS, LC, RPT, WR, false, true, true, GRAD>
+                      : qdq_tile_kernel<ESZ, BS, LC, RPT, WR, false, true, false, GRAD>;
+    return qdq_tile_kernel<ESZ, BS, LC, RPT, WR, true, false, false, GRAD>;
+}
+
+// Tile shape per (element size, block): LC lanes across, RPT rows per thread,
+// WR warps down the tile.
+template <int ESZ, int BS>
+struct TileShape;
+template <> struct TileShape<2, 32> { static constexpr int LC = 8, RPT = 8, WR = 1; };
+template <> struct TileShape<2, 128> { static constexpr int LC = 16, RPT = 8, WR = 8; };
+template <> struct TileShape<4, 32> { static constexpr int LC = 8, RPT = 8, WR = 1; };
+template <> struct TileShape<4, 128> { static constexpr int LC = 32, RPT = 16, WR = 8; };
+
+template <int ESZ, int BS>
+static KernelFn pick_tile_shape(bool row, bool col, bool groups, bool grad, int& tc, int& nwg)
+{
+    using TS = TileShape<ESZ, BS>;
+    tc = TS::LC * (16 / ESZ);
+    nwg = (NTHREADS / 32) / TS::WR;
+    return grad ? pick_tile<ESZ, BS, TS::LC, TS::RPT, TS::WR, true>(row, col, groups)
+                : pick_tile<ESZ, BS, TS::LC, TS::RPT, TS::WR, false>(row, col, groups);
+}
+
+static KernelFn pick_generic_row(int esz, int bs, bool grad)
+{
+    if (esz == 2)
+        return bs == 32 ? (grad ? generic_row_kernel<2, 32, true> : generic_row_kernel<2, 32, false>)
+                        : (grad ? generic_row_kernel<2, 128, true> : generic_row_kernel<2, 128, false>);
+    return bs == 32 ? (grad ? generic_row_kernel<4, 32, true> : generic_row_kernel<4, 32, false>)
+                    : (grad ? generic_row_kernel<4, 128, true> : generic_row_kernel<4, 128, false>);
+}
+
+template <int ESZ, int BS>
+static KernelFn pick_generic_col_bs(bool groups, bool grad)
+{
+    if (groups)
+        return grad ? generic_col_kernel<ESZ, BS, true, true> : generic_col_kernel<ESZ, BS, true, false>;
+    return grad ? generic_col_kernel<ESZ, BS, false, true> : generic_col_kernel<ESZ, BS, false, false>;
+}
+
+static KernelFn pick_generic_col(int esz, int bs, bool groups, bool grad)
+{
+    if (esz == 2)
+        return bs == 32 ? pick_generic_col_bs<2, 32>(groups, grad) : pick_generic_col_bs<2, 128>(groups, grad);
+    return bs == 32 ? pick_generic_col_bs<4, 32>(groups, grad) : pick_generic_col_bs<4, 128>(groups, grad);
+}
+
+static mxfp4_status launch(KernelFn fn, int64_t work_units, size_t smem, const KArgs& k, cudaStream_t s)
+{
+    const int sms = device_sms();
+    const int occ = occupancy((const void*)fn, smem);
+    if (sms <= 0 || occ <= 0)
+        return MXFP4_ECUDA;
+    int64_t grid = (int64_t)sms * occ;
+    if (work_units < grid)
+        grid = work_units < 1 ? 1 : work_units;
+    fn<<<(unsigned)grid, NTHREADS, smem, s>>>(k);
+    return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
+}
+
+static mxfp4_status check_geometry(const mxfp4_qdq_args* a)
+{
+    if (!a)
+        return MXFP4_EINVAL;
+    if (a->dtype != MXFP4_F32 && a->dtype != MXFP4_BF16)
+        return MXFP4_EINVAL;
+    if (a->block <= 0)
+        return MXFP4_EINVAL;
+    if (a->block != 32 && a->block != 128)
+        return MXFP4_EUNSUPPORTED;
+    if (!(a->scale_factor > 0.0f) || !isfinite(a->scale_factor))
+        return MXFP4_EINVAL;
+    if (a->scale_mode != MXFP4_SCALE_PAGE && a->scale_mode != MXFP4_SCALE_FLOOR)
+        return MXFP4_EINVAL;
+    if (a->rows < 0 || a->cols < 0)
+        return MXFP4_EINVAL;
+    if (a->rows > INT32_MAX || a->cols > INT32_MAX)
+        return MXFP4_EUNSUPPORTED;
+    if (a->dirs == 0 || (a->dirs & ~(MXFP4_ROWWISE | MXFP4_COLWISE)))
+        return MXFP4_EINVAL;
+    if (a->group_list) {
+        if (a->num_groups < 1)
+            return MXFP4_EINVAL;
+        if (a->num_groups > MXFP4_MAX_GROUPS)
+            return MXFP4_EUNSUPPORTED;
+        if (a->group_list_type != 0 && a->group_list_type != 1)
+            return MXFP4_EINVAL;
+        if (!aligned(a->group_list, 8))
+            return MXFP4_EINVAL;
+    }
+    return MXFP4_OK;
+}
+
+// Validates, then queues the forward (and the fused backward when g_in is set).
+static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_in, int64_t ld_g,
+                            uint32_t grad_dir, cudaStream_t s)
+{
+    mxfp4_status st = check_geometry(A);
+    if (st != MXFP4_OK)
+        return st;
+    const bool row = A->dirs & MXFP4_ROWWISE, col = A->dirs & MXFP4_COLWISE;
+    const bool grad = g_in != nullptr;
+    const int esz = A->dtype == MXFP4_BF16 ? 2 : 4;
+    if (grad) {
+        if (!g_out || (grad_dir != MXFP4_ROWWISE && grad_dir != MXFP4_COLWISE) || !(A->dirs & grad_dir))
+            return MXFP4_EINVAL;
+        if (ld_g < A->cols || !aligned(g_out, esz) || !aligned(g_in, esz))
+            return MXFP4_EINVAL;
+    }
+    const bool groups = col && A->group_list != nullptr;
+    if (A->rows == 0 || A->cols == 0) {
+        if (A->status && cudaMemsetAsync(A->status, 0, sizeof(int32_t), s) != cudaSuccess)
+            return MXFP4_ECUDA;
+        return MXFP4_OK;
+    }
+    if (!A->x || A->ld < A->cols || !aligned(A->x, esz))
+        return MXFP4_EINVAL;
+
+    KArgs k;
+    memset(&k, 0, sizeof(k));
+    k.x = A->x;
+    k.rows = A->rows;
+    k.cols = A->cols;
+    k.ld = A->ld;
+    k.sf = A->scale_factor;
+    k.mode = A->scale_mode;
+    k.grad_dir = grad ? (int32_t)grad_dir : 0;
+    if (row) {
+        k.y_row = A->y_row;
+        k.codes_row = A->codes_row;
+        k.scales_row = A->scales_row;
+        k.mask_row = A->mask_row;
+    }
+    if (col) {
+        k.y_col = A->y_col;
+        k.codes_col = A->codes_col;
+        k.scales_col = A->scales_col;
+        k.mask_col = A->mask_col;
+    }
+    k.ld_y = A->ld_y;
+    if ((k.y_row || k.y_col) && A->ld_y < A->cols)
+        return MXFP4_EINVAL;
+    if ((k.y_row && !aligned(k.y_row, esz)) || (k.y_col && !aligned(k.y_col, esz)))
+        return MXFP4_EINVAL;
+    k.g_out = g_out;
+    k.g_in = g_in;
+    k.ld_g = ld_g;
+    k.group_list = groups ? A->group_list : nullptr;
+    k.num_groups = groups ? (int32_t)A->num_groups : 0;
+    k.gl_type = A->group_list_type;
+    k.status = A->status;
+    if (A->status && !groups && cudaMemsetAsync(A->status, 0, sizeof(int32_t), s) != cudaSuccess)
+        return MXFP4_ECUDA;
+
+    const int vec = 16 / esz;
+    bool fast = aligned(A->x, 16) && A->ld % vec == 0 && A->cols % vec == 0;
+    for (void* y : {k.y_row, k.y_col})
+        if (y)
+            fast = fast && aligned(y, 16) && A->ld_y % vec == 0;
+    for (uint8_t* c : {k.codes_row, k.codes_col})
+        if (c)
+            fast = fast && aligned(c, vec / 2);
+    if (k.scales_col)
+        fast = fast && aligned(k.scales_col, vec);
+    if (grad)
+        fast = fast && aligned(g_out, 16) && aligned(g_in, 16) && ld_g % vec == 0;
+
+    const int bs = A->block;
+    const size_t plan_smem = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
+    const int64_t s_bound = groups ? A->rows / bs + A->num_groups : (A->rows + bs - 1) / bs;
+
+    if (fast) {
+        int tc = 0, nwg = 1;
+        KernelFn fn;
+        if (esz == 2)
+            fn = bs == 32 ? pick_tile_shape<2, 32>(row, col, groups, grad, tc, nwg)
+                          : pick_tile_shape<2, 128>(row, col, groups, grad, tc, nwg);
+        else
+            fn = bs == 32 ? pick_tile_shape<4, 32>(row, col, groups, grad, tc, nwg)
+                          : pick_tile_shape<4, 128>(row, col, groups, grad, tc, nwg);
+        const int64_t n_ct = (A->cols + tc - 1) / tc;
+        if (s_bound * n_ct >= (int64_t)INT32_MAX)
+            return MXFP4_EUNSUPPORTED;
+        k.n_ct = (uint32_t)n_ct;
+        return launch(fn, (s_bound * n_ct + nwg - 1) / nwg, plan_smem, k, s);
+    }
+
+    // generic path: one kernel per direction
+    if (row) {
+        KArgs kr = k;
+        kr.y_col = nullptr;
+        st = launch(pick_generic_row(esz, bs, grad && grad_dir == MXFP4_ROWWISE),
+                    (A->rows * ((A->cols + bs - 1) / bs) + NTHREADS - 1) / NTHREADS, 0, kr, s);
+        if (st != MXFP4_OK)
+            return st;
+    }
+    if (col) {
+        const int64_t units = s_bound * ((A->cols + 7) / 8);
+        st = launch(pick_generic_col(esz, bs, groups, grad && grad_dir == MXFP4_COLWISE),
+                    (units + NTHREADS - 1) / NTHREADS, plan_smem, k, s);
+    }
+    return st;
+}
+
+}  // namespace mxfp4
+
+using namespace mxfp4;
+
+extern "C" {
+
+mxfp4_status mxfp4_qdq_fwd(const mxfp4_qdq_args* args, mxfp4_stream_t stream)
+{
+    return run_qdq(args, nullptr, nullptr, 0, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mxfp4_status mxfp4_qdq_fwd_bwd(const mxfp4_qdq_args* args, const void* grad_out, void* grad_in,
+                               int64_t ld_grad, uint32_t grad_dir, mxfp4_stream_t stream)
+{
+    if (!grad_in)
+        return MXFP4_EINVAL;
+    return run_qdq(args, grad_out, grad_in, ld_grad, grad_dir, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mxfp4_status mxfp4_ste_bwd(const mxfp4_qdq_args* geom, const void* grad_out, void* grad_in,
+                           int64_t ld_grad, const uint8_t* saved_mask, int32_t clip_grad,
+                           mxfp4_stream_t stream)
+{
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (!geom || (geom->dirs != MXFP4_ROWWISE && geom->dirs != MXFP4_COLWISE))
+        return MXFP4_EINVAL;
+    if (geom->dtype != MXFP4_F32 && geom->dtype != MXFP4_BF16)
+        return MXFP4_EINVAL;
+    if (geom->rows < 0 || geom->cols < 0)
+        return MXFP4_EINVAL;
+    if (geom->rows > INT32_MAX || geom->cols > INT32_MAX)
+        return MXFP4_EUNSUPPORTED;
+    if (geom->rows == 0 || geom->cols == 0)
+        return MXFP4_OK;
+    const int esz = geom->dtype == MXFP4_BF16 ? 2 : 4;
+    if (!grad_out || !grad_in || ld_grad < geom->cols || !aligned(grad_out, esz) || !aligned(grad_in, esz))
+        return MXFP4_EINVAL;
+    if (clip_grad && !saved_mask) {
+        // saved-free: recompute the saturation of x in the same pass
+        mxfp4_qdq_args g = *geom;
+        g.y_row = g.y_col = nullptr;
+        g.codes_row = g.scales_row = g.mask_row = nullptr;
+        g.codes_col = g.scales_col = g.mask_col = nullptr;
+        return run_qdq(&g, grad_out, grad_in, ld_grad, geom->dirs, s);
+    }
+    if (!clip_grad && grad_in == grad_out)
+        return MXFP4_OK;
+    const int vec = (((uintptr_t)grad_out | (uintptr_t)grad_in) % 16 == 0) && (ld_grad % 8 == 0) &&
+                    (geom->cols % 8 == 0);
+    const int64_t units = geom->rows * ((geom->cols + 7) / 8);
+    const uint8_t* m = clip_grad ? saved_mask : nullptr;
+    const int sms = device_sms();
+    if (sms <= 0)
+        return MXFP4_ECUDA;
+    const void* fn = esz == 2 ? (const void*)ste_mask_kernel<2> : (const void*)ste_mask_kernel<4>;
+    const int occ = occupancy(fn, 0);
+    if (occ <= 0)
+        return MXFP4_ECUDA;
+    int64_t grid = (int64_t)sms * occ;
+    const int64_t need = (units + NTHREADS - 1) / NTHREADS;
+    if (need < grid)
+        grid = need;
+    if (esz == 2)
+        ste_mask_kernel<2><<<(unsigned)grid, NTHREADS, 0, s>>>(geom->rows, geom->cols, grad_out, grad_in,
+                                                              ld_grad, m, vec);
+    else
+        ste_mask_kernel<4><<<(unsigned)grid, NTHREADS, 0, s>>>(geom->rows, geom->cols, grad_out, grad_in,
+                                                              ld_grad, m, vec);
+    return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
+}
+
+int64_t mxfp4_colwise_scale_rows(const int64_t* host_group_list, int64_t num_groups,
+                                 int32_t group_list_type, int64_t rows, int32_t block)
+{
+    if (block <= 0 || rows < 0)
+        return -1;
+    if (!host_group_list)
+        return (rows + block - 1) / block;
+    if (num_groups < 1 || (group_list_type != 0 && group_list_type != 1))
+        return -1;
+    int64_t total = 0, prev = 0, s = 0;
+    for (int64_t g = 0; g < num_groups; ++g) {
+        const int64_t v = host_group_list[g];
+        const int64_t n = group_list_type == 1 ? v : v - prev;
+        prev = v;
+        if (n < 0 || n > rows)
+            return -1;
+        total += n;
+        s += (n + block - 1) / block;
+    }
+    return total == rows ? s : -1;
+}
+
+int64_t mxfp4_colwise_scale_rows_bound(int64_t rows, int64_t num_groups, int32_t block)
+{
+    if (block <= 0 || rows < 0)
+        return -1;
+    if (num_groups <= 0)
+        return (rows + block - 1) / block;
+    return rows / block + num_groups;
+}
+
+const char* mxfp4_status_string(mxfp4_status status)
+{
+    switch (status) {
+    case MXFP4_OK: return "ok";
+    case MXFP4_EINVAL: return "invalid argument";
+    case MXFP4_EUNSUPPORTED: return "unsupported argument";
+    case MXFP4_ECUDA: return "CUDA error";
+    }
+    return "unknown status";
+}
+
+int32_t mxfp4_abi_version(void) { return MXFP4_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,229 @@
+"""Torch-facing binding of libmxfp4: the C entry points under the same names.
+
+torch supplies device memory (output allocation) and the current CUDA stream;
+every byte of the computation runs in the library's kernels. Inputs must be
+CUDA tensors: there is no CPU path.
+
+Tensor conventions follow include/mxfp4.h: x is 2-D [rows, cols] with unit
+stride along cols (a 1-D tensor is one row); outputs are contiguous; masks are
+bit-packed [rows, ceil(cols/8)] uint8; codes are nibble pairs
+[rows, ceil(cols/2)] uint8; row-wise scales [rows, ceil(cols/block)] uint8;
+column-wise scales [S_bound, cols] uint8 (only the first S rows are written,
+S = mxfp4_colwise_scale_rows(...)).
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+from . import _abi
+
+_DTYPES = {torch.float32: _abi.F32, torch.bfloat16: _abi.BF16}
+_MODES = {"page": _abi.SCALE_PAGE, "floor": _abi.SCALE_FLOOR}
+_DIRS = {"rowwise": _abi.ROWWISE, "colwise": _abi.COLWISE}
+
+
+@dataclasses.dataclass
+class QDQResult:
+    y_row: torch.Tensor | None = None
+    y_col: torch.Tensor | None = None
+    codes_row: torch.Tensor | None = None
+    scales_row: torch.Tensor | None = None
+    mask_row: torch.Tensor | None = None
+    codes_col: torch.Tensor | None = None
+    scales_col: torch.Tensor | None = None
+    mask_col: torch.Tensor | None = None
+    status: torch.Tensor | None = None
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _as_2d(x: torch.Tensor, name: str = "x") -> torch.Tensor:
+    if x.ndim == 0:
+        raise ValueError(f"{name} must have at least 1 dimension")
+    if not x.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libmxfp4 has no CPU path)")
+    if x.dtype not in _DTYPES:
+        raise TypeError(f"{name} must be float32 or bfloat16, got {x.dtype}")
+    if x.ndim == 1:
+        x = x.unsqueeze(0)
+    elif x.ndim > 2:
+        x = x.reshape(-1, x.shape[-1])
+    if x.shape[-1] > 1 and x.stride(-1) != 1:
+        x = x.contiguous()
+    return x
+
+
+def _ld(t: torch.Tensor) -> int:
+    return max(t.stride(0), t.shape[1]) if t.shape[0] > 1 else t.shape[1]
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _group_args(group_list, group_list_type: int, device):
+    if group_list is None:
+        return None, 0
+    gl = group_list
+    if not isinstance(gl, torch.Tensor):
+        gl = torch.tensor(list(gl), dtype=torch.int64, device=device)
+    if gl.dtype != torch.int64 or not gl.is_cuda or gl.ndim != 1:
+        raise ValueError("group_list must be a 1-D int64 CUDA tensor")
+    return gl.contiguous(), gl.numel()
+
+
+def make_args(x: torch.Tensor, *, block: int, scale_factor: float, scale_mode: str, dirs: int,
+              group_list=None, group_list_type: int = 0, status: torch.Tensor | None = None) -> _abi.QdqArgs:
+    a = _abi.QdqArgs()
+    a.x = x.data_ptr()
+    a.dtype = _DTYPES[x.dtype]
+    a.block = int(block)
+    a.rows, a.cols = int(x.shape[0]), int(x.shape[1])
+    a.ld = _ld(x)
+    a.scale_factor = float(scale_factor)
+    if scale_mode not in _MODES:
+        raise ValueError(f"scale_mode must be one of {tuple(_MODES)}, got {scale_mode!r}")
+    a.scale_mode = _MODES[scale_mode]
+    a.dirs = dirs
+    if group_list is not None:
+        a.group_list = group_list.data_ptr()
+        a.num_groups = group_list.numel()
+        a.group_list_type = int(group_list_type)
+    a.status = _ptr(status)
+    return a
+
+
+def colwise_scale_rows_bound(rows: int, num_groups: int, block: int) -> int:
+    return _abi.mxfp4_colwise_scale_rows_bound(rows, num_groups, block)
+
+
+def mxfp4_colwise_scale_rows(group_list, group_list_type: int, rows: int, block: int) -> int:
+    """Exact number of column-wise scale rows (copies a device group_list to the host)."""
+    if isinstance(group_list, torch.Tensor):
+        group_list = group_list.cpu().tolist()
+    return _abi.mxfp4_colwise_scale_rows(group_list, group_list_type, rows, block)
+
+
+def alloc_outputs(x: torch.Tensor, *, block: int, rowwise: bool, colwise: bool, num_groups: int,
+                  emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
+                  with_status: bool = False) -> QDQResult:
+    rows, cols = x.shape
+    dev = x.device
+    r = QDQResult()
+    u8 = dict(dtype=torch.uint8, device=dev)
+    if rowwise:
+        if emit_values:
+            r.y_row = torch.empty((rows, cols), dtype=x.dtype, device=dev)
+        if emit_codes:
+            r.codes_row = torch.empty((rows, (cols + 1) // 2), **u8)
+            r.scales_row = torch.empty((rows, (cols + block - 1) // block), **u8)
+        if emit_mask:
+            r.mask_row = torch.empty((rows, (cols + 7) // 8), **u8)
+    if colwise:
+        if emit_values:
+            r.y_col = torch.empty((rows, cols), dtype=x.dtype, device=dev)
+        if emit_codes:
+            r.codes_col = torch.empty((rows, (cols + 1) // 2), **u8)
+            r.scales_col = torch.empty((colwise_scale_rows_bound(rows, num_groups, block), cols), **u8)
+        if emit_mask:
+            r.mask_col = torch.empty((rows, (cols + 7) // 8), **u8)
+    if with_status:
+        r.status = torch.empty((1,), dtype=torch.int32, device=dev)
+    return r
+
+
+def _fill_outputs(a: _abi.QdqArgs, r: QDQResult) -> None:
+    a.y_row, a.y_col = _ptr(r.y_row), _ptr(r.y_col)
+    ys = [t for t in (r.y_row, r.y_col) if t is not None]
+    a.ld_y = _ld(ys[0]) if ys else a.cols
+    a.codes_row, a.scales_row, a.mask_row = _ptr(r.codes_row), _ptr(r.scales_row), _ptr(r.mask_row)
+    a.codes_col, a.scales_col, a.mask_col = _ptr(r.codes_col), _ptr(r.scales_col), _ptr(r.mask_col)
+
+
+def _check_status(r: QDQResult, where: str) -> None:
+    if r.status is not None:
+        st = int(r.status.item())
+        _abi.check(st, where + " (group_list)")
+
+
+def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0, scale_mode: str = "page",
+                  rowwise: bool = True, colwise: bool = False, group_list=None, group_list_type: int = 0,
+                  emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
+                  check: bool = False, out: QDQResult | None = None) -> QDQResult:
+    """QDQ forward; returns the requested outputs. check=True synchronises and
+    raises on an invalid group_list."""
+    x = _as_2d(x)
+    gl, ng = _group_args(group_list, group_list_type, x.device)
+    dirs = (_abi.ROWWISE if rowwise else 0) | (_abi.COLWISE if colwise else 0)
+    if dirs == 0:
+        raise ValueError("at least one of rowwise / colwise must be set")
+    r = out if out is not None else alloc_outputs(
+        x, block=block, rowwise=rowwise, colwise=colwise, num_groups=ng, emit_values=emit_values,
+        emit_codes=emit_codes, emit_mask=emit_mask, with_status=check or gl is not None)
+    a = make_args(x, block=block, scale_factor=scale_factor, scale_mode=scale_mode, dirs=dirs,
+                  group_list=gl, group_list_type=group_list_type, status=r.status)
+    _fill_outputs(a, r)
+    _abi.check(_abi.mxfp4_qdq_fwd(a, _stream(x.device)), "mxfp4_qdq_fwd")
+    if check:
+        _check_status(r, "mxfp4_qdq_fwd")
+    return r
+
+
+def mxfp4_ste_bwd(grad_out: torch.Tensor, *, saved_mask: torch.Tensor | None = None,
+                  x: torch.Tensor | None = None, clip_grad: bool = True, block: int = 32,
+                  scale_factor: float = 6.0, scale_mode: str = "page", direction: str = "rowwise",
+                  group_list=None, group_list_type: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Plain / clipped STE backward. With clip_grad and no saved_mask the mask
+    is recomputed from x in the same pass."""
+    shape = grad_out.shape
+    g = _as_2d(grad_out, "grad_out")
+    if not g.is_contiguous():
+        g = g.contiguous()
+    gi = out if out is not None else torch.empty_like(g)
+    gi2 = gi.view(g.shape)
+    if x is not None:
+        x2 = _as_2d(x)
+        if x2.shape != g.shape or x2.dtype != g.dtype:
+            raise ValueError("x and grad_out must have the same shape and dtype")
+    else:
+        x2 = g  # geometry only; x is not read when the mask is saved
+        if clip_grad and saved_mask is None:
+            raise ValueError("clip_grad without saved_mask needs x to recompute the mask")
+    gl, _ = _group_args(group_list, group_list_type, g.device)
+    a = make_args(x2, block=block, scale_factor=scale_factor, scale_mode=scale_mode,
+                  dirs=_DIRS[direction], group_list=gl, group_list_type=group_list_type)
+    if x is None:
+        a.x = None
+    st = _abi.mxfp4_ste_bwd(a, g.data_ptr(), gi2.data_ptr(), g.shape[1], _ptr(saved_mask),
+                            int(bool(clip_grad)), _stream(g.device))
+    _abi.check(st, "mxfp4_ste_bwd")
+    return gi.view(shape)
+
+
+def mxfp4_qdq_fwd_bwd(x: torch.Tensor, grad_out: torch.Tensor, *, grad_direction: str = "rowwise",
+                      block: int = 32, scale_factor: float = 6.0, scale_mode: str = "page",
+                      rowwise: bool = True, colwise: bool = False, group_list=None, group_list_type: int = 0,
+                      emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
+                      out: QDQResult | None = None, grad_in: torch.Tensor | None = None):
+    """Fused forward + clipped-STE backward; returns (QDQResult, grad_in)."""
+    x = _as_2d(x)
+    g = _as_2d(grad_out, "grad_out").contiguous()
+    if g.shape != x.shape or g.dtype != x.dtype:
+        raise ValueError("x and grad_out must have the same shape and dtype")
+    gl, ng = _group_args(group_list, group_list_type, x.device)
+    dirs = (_abi.ROWWISE if rowwise else 0) | (_abi.COLWISE if colwise else 0)
+    r = out if out is not None else alloc_outputs(
+        x, block=block, rowwise=rowwise, colwise=colwise, num_groups=ng, emit_values=emit_values,
+        emit_codes=emit_codes, emit_mask=emit_mask, with_status=gl is not None)
+    gi = grad_in if grad_in is not None else torch.empty_like(g)
+    a = make_args(x, block=block, scale_factor=scale_factor, scale_mode=scale_mode, dirs=dirs,
+                  group_list=gl, group_list_type=group_list_type, status=r.status)
+    _fill_outputs(a, r)
+    st = _abi.mxfp4_qdq_fwd_bwd(a, g.data_ptr(), gi.data_ptr(), g.shape[1], _DIRS[grad_direction],
+                                _stream(x.device))
+    _abi.check(st, "mxfp4_qdq_fwd_bwd")
+    return r, gi

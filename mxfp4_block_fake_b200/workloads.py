@@ -84,6 +84,12 @@ def train_step(rows: int = 16384, cols: int = 4096, seed: int = 3, block: int = 
     return xb, grad.to(torch.bfloat16)
 
 
+def train_step_grad(rows: int, cols: int, seed: int = 5, sigma: float = 1e-3) -> torch.Tensor:
+    """Incoming gradient of the training-step workloads: bf16 ~ N(0, sigma^2)."""
+    g = _gen(seed)
+    return (torch.randn(rows, cols, generator=g, dtype=torch.float32) * sigma).to(torch.bfloat16)
+
+
 def moe_group_counts(rows: int, groups: int = 256, seed: int = 4, empty=(0, 100, 255)):
     """Multinomial group sizes over p ~ u^4; the listed groups are emptied into
     their neighbours (0 -> 1, 100 -> 101, 255 -> 254)."""
@@ -107,6 +113,42 @@ def moe_grouped(rows: int = 65536, cols: int = 7168, groups: int = 256, seed: in
     x = torch.randn(rows, cols, generator=g, dtype=torch.float32).to(torch.bfloat16)
     counts = moe_group_counts(rows, groups, seed)
     return x, counts, torch.cumsum(counts, 0)
+
+
+def mixed(rows: int, cols: int, dtype=torch.bfloat16, seed: int = 9, specials: bool = True) -> torch.Tensor:
+    """Parity-test input mixing every regime a block can be in: N(0,1) rows
+    scaled by 2^U(-40, 40), a few x50 outlier columns, exact codebook values
+    and midpoints times a power of two, all-zero and -0 blocks, bf16/fp32
+    subnormals, and (with specials) scattered +inf, -inf and NaN."""
+    g = _gen(seed)
+    x = torch.randn(rows, cols, generator=g, dtype=torch.float32)
+    x *= torch.exp2(torch.randint(-40, 41, (rows, 1), generator=g).float())
+    if cols >= 8:
+        x[:, torch.randperm(cols, generator=g)[: max(1, cols // 200)]] *= 50
+    n = rows * cols
+    flat = x.view(-1)
+    grid = torch.tensor([0.0, 0.25, 0.5, 0.75, 1.0, 1.25, 1.5, 1.75, 2.0, 2.5, 3.0, 3.5, 4.0, 5.0, 6.0, 7.0])
+    idx = torch.randint(0, n, (n // 16,), generator=g)
+    pick = grid[torch.randint(0, len(grid), (idx.numel(),), generator=g)]
+    sgn = torch.where(torch.rand(idx.numel(), generator=g) < 0.5, -1.0, 1.0)
+    flat[idx] = sgn * pick * torch.exp2(torch.randint(-10, 11, (idx.numel(),), generator=g).float())
+    idx = torch.randint(0, n, (n // 64,), generator=g)
+    flat[idx] = torch.where(torch.rand(idx.numel(), generator=g) < 0.5, 0.0, -0.0)
+    if rows >= 4 and cols >= 64:
+        r0 = int(torch.randint(0, rows - 3, (1,), generator=g))
+        x[r0: r0 + 3, 0:64] = 0.0
+        x[r0 + 1, 3] = -0.0
+    tiny = 2.0 ** -133 if dtype == torch.bfloat16 else 2.0 ** -149
+    idx = torch.randint(0, n, (n // 128,), generator=g)
+    flat[idx] = torch.randint(-16, 17, (idx.numel(),), generator=g).float() * tiny
+    if rows >= 2 and cols >= 64:
+        r1 = int(torch.randint(0, rows, (1,), generator=g))
+        x[r1, 32:64] = torch.randint(-127, 128, (32,), generator=g).float() * tiny
+    if specials:
+        for v in (float("inf"), float("-inf"), float("nan")):
+            idx = torch.randint(0, n, (max(1, n // 20000),), generator=g)
+            flat[idx] = v
+    return x.to(dtype)
 
 
 WORKLOADS = {

@@ -1,0 +1,165 @@
+"""CPU checks of the C ABI boundary (no GPU needed).
+
+* libmxfp4.so builds, loads and exports every function include/mxfp4.h declares;
+* the ctypes mirror of mxfp4_qdq_args has the C layout (sizeof/offsetof taken
+  from a C program compiled against the header);
+* host-only entry points (scale-row counting, status strings) agree with the
+  oracle's group_list normalisation (the MindSpore fake_w4a8_gmm_func.py page,
+  normalize_group_list);
+* argument errors are rejected on the host before any CUDA call.
+"""
+from __future__ import annotations
+
+import os
+import re
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "mxfp4.h")
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from mxfp4_block_fake_b200 import build
+    build.build()
+    from mxfp4_block_fake_b200 import _abi
+    _abi.lib()
+    return _abi
+
+
+def declared_functions() -> list[str]:
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports(abi):
+    assert declared_functions() == sorted(abi.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(abi):
+    out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\sT\s(\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(abi.lib(), name)
+
+
+def test_struct_layout_matches_c(abi, tmp_path):
+    fields = [f for f, _ in abi.QdqArgs._fields_]
+    src = tmp_path / "layout.c"
+    body = "\n".join(f'  printf("{f} %zu\\n", offsetof(mxfp4_qdq_args, {f}));' for f in fields)
+    src.write_text(
+        "#include <stdio.h>\n#include <stddef.h>\n#include \"mxfp4.h\"\n"
+        "int main(void) {\n" + body + '\n  printf("sizeof %zu\\n", sizeof(mxfp4_qdq_args));\n  return 0;\n}\n'
+    )
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), "-o", str(exe), str(src)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                      check=True).stdout.splitlines())
+    import ctypes
+    for f in fields:
+        assert int(got[f]) == getattr(abi.QdqArgs, f).offset, f
+    assert int(got["sizeof"]) == ctypes.sizeof(abi.QdqArgs)
+
+
+def test_header_compiles_as_c_and_cpp(tmp_path):
+    src = tmp_path / "inc.c"
+    src.write_text('#include "mxfp4.h"\nint f(void) { return MXFP4_ABI_VERSION + MXFP4_MAX_GROUPS; }\n')
+    for comp, std in (("gcc", "-std=c99"), ("g++", "-std=c++11")):
+        subprocess.run([comp, std, "-Wall", "-Werror", "-c", "-I", os.path.dirname(HEADER), "-x",
+                        "c" if comp == "gcc" else "c++", str(src), "-o", str(tmp_path / "o.o")], check=True)
+
+
+def test_status_strings(abi):
+    assert abi.status_string(abi.OK) == "ok"
+    assert abi.status_string(abi.EINVAL) == "invalid argument"
+    assert abi.status_string(abi.EUNSUPPORTED) == "unsupported argument"
+    assert abi.status_string(abi.ECUDA) == "CUDA error"
+    assert abi.status_string(77) == "unknown status"
+    assert abi.lib().mxfp4_abi_version() == abi.ABI_VERSION
+
+
+@pytest.mark.parametrize("block", [32, 128])
+def test_colwise_scale_rows_matches_oracle(abi, oracle_mod, block):
+    rng = np.random.default_rng(3)
+    for trial in range(200):
+        g = int(rng.integers(1, 40))
+        counts = rng.integers(0, 300, g)
+        counts[rng.random(g) < 0.3] = 0
+        rows = int(counts.sum())
+        ends = oracle_mod.group_ends(counts, 1, rows)
+        exp = oracle_mod.colwise_scale_rows(ends, block)
+        assert abi.mxfp4_colwise_scale_rows(counts.tolist(), 1, rows, block) == exp
+        assert abi.mxfp4_colwise_scale_rows(ends.tolist(), 0, rows, block) == exp
+        assert abi.mxfp4_colwise_scale_rows_bound(rows, g, block) >= exp
+    # invalid lists
+    assert abi.mxfp4_colwise_scale_rows([3, 2, 8], 0, 8, 32) == -1
+    assert abi.mxfp4_colwise_scale_rows([3, 3, 7], 0, 8, 32) == -1
+    assert abi.mxfp4_colwise_scale_rows([3, -1, 6], 1, 8, 32) == -1
+    assert abi.mxfp4_colwise_scale_rows(None, 0, 100, 32) == 4
+
+
+def _args(abi, **kw):
+    a = abi.QdqArgs()
+    a.dtype, a.block, a.rows, a.cols, a.ld = abi.BF16, 32, 4, 64, 64
+    a.scale_factor, a.scale_mode, a.dirs = 6.0, abi.SCALE_PAGE, abi.ROWWISE
+    a.x = 4096  # never dereferenced: every case below fails host validation first
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(block=0), 1), (dict(block=-32), 1), (dict(block=64), 2), (dict(block=16), 2),
+    (dict(scale_factor=0.0), 1), (dict(scale_factor=-6.0), 1), (dict(scale_factor=float("nan")), 1),
+    (dict(scale_factor=float("inf")), 1), (dict(dtype=7), 1), (dict(scale_mode=5), 1),
+    (dict(dirs=0), 1), (dict(dirs=4), 1), (dict(rows=-1), 1), (dict(cols=-3), 1),
+    (dict(rows=2 ** 31), 2), (dict(x=None), 1), (dict(ld=32), 1), (dict(x=4097), 1),
+    (dict(dirs=2, group_list=4096, num_groups=0), 1),
+    (dict(dirs=2, group_list=4096, num_groups=5000), 2),
+    (dict(dirs=2, group_list=4096, num_groups=3, group_list_type=2), 1),
+    (dict(dirs=2, group_list=4097, num_groups=3), 1),
+])
+def test_fwd_rejects_bad_arguments_on_host(abi, kw, expected):
+    assert abi.mxfp4_qdq_fwd(_args(abi, **kw), None) == expected
+
+
+def test_null_args_and_bad_bwd_arguments(abi):
+    import ctypes
+    L = abi.lib()
+    assert L.mxfp4_qdq_fwd(None, None) == abi.EINVAL
+    assert L.mxfp4_ste_bwd(None, 4096, 4096, 64, None, 1, None) == abi.EINVAL
+    a = _args(abi, dirs=3)
+    assert abi.mxfp4_ste_bwd(a, 4096, 4096, 64, None, 1, None) == abi.EINVAL  # two directions
+    a = _args(abi)
+    assert abi.mxfp4_ste_bwd(a, None, 4096, 64, None, 1, None) == abi.EINVAL
+    assert abi.mxfp4_ste_bwd(a, 4096, 4096, 32, None, 1, None) == abi.EINVAL  # ld_grad < cols
+    assert abi.mxfp4_qdq_fwd_bwd(a, 4096, None, 64, 1, None) == abi.EINVAL
+    assert abi.mxfp4_qdq_fwd_bwd(a, 4096, 4096, 64, 2, None) == abi.EINVAL  # grad dir not computed
+    assert abi.mxfp4_qdq_fwd_bwd(a, 4096, 4096, 64, 3, None) == abi.EINVAL
+    _ = ctypes
+
+
+def test_product_path_has_no_cpu_fallback():
+    torch = pytest.importorskip("torch")
+    from mxfp4_block_fake_b200 import mxfp4_quant_dequant
+    with pytest.raises(ValueError, match="CUDA"):
+        mxfp4_quant_dequant(torch.ones(4, 64))
+
+
+def test_product_code_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "mxfp4_block_fake_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
+                assert "liboracle" not in text and "mxfp4_oracle" not in text, f
+    _ = sys

@@ -1,0 +1,355 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the CPU oracle.
+
+Tolerance: 0 ULP. Every dequantised value is exactly representable, so the bf16
+/ fp32 outputs, the packed E2M1 codes, the E8M0 scales, the saturation
+bitmasks and the STE gradients must match the oracle byte for byte.
+
+Shapes span several tiles plus ragged tails (rows not a multiple of the block,
+cols not a multiple of the block, of 8, or of the tile width), strided and
+unaligned inputs (the generic kernels), empty tensors, group lists with empty
+groups and partial tail blocks, every finite bf16 value as element and as
+block maximum, and (test_full_size_sampled) the full sizes of the workloads
+in the launch configuration the benchmark times, checked on sampled rows and
+columns.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from mxfp4_block_fake_b200 import MXFP4ArgumentError, ops, workloads as W
+
+pytestmark = pytest.mark.gpu
+
+MODES = {"page": O.SCALE_PAGE, "floor": O.SCALE_FLOOR}
+
+
+def np_bits(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float32:
+        return t.numpy().view(np.uint32)
+    return t.numpy()
+
+
+def oracle_in(x: torch.Tensor) -> np.ndarray:
+    x = x.contiguous()
+    return np_bits(x) if x.dtype == torch.bfloat16 else x.numpy()
+
+
+def ora_bits(a: np.ndarray) -> np.ndarray:
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
+def check_dir(res: ops.QDQResult, ora: dict, d: str, cols: int, srows: int | None = None, label=""):
+    y, codes, scales, mask = (getattr(res, f"{k}_{d}") for k in ("y", "codes", "scales", "mask"))
+    if y is not None:
+        g = np_bits(y)
+        e = ora_bits(ora["y"])
+        bad = np.argwhere(g != e)
+        assert bad.size == 0, f"{label} y_{d}: {len(bad)} mismatches, first {bad[:3].tolist()} " \
+                              f"gpu {g[tuple(bad[0])]:#x} oracle {e[tuple(bad[0])]:#x}"
+    if codes is not None:
+        assert np.array_equal(np_bits(codes), ora["codes"]), f"{label} codes_{d}"
+    if scales is not None:
+        s = ora["scales"].shape[0] if srows is None else srows
+        assert np.array_equal(np_bits(scales)[:s], ora["scales"][:s]), f"{label} scales_{d}"
+    if mask is not None:
+        assert np.array_equal(np_bits(mask), ora["mask"]), f"{label} mask_{d}"
+
+
+def run_both(x: torch.Tensor, *, block: int, mode: str, rowwise: bool, colwise: bool, counts=None,
+             gl_type: int = 0, sf: float = 6.0, xdev: torch.Tensor | None = None):
+    xd = x.cuda() if xdev is None else xdev
+    gl = None
+    ends = None
+    if counts is not None:
+        counts = np.asarray(counts, np.int64)
+        ends = np.cumsum(counts)
+        gl = torch.tensor(counts if gl_type == 1 else ends, dtype=torch.int64, device="cuda")
+    res = ops.mxfp4_qdq_fwd(xd, block=block, scale_factor=sf, scale_mode=mode, rowwise=rowwise, colwise=colwise,
+                            group_list=gl, group_list_type=gl_type, emit_codes=True, emit_mask=True, check=True)
+    torch.cuda.synchronize()
+    xo = oracle_in(x)
+    out = {}
+    if rowwise:
+        out["row"] = O.qdq_rowwise(xo, block, sf, MODES[mode])
+    if colwise:
+        out["col"] = O.qdq_colwise(xo, block, sf, MODES[mode], ends=ends)
+    return res, out
+
+
+SHAPES = [(300, 1024), (37, 1000), (129, 136), (1, 64), (64, 4096), (5, 999), (33, 77), (2, 8)]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("block", [32, 128])
+@pytest.mark.parametrize("mode", ["page", "floor"])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_rowwise(dtype, block, mode, shape):
+    x = W.mixed(*shape, dtype=dtype, seed=hash(shape) % 1000)
+    res, ora = run_both(x, block=block, mode=mode, rowwise=True, colwise=False)
+    check_dir(res, ora["row"], "row", shape[1], label=f"{shape}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("block", [32, 128])
+@pytest.mark.parametrize("mode", ["page", "floor"])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_colwise_and_dual(dtype, block, mode, shape):
+    x = W.mixed(*shape, dtype=dtype, seed=1 + hash(shape) % 1000)
+    res, ora = run_both(x, block=block, mode=mode, rowwise=False, colwise=True)
+    check_dir(res, ora["col"], "col", shape[1], label=f"col {shape}")
+    res, ora = run_both(x, block=block, mode=mode, rowwise=True, colwise=True)
+    check_dir(res, ora["row"], "row", shape[1], label=f"dual {shape}")
+    check_dir(res, ora["col"], "col", shape[1], label=f"dual {shape}")
+
+
+GROUPS = [
+    [0, 45, 32, 0, 1, 70, 0],          # empty groups, partial tails, a 1-row group
+    [300],                               # one group
+    [0, 0, 300],
+    [31, 33, 64, 128, 44],
+    [1] * 40 + [260],
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("block", [32, 128])
+@pytest.mark.parametrize("gl_type", [0, 1])
+@pytest.mark.parametrize("gi", range(len(GROUPS)))
+@pytest.mark.parametrize("cols", [256, 200, 99])
+def test_grouped_colwise_and_dual(dtype, block, gl_type, gi, cols):
+    counts = GROUPS[gi]
+    rows = sum(counts)
+    x = W.mixed(rows, cols, dtype=dtype, seed=100 + gi)
+    mode = "page" if gi % 2 == 0 else "floor"
+    res, ora = run_both(x, block=block, mode=mode, rowwise=True, colwise=True, counts=counts, gl_type=gl_type)
+    check_dir(res, ora["row"], "row", cols, label="grouped")
+    check_dir(res, ora["col"], "col", cols, label="grouped")
+    assert int(res.status.item()) == 0
+
+
+def test_moe_group_recipe_reduced():
+    counts = W.moe_group_counts(4096, 256, seed=4).numpy()
+    x = W.moe_grouped(4096, 512, 256, seed=4)[0]
+    res, ora = run_both(x, block=32, mode="page", rowwise=True, colwise=True, counts=counts)
+    check_dir(res, ora["row"], "row", 512)
+    check_dir(res, ora["col"], "col", 512)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dirs", [(True, False), (False, True), (True, True)])
+def test_strided_and_unaligned_inputs(dtype, dirs):
+    big = W.mixed(70, 272, dtype=dtype, seed=5).cuda()
+    for view in (big[:, 8:264], big[:, 3:259], big[1:, 1:200]):
+        x = view.cpu()
+        res, ora = run_both(x, block=32, mode="page", rowwise=dirs[0], colwise=dirs[1], xdev=view)
+        if dirs[0]:
+            check_dir(res, ora["row"], "row", x.shape[1], label="strided")
+        if dirs[1]:
+            check_dir(res, ora["col"], "col", x.shape[1], label="strided")
+
+
+@pytest.mark.parametrize("sf", [1.0, 4.0, 7.5, 0.75, 3.0e-38, 1.0e30])
+def test_scale_factors_page_mode(sf):
+    x = W.mixed(64, 512, seed=6)
+    res, ora = run_both(x, block=32, mode="page", rowwise=True, colwise=True, sf=sf)
+    check_dir(res, ora["row"], "row", 512)
+    check_dir(res, ora["col"], "col", 512)
+
+
+@pytest.mark.parametrize("mode", ["page", "floor"])
+def test_every_bf16_value_as_element_and_as_block_max(mode):
+    allv = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    # as block maximum: row = [v, v/2-ish neighbours...] -> every amax pattern incl. inf / NaN
+    rows = []
+    for shift in (0, 1, 3):
+        blk = np.zeros((65536, 32), np.uint16)
+        blk[:, 0] = allv
+        blk[:, 1] = np.where((allv & 0x7F80) >= (shift << 7), allv - (shift << 7), allv)
+        blk[:, 2] = allv ^ 0x8000
+        blk[:, 5] = 0x3F80
+        rows.append(blk)
+    # as element under fixed maxima
+    for mx in (0x40C0, 0x4090, 0x3F80, 0x40F8, 0x0010, 0x7F7F):
+        blk = np.zeros((65536, 32), np.uint16)
+        blk[:, 0] = mx
+        blk[:, 7] = allv
+        rows.append(blk)
+    xb = np.concatenate(rows)
+    x = torch.from_numpy(xb.view(np.int16).copy()).view(torch.bfloat16)
+    res, ora = run_both(x, block=32, mode=mode, rowwise=True, colwise=False)
+    check_dir(res, ora["row"], "row", 32, label="bf16 sweep")
+
+
+def test_fp32_random_patterns():
+    rng = np.random.default_rng(7)
+    bits = rng.integers(0, 2 ** 32, (4096, 256), dtype=np.uint64).astype(np.uint32)
+    bits[:1024] &= 0x807FFFFF  # subnormal-heavy rows
+    bits[1024:2048] = (bits[1024:2048] & 0x80FFFFFF) | 0x3F000000  # values near 0.5..2
+    x = torch.from_numpy(bits.view(np.float32).copy())
+    for mode in ("page", "floor"):
+        res, ora = run_both(x, block=32, mode=mode, rowwise=True, colwise=True)
+        check_dir(res, ora["row"], "row", 256, label="fp32 patterns")
+        check_dir(res, ora["col"], "col", 256, label="fp32 patterns")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("direction", ["rowwise", "colwise"])
+@pytest.mark.parametrize("shape", [(300, 1024), (37, 1000), (5, 999)])
+def test_ste_backward(dtype, direction, shape):
+    x = W.mixed(*shape, dtype=dtype, seed=11)
+    g = W.mixed(*shape, dtype=dtype, seed=12, specials=False)
+    counts = [shape[0] // 3, 0, shape[0] - shape[0] // 3] if direction == "colwise" else None
+    ends = None if counts is None else np.cumsum(counts)
+    gl = None if counts is None else torch.tensor(counts, dtype=torch.int64, device="cuda")
+    xd, gd = x.cuda(), g.cuda()
+    xo, go = oracle_in(x), oracle_in(g)
+    if direction == "rowwise":
+        ora = O.qdq_rowwise(xo, 32, 6.0, O.SCALE_PAGE)
+    else:
+        ora = O.qdq_colwise(xo, 32, 6.0, O.SCALE_PAGE, ends=ends)
+    exp = ora_bits(O.ste_bwd(go, ora["mask"], True))
+    # 1) forward writes the mask, backward reads it
+    res = ops.mxfp4_qdq_fwd(xd, rowwise=direction == "rowwise", colwise=direction == "colwise",
+                            group_list=gl, group_list_type=1, emit_mask=True)
+    m = res.mask_row if direction == "rowwise" else res.mask_col
+    gi = ops.mxfp4_ste_bwd(gd, saved_mask=m, clip_grad=True)
+    assert np.array_equal(np_bits(gi), exp)
+    # 2) saved-free: recompute the mask from x
+    gi = ops.mxfp4_ste_bwd(gd, x=xd, clip_grad=True, direction=direction, group_list=gl, group_list_type=1)
+    assert np.array_equal(np_bits(gi), exp)
+    # 3) fused forward + backward in one pass
+    res, gi = ops.mxfp4_qdq_fwd_bwd(xd, gd, grad_direction=direction, rowwise=True, colwise=True,
+                                    group_list=gl, group_list_type=1, emit_codes=True, emit_mask=True)
+    assert np.array_equal(np_bits(gi), exp)
+    check_dir(res, ora, "row" if direction == "rowwise" else "col", shape[1], label="fused")
+    # 4) plain STE is the identity
+    gi = ops.mxfp4_ste_bwd(gd, clip_grad=False)
+    assert np.array_equal(np_bits(gi), np_bits(g))
+
+
+def test_invalid_group_list_writes_nothing_and_reports():
+    x = W.mixed(100, 128, seed=13).cuda()
+    for gl, t in (([50, 40, 60], 0), ([50, 60, 90], 0), ([50, -10, 60], 1), ([-1, 100], 0)):
+        r = ops.alloc_outputs(x, block=32, rowwise=False, colwise=True, num_groups=len(gl), emit_codes=True,
+                              emit_mask=True, with_status=True)
+        for t_ in (r.y_col, r.codes_col, r.scales_col, r.mask_col):
+            t_.view(torch.uint8).fill_(0xA5)
+        glt = torch.tensor(gl, dtype=torch.int64, device="cuda")
+        with pytest.raises(MXFP4ArgumentError):
+            ops.mxfp4_qdq_fwd(x, rowwise=False, colwise=True, group_list=glt, group_list_type=t, out=r,
+                              check=True)
+        for t_ in (r.y_col, r.codes_col, r.scales_col, r.mask_col):
+            assert bool((t_.view(torch.uint8) == 0xA5).all())
+
+
+def test_empty_inputs():
+    for shape in ((0, 64), (16, 0)):
+        x = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+        r = ops.mxfp4_qdq_fwd(x, rowwise=True, colwise=True, emit_codes=True, emit_mask=True)
+        assert r.y_row.shape == shape
+    with pytest.raises(ValueError):
+        ops.mxfp4_qdq_fwd(torch.tensor(1.0, device="cuda"))
+
+
+def test_qat_linear_tiny_fwd_bwd():
+    """Tiny QAT linear, fp32 x [4,64] and W [32,64], block 32 along the last dim:
+    forward y = Q(x) Q(W)^T, clipped-STE grads for grad_out = ones."""
+    from mxfp4_block_fake_b200 import MXFP4QATConfig, MXFP4QATLinear
+    torch.backends.cuda.matmul.allow_tf32 = False
+    x, w = W.qat_linear_tiny()
+    for clip in (False, True):
+        lin = MXFP4QATLinear(64, 32, bias=False, config=MXFP4QATConfig(quantize_input=True, clip_grad=clip))
+        with torch.no_grad():
+            lin.weight.copy_(w)
+        lin = lin.cuda()
+        xd = x.cuda().requires_grad_(True)
+        y = lin(xd)
+        y.backward(torch.ones_like(y))
+        qx = O.qdq_rowwise(x.numpy(), 32, 6.0, O.SCALE_PAGE)
+        qw = O.qdq_rowwise(w.numpy(), 32, 6.0, O.SCALE_PAGE)
+        # products of <=2-significant-bit values summed over 64 terms: exact in float64
+        y_exp = qx["y"].astype(np.float64) @ qw["y"].astype(np.float64).T
+        np.testing.assert_allclose(y.detach().cpu().numpy(), y_exp, rtol=2e-7, atol=0)
+        ones = np.ones((4, 32))
+        dx = ones @ qw["y"].astype(np.float64)
+        dw = ones.T @ qx["y"].astype(np.float64)
+        if clip:
+            dx = np.where(O.unpack_bits(qx["mask"], 64), 0.0, dx)
+            dw = np.where(O.unpack_bits(qw["mask"], 64), 0.0, dw)
+        np.testing.assert_allclose(xd.grad.cpu().numpy(), dx, rtol=2e-7, atol=0)
+        np.testing.assert_allclose(lin.weight.grad.cpu().numpy(), dw, rtol=2e-7, atol=0)
+
+
+def _sample_full(x: torch.Tensor, xd: torch.Tensor, res: ops.QDQResult, rowwise: bool, colwise: bool,
+                 mode: str, block: int, ends=None, nsamp: int = 256, seed: int = 0):
+    """Compare sampled rows (row-wise) and sampled columns (column-wise, all
+    row-blocks) of full-size outputs with the oracle run on those slices."""
+    rng = np.random.default_rng(seed)
+    rows, cols = x.shape
+    if rowwise:
+        ri = np.sort(rng.choice(rows, size=min(nsamp, rows), replace=False))
+        rit = torch.from_numpy(ri).cuda()
+        ora = O.qdq_rowwise(oracle_in(x[torch.from_numpy(ri)]), block, 6.0, MODES[mode])
+        sub = ops.QDQResult(y_row=res.y_row[rit], codes_row=None if res.codes_row is None else res.codes_row[rit],
+                            scales_row=None if res.scales_row is None else res.scales_row[rit],
+                            mask_row=None if res.mask_row is None else res.mask_row[rit])
+        check_dir(sub, ora, "row", cols, label="full-size rows")
+    if colwise:
+        # whole aligned octets of columns so that mask and code bytes compare directly
+        oc = np.sort(rng.choice(cols // 8, size=min(nsamp // 8, cols // 8), replace=False))
+        ci = (oc[:, None] * 8 + np.arange(8)).reshape(-1)
+        cit = torch.from_numpy(ci).cuda()
+        ora = O.qdq_colwise(oracle_in(x[:, torch.from_numpy(ci)]), block, 6.0, MODES[mode], ends=ends)
+        s = ora["scales"].shape[0]
+        assert np.array_equal(np_bits(res.y_col[:, cit]), ora_bits(ora["y"]))
+        if res.codes_col is not None:
+            bc = torch.from_numpy((oc[:, None] * 4 + np.arange(4)).reshape(-1)).cuda()
+            assert np.array_equal(np_bits(res.codes_col[:, bc]), ora["codes"])
+            assert np.array_equal(np_bits(res.scales_col[:s][:, cit]), ora["scales"])
+        if res.mask_col is not None:
+            assert np.array_equal(np_bits(res.mask_col[:, torch.from_numpy(oc).cuda()]), ora["mask"])
+
+
+@pytest.mark.parametrize("name", ["act_rowwise", "weight_dual", "train_step", "moe_grouped"])
+def test_full_size_sampled(name):
+    """Full workload sizes, launched exactly as the benchmark launches them."""
+    torch.cuda.empty_cache()
+    if name == "act_rowwise":
+        x = W.act_rowwise()
+        xd = x.cuda()
+        res = ops.mxfp4_qdq_fwd(xd, emit_codes=True)
+        _sample_full(x, xd, res, True, False, "page", 32)
+    elif name == "weight_dual":
+        x = W.weight_dual()
+        xd = x.cuda()
+        for block in (32, 128):
+            res = ops.mxfp4_qdq_fwd(xd, block=block, rowwise=True, colwise=True, emit_codes=True)
+            _sample_full(x, xd, res, True, True, "page", block)
+    elif name == "train_step":
+        x, g = W.train_step()
+        xd, gd = x.cuda(), g.cuda()
+        res = ops.mxfp4_qdq_fwd(xd, emit_mask=True)
+        gi = ops.mxfp4_ste_bwd(gd, x=xd, clip_grad=True)
+        gi2 = ops.mxfp4_ste_bwd(gd, saved_mask=res.mask_row, clip_grad=True)
+        _sample_full(x, xd, res, True, False, "page", 32)
+        assert torch.equal(gi.view(torch.int16), gi2.view(torch.int16))
+        rng = np.random.default_rng(1)
+        ri = torch.from_numpy(np.sort(rng.choice(x.shape[0], 256, replace=False)))
+        ora = O.qdq_rowwise(oracle_in(x[ri]), 32, 6.0, O.SCALE_PAGE)
+        exp = O.ste_bwd(oracle_in(g[ri]), ora["mask"], True)
+        assert np.array_equal(np_bits(gi[ri.cuda()]), exp)
+    else:
+        x, counts, offsets = W.moe_grouped()
+        xd = x.cuda()
+        gl = offsets.cuda()
+        for mode in ("page", "floor"):
+            res = ops.mxfp4_qdq_fwd(xd, scale_mode=mode, rowwise=True, colwise=True, group_list=gl,
+                                    emit_codes=True, emit_mask=True, check=True)
+            _sample_full(x, xd, res, True, True, mode, 32, ends=offsets.numpy(), seed=3)
+    torch.cuda.synchronize()
