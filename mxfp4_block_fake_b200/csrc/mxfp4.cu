@@ -64,6 +64,7 @@ struct KArgs {
     int32_t gl_type;
     int32_t* status;
     uint32_t n_ct;  // column tiles of the tile kernel
+    uint32_t thr;   // PAGE mode: fp32 bits of T0 (see qparams)
 };
 
 // ---------------------------------------------------------------------------
@@ -310,7 +311,155 @@ __device__ __forceinline__ void plan_lookup(const int32_t* s_bpre, const int32_t
 // Tile kernel (vector path)
 // ---------------------------------------------------------------------------
 
-// T-size: 2 (bf16) or 4 (fp32) bytes. LC lanes across columns (16 bytes each),
+// Per-block parameters of the vector path: only 2^-k and 2^k are kept. A
+// non-finite block (a NaN or inf element, or 2^k overflowing fp32) gets
+// scale = NaN (0x7FC00000) and inv = 0, so that
+//   E8M0 byte  = scale_bits >> 23   (0xFF for NaN; 0 for the subnormal 2^-127)
+//   rare block = scale_bits >= 0x7E800000 (non-finite, or k >= 126 where
+//                fl(6 * 2^k) overflows and nothing saturates)
+struct QP {
+    float inv;
+    float scale;
+};
+
+// Scale exponent without a divide. PAGE mode: with T0 the smallest fp32 a for
+// which fl(a / scale_factor) >= C (C = 0x3FB504F4, the first fp32 above
+// sqrt 2), round(log2(fl(amax / sf))) >= j + 1 exactly when amax >= T0 * 2^j,
+// because dividing by sf commutes with power-of-two scaling while the results
+// stay normal. So k = floor(log2(amax / T0)) + 1, an exponent difference
+// corrected by a significand compare, then clamped at -30 (the 2^-30 floor of
+// the raw scale). The host computes T0 and limits scale_factor to
+// [2^-64, 11] on this path so that every threshold used is a normal number.
+__device__ __forceinline__ QP qparams(uint32_t A, int mode, uint32_t thr)
+{
+    int k;
+    if (mode == MXFP4_SCALE_FLOOR) {
+        k = max((int)(A >> 23) - 129, -127);
+    } else {
+        k = (int)(A >> 23) - (int)(thr >> 23) + 1 - ((A & 0x7FFFFFu) < (thr & 0x7FFFFFu) ? 1 : 0);
+        k = max(k, -30);
+    }
+    QP p;
+    if (A >= 0x7F800000u || k > 127) {
+        p.inv = 0.0f;
+        p.scale = __uint_as_float(QNAN32);
+    } else {
+        p.inv = __uint_as_float(pow2_bits(-k));
+        p.scale = __uint_as_float(pow2_bits(k));
+    }
+    return p;
+}
+
+__device__ __forceinline__ uint32_t qp_e8(const QP& p) { return __float_as_uint(p.scale) >> 23; }
+__device__ __forceinline__ bool qp_rare(const QP& p) { return __float_as_uint(p.scale) >= 0x7E800000u; }
+__device__ __forceinline__ bool qp_nonfinite(const QP& p) { return __float_as_uint(p.scale) > 0x7F800000u; }
+
+// E8M0 bytes of four blocks, first block in the low byte.
+__device__ __forceinline__ uint32_t pack_e8(const QP& a, const QP& b, const QP& c, const QP& d)
+{
+    return qp_e8(a) | (qp_e8(b) << 8) | (qp_e8(c) << 16) | (qp_e8(d) << 24);
+}
+
+// Lookup entry for u = floor(4 |y|), u < 64: the code magnitude as fp32 bits
+// (two significant bits, so the low half is zero) with the code index in the
+// low 3 bits. The index is the number of midpoints m with 4m <= u, i.e. with
+// m <= |y| since every 4m is an integer (ties go to the larger code).
+__device__ __forceinline__ uint32_t lut_entry(uint32_t u)
+{
+    const uint32_t i = (u >= 1) + (u >= 3) + (u >= 5) + (u >= 7) + (u >= 10) + (u >= 14) + (u >= 20);
+    const uint32_t cb = i >= 2u ? (i << 22) + 0x3F000000u : (i == 1u ? 0x3F000000u : 0u);
+    return cb | i;
+}
+
+// One element. y = fl(x / 2^k); t = 2^23 + floor(4|y|) (one fma rounding
+// down: the sum is exact below 2^24); the lookup address is
+// lut_base + 4 * (t_bits - 0x4B000000) folded into one shift-add (lutb holds
+// lut_base - 0x2C000000). |y| < 16 in every finite block on this path; the
+// clamp (which also maps NaN to 15.75) keeps the table index inside [0, 63]
+// for the non-finite blocks, whose outputs are then replaced. The sign follows
+// sign(y): set only for y < 0, not for -0 (y & (0x80000000 - y) has bit 31
+// set exactly then).
+__device__ __forceinline__ void qfast(uint32_t xb, const QP& p, uint32_t lutb, float& cs, float& o, bool& sat)
+{
+    const float y = __fmul_rn(__uint_as_float(xb), p.inv);
+    const float t = __fmaf_rd(fminf(fabsf(y), 15.75f), 4.0f, 8388608.0f);
+    uint32_t e;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(e) : "r"(lutb + (__float_as_uint(t) << 2)));
+    const uint32_t yb = __float_as_uint(y);
+    const uint32_t s = yb & (0x80000000u - yb) & 0x80000000u;
+    cs = __uint_as_float((e & 0xFFFF0000u) | s);
+    o = __fmul_rn(cs, p.scale);
+    sat = fabsf(y) > 6.0f;
+}
+
+// 8 signed code values (exact E2M1 values, so the conversion rounds nothing)
+// -> 8 nibbles, element 2j in the low nibble of byte j.
+__device__ __forceinline__ uint32_t e2m1x8(const float (&c)[8])
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]), "f"(c[4]), "f"(c[5]), "f"(c[6]), "f"(c[7]));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t e2m1x4(const float (&c)[4])
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "mov.b32 %0, {b0, b1, 0, 0};\n\t}"
+        : "=r"(r)
+        : "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
+    return r;
+}
+
+template <int VEC>
+__device__ __forceinline__ uint32_t nibbles(const float (&c)[VEC]);
+template <>
+__device__ __forceinline__ uint32_t nibbles<8>(const float (&c)[8]) { return e2m1x8(c); }
+template <>
+__device__ __forceinline__ uint32_t nibbles<4>(const float (&c)[4]) { return e2m1x4(c); }
+
+// Quantise the VEC elements of one 16-byte chunk with one parameter set
+// (row-wise: the chunk's block) or one per element (column-wise).
+template <int VEC, bool PER_ELEM>
+__device__ __forceinline__ void quant_chunk(const uint32_t (&xb)[VEC], const QP* p, uint32_t lutb,
+                                            uint32_t (&ob)[VEC], uint32_t& nibs, uint32_t& sats)
+{
+    float cs[VEC];
+    sats = 0;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        float o;
+        bool sat;
+        qfast(xb[e], p[PER_ELEM ? e : 0], lutb, cs[e], o, sat);
+        ob[e] = __float_as_uint(o);
+        sats |= (sat ? 1u : 0u) << e;
+    }
+    nibs = nibbles<VEC>(cs);
+}
+
+// Fix-up for rare blocks (non-finite, or k >= 126): every output NaN with code
+// 0 and no saturation for a non-finite block; no saturation when 6 * 2^k
+// overflows fp32.
+template <int VEC>
+__device__ __forceinline__ void rare_fixup(const QP& p, int e, uint32_t (&ob)[VEC], uint32_t& nibs, uint32_t& sats)
+{
+    if (qp_nonfinite(p)) {
+        ob[e] = QNAN32;
+        nibs &= ~(0xFu << (4 * e));
+    }
+    sats &= ~(1u << e);
+}
+
+// ESZ: 2 (bf16) or 4 (fp32) bytes. LC lanes across columns (16 bytes each),
 // LR = 32/LC lanes across rows, RPT rows per thread, WR warps down the tile.
 // A tile is BS rows (one column-wise block; a group tail may be shorter) by
 // LC*VEC columns.
@@ -329,24 +478,29 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
 
     extern __shared__ int32_t s_plan[];
     __shared__ uint32_t s_am[(COL && WR > 1) ? WR * TC : 1];
+    __shared__ uint32_t s_lut[64];
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int wg = warp / WR, wr = warp - wg * WR;
     const int lc = lane % LC, lr = lane / LC;
 
+    if (threadIdx.x < 64)
+        s_lut[threadIdx.x] = lut_entry(threadIdx.x);
     uint32_t S;
     int32_t* s_bpre = s_plan;
     int32_t* s_rst = s_plan + (GROUPS ? a.num_groups + 1 : 0);
     if constexpr (GROUPS) {
-        const int64_t s = build_plan<BS>(a, s_bpre, s_rst);
+        const int64_t s = build_plan<BS>(a, s_bpre, s_rst);  // contains __syncthreads
         if (blockIdx.x == 0 && threadIdx.x == 0 && a.status)
             *a.status = s < 0 ? MXFP4_EINVAL : MXFP4_OK;
         if (s < 0)
             return;
         S = (uint32_t)s;
     } else {
+        __syncthreads();
         S = (uint32_t)((a.rows + BS - 1) / BS);
     }
+    const uint32_t lutb = (uint32_t)__cvta_generic_to_shared(s_lut) - 0x2C000000u;
 
     const char* xp = static_cast<const char*>(a.x);
     const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8, nblk = (a.cols + BS - 1) / BS;
@@ -381,59 +535,10 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
             }
         }
 
-        uint32_t satr[ROW ? RPT : 1];
-        uint32_t satc[COL ? RPT : 1];
-
-        if constexpr (ROW) {
-#pragma unroll
-            for (int i = 0; i < RPT; ++i) {
-                const int r = i * (LR * WR) + wr * LR + lr;
-                const bool ok = colok && r < nrows;
-                const int64_t row = row0 + r;
-                uint32_t xb[VEC];
-                V::unpack(d[i], xb);
-                uint32_t am = 0;
-#pragma unroll
-                for (int e = 0; e < VEC; ++e)
-                    am = max(am, xb[e] & 0x7FFFFFFFu);
-#pragma unroll
-                for (int o = 1; o < BL; o <<= 1)
-                    am = max(am, __shfl_xor_sync(FULL, am, o));
-                const BP p = block_params(am, a.mode, a.sf);
-                uint32_t ob[VEC];
-                uint32_t nibs = 0, sats = 0;
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    uint32_t nb, st;
-                    ob[e] = qdq_elem(xb[e], p, nb, st);
-                    ob[e] = p.nanm ? QNAN32 : ob[e];
-                    nibs |= nb << (4 * e);
-                    sats |= st << e;
-                }
-                nibs &= ~p.nanm;
-                sats &= ~p.nanm;
-                satr[i] = sats;
-                if constexpr (VEC == 4) {  // two lanes form one mask byte
-                    const uint32_t other = __shfl_xor_sync(FULL, sats, 1);
-                    sats = (lc & 1) ? 0u : (sats | (other << 4));
-                }
-                if (ok) {
-                    if (a.y_row)
-                        st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * ESZ, V::pack(ob));
-                    if (a.codes_row) {
-                        if constexpr (VEC == 8)
-                            *reinterpret_cast<uint32_t*>(a.codes_row + row * cstride + col / 2) = nibs;
-                        else
-                            *reinterpret_cast<uint16_t*>(a.codes_row + row * cstride + col / 2) = (uint16_t)nibs;
-                    }
-                    if (a.mask_row && (VEC == 8 || !(lc & 1)))
-                        a.mask_row[row * mstride + col / 8] = (uint8_t)sats;
-                    if (a.scales_row && (lc % BL) == 0)
-                        a.scales_row[row * nblk + col / BS] = (uint8_t)p.e8;
-                }
-            }
-        }
-
+        // column-wise block parameters first (a register max down the thread's
+        // rows, a shuffle across the LR row lanes, shared memory across warps)
+        QP pc[COL ? VEC : 1];
+        bool crare = false;
         if constexpr (COL) {
             uint32_t amc[VEC];
 #pragma unroll
@@ -468,29 +573,84 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
                         m = max(m, s_am[w * TC + lc * VEC + e]);
                     amc[e] = m;
                 }
+                __syncthreads();  // s_am is rewritten by the next tile
             }
-            BP pc[VEC];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e)
-                pc[e] = block_params(amc[e], a.mode, a.sf);
-#pragma unroll
-            for (int i = 0; i < RPT; ++i) {
-                const int r = i * (LR * WR) + wr * LR + lr;
-                const bool ok = colok && r < nrows;
-                const int64_t row = row0 + r;
-                uint32_t xb[VEC];
-                V::unpack(d[i], xb);
-                uint32_t ob[VEC];
-                uint32_t nibs = 0, sats = 0;
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    uint32_t nb, st;
-                    ob[e] = qdq_elem(xb[e], pc[e], nb, st);
-                    ob[e] = pc[e].nanm ? QNAN32 : ob[e];
-                    nibs |= (nb & ~pc[e].nanm) << (4 * e);
-                    sats |= (st & ~pc[e].nanm) << e;
+            for (int e = 0; e < VEC; ++e) {
+                pc[e] = qparams(amc[e], a.mode, a.thr);
+                crare = crare || qp_rare(pc[e]);
+            }
+            if (a.scales_col && lr == 0 && wr == 0 && colok) {
+                uint8_t* sp = a.scales_col + (int64_t)rb * a.cols + col;
+                if constexpr (VEC == 8) {
+                    uint2 v;
+                    v.x = pack_e8(pc[0], pc[1], pc[2], pc[3]);
+                    v.y = pack_e8(pc[4 % VEC], pc[5 % VEC], pc[6 % VEC], pc[7 % VEC]);
+                    *reinterpret_cast<uint2*>(sp) = v;
+                } else {
+                    *reinterpret_cast<uint32_t*>(sp) = pack_e8(pc[0], pc[1], pc[2], pc[3 % VEC]);
                 }
-                satc[i] = sats;
+            }
+        }
+
+        // then one pass over the rows: both directions of row i, and the
+        // gradient of row i, before moving on
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) {
+            const int r = i * (LR * WR) + wr * LR + lr;
+            const bool ok = colok && r < nrows;
+            const int64_t row = row0 + r;
+            uint32_t xb[VEC];
+            V::unpack(d[i], xb);
+            uint32_t gmask = 0;
+            if constexpr (ROW) {
+                uint32_t am = 0;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    am = max(am, xb[e] & 0x7FFFFFFFu);
+#pragma unroll
+                for (int o = 1; o < BL; o <<= 1)
+                    am = max(am, __shfl_xor_sync(FULL, am, o));
+                const QP p = qparams(am, a.mode, a.thr);
+                uint32_t ob[VEC], nibs, sats;
+                quant_chunk<VEC, false>(xb, &p, lutb, ob, nibs, sats);
+                if (qp_rare(p)) {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e)
+                        rare_fixup<VEC>(p, e, ob, nibs, sats);
+                }
+                if (a.grad_dir == MXFP4_ROWWISE)
+                    gmask = sats;
+                if constexpr (VEC == 4) {  // two lanes form one mask byte
+                    const uint32_t other = __shfl_xor_sync(FULL, sats, 1);
+                    sats = (lc & 1) ? 0u : (sats | (other << 4));
+                }
+                if (ok) {
+                    if (a.y_row)
+                        st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * ESZ, V::pack(ob));
+                    if (a.codes_row) {
+                        if constexpr (VEC == 8)
+                            *reinterpret_cast<uint32_t*>(a.codes_row + row * cstride + col / 2) = nibs;
+                        else
+                            *reinterpret_cast<uint16_t*>(a.codes_row + row * cstride + col / 2) = (uint16_t)nibs;
+                    }
+                    if (a.mask_row && (VEC == 8 || !(lc & 1)))
+                        a.mask_row[row * mstride + col / 8] = (uint8_t)sats;
+                    if (a.scales_row && (lc % BL) == 0)
+                        a.scales_row[row * nblk + col / BS] = (uint8_t)qp_e8(p);
+                }
+            }
+            if constexpr (COL) {
+                uint32_t ob[VEC], nibs, sats;
+                quant_chunk<VEC, true>(xb, pc, lutb, ob, nibs, sats);
+                if (crare) {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e)
+                        if (qp_rare(pc[e]))
+                            rare_fixup<VEC>(pc[e], e, ob, nibs, sats);
+                }
+                if (a.grad_dir == MXFP4_COLWISE)
+                    gmask = sats;
                 if constexpr (VEC == 4) {
                     const uint32_t other = __shfl_xor_sync(FULL, sats, 1);
                     sats = (lc & 1) ? 0u : (sats | (other << 4));
@@ -508,36 +668,9 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
                         a.mask_col[row * mstride + col / 8] = (uint8_t)sats;
                 }
             }
-            if (a.scales_col && lr == 0 && wr == 0 && colok) {
-                uint8_t* sp = a.scales_col + (int64_t)rb * a.cols + col;
-                if constexpr (VEC == 8) {
-                    uint2 v;
-                    v.x = pc[0].e8 | (pc[1].e8 << 8) | (pc[2].e8 << 16) | (pc[3].e8 << 24);
-                    v.y = pc[4].e8 | (pc[5].e8 << 8) | (pc[6].e8 << 16) | (pc[7].e8 << 24);
-                    *reinterpret_cast<uint2*>(sp) = v;
-                } else {
-                    *reinterpret_cast<uint32_t*>(sp) =
-                        pc[0].e8 | (pc[1].e8 << 8) | (pc[2].e8 << 16) | (pc[3].e8 << 24);
-                }
-            }
-            if constexpr (WR > 1)
-                __syncthreads();  // s_am is rewritten by the next tile
-        }
-
-        if constexpr (GRAD) {
-#pragma unroll
-            for (int i = 0; i < RPT; ++i) {
-                const int r = i * (LR * WR) + wr * LR + lr;
-                if (!(colok && r < nrows))
-                    continue;
-                uint32_t m = 0;
-                if constexpr (ROW)
-                    if (a.grad_dir == MXFP4_ROWWISE)
-                        m = satr[i];
-                if constexpr (COL)
-                    if (a.grad_dir == MXFP4_COLWISE)
-                        m = satc[i];
-                st_stream(static_cast<char*>(a.g_in) + ((row0 + r) * a.ld_g + col) * ESZ, V::mask_out(gv[i], m));
+            if constexpr (GRAD) {
+                if (ok)
+                    st_stream(static_cast<char*>(a.g_in) + (row * a.ld_g + col) * ESZ, V::mask_out(gv[i], gmask));
             }
         }
     }
@@ -791,6 +924,48 @@ static int occupancy(const void* fn, size_t smem)
 
 static inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
+static float f32_of(uint32_t u)
+{
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+static uint32_t u32_of(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return u;
+}
+
+// PAGE-mode scale_factor range of the vector path: every threshold T0 * 2^j it
+// uses stays a normal fp32 number, and |x / 2^k| < 16 keeps floor(4|y|) inside
+// the 64-entry lookup table.
+static bool page_fast_ok(float sf) { return sf >= 0x1p-64f && sf <= 11.0f; }
+
+// T0 = the smallest fp32 a with fl(a / sf) >= C, C = 0x3FB504F4 (the first fp32
+// above sqrt 2), found by stepping from fl(C * sf) one ulp at a time with IEEE
+// fp32 host division (a -> fl(a / sf) is monotone).
+static uint32_t page_threshold(float sf)
+{
+    const float C = f32_of(0x3FB504F4u);
+    volatile float a = C * sf;
+    for (int i = 0; i < 64; ++i) {
+        volatile float prev = nextafterf(a, 0.0f);
+        volatile float q = prev / sf;
+        if (!(q >= C))
+            break;
+        a = prev;
+    }
+    for (int i = 0; i < 64; ++i) {
+        volatile float q = a / sf;
+        if (q >= C)
+            break;
+        a = nextafterf(a, INFINITY);
+    }
+    return u32_of(a);
+}
+
 typedef void (*KernelFn)(const KArgs);
 
 template <int ESZ, int BS, int LC, int RPT, int WR, bool GRAD>
@@ -967,6 +1142,11 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
         fast = fast && aligned(k.scales_col, vec);
     if (grad)
         fast = fast && aligned(g_out, 16) && aligned(g_in, 16) && ld_g % vec == 0;
+    if (A->scale_mode == MXFP4_SCALE_PAGE) {
+        fast = fast && page_fast_ok(A->scale_factor);
+        if (fast)
+            k.thr = page_threshold(A->scale_factor);
+    }
 
     const int bs = A->block;
     const size_t plan_smem = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
