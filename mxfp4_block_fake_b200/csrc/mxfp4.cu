@@ -459,6 +459,84 @@ __device__ __forceinline__ void rare_fixup(const QP& p, int e, uint32_t (&ob)[VE
     sats &= ~(1u << e);
 }
 
+// ---- bf16 fast path: two elements per 32-bit word ---------------------------
+
+// Packed unsigned 16-bit max of two words.
+__device__ __forceinline__ uint32_t vmax2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// A block takes the bf16 fast path when 2^-126 <= 2^k <= 2^16. k <= 16 keeps
+// every nonzero bf16 x clear of the fp32 underflow of x / 2^k (|x| >= 2^-133
+// > 2^(k-150)), so sign(y) is the sign of x; k >= -126 keeps 2^k normal, so
+// the bf16 bits of 6 * 2^k = 1.5 * 2^(k+2) are (scale_bits >> 16) + 0x140.
+// Non-finite blocks (scale NaN) and every other k take the general path.
+__device__ __forceinline__ bool qp_fast16(const QP& p)
+{
+    return (__float_as_uint(p.scale) - 0x00800000u) <= 0x47000000u;
+}
+
+__device__ __forceinline__ uint32_t qp_lim16(const QP& p) { return (__float_as_uint(p.scale) >> 16) + 0x140u; }
+
+// Code of one bf16 element on the fast path, signed like x. xw holds the
+// element in its top 16 bits; its low 16 bits may hold the other element of
+// the word: that perturbs |x| by less than one bf16 ulp, and every quarter of
+// 2^k that the rounding compares against is a bf16 number, so floor(4|y|) is
+// unchanged. t = 2^21 + |x| * 2^-k rounded down once: fp32 spacing on
+// [2^21, 2^22) is 1/4, so t's bit pattern is 0x4A000000 + floor(4|y|) and the
+// table address is lut_base + 4 * that, folded into one shift-add (lutb16 =
+// lut_base - 0x28000000). -0 inputs were cleared to +0 beforehand.
+__device__ __forceinline__ float qcode16(uint32_t xw, float inv, uint32_t lutb16)
+{
+    const float t = __fmaf_rd(fabsf(__uint_as_float(xw)), inv, 0x1p21f);
+    uint32_t e;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(e) : "r"(lutb16 + (__float_as_uint(t) << 2)));
+    return __uint_as_float(e | (xw & 0x80000000u));
+}
+
+// Quantise 8 bf16 elements (4 cleaned words) on the fast path: packed bf16
+// outputs and nibbles. One parameter set (row-wise) or one per element.
+template <bool PER_ELEM>
+__device__ __forceinline__ void quant16(const uint32_t (&wc)[4], const QP* p, uint32_t lutb16, uint32_t (&packed)[4],
+                                        uint32_t& nibs)
+{
+    float cs[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const QP& pl = p[PER_ELEM ? 2 * j : 0];
+        const QP& ph = p[PER_ELEM ? 2 * j + 1 : 0];
+        cs[2 * j] = qcode16(wc[j] << 16, pl.inv, lutb16);
+        cs[2 * j + 1] = qcode16(wc[j], ph.inv, lutb16);
+        const float o0 = __fmul_rn(cs[2 * j], pl.scale);
+        const float o1 = __fmul_rn(cs[2 * j + 1], ph.scale);
+        packed[j] = __byte_perm(__float_as_uint(o0), __float_as_uint(o1), 0x7632);
+    }
+    nibs = e2m1x8(cs);
+}
+
+// Saturation bits of 8 elements from their abs bits (4 words) against packed
+// limits: per half, 0x8000 + lim - a keeps bit 15 set exactly when a <= lim
+// (no borrow crosses halves since the result stays positive). The four bytes
+// holding those bits are gathered and their top bits collected by a multiply.
+__device__ __forceinline__ uint32_t sat8(const uint32_t (&aw)[4], const uint32_t (&limx)[4])
+{
+    const uint32_t b01 = __byte_perm(limx[0] - aw[0], limx[1] - aw[1], 0x7531);
+    const uint32_t b23 = __byte_perm(limx[2] - aw[2], limx[3] - aw[3], 0x7531);
+    const uint32_t g01 = (((b01 >> 7) & 0x01010101u) * 0x10204080u) >> 28;
+    const uint32_t g23 = (((b23 >> 7) & 0x01010101u) * 0x10204080u) >> 28;
+    return ~(g01 | (g23 << 4)) & 0xFFu;
+}
+
+// |x| bits of a word and the word with -0 halves cleared to +0.
+__device__ __forceinline__ void prep16(uint32_t w, uint32_t& aw, uint32_t& wc)
+{
+    aw = w & 0x7FFF7FFFu;
+    wc = w & ((aw + 0x7FFF7FFFu) | 0x7FFF7FFFu);
+}
+
 // ESZ: 2 (bf16) or 4 (fp32) bytes. LC lanes across columns (16 bytes each),
 // LR = 32/LC lanes across rows, RPT rows per thread, WR warps down the tile.
 // A tile is BS rows (one column-wise block; a group tail may be shorter) by
@@ -535,50 +613,81 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
             }
         }
 
-        // column-wise block parameters first (a register max down the thread's
-        // rows, a shuffle across the LR row lanes, shared memory across warps)
+        // Column-wise block parameters first: a max down the thread's rows, a
+        // shuffle across the LR row lanes, shared memory across warps.
         QP pc[COL ? VEC : 1];
-        bool crare = false;
+        bool cgen = false;                  // some column block needs the general path
+        uint32_t limxc[(COL && VEC == 8) ? 4 : 1];
+        bool csat = false;                  // some column block may saturate
         if constexpr (COL) {
-            uint32_t amc[VEC];
+            constexpr int NW = (VEC == 8) ? 4 : VEC;  // words (bf16 pairs) or elements (fp32)
+            uint32_t mc[NW];
 #pragma unroll
-            for (int e = 0; e < VEC; ++e)
-                amc[e] = 0;
+            for (int j = 0; j < NW; ++j)
+                mc[j] = 0;
 #pragma unroll
             for (int i = 0; i < RPT; ++i) {
-                uint32_t xb[VEC];
-                V::unpack(d[i], xb);
+                const uint32_t w[4] = {d[i].x, d[i].y, d[i].z, d[i].w};
 #pragma unroll
-                for (int e = 0; e < VEC; ++e)
-                    amc[e] = max(amc[e], xb[e] & 0x7FFFFFFFu);
+                for (int j = 0; j < NW; ++j) {
+                    if constexpr (VEC == 8)
+                        mc[j] = vmax2(mc[j], w[j] & 0x7FFF7FFFu);
+                    else
+                        mc[j] = max(mc[j], w[j] & 0x7FFFFFFFu);
+                }
             }
 #pragma unroll
             for (int o = LC; o < 32; o <<= 1) {
 #pragma unroll
-                for (int e = 0; e < VEC; ++e)
-                    amc[e] = max(amc[e], __shfl_xor_sync(FULL, amc[e], o));
+                for (int j = 0; j < NW; ++j) {
+                    const uint32_t v = __shfl_xor_sync(FULL, mc[j], o);
+                    if constexpr (VEC == 8)
+                        mc[j] = vmax2(mc[j], v);
+                    else
+                        mc[j] = max(mc[j], v);
+                }
             }
             if constexpr (WR > 1) {
                 if (lr == 0) {
 #pragma unroll
-                    for (int e = 0; e < VEC; ++e)
-                        s_am[wr * TC + lc * VEC + e] = amc[e];
+                    for (int j = 0; j < NW; ++j)
+                        s_am[wr * TC + lc * VEC + j] = mc[j];
                 }
                 __syncthreads();
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) {
+                for (int j = 0; j < NW; ++j) {
                     uint32_t m = 0;
 #pragma unroll
-                    for (int w = 0; w < WR; ++w)
-                        m = max(m, s_am[w * TC + lc * VEC + e]);
-                    amc[e] = m;
+                    for (int w = 0; w < WR; ++w) {
+                        const uint32_t v = s_am[w * TC + lc * VEC + j];
+                        if constexpr (VEC == 8)
+                            m = vmax2(m, v);
+                        else
+                            m = max(m, v);
+                    }
+                    mc[j] = m;
                 }
                 __syncthreads();  // s_am is rewritten by the next tile
             }
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
-                pc[e] = qparams(amc[e], a.mode, a.thr);
-                crare = crare || qp_rare(pc[e]);
+                uint32_t A;
+                if constexpr (VEC == 8)
+                    A = (e & 1) ? (mc[e / 2] & 0xFFFF0000u) : (mc[e / 2] << 16);
+                else
+                    A = mc[e];
+                pc[e] = qparams(A, a.mode, a.thr);
+            }
+            if constexpr (VEC == 8) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    cgen = cgen || !qp_fast16(pc[2 * j]) || !qp_fast16(pc[2 * j + 1]);
+                    limxc[j] = (0x8000u + qp_lim16(pc[2 * j])) | ((0x8000u + qp_lim16(pc[2 * j + 1])) << 16);
+                    // both halves of limx - amax keep bit 15 set when nothing in the column can saturate
+                    csat = csat || (((limxc[j] - mc[j]) & 0x80008000u) != 0x80008000u);
+                }
+            } else {
+                cgen = true;
             }
             if (a.scales_col && lr == 0 && wr == 0 && colok) {
                 uint8_t* sp = a.scales_col + (int64_t)rb * a.cols + col;
@@ -593,31 +702,62 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
             }
         }
 
-        // then one pass over the rows: both directions of row i, and the
-        // gradient of row i, before moving on
+        // Then one pass over the rows: both directions of row i, and the
+        // gradient of row i, before moving on.
 #pragma unroll
         for (int i = 0; i < RPT; ++i) {
             const int r = i * (LR * WR) + wr * LR + lr;
             const bool ok = colok && r < nrows;
             const int64_t row = row0 + r;
-            uint32_t xb[VEC];
-            V::unpack(d[i], xb);
+            const uint32_t w[4] = {d[i].x, d[i].y, d[i].z, d[i].w};
+            uint32_t aw[4], wc[4];
+            if constexpr (VEC == 8) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    prep16(w[j], aw[j], wc[j]);
+            }
             uint32_t gmask = 0;
             if constexpr (ROW) {
-                uint32_t am = 0;
-#pragma unroll
-                for (int e = 0; e < VEC; ++e)
-                    am = max(am, xb[e] & 0x7FFFFFFFu);
+                uint32_t am;
+                if constexpr (VEC == 8) {
+                    const uint32_t m2 = vmax2(vmax2(aw[0], aw[1]), vmax2(aw[2], aw[3]));
+                    am = max(m2 & 0xFFFFu, m2 >> 16);
+                } else {
+                    am = max(max(w[0] & 0x7FFFFFFFu, w[1] & 0x7FFFFFFFu), max(w[2] & 0x7FFFFFFFu, w[3] & 0x7FFFFFFFu));
+                }
 #pragma unroll
                 for (int o = 1; o < BL; o <<= 1)
                     am = max(am, __shfl_xor_sync(FULL, am, o));
-                const QP p = qparams(am, a.mode, a.thr);
-                uint32_t ob[VEC], nibs, sats;
-                quant_chunk<VEC, false>(xb, &p, lutb, ob, nibs, sats);
-                if (qp_rare(p)) {
+                const QP p = qparams(VEC == 8 ? am << 16 : am, a.mode, a.thr);
+                uint32_t packed[4], nibs, sats;
+                bool general = true;
+                if constexpr (VEC == 8) {
+                    if (qp_fast16(p)) {
+                        general = false;
+                        quant16<false>(wc, &p, lutb - 0x28000000u + 0x2C000000u, packed, nibs);
+                        const uint32_t lim = qp_lim16(p);
+                        sats = 0;
+                        if (am > lim) {
+                            const uint32_t lx = (0x8000u + lim) * 0x10001u;
+                            const uint32_t limx[4] = {lx, lx, lx, lx};
+                            sats = sat8(aw, limx);
+                        }
+                    }
+                }
+                if (general) {
+                    uint32_t xb[VEC], ob[VEC];
+                    V::unpack(d[i], xb);
+                    quant_chunk<VEC, false>(xb, &p, lutb, ob, nibs, sats);
+                    if (qp_rare(p)) {
 #pragma unroll
-                    for (int e = 0; e < VEC; ++e)
-                        rare_fixup<VEC>(p, e, ob, nibs, sats);
+                        for (int e = 0; e < VEC; ++e)
+                            rare_fixup<VEC>(p, e, ob, nibs, sats);
+                    }
+                    const uint4 pk = V::pack(ob);
+                    packed[0] = pk.x;
+                    packed[1] = pk.y;
+                    packed[2] = pk.z;
+                    packed[3] = pk.w;
                 }
                 if (a.grad_dir == MXFP4_ROWWISE)
                     gmask = sats;
@@ -627,7 +767,8 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
                 }
                 if (ok) {
                     if (a.y_row)
-                        st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * ESZ, V::pack(ob));
+                        st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * ESZ,
+                                  make_uint4(packed[0], packed[1], packed[2], packed[3]));
                     if (a.codes_row) {
                         if constexpr (VEC == 8)
                             *reinterpret_cast<uint32_t*>(a.codes_row + row * cstride + col / 2) = nibs;
@@ -641,13 +782,25 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
                 }
             }
             if constexpr (COL) {
-                uint32_t ob[VEC], nibs, sats;
-                quant_chunk<VEC, true>(xb, pc, lutb, ob, nibs, sats);
-                if (crare) {
+                uint32_t packed[4], nibs, sats;
+                if (!cgen) {
+                    if constexpr (VEC == 8) {
+                        quant16<true>(wc, pc, lutb - 0x28000000u + 0x2C000000u, packed, nibs);
+                        sats = csat ? sat8(aw, limxc) : 0u;
+                    }
+                } else {
+                    uint32_t xb[VEC], ob[VEC];
+                    V::unpack(d[i], xb);
+                    quant_chunk<VEC, true>(xb, pc, lutb, ob, nibs, sats);
 #pragma unroll
                     for (int e = 0; e < VEC; ++e)
                         if (qp_rare(pc[e]))
                             rare_fixup<VEC>(pc[e], e, ob, nibs, sats);
+                    const uint4 pk = V::pack(ob);
+                    packed[0] = pk.x;
+                    packed[1] = pk.y;
+                    packed[2] = pk.z;
+                    packed[3] = pk.w;
                 }
                 if (a.grad_dir == MXFP4_COLWISE)
                     gmask = sats;
@@ -657,7 +810,8 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
                 }
                 if (ok) {
                     if (a.y_col)
-                        st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * ESZ, V::pack(ob));
+                        st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * ESZ,
+                                  make_uint4(packed[0], packed[1], packed[2], packed[3]));
                     if (a.codes_col) {
                         if constexpr (VEC == 8)
                             *reinterpret_cast<uint32_t*>(a.codes_col + row * cstride + col / 2) = nibs;
