@@ -517,17 +517,50 @@ __device__ __forceinline__ void quant16(const uint32_t (&wc)[4], const QP* p, ui
     nibs = e2m1x8(cs);
 }
 
+// Scale exponent k of a block from its amax bits, by the same rule as
+// qparams but without building 2^k: non-finite amax yields k >= 125 here
+// (scale_factor <= 11 on the vector path), which the fast-path range test
+// below rejects.
+__device__ __forceinline__ int block_k(uint32_t A, int mode, uint32_t thr)
+{
+    if (mode == MXFP4_SCALE_FLOOR)
+        return max((int)(A >> 23) - 129, -127);
+    const int k = (int)(A >> 23) - (int)(thr >> 23) + 1 - ((A & 0x7FFFFFu) < (thr & 0x7FFFFFu) ? 1 : 0);
+    return max(k, -30);
+}
+
+// bf16 fast-path range: -126 <= k <= 16 (see qp_fast16).
+__device__ __forceinline__ bool k_fast16(int k) { return (uint32_t)(k + 126) <= 142u; }
+
+// 2^-k and 2^k for a fast-path k (both normal), as exponent-field arithmetic.
+__device__ __forceinline__ QP qp_of_k(int k)
+{
+    QP p;
+    p.inv = __uint_as_float(0x3F800000u - ((uint32_t)k << 23));
+    p.scale = __uint_as_float(0x3F800000u + ((uint32_t)k << 23));
+    return p;
+}
+
+// bf16 bits of 6 * 2^k = 1.5 * 2^(k+2) for a fast-path k.
+__device__ __forceinline__ uint32_t lim16_of_k(int k) { return ((uint32_t)k << 7) + 0x40C0u; }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
 // Saturation bits of 8 elements from their abs bits (4 words) against packed
-// limits: per half, 0x8000 + lim - a keeps bit 15 set exactly when a <= lim
-// (no borrow crosses halves since the result stays positive). The four bytes
-// holding those bits are gathered and their top bits collected by a multiply.
+// limits: per half, 0x8000 + lim - a keeps bit 15 set exactly when a <= lim.
+// A sign-replicating byte permute turns those bits into 0x00/0xFF bytes, a
+// mask keeps a different bit per element, and one multiply ORs the four bytes.
 __device__ __forceinline__ uint32_t sat8(const uint32_t (&aw)[4], const uint32_t (&limx)[4])
 {
-    const uint32_t b01 = __byte_perm(limx[0] - aw[0], limx[1] - aw[1], 0x7531);
-    const uint32_t b23 = __byte_perm(limx[2] - aw[2], limx[3] - aw[3], 0x7531);
-    const uint32_t g01 = (((b01 >> 7) & 0x01010101u) * 0x10204080u) >> 28;
-    const uint32_t g23 = (((b23 >> 7) & 0x01010101u) * 0x10204080u) >> 28;
-    return ~(g01 | (g23 << 4)) & 0xFFu;
+    const uint32_t m01 = prmt(limx[0] - aw[0], limx[1] - aw[1], 0xFDB9u);
+    const uint32_t m23 = prmt(limx[2] - aw[2], limx[3] - aw[3], 0xFDB9u);
+    const uint32_t keep = (m01 & 0x08040201u) | (m23 & 0x80402010u);
+    return ~(keep * 0x01010101u) >> 24;
 }
 
 // |x| bits of a word and the word with -0 halves cleared to +0.
@@ -537,12 +570,49 @@ __device__ __forceinline__ void prep16(uint32_t w, uint32_t& aw, uint32_t& wc)
     wc = w & ((aw + 0x7FFF7FFFu) | 0x7FFF7FFFu);
 }
 
+// General path for the VEC elements of one chunk, out of line so that the
+// fast path keeps its registers: exact block parameters (subnormal 2^k,
+// non-finite blocks, any scale_factor within the vector-path range), the
+// clamped lookup of qfast, and the rare-block fix-ups. ROWWISE: one block
+// with amax bits A[0]; COLWISE: one block per element with amax bits A[e].
+struct ChunkOut {
+    uint4 packed;
+    uint32_t nibs;
+    uint32_t sats;
+};
+
+template <int VEC, bool PER_ELEM>
+__device__ __noinline__ ChunkOut general_chunk(uint4 dv, const uint32_t* A, int mode, uint32_t thr, uint32_t lutb)
+{
+    QP p[PER_ELEM ? VEC : 1];
+#pragma unroll
+    for (int e = 0; e < (PER_ELEM ? VEC : 1); ++e)
+        p[e] = qparams(A[e], mode, thr);
+    uint32_t xb[VEC], ob[VEC];
+    Vec<VEC>::unpack(dv, xb);
+    ChunkOut r;
+    quant_chunk<VEC, PER_ELEM>(xb, p, lutb, ob, r.nibs, r.sats);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e)
+        if (qp_rare(p[PER_ELEM ? e : 0]))
+            rare_fixup<VEC>(p[PER_ELEM ? e : 0], e, ob, r.nibs, r.sats);
+    r.packed = Vec<VEC>::pack(ob);
+    return r;
+}
+
+// E8M0 byte of a block from its amax bits and k: 0xFF for a non-finite block
+// (a NaN or inf element, or 2^k beyond fp32), else k + 127.
+__device__ __forceinline__ uint32_t e8_of(uint32_t A, int k)
+{
+    return (A >= 0x7F800000u || k > 127) ? 0xFFu : (uint32_t)(k + 127);
+}
+
 // ESZ: 2 (bf16) or 4 (fp32) bytes. LC lanes across columns (16 bytes each),
 // LR = 32/LC lanes across rows, RPT rows per thread, WR warps down the tile.
 // A tile is BS rows (one column-wise block; a group tail may be shorter) by
 // LC*VEC columns.
 template <int ESZ, int BS, int LC, int RPT, int WR, bool ROW, bool COL, bool GROUPS, bool GRAD>
-__global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
+__global__ void __launch_bounds__(NTHREADS, COL ? 2 : 1) qdq_tile_kernel(const KArgs a)
 {
     constexpr int VEC = 16 / ESZ;
     constexpr int LR = 32 / LC;
@@ -579,6 +649,7 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
         S = (uint32_t)((a.rows + BS - 1) / BS);
     }
     const uint32_t lutb = (uint32_t)__cvta_generic_to_shared(s_lut) - 0x2C000000u;
+    const uint32_t lutb16 = lutb + 0x04000000u;  // lut_base - 0x28000000
 
     const char* xp = static_cast<const char*>(a.x);
     const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8, nblk = (a.cols + BS - 1) / BS;
@@ -615,13 +686,13 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
 
         // Column-wise block parameters first: a max down the thread's rows, a
         // shuffle across the LR row lanes, shared memory across warps.
-        QP pc[COL ? VEC : 1];
-        bool cgen = false;                  // some column block needs the general path
+        constexpr int NW = (VEC == 8) ? 4 : VEC;  // words (bf16 pairs) or elements (fp32)
+        uint32_t mc[COL ? NW : 1];
+        QP pc[COL ? VEC : 1];                      // fast-path 2^-k, 2^k per column
         uint32_t limxc[(COL && VEC == 8) ? 4 : 1];
-        bool csat = false;                  // some column block may saturate
+        bool cgen = false;                         // some column block needs the general path
+        bool csat = false;                         // some column block may saturate
         if constexpr (COL) {
-            constexpr int NW = (VEC == 8) ? 4 : VEC;  // words (bf16 pairs) or elements (fp32)
-            uint32_t mc[NW];
 #pragma unroll
             for (int j = 0; j < NW; ++j)
                 mc[j] = 0;
@@ -669,6 +740,7 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
                 }
                 __syncthreads();  // s_am is rewritten by the next tile
             }
+            uint32_t e8[VEC];
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
                 uint32_t A;
@@ -676,29 +748,33 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
                     A = (e & 1) ? (mc[e / 2] & 0xFFFF0000u) : (mc[e / 2] << 16);
                 else
                     A = mc[e];
-                pc[e] = qparams(A, a.mode, a.thr);
+                const int k = block_k(A, a.mode, a.thr);
+                e8[e] = e8_of(A, k);
+                if constexpr (VEC == 8) {
+                    cgen = cgen || !k_fast16(k);
+                    pc[e] = qp_of_k(k);
+                    const uint32_t lim = lim16_of_k(k);
+                    if (e & 1)
+                        limxc[e / 2] |= (0x8000u + lim) << 16;
+                    else
+                        limxc[e / 2] = 0x8000u + lim;
+                }
             }
             if constexpr (VEC == 8) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    cgen = cgen || !qp_fast16(pc[2 * j]) || !qp_fast16(pc[2 * j + 1]);
-                    limxc[j] = (0x8000u + qp_lim16(pc[2 * j])) | ((0x8000u + qp_lim16(pc[2 * j + 1])) << 16);
-                    // both halves of limx - amax keep bit 15 set when nothing in the column can saturate
+                for (int j = 0; j < 4; ++j)  // both halves of limx - amax keep bit 15 when nothing saturates
                     csat = csat || (((limxc[j] - mc[j]) & 0x80008000u) != 0x80008000u);
-                }
             } else {
                 cgen = true;
             }
             if (a.scales_col && lr == 0 && wr == 0 && colok) {
                 uint8_t* sp = a.scales_col + (int64_t)rb * a.cols + col;
-                if constexpr (VEC == 8) {
-                    uint2 v;
-                    v.x = pack_e8(pc[0], pc[1], pc[2], pc[3]);
-                    v.y = pack_e8(pc[4 % VEC], pc[5 % VEC], pc[6 % VEC], pc[7 % VEC]);
-                    *reinterpret_cast<uint2*>(sp) = v;
-                } else {
-                    *reinterpret_cast<uint32_t*>(sp) = pack_e8(pc[0], pc[1], pc[2], pc[3 % VEC]);
-                }
+                const uint32_t lo = e8[0] | (e8[1] << 8) | (e8[2] << 16) | (e8[3] << 24);
+                if constexpr (VEC == 8)
+                    *reinterpret_cast<uint2*>(sp) =
+                        make_uint2(lo, e8[4 % VEC] | (e8[5 % VEC] << 8) | (e8[6 % VEC] << 16) | (e8[7 % VEC] << 24));
+                else
+                    *reinterpret_cast<uint32_t*>(sp) = lo;
             }
         }
 
@@ -728,36 +804,27 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
 #pragma unroll
                 for (int o = 1; o < BL; o <<= 1)
                     am = max(am, __shfl_xor_sync(FULL, am, o));
-                const QP p = qparams(VEC == 8 ? am << 16 : am, a.mode, a.thr);
+                const uint32_t A = VEC == 8 ? am << 16 : am;
+                const int k = block_k(A, a.mode, a.thr);
                 uint32_t packed[4], nibs, sats;
-                bool general = true;
-                if constexpr (VEC == 8) {
-                    if (qp_fast16(p)) {
-                        general = false;
-                        quant16<false>(wc, &p, lutb - 0x28000000u + 0x2C000000u, packed, nibs);
-                        const uint32_t lim = qp_lim16(p);
-                        sats = 0;
-                        if (am > lim) {
-                            const uint32_t lx = (0x8000u + lim) * 0x10001u;
-                            const uint32_t limx[4] = {lx, lx, lx, lx};
-                            sats = sat8(aw, limx);
-                        }
+                if (VEC == 8 && k_fast16(k)) {
+                    const QP p = qp_of_k(k);
+                    quant16<false>(wc, &p, lutb16, packed, nibs);
+                    const uint32_t lim = lim16_of_k(k);
+                    sats = 0;
+                    if (am > lim) {
+                        const uint32_t lx = (0x8000u + lim) * 0x10001u;
+                        const uint32_t limx[4] = {lx, lx, lx, lx};
+                        sats = sat8(aw, limx);
                     }
-                }
-                if (general) {
-                    uint32_t xb[VEC], ob[VEC];
-                    V::unpack(d[i], xb);
-                    quant_chunk<VEC, false>(xb, &p, lutb, ob, nibs, sats);
-                    if (qp_rare(p)) {
-#pragma unroll
-                        for (int e = 0; e < VEC; ++e)
-                            rare_fixup<VEC>(p, e, ob, nibs, sats);
-                    }
-                    const uint4 pk = V::pack(ob);
-                    packed[0] = pk.x;
-                    packed[1] = pk.y;
-                    packed[2] = pk.z;
-                    packed[3] = pk.w;
+                } else {
+                    const ChunkOut g = general_chunk<VEC, false>(d[i], &A, a.mode, a.thr, lutb);
+                    packed[0] = g.packed.x;
+                    packed[1] = g.packed.y;
+                    packed[2] = g.packed.z;
+                    packed[3] = g.packed.w;
+                    nibs = g.nibs;
+                    sats = g.sats;
                 }
                 if (a.grad_dir == MXFP4_ROWWISE)
                     gmask = sats;
@@ -778,29 +845,32 @@ __global__ void __launch_bounds__(NTHREADS) qdq_tile_kernel(const KArgs a)
                     if (a.mask_row && (VEC == 8 || !(lc & 1)))
                         a.mask_row[row * mstride + col / 8] = (uint8_t)sats;
                     if (a.scales_row && (lc % BL) == 0)
-                        a.scales_row[row * nblk + col / BS] = (uint8_t)qp_e8(p);
+                        a.scales_row[row * nblk + col / BS] = (uint8_t)e8_of(A, k);
                 }
             }
             if constexpr (COL) {
                 uint32_t packed[4], nibs, sats;
                 if (!cgen) {
                     if constexpr (VEC == 8) {
-                        quant16<true>(wc, pc, lutb - 0x28000000u + 0x2C000000u, packed, nibs);
+                        quant16<true>(wc, pc, lutb16, packed, nibs);
                         sats = csat ? sat8(aw, limxc) : 0u;
                     }
                 } else {
-                    uint32_t xb[VEC], ob[VEC];
-                    V::unpack(d[i], xb);
-                    quant_chunk<VEC, true>(xb, pc, lutb, ob, nibs, sats);
+                    uint32_t Ac[VEC];
 #pragma unroll
-                    for (int e = 0; e < VEC; ++e)
-                        if (qp_rare(pc[e]))
-                            rare_fixup<VEC>(pc[e], e, ob, nibs, sats);
-                    const uint4 pk = V::pack(ob);
-                    packed[0] = pk.x;
-                    packed[1] = pk.y;
-                    packed[2] = pk.z;
-                    packed[3] = pk.w;
+                    for (int e = 0; e < VEC; ++e) {
+                        if constexpr (VEC == 8)
+                            Ac[e] = (e & 1) ? (mc[e / 2] & 0xFFFF0000u) : (mc[e / 2] << 16);
+                        else
+                            Ac[e] = mc[e];
+                    }
+                    const ChunkOut g = general_chunk<VEC, true>(d[i], Ac, a.mode, a.thr, lutb);
+                    packed[0] = g.packed.x;
+                    packed[1] = g.packed.y;
+                    packed[2] = g.packed.z;
+                    packed[3] = g.packed.w;
+                    nibs = g.nibs;
+                    sats = g.sats;
                 }
                 if (a.grad_dir == MXFP4_COLWISE)
                     gmask = sats;
