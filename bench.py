@@ -75,6 +75,27 @@ def step_bytes(rows: int, cols: int, s_col: int, esz: int = 2, block: int = 32) 
     return {"fwd": fwd, "bwd": bwd, "step": fwd + bwd}
 
 
+def rank_seed(base: int, rank: int) -> int:
+    """Every rank quantises its own batch (weak scaling): distinct seeds per rank."""
+    return base + 1000 * rank
+
+
+def reduce_max(values, world: int, device) -> list:
+    """Max over ranks of per-rank timings (a no-op for one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weak_value(bytes_per_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job GB/s: the bytes every rank moved over the slowest rank's time."""
+    return bytes_per_step * world * steps / (ms / 1e3) / 1e9
+
+
 def workload_desc(a, s_col: int) -> dict:
     return {
         "workload": "moe_grouped_dual_qdq_fwd_ste_bwd",
@@ -187,8 +208,8 @@ def run_ours(a, rank: int, world: int):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
 
-    x_h, counts, offsets = W.moe_grouped(a.rows, a.cols, a.groups, seed=4 + 1000 * rank)
-    g_h = W.train_step_grad(a.rows, a.cols, seed=5 + 1000 * rank)
+    x_h, counts, offsets = W.moe_grouped(a.rows, a.cols, a.groups, seed=rank_seed(4, rank))
+    g_h = W.train_step_grad(a.rows, a.cols, seed=rank_seed(5, rank))
     s_col = ops.mxfp4_colwise_scale_rows(offsets.tolist(), 0, a.rows, 32)
     xd, gd, gl = x_h.cuda(), g_h.cuda(), offsets.cuda()
 
@@ -244,12 +265,8 @@ def run_ours(a, rank: int, world: int):
         end.record(stream)
         torch.cuda.synchronize()
     barrier()
-    ms = start.elapsed_time(end)
-    fwd_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
-    t = torch.tensor([ms, fwd_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, fwd_ms = float(t[0]), float(t[1])
+    ms, fwd_ms = reduce_max([start.elapsed_time(end), statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)],
+                            world, "cuda")
 
     # e2e: same step through the public entry points with host buffers
     e2e = None
@@ -280,10 +297,7 @@ def run_ours(a, rank: int, world: int):
         s1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        te = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = (float(te[0]), h2d, d2h)
+        e2e = (reduce_max([s0.elapsed_time(s1)], world, "cuda")[0], h2d, d2h)
 
     return dict(ms=ms, fwd_ms=fwd_ms, s_col=s_col, clocks=sampler.summary(), e2e=e2e,
                 x_h=x_h, g_h=g_h, offsets=offsets, np=np)
@@ -335,7 +349,7 @@ def main():
         if rank == 0:
             peak, peak_kind = measured_peaks()
             b = step_bytes(a.rows, a.cols, r["s_col"])
-            value = b["step"] * world * a.steps / (r["ms"] / 1e3) / 1e9
+            value = weak_value(b["step"], a.steps, world, r["ms"])
             achieved = b["fwd"] / (r["fwd_ms"] / 1e3) / 1e9
             src = os.path.join(ROOT, "mxfp4_block_fake_b200", "csrc", "mxfp4.cu")
             line = {
@@ -359,7 +373,7 @@ def main():
             }
             if r["e2e"] is not None:
                 ms_e, h2d, d2h = r["e2e"]
-                line["e2e"] = {"value": round(b["step"] * world * a.steps / (ms_e / 1e3) / 1e9, 2),
+                line["e2e"] = {"value": round(weak_value(b["step"], a.steps, world, ms_e), 2),
                                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                                "ms_per_step": round(ms_e / a.steps, 3)}
             if world == 1 and not a.no_cpu_baseline:
