@@ -32,7 +32,8 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(p) > t for p in (SRC, HDR, __file__))
+    deps = (SRC, HDR, __file__, os.path.join(PKG, "csrc", "mxfp4_staged.cuh"))
+    return any(os.path.getmtime(p) > t for p in deps)
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:

@@ -25,6 +25,7 @@
 //  * generic kernels (one thread per block, scalar accesses) serve shapes and
 //    pointers the vector path cannot (cols or ld not a multiple of 16 bytes,
 //    unaligned buffers).
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <math.h>
@@ -361,14 +362,13 @@ __device__ __forceinline__ uint32_t pack_e8(const QP& a, const QP& b, const QP& 
 }
 
 // Lookup entry for u = floor(4 |y|), u < 64: the code magnitude as fp32 bits
-// (two significant bits, so the low half is zero) with the code index in the
-// low 3 bits. The index is the number of midpoints m with 4m <= u, i.e. with
-// m <= |y| since every 4m is an integer (ties go to the larger code).
+// (two significant bits, so the low half is zero). The code index is the
+// number of midpoints m with 4m <= u, i.e. with m <= |y| since every 4m is an
+// integer (ties go to the larger code).
 __device__ __forceinline__ uint32_t lut_entry(uint32_t u)
 {
     const uint32_t i = (u >= 1) + (u >= 3) + (u >= 5) + (u >= 7) + (u >= 10) + (u >= 14) + (u >= 20);
-    const uint32_t cb = i >= 2u ? (i << 22) + 0x3F000000u : (i == 1u ? 0x3F000000u : 0u);
-    return cb | i;
+    return i >= 2u ? (i << 22) + 0x3F000000u : (i == 1u ? 0x3F000000u : 0u);
 }
 
 // One element. y = fl(x / 2^k); t = 2^23 + floor(4|y|) (one fma rounding
@@ -1087,6 +1087,12 @@ __global__ void __launch_bounds__(NTHREADS)
     }
 }
 
+}  // namespace mxfp4
+
+#include "mxfp4_staged.cuh"
+
+namespace mxfp4 {
+
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
@@ -1260,6 +1266,78 @@ static mxfp4_status launch(KernelFn fn, int64_t work_units, size_t smem, const K
     return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
 }
 
+// ---- staged path: TMA tensor maps ------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the library
+// does not link libcuda directly); nullptr when unavailable.
+static EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            (void)cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D bf16 map of x: inner dimension cols, outer rows, row pitch ld * 2
+// bytes; 64 x 32 boxes with the 128-byte swizzle; out-of-range elements read
+// as zero.
+static bool make_tmap(CUtensorMap* tm, const mxfp4_qdq_args* A)
+{
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)A->cols, (cuuint64_t)A->rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)A->ld * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)SG_SLAB_COLS, (cuuint32_t)SG_ROWS};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(A->x), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+typedef void (*StagedFn)(const CUtensorMap, const KArgs);
+
+template <bool ALL>
+static StagedFn pick_staged(bool row, bool groups)
+{
+    return row ? (groups ? qdq_staged_kernel<true, true, ALL> : qdq_staged_kernel<true, false, ALL>)
+               : (groups ? qdq_staged_kernel<false, true, ALL> : qdq_staged_kernel<false, false, ALL>);
+}
+
+static mxfp4_status launch_staged(bool row, bool groups, const CUtensorMap& tm, const KArgs& k, int64_t tiles,
+                                  size_t plan_smem, cudaStream_t s)
+{
+    const bool all = k.y_col && k.codes_col && k.scales_col && k.mask_col &&
+                     (!row || (k.y_row && k.codes_row && k.scales_row && k.mask_row));
+    StagedFn fn = all ? pick_staged<true>(row, groups) : pick_staged<false>(row, groups);
+    const size_t smem = sizeof(StagedSmem) + 1024 + plan_smem;
+    if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MXFP4_ECUDA;
+    const int sms = device_sms();
+    const int occ = occupancy((const void*)fn, smem);
+    if (sms <= 0 || occ <= 0)
+        return MXFP4_ECUDA;
+    int64_t grid = (int64_t)sms * occ;
+    if (tiles < grid)
+        grid = tiles < 1 ? 1 : tiles;
+    fn<<<(unsigned)grid, NTHREADS, smem, s>>>(tm, k);
+    return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
+}
+
 static mxfp4_status check_geometry(const mxfp4_qdq_args* a)
 {
     if (!a)
@@ -1376,6 +1454,16 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     const size_t plan_smem = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
     const int64_t s_bound = groups ? A->rows / bs + A->num_groups : (A->rows + bs - 1) / bs;
 
+    if (fast && esz == 2 && bs == 32 && col && !grad) {
+        CUtensorMap tm;
+        if (make_tmap(&tm, A)) {
+            const int64_t n_ct = (A->cols + SG_COLS - 1) / SG_COLS;
+            if (s_bound * n_ct >= (int64_t)INT32_MAX)
+                return MXFP4_EUNSUPPORTED;
+            k.n_ct = (uint32_t)n_ct;
+            return launch_staged(row, groups, tm, k, s_bound * n_ct, plan_smem, s);
+        }
+    }
     if (fast) {
         int tc = 0, nwg = 1;
         KernelFn fn;
