@@ -66,6 +66,7 @@ struct KArgs {
     int32_t* status;
     uint32_t n_ct;  // column tiles of the tile kernel
     uint32_t thr;   // PAGE mode: fp32 bits of T0 (see qparams)
+    uint32_t ts_flags;  // staged kernel: column-wise outputs written by TMA stores (SG_TS_*)
 };
 
 // ---------------------------------------------------------------------------
@@ -1292,38 +1293,69 @@ static EncodeTiledFn encode_tiled()
     return fn;
 }
 
-// 2-D bf16 map of x: inner dimension cols, outer rows, row pitch ld * 2
-// bytes; 64 x 32 boxes with the 128-byte swizzle; out-of-range elements read
-// as zero.
-static bool make_tmap(CUtensorMap* tm, const mxfp4_qdq_args* A)
+// One 2-D tiled map: inner dimension d0 (elements of esz bytes), outer d1,
+// row pitch bytes, box b0 x b1.
+static bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, void* base, uint64_t d0, uint64_t d1, uint64_t pitch,
+                      uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw)
 {
     EncodeTiledFn fn = encode_tiled();
     if (!fn)
         return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)A->cols, (cuuint64_t)A->rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)A->ld * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)SG_SLAB_COLS, (cuuint32_t)SG_ROWS};
+    const cuuint64_t dims[2] = {(cuuint64_t)d0, (cuuint64_t)d1};
+    const cuuint64_t strides[1] = {(cuuint64_t)pitch};
+    const cuuint32_t box[2] = {(cuuint32_t)b0, (cuuint32_t)b1};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(A->x), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(tm, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-typedef void (*StagedFn)(const CUtensorMap, const KArgs);
-
-template <bool ALL>
-static StagedFn pick_staged(bool row, bool groups)
+// Maps of the staged kernel. x: bf16 [rows, cols] with row pitch ld * 2
+// bytes, 64 x 32 boxes with the 128-byte swizzle (out-of-range elements read
+// as zero). Column-wise outputs, each only where TMA can address it (16-byte
+// aligned base and row pitch) and the tensor holds at least one full tile:
+// y_col as x (pitch ld_y * 2), codes_col [rows, cols/2] bytes in 128 x 32
+// boxes with the 128-byte swizzle, mask_col [rows, cols/8] bytes in 32 x 32
+// boxes. Returns false when the input map cannot be built.
+static bool make_staged_maps(StagedMaps* m, const KArgs& k, uint32_t* ts_flags)
 {
-    return row ? (groups ? qdq_staged_kernel<true, true, ALL> : qdq_staged_kernel<true, false, ALL>)
-               : (groups ? qdq_staged_kernel<false, true, ALL> : qdq_staged_kernel<false, false, ALL>);
+    memset(m, 0, sizeof(*m));
+    *ts_flags = 0;
+    if (!encode_2d(&m->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(k.x), (uint64_t)k.cols,
+                   (uint64_t)k.rows, (uint64_t)k.ld * 2, SG_SLAB_COLS, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        return false;
+    if (k.cols < SG_COLS || k.rows < SG_ROWS)
+        return true;
+    if (k.y_col && aligned(k.y_col, 16) && (k.ld_y * 2) % 16 == 0 &&
+        encode_2d(&m->y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.y_col, (uint64_t)k.cols, (uint64_t)k.rows,
+                  (uint64_t)k.ld_y * 2, SG_SLAB_COLS, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        *ts_flags |= SG_TS_Y;
+    if (k.codes_col && aligned(k.codes_col, 16) && (k.cols / 2) % 16 == 0 &&
+        encode_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.codes_col, (uint64_t)k.cols / 2, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 2, SG_COLS / 2, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        *ts_flags |= SG_TS_CODES;
+    if (k.mask_col && aligned(k.mask_col, 16) && (k.cols / 8) % 16 == 0 &&
+        encode_2d(&m->mask, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.mask_col, (uint64_t)k.cols / 8, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 8, SG_COLS / 8, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+        *ts_flags |= SG_TS_MASK;
+    return true;
 }
 
-static mxfp4_status launch_staged(bool row, bool groups, const CUtensorMap& tm, const KArgs& k, int64_t tiles,
+typedef void (*StagedFn)(const StagedMaps, const KArgs);
+
+static mxfp4_status launch_staged(bool row, bool groups, const StagedMaps& maps, const KArgs& k, int64_t tiles,
                                   size_t plan_smem, cudaStream_t s)
 {
-    const bool all = k.y_col && k.codes_col && k.scales_col && k.mask_col &&
-                     (!row || (k.y_row && k.codes_row && k.scales_row && k.mask_row));
-    StagedFn fn = all ? pick_staged<true>(row, groups) : pick_staged<false>(row, groups);
+    StagedFn fn;
+    if (k.mode == MXFP4_SCALE_FLOOR)
+        fn = row ? (groups ? qdq_staged_kernel<true, true, MXFP4_SCALE_FLOOR>
+                           : qdq_staged_kernel<true, false, MXFP4_SCALE_FLOOR>)
+                 : (groups ? qdq_staged_kernel<false, true, MXFP4_SCALE_FLOOR>
+                           : qdq_staged_kernel<false, false, MXFP4_SCALE_FLOOR>);
+    else
+        fn = row ? (groups ? qdq_staged_kernel<true, true, MXFP4_SCALE_PAGE>
+                           : qdq_staged_kernel<true, false, MXFP4_SCALE_PAGE>)
+                 : (groups ? qdq_staged_kernel<false, true, MXFP4_SCALE_PAGE>
+                           : qdq_staged_kernel<false, false, MXFP4_SCALE_PAGE>);
     const size_t smem = sizeof(StagedSmem) + 1024 + plan_smem;
     if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MXFP4_ECUDA;
@@ -1334,7 +1366,7 @@ static mxfp4_status launch_staged(bool row, bool groups, const CUtensorMap& tm, 
     int64_t grid = (int64_t)sms * occ;
     if (tiles < grid)
         grid = tiles < 1 ? 1 : tiles;
-    fn<<<(unsigned)grid, NTHREADS, smem, s>>>(tm, k);
+    fn<<<(unsigned)grid, NTHREADS, smem, s>>>(maps, k);
     return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
 }
 
@@ -1454,14 +1486,16 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     const size_t plan_smem = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
     const int64_t s_bound = groups ? A->rows / bs + A->num_groups : (A->rows + bs - 1) / bs;
 
-    if (fast && esz == 2 && bs == 32 && col && !grad) {
-        CUtensorMap tm;
-        if (make_tmap(&tm, A)) {
+    // TMA coordinates and the staged kernel's tile bookkeeping are 32-bit
+    if (fast && esz == 2 && bs == 32 && col && !grad && A->rows <= INT32_MAX - 2 * SG_ROWS &&
+        A->cols <= INT32_MAX - 2 * SG_COLS) {
+        StagedMaps maps;
+        if (make_staged_maps(&maps, k, &k.ts_flags)) {
             const int64_t n_ct = (A->cols + SG_COLS - 1) / SG_COLS;
             if (s_bound * n_ct >= (int64_t)INT32_MAX)
                 return MXFP4_EUNSUPPORTED;
             k.n_ct = (uint32_t)n_ct;
-            return launch_staged(row, groups, tm, k, s_bound * n_ct, plan_smem, s);
+            return launch_staged(row, groups, maps, k, s_bound * n_ct, plan_smem, s);
         }
     }
     if (fast) {

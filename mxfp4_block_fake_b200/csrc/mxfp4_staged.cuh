@@ -2,40 +2,71 @@
 // column-wise or both directions (included by mxfp4.cu; shares its helpers).
 //
 // A tile is one column-wise block of 32 rows (shorter at a group tail) by 256
-// columns. TMA (cp.async.bulk.tensor, 2-D, no multicast) brings each tile into
-// shared memory as four 64-column slabs with the 128-byte swizzle, four tiles
-// ahead of the computation, so the bytes in flight do not depend on registers.
+// columns. Each CTA walks a contiguous range of tiles (row block major, so
+// consecutive tiles are neighbours along the row). TMA (cp.async.bulk.tensor,
+// 2-D, no multicast) brings each tile into shared memory as four 64-column
+// slabs with the 128-byte swizzle, SG_STAGES tiles ahead of the computation.
+// Thread 0 also writes the tile's coordinates next to the stage, so the other
+// threads never search the group plan.
+//
 // Per tile every one of the 256 threads owns
-//   * one row-wise block (32 elements of one row): amax, exponent and
-//     parameters once per block, no shuffles; and
-//   * one column octet over four rows (32 elements) of the column-wise pass:
-//     warp w owns tile columns 32w..32w+31 over all 32 rows, so the column
-//     amax is a three-step shuffle, each lane computes the parameters of one
-//     column of its octet and the octet's eight lanes share them by shuffles;
-//     no CTA barrier is needed except the one that frees a stage.
-// Shared-memory reads are conflict-free by construction: in both passes the
-// eight lanes of a quarter-warp read eight distinct 16-byte chunks of the same
-// 1024-byte swizzle atom. Every wait on an mbarrier is bounded; on expiry the
-// kernel records MXFP4_ECUDA in the caller's status word (when given) and
-// returns.
+//   * one row-wise block (32 elements of one row), stored straight to global
+//     memory with 32- and 16-byte stores; and
+//   * one column pair over 16 of the 32 rows of the column-wise pass: lanes
+//     l and l ^ 16 of a warp share the pair (rows with bit 2 clear / set), so
+//     the column amax takes one shuffle and each thread derives the two
+//     columns' parameters itself. Its column-wise outputs go to a staging
+//     tile in shared memory (same swizzled layout as the input), which TMA
+//     stores (cp.async.bulk.tensor ... bulk_group) write to global memory
+//     once the tile is complete. Group-tail and ragged tiles, and outputs
+//     whose layout TMA cannot address, are copied out by the threads instead.
+// Shared-memory accesses are conflict-free by construction: the two
+// half-warps of the column pass read and write rows whose swizzle phases
+// differ by 4, i.e. disjoint 64-byte halves of the bank space.
+//
+// One CTA barrier per tile. Before it, thread 0 waits until the previous
+// tile's TMA stores have read their staging buffer (double-buffered), so the
+// next tile may write it; after it, thread 0 issues this tile's stores and
+// refills the freed input stage. Every wait on an mbarrier is bounded; on
+// expiry the CTA records MXFP4_ECUDA in the caller's status word (when
+// given), waits (bounded) for its own loads still in flight and for its
+// stores, and returns.
 
 namespace mxfp4 {
 
-constexpr int SG_ROWS = 32;                      // rows per tile (= the block)
-constexpr int SG_COLS = 256;                     // columns per tile
-constexpr int SG_SLAB_COLS = 64;                 // columns per TMA box (128 bytes of bf16)
+constexpr int SG_ROWS = 32;                                // rows per tile (= the block)
+constexpr int SG_COLS = 256;                               // columns per tile
+constexpr int SG_SLAB_COLS = 64;                           // columns per TMA box (128 bytes of bf16)
 constexpr int SG_SLAB_BYTES = SG_SLAB_COLS * 2 * SG_ROWS;  // 4096
 constexpr int SG_TILE_BYTES = 4 * SG_SLAB_BYTES;           // 16384
-constexpr int SG_STAGES = 4;
-constexpr uint32_t SG_WAIT_LIMIT = 1u << 22;     // try_wait polls before giving up
+constexpr int SG_CODE_BYTES = SG_ROWS * SG_COLS / 2;       // 4096: e2m1 codes of a tile
+constexpr int SG_MASK_WORDS = SG_ROWS * SG_COLS / 32;      // 256: saturation bits of a tile
+constexpr int SG_STAGES = 3;
+constexpr uint32_t SG_WAIT_LIMIT = 1u << 22;               // try_wait polls before giving up
+
+// which column-wise outputs leave through TMA stores on full tiles
+constexpr uint32_t SG_TS_Y = 1u, SG_TS_CODES = 2u, SG_TS_MASK = 4u;
 
 struct __align__(1024) StagedSmem {
-    uint8_t tiles[SG_STAGES][SG_TILE_BYTES];     // 1024-aligned slabs (swizzle atoms)
+    uint8_t tiles[SG_STAGES][SG_TILE_BYTES];  // input stages (1024-aligned swizzle atoms)
+    uint8_t ycol[2][SG_TILE_BYTES];           // column-wise y staging, input layout
+    uint8_t ccol[2][SG_CODE_BYTES];           // column-wise codes staging, 128-byte rows, swizzled
+    uint32_t mcol[2][SG_MASK_WORDS];          // column-wise saturation bits, 32-byte rows
+    uint32_t limw[8][16];                     // per warp and column pair: 0x8000 + limit bits of each column
+    int4 info[SG_STAGES];                     // row0, nrows, col0, row block of each stage's tile
     uint32_t lut[64];
-    unsigned long long full[SG_STAGES];          // mbarriers, one per stage
+    unsigned long long full[SG_STAGES];       // mbarriers, one per stage
+    int err;
+};
+
+// TMA descriptors: the input and the three column-wise outputs (the output
+// maps are only read when the matching SG_TS_* flag is set).
+struct StagedMaps {
+    CUtensorMap x, y, codes, mask;
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
@@ -74,68 +105,130 @@ __device__ __forceinline__ void tma_load_slab(uint32_t dst, const CUtensorMap* m
         : "memory");
 }
 
-// Byte offset of 16-byte chunk c (0..7) of tile row r inside a slab laid out
-// with the 128-byte swizzle: the chunk index is XORed with r mod 8.
-__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr)
+// One box from shared memory to global memory (bulk-group completion). The
+// box lies wholly inside the tensor and its inner coordinate is a multiple of
+// 16 bytes.
+__device__ __forceinline__ void tma_store_box(const CUtensorMap* map, uint32_t src, int x, int y)
 {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map), "r"(src),
+                 "r"(x), "r"(y)
+                 : "memory");
 }
 
-// ---- packed fp32 pairs (f32x2) ------------------------------------------------
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ __forceinline__ uint64_t pk2(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
-__device__ __forceinline__ uint32_t lo32(uint64_t v) { return (uint32_t)v; }
-__device__ __forceinline__ uint32_t hi32(uint64_t v) { return (uint32_t)(v >> 32); }
-
-__device__ __forceinline__ uint64_t fma_rm2(uint64_t a, uint64_t b, uint64_t c)
-{
-    uint64_t r;
-    asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
-__device__ __forceinline__ uint64_t mul_rn2(uint64_t a, uint64_t b)
-{
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t lds32(uint32_t addr)
+// A code-table entry. Not volatile: the table does not change once built, so
+// the compiler may schedule these loads freely among the surrounding work.
+__device__ __forceinline__ uint32_t lut_load(uint32_t addr)
 {
     uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
 
-// 8 bf16 elements (4 words) of fast-path blocks, two elements per packed fp32
-// instruction. aw: |x| bits, from which the index is formed (the high element
-// carries the low one's magnitude below its own last bit, less than one bf16
-// ulp, which cannot carry it across a quarter of 2^k); wc: x with -0 cleared,
-// which supplies the signs. t = 2^21 + |x| * 2^-k rounded down (fp32 spacing
-// on [2^21, 2^22) is 1/4), so t's bits are 0x4A000000 + floor(4|y|); lutb16 =
-// table base - 0x28000000 folds the offset into the address shift-add.
-template <bool PER_WORD>
-__device__ __forceinline__ void quant16x2(const uint32_t* aw, const uint32_t* wc, const uint64_t* inv2,
-                                          const uint64_t* scale2, uint32_t lutb16, uint32_t* packed, uint32_t& nibs)
+// Typed views of shared memory by byte offset (ordinary loads and stores, so
+// that the compiler orders them against the barriers and schedules them
+// freely among themselves).
+__device__ __forceinline__ uint32_t sm_ld32(const uint8_t* base, uint32_t off)
 {
-    constexpr uint64_t MAGIC2 = 0x4A0000004A000000ull;  // 2^21 in both halves
-    float cs[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint64_t t = fma_rm2(pk2(aw[j] << 16, aw[j]), inv2[PER_WORD ? j : 0], MAGIC2);
-        const uint32_t clo = lds32(lutb16 + (lo32(t) << 2)) | ((wc[j] << 16) & 0x80000000u);
-        const uint32_t chi = lds32(lutb16 + (hi32(t) << 2)) | (wc[j] & 0x80000000u);
-        const uint64_t o = mul_rn2(pk2(clo, chi), scale2[PER_WORD ? j : 0]);
-        packed[j] = __byte_perm(lo32(o), hi32(o), 0x7632);
-        cs[2 * j] = __uint_as_float(clo);
-        cs[2 * j + 1] = __uint_as_float(chi);
+    return *reinterpret_cast<const uint32_t*>(base + off);
+}
+__device__ __forceinline__ uint4 sm_ld128(const uint8_t* base, uint32_t off)
+{
+    return *reinterpret_cast<const uint4*>(base + off);
+}
+__device__ __forceinline__ void sm_st32(uint8_t* base, uint32_t off, uint32_t v)
+{
+    *reinterpret_cast<uint32_t*>(base + off) = v;
+}
+
+__device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// E2M1 byte of one word of signed packed bf16 codes (low element in the low
+// nibble). The high element is converted from the whole word read as fp32:
+// the low element's bits sit below its last bf16 bit and cannot move it to
+// another E2M1 value (a code of zero gives a subnormal of the same sign).
+__device__ __forceinline__ uint32_t e2m1_byte(uint32_t P)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+        "cvt.u32.u8 %0, b;\n\t}"
+        : "=r"(r)
+        : "f"(__uint_as_float(P)), "f"(__uint_as_float(P << 16)));
+    return r;
+}
+
+// E2M1 nibbles of four words of signed packed bf16 codes (8 elements).
+__device__ __forceinline__ uint32_t e2m1_word(const uint32_t* P)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %1, %2;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %3, %4;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %5, %6;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %7, %8;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(__uint_as_float(P[0])), "f"(__uint_as_float(P[0] << 16)), "f"(__uint_as_float(P[1])),
+          "f"(__uint_as_float(P[1] << 16)), "f"(__uint_as_float(P[2])), "f"(__uint_as_float(P[2] << 16)),
+          "f"(__uint_as_float(P[3])), "f"(__uint_as_float(P[3] << 16)));
+    return r;
+}
+
+// Block exponent for a scale mode fixed at compile time (block_k's rule).
+template <int MODE>
+__device__ __forceinline__ int block_kt(uint32_t A, uint32_t thr)
+{
+    if constexpr (MODE == MXFP4_SCALE_FLOOR) {
+        return max((int)(A >> 23) - 129, -127);
+    } else {
+        const int k = (int)(A >> 23) - (int)(thr >> 23) + 1 - ((A & 0x7FFFFFu) < (thr & 0x7FFFFFu) ? 1 : 0);
+        return max(k, -30);
     }
-    nibs = e2m1x8(cs);
+}
+
+// Fast-path exponent range of this kernel: 2^k and every code * 2^k are
+// normal bf16 numbers (k >= -125), and the limit bits of lim16_of_k stay
+// below 0x8000 (k <= 16).
+__device__ __forceinline__ bool k_fast_bf(int k) { return (uint32_t)(k + 125) <= 141u; }
+
+// bf16 bits of 2^k for a fast-path k.
+__device__ __forceinline__ uint32_t bf16_pow2(int k) { return (uint32_t)(k + 127) << 7; }
+
+// One word (two bf16 elements) of fast-path blocks. aw: |x| bits; sg: the
+// sign bits to keep (those of nonzero elements). inv_*: 2^-k of each
+// element's block; s2: packed bf16 2^k of each element's block.
+// t = 2^21 + |x| * 2^-k rounded down (fp32 spacing on [2^21, 2^22) is 1/4),
+// so t's bits are 0x4A000000 + floor(4|y|); lutb16 = table base - 0x28000000
+// folds that offset into the address shift-add. The high element is indexed
+// from the whole word: the low element's magnitude lies below its last bf16
+// bit and cannot carry it across a quarter of 2^k. Returns the dequantised
+// packed bf16 pair; P receives the signed codes.
+__device__ __forceinline__ uint32_t qword(uint32_t aw, uint32_t sg, float inv_lo, float inv_hi, uint32_t s2,
+                                          uint32_t lutb16, uint32_t& P)
+{
+    const float tl = __fmaf_rd(__uint_as_float(aw << 16), inv_lo, 0x1p21f);
+    const float th = __fmaf_rd(__uint_as_float(aw), inv_hi, 0x1p21f);
+    const uint32_t el = lut_load(lutb16 + (__float_as_uint(tl) << 2));
+    const uint32_t eh = lut_load(lutb16 + (__float_as_uint(th) << 2));
+    P = __byte_perm(el, eh, 0x7632) | sg;
+    return hmul2_bf16(P, s2);
+}
+
+// |x| bits of a word and the sign bits of its nonzero halves (-0 gives +0).
+__device__ __forceinline__ void prep_bf(uint32_t w, uint32_t& aw, uint32_t& sg)
+{
+    aw = w & 0x7FFF7FFFu;
+    sg = w & (aw + 0x7FFF7FFFu) & 0x80008000u;
 }
 
 __device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v)
@@ -145,25 +238,9 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v)
                  : "memory");
 }
 
-// Tile t -> first row, row count, first column (group plan or uniform blocks).
-template <bool GROUPS>
-__device__ __forceinline__ void staged_tile(const KArgs& a, const int32_t* s_bpre, const int32_t* s_rst, uint32_t t,
-                                            int64_t& row0, int& nrows, int64_t& col0, uint32_t& rb)
-{
-    rb = t / a.n_ct;
-    const uint32_t ct = t - rb * a.n_ct;
-    if constexpr (GROUPS) {
-        plan_lookup(s_bpre, s_rst, a.num_groups, rb, SG_ROWS, row0, nrows);
-    } else {
-        row0 = (int64_t)rb * SG_ROWS;
-        nrows = (int)min((int64_t)SG_ROWS, a.rows - row0);
-    }
-    col0 = (int64_t)ct * SG_COLS;
-}
-
-// Stores of one row-wise block (32 elements) for any tile: null outputs are
-// skipped and a row's last block may hold only 8, 16 or 24 real elements
-// (cols is a multiple of 8 here).
+// Stores of one row-wise block (32 elements): null outputs are skipped and a
+// row's last block may hold only 8, 16 or 24 real elements (cols is a
+// multiple of 8 here).
 __device__ __forceinline__ void store_row_block(const KArgs& a, int64_t row, int64_t col, const uint32_t* packed,
                                                 const uint32_t* nib, uint32_t sats, uint32_t e8, bool v8y, bool a16,
                                                 bool a4, int64_t cstride, int64_t mstride, int64_t nblk)
@@ -209,10 +286,108 @@ __device__ __forceinline__ void store_row_block(const KArgs& a, int64_t row, int
         a.scales_row[row * nblk + col / 32] = (uint8_t)e8;
 }
 
-// ALL: every output of the computed directions is present (the common case),
-// so the full-tile fast paths store without null checks.
-template <bool ROW, bool GROUPS, bool ALL>
-__global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_constant__ CUtensorMap tmap, const KArgs a)
+// Tile sequence of one CTA: row block rb and column tile ct, advanced in
+// order; g tracks the group that holds rb (largest g with s_bpre[g] <= rb,
+// which skips empty groups).
+template <bool GROUPS>
+struct TileWalk {
+    uint32_t rb, ct;
+    int g;
+
+    __device__ void start(const KArgs& a, const int32_t* s_bpre, uint32_t t)
+    {
+        rb = t / a.n_ct;
+        ct = t - rb * a.n_ct;
+        g = 0;
+        if constexpr (GROUPS) {
+            int lo = 0, hi = a.num_groups - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if ((uint32_t)s_bpre[mid] <= rb)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            g = lo;
+        }
+    }
+
+    __device__ void next(const KArgs& a, const int32_t* s_bpre)
+    {
+        if (++ct == a.n_ct) {
+            ct = 0;
+            ++rb;
+            if constexpr (GROUPS) {
+                while (g + 1 < a.num_groups && (uint32_t)s_bpre[g + 1] <= rb)
+                    ++g;
+            }
+        }
+    }
+
+    // row0, nrows, col0, rb
+    __device__ int4 info(const KArgs& a, const int32_t* s_bpre, const int32_t* s_rst) const
+    {
+        int r0, nr;
+        if constexpr (GROUPS) {
+            r0 = s_rst[g] + (int)(rb - (uint32_t)s_bpre[g]) * SG_ROWS;
+            nr = min(SG_ROWS, s_rst[g + 1] - r0);
+        } else {
+            r0 = (int)rb * SG_ROWS;
+            nr = (int)min((int64_t)SG_ROWS, a.rows - r0);
+        }
+        return make_int4(r0, nr, (int)ct * SG_COLS, (int)rb);
+    }
+};
+
+// Copy the staged column-wise outputs of a tile to global memory with the
+// threads (group tails, ragged tiles, outputs TMA cannot address).
+__device__ __forceinline__ void copy_col_outputs(const KArgs& a, const StagedSmem& sm, int buf, int row0, int nrows,
+                                                 int col0, bool cy, bool cc, bool cm)
+{
+    const int tid = threadIdx.x;
+    const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8;
+    const uint8_t* yb = sm.ycol[buf];
+    const uint8_t* cb = sm.ccol[buf];
+    const uint8_t* mb = reinterpret_cast<const uint8_t*>(sm.mcol[buf]);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int q = tid + NTHREADS * m;  // 0..1023
+        const int r = q >> 5, u = q & 31;
+        if (r >= nrows)
+            continue;
+        const int64_t row = row0 + r;
+        const int col = col0 + 8 * u;  // y chunk u / codes word u / mask byte u: columns col..col+7
+        if (col >= a.cols)
+            continue;
+        if (cy) {
+            const uint4 v = sm_ld128(yb, (u >> 3) * SG_SLAB_BYTES + r * 128 + (((u & 7) ^ (r & 7)) << 4));
+            st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * 2, v);
+        }
+        if (cc) {
+            const uint32_t v = sm_ld32(cb, r * 128 + (((u >> 2) ^ (r & 7)) << 4) + 4 * (u & 3));
+            *reinterpret_cast<uint32_t*>(a.codes_col + row * cstride + col / 2) = v;
+        }
+        if (cm)
+            a.mask_col[row * mstride + col / 8] = mb[r * 32 + u];
+    }
+}
+
+// ORs a warp's column-pass saturation bits into the staged mask words (one
+// 32-bit word per tile row and warp, bit 2p + e for column pair p). Called
+// by the whole warp: the words were zeroed by other lanes.
+__device__ __forceinline__ void col_sat_store(uint32_t* mwords, uint32_t bits, int h, int p, int warp)
+{
+    __syncwarp();
+    while (bits) {
+        const int i = (__ffs(bits) - 1) >> 1;
+        const uint32_t two = (bits >> (2 * i)) & 3u;
+        bits &= ~(3u << (2 * i));
+        atomicOr(&mwords[(8 * (i >> 2) + 4 * h + (i & 3)) * 8 + warp], two << (2 * p));
+    }
+}
+
+template <bool ROW, bool GROUPS, int MODE>
+__global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_constant__ StagedMaps maps, const KArgs a)
 {
     extern __shared__ __align__(1024) uint8_t s_dyn[];
     // the swizzle pattern follows absolute shared-memory address bits, so the
@@ -227,6 +402,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
     if (tid < 64)
         sm.lut[tid] = lut_entry(tid);
     if (tid == 0) {
+        sm.err = 0;
         for (int s = 0; s < SG_STAGES; ++s)
             mbar_init(smem_addr(&sm.full[s]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -244,271 +420,308 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
         S = (uint32_t)((a.rows + SG_ROWS - 1) / SG_ROWS);
     }
     const uint32_t ntiles = S * a.n_ct;
+    const uint32_t t_begin = (uint32_t)(((uint64_t)blockIdx.x * ntiles) / gridDim.x);
+    const uint32_t t_end = (uint32_t)(((uint64_t)(blockIdx.x + 1) * ntiles) / gridDim.x);
     const uint32_t lutb = smem_addr(sm.lut) - 0x2C000000u;
     const uint32_t lutb16 = lutb + 0x04000000u;
     const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8, nblk = (a.cols + 31) / 32;
-    const bool v8y = ((a.ld_y * 2) % 32 == 0) && (((uintptr_t)a.y_row | (uintptr_t)a.y_col) % 32 == 0);
+    const bool v8y = ((a.ld_y * 2) % 32 == 0) && ((uintptr_t)a.y_row % 32 == 0);
     const bool a16 = (cstride % 16 == 0) && ((uintptr_t)a.codes_row % 16 == 0);
     const bool a4 = (mstride % 4 == 0) && ((uintptr_t)a.mask_row % 4 == 0);
-    const bool wide = v8y && a16 && a4;  // full-tile row stores may use the widest forms
 
-    auto issue = [&](uint32_t t, int s) {
-        int64_t row0, col0;
-        int nrows;
-        uint32_t rb;
-        staged_tile<GROUPS>(a, s_bpre, s_rst, t, row0, nrows, col0, rb);
+    // producer state (thread 0): the next tile to load
+    TileWalk<GROUPS> pw;
+    uint32_t t_issue = t_begin;
+    auto issue = [&](int s) {
+        const int4 inf = pw.info(a, s_bpre, s_rst);
+        sm.info[s] = inf;
         const uint32_t bar = smem_addr(&sm.full[s]);
         mbar_expect_tx(bar, SG_TILE_BYTES);
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl)
-            tma_load_slab(smem_addr(sm.tiles[s] + sl * SG_SLAB_BYTES), &tmap, (int)(col0 + sl * SG_SLAB_COLS),
-                          (int)row0, bar);
+            tma_load_slab(smem_addr(sm.tiles[s] + sl * SG_SLAB_BYTES), &maps.x, inf.z + sl * SG_SLAB_COLS, inf.x, bar);
+        ++t_issue;
+        pw.next(a, s_bpre);
     };
-    if (tid == 0) {
-        for (int s = 0; s < SG_STAGES; ++s) {
-            const uint32_t t = blockIdx.x + (uint32_t)s * gridDim.x;
-            if (t < ntiles)
-                issue(t, s);
+    if (tid == 0 && t_begin < t_end) {
+        pw.start(a, s_bpre, t_begin);
+        for (int s = 0; s < SG_STAGES && t_issue < t_end; ++s)
+            issue(s);
+    }
+
+    // column pass: warp w owns tile columns 32w..32w+31 (slab w/2); lane =
+    // column pair p (columns 32w+2p, +1) x row half h: rows 8i'+4h+q for
+    // i' = 0..3, q = 0..3 (word i = 4i' + q)
+    const int p = lane & 15, h = lane >> 4;
+    const int cpair = 32 * warp + 2 * p;  // first tile column of the pair
+    const uint32_t cchunk = 4 * (warp & 1) + (p >> 2);
+    uint32_t yo[4], co[4];  // per q: byte offset of word (i' = 0) in a y tile / in a codes tile
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t rq = 4 * h + q;  // row mod 8 (and row for i' = 0)
+        yo[q] = (uint32_t)(warp >> 1) * SG_SLAB_BYTES + rq * 128 + ((cchunk ^ rq) << 4) + 4 * (p & 3);
+        co[q] = rq * 128 + (((uint32_t)warp ^ rq) << 4) + p;
+    }
+    // row pass: warp w takes the row-wise blocks of columns 32w..32w+31 (the
+    // columns of its column pass), one tile row per lane; per-chunk byte
+    // offsets of the lane's block in a y tile
+    const int rr = lane, bb = warp;
+    uint32_t ro[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+        ro[jj] = (uint32_t)(bb >> 1) * SG_SLAB_BYTES + rr * 128 + ((uint32_t)((4 * (bb & 1) + jj) ^ (rr & 7)) << 4);
+    // full tiles with every row-wise output present and wide-store aligned:
+    // the thread's outputs sit at fixed offsets from the tile's corner
+    const bool row_wide = ROW && a.y_row && a.codes_row && a.mask_row && a.scales_row && v8y && a16 && a4;
+    const int64_t ry = (int64_t)rr * a.ld_y * 2 + 64 * bb, rc = (int64_t)rr * cstride + 16 * bb,
+                  rm = (int64_t)rr * mstride + 4 * bb, rs = (int64_t)rr * nblk + bb;
+
+    int s = 0;
+    uint32_t phase = 0;
+    for (uint32_t t = t_begin, j = 0; t < t_end; ++t, ++j) {
+        const int buf = (int)(j & 1);
+        bool full = false;
+        int row0 = 0, nrows = 0, col0 = 0;
+        // the warp decides together, so that its shuffles and votes below
+        // always see all 32 lanes
+        if (!__all_sync(FULL, mbar_wait(smem_addr(&sm.full[s]), phase))) {
+            sm.err = 1;
+        } else {
+            const int4 inf = sm.info[s];
+            row0 = inf.x;
+            nrows = inf.y;
+            col0 = inf.z;
+            const uint32_t rb = (uint32_t)inf.w;
+            full = nrows == SG_ROWS && col0 + SG_COLS <= a.cols;  // the same for the whole CTA
+            const uint8_t* tile = sm.tiles[s];
+
+            // ---- column pass: y and codes of this thread's column pair
+            uint32_t gsat = 0;  // saturation bits of general-path column pairs (bits 2i, 2i+1: word i)
+            {
+                // per q (row mod 4 of the word): the word's address for i' = 0;
+                // word i = 4i' + q lies i' * 1024 bytes further
+                const uint32_t* tq[4];
+                uint32_t* yq[4];
+                uint8_t* cq[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    tq[q] = reinterpret_cast<const uint32_t*>(tile + yo[q]);
+                    yq[q] = reinterpret_cast<uint32_t*>(sm.ycol[buf] + yo[q]);
+                    cq[q] = sm.ccol[buf] + co[q];
+                }
+                uint32_t aw[16], sg[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    prep_bf(tq[i & 3][(i >> 2) * 256], aw[i], sg[i]);
+                if (!full) {
+                    // rows past a group tail belong to the next group: neither
+                    // their values nor their amax take part
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (8 * (i >> 2) + 4 * h + (i & 3) >= nrows)
+                            aw[i] = sg[i] = 0u;
+                }
+                uint32_t m2 = vmax2(vmax2(vmax2(aw[0], aw[1]), vmax2(aw[2], aw[3])),
+                                    vmax2(vmax2(aw[4], aw[5]), vmax2(aw[6], aw[7])));
+                m2 = vmax2(m2, vmax2(vmax2(vmax2(aw[8], aw[9]), vmax2(aw[10], aw[11])),
+                                     vmax2(vmax2(aw[12], aw[13]), vmax2(aw[14], aw[15]))));
+                m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 16));
+                const uint32_t A_lo = m2 << 16, A_hi = m2 & 0xFFFF0000u;
+                const int k_lo = block_kt<MODE>(A_lo, a.thr), k_hi = block_kt<MODE>(A_hi, a.thr);
+                const bool fast = k_fast_bf(k_lo) && k_fast_bf(k_hi);
+                if (h == 0) {
+                    // the row pass of this warp tests its elements against these
+                    // limits (0xFFFF: never; the general path reports its own)
+                    sm.limw[warp][p] = fast ? (0x8000u + lim16_of_k(k_lo)) | ((0x8000u + lim16_of_k(k_hi)) << 16)
+                                            : 0xFFFFFFFFu;
+                    if (a.scales_col && (full || col0 + cpair < a.cols)) {
+                        // fast-path blocks are finite with k <= 16: the byte is k + 127
+                        const uint32_t e8p = fast ? (uint32_t)(k_lo + 127) | ((uint32_t)(k_hi + 127) << 8)
+                                                  : e8_of(A_lo, k_lo) | (e8_of(A_hi, k_hi) << 8);
+                        *reinterpret_cast<uint16_t*>(a.scales_col + (int64_t)rb * a.cols + col0 + cpair) =
+                            (uint16_t)e8p;
+                    }
+                }
+                auto col_fast = [&]() {
+                    const float inv_lo = __uint_as_float(0x3F800000u - ((uint32_t)k_lo << 23));
+                    const float inv_hi = __uint_as_float(0x3F800000u - ((uint32_t)k_hi << 23));
+                    const uint32_t s2 = bf16_pow2(k_lo) | (bf16_pow2(k_hi) << 16);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        uint32_t P;
+                        const uint32_t o = qword(aw[i], sg[i], inv_lo, inv_hi, s2, lutb16, P);
+                        yq[i & 3][(i >> 2) * 256] = o;
+                        cq[i & 3][(i >> 2) * 1024] = (uint8_t)e2m1_byte(P);
+                    }
+                };
+                if (__all_sync(FULL, fast)) {
+                    col_fast();  // the common case, straight-line
+                } else if (fast) {
+                    col_fast();
+                } else {
+                    const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
+#pragma unroll
+                    for (int i0 = 0; i0 < 16; i0 += 4) {
+                        // the general path takes x itself; -0 halves may enter as +0
+                        uint4 dv;
+                        dv.x = aw[i0] | sg[i0];
+                        dv.y = aw[i0 + 1] | sg[i0 + 1];
+                        dv.z = aw[i0 + 2] | sg[i0 + 2];
+                        dv.w = aw[i0 + 3] | sg[i0 + 3];
+                        const ChunkOut gch = general_chunk<8, true>(dv, Ac, a.mode, a.thr, lutb);
+                        gsat |= (gch.sats & 0xFFu) << (2 * i0);
+                        const uint32_t ov[4] = {gch.packed.x, gch.packed.y, gch.packed.z, gch.packed.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int i = i0 + u;
+                            yq[i & 3][(i >> 2) * 256] = ov[u];
+                            cq[i & 3][(i >> 2) * 1024] = (uint8_t)(gch.nibs >> (8 * u));
+                        }
+                    }
+                }
+            }
+            __syncwarp();  // limw of this warp
+
+            // ---- row pass: the lane's row-wise block (tile row rr, columns
+            // 32w..32w+31): row-wise outputs, and the column-wise saturation
+            // word of the same 32 elements
+            {
+                uint32_t aw[16], sg[16];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint4 c = sm_ld128(tile, ro[jj]);
+                    prep_bf(c.x, aw[4 * jj + 0], sg[4 * jj + 0]);
+                    prep_bf(c.y, aw[4 * jj + 1], sg[4 * jj + 1]);
+                    prep_bf(c.z, aw[4 * jj + 2], sg[4 * jj + 2]);
+                    prep_bf(c.w, aw[4 * jj + 3], sg[4 * jj + 3]);
+                }
+                if (a.mask_col) {
+                    // rows past a group tail are not copied out; their word is don't-care
+                    uint32_t cm = 0;
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const uint4 L = *reinterpret_cast<const uint4*>(&sm.limw[warp][4 * jj]);
+                        const uint32_t lx[4] = {L.x, L.y, L.z, L.w};
+                        const uint32_t a4w[4] = {aw[4 * jj], aw[4 * jj + 1], aw[4 * jj + 2], aw[4 * jj + 3]};
+                        cm |= sat8(a4w, lx) << (8 * jj);
+                    }
+                    sm.mcol[buf][rr * 8 + warp] = cm;
+                }
+                if constexpr (ROW) {
+                    uint32_t m2 = vmax2(vmax2(vmax2(aw[0], aw[1]), vmax2(aw[2], aw[3])),
+                                        vmax2(vmax2(aw[4], aw[5]), vmax2(aw[6], aw[7])));
+                    m2 = vmax2(m2, vmax2(vmax2(vmax2(aw[8], aw[9]), vmax2(aw[10], aw[11])),
+                                         vmax2(vmax2(aw[12], aw[13]), vmax2(aw[14], aw[15]))));
+                    const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
+                    const uint32_t A = am << 16;
+                    const int k = block_kt<MODE>(A, a.thr);
+                    const bool fast = k_fast_bf(k);
+                    uint32_t packed[16], nib[4], sats = 0;
+                    auto row_fast = [&]() {
+                        const float inv = __uint_as_float(0x3F800000u - ((uint32_t)k << 23));
+                        const uint32_t s2 = bf16_pow2(k) * 0x10001u;
+                        const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
+                        const uint32_t limx[4] = {lx, lx, lx, lx};
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            uint32_t P[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                packed[4 * jj + u] = qword(aw[4 * jj + u], sg[4 * jj + u], inv, inv, s2, lutb16, P[u]);
+                            nib[jj] = e2m1_word(P);
+                            const uint32_t a4w[4] = {aw[4 * jj], aw[4 * jj + 1], aw[4 * jj + 2], aw[4 * jj + 3]};
+                            sats |= sat8(a4w, limx) << (8 * jj);
+                        }
+                    };
+                    // the lane's block lies in the tile unless the tile is a
+                    // group tail or the row's ragged end
+                    if (full && __all_sync(FULL, fast)) {
+                        row_fast();
+                        // fast-path blocks are finite with k <= 16: the byte is k + 127
+                        if (row_wide) {
+                            char* yp = static_cast<char*>(a.y_row) + ((int64_t)row0 * a.ld_y + col0) * 2 + ry;
+                            st_global_v8(yp, packed);
+                            st_global_v8(yp + 32, packed + 8);
+                            *reinterpret_cast<uint4*>(a.codes_row + (int64_t)row0 * cstride + col0 / 2 + rc) =
+                                make_uint4(nib[0], nib[1], nib[2], nib[3]);
+                            *reinterpret_cast<uint32_t*>(a.mask_row + (int64_t)row0 * mstride + col0 / 8 + rm) = sats;
+                            a.scales_row[(int64_t)row0 * nblk + col0 / 32 + rs] = (uint8_t)(k + 127);
+                        } else {
+                            store_row_block(a, (int64_t)row0 + rr, (int64_t)col0 + 32 * bb, packed, nib, sats,
+                                            (uint32_t)(k + 127), v8y, a16, a4, cstride, mstride, nblk);
+                        }
+                    } else if (rr < nrows && col0 + 32 * bb < a.cols) {
+                        if (fast) {
+                            row_fast();
+                        } else {
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj) {
+                                uint4 dv;
+                                dv.x = aw[4 * jj] | sg[4 * jj];
+                                dv.y = aw[4 * jj + 1] | sg[4 * jj + 1];
+                                dv.z = aw[4 * jj + 2] | sg[4 * jj + 2];
+                                dv.w = aw[4 * jj + 3] | sg[4 * jj + 3];
+                                const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
+                                packed[4 * jj + 0] = gch.packed.x;
+                                packed[4 * jj + 1] = gch.packed.y;
+                                packed[4 * jj + 2] = gch.packed.z;
+                                packed[4 * jj + 3] = gch.packed.w;
+                                nib[jj] = gch.nibs;
+                                sats |= gch.sats << (8 * jj);
+                            }
+                        }
+                        store_row_block(a, (int64_t)row0 + rr, (int64_t)col0 + 32 * bb, packed, nib, sats,
+                                        fast ? (uint32_t)(k + 127) : e8_of(A, k), v8y, a16, a4, cstride, mstride,
+                                        nblk);
+                    }
+                }
+            }
+            // column pairs of the general path add their exact saturation bits
+            if (__any_sync(FULL, gsat != 0u))
+                col_sat_store(sm.mcol[buf], gsat, h, p, warp);
+            fence_async_smem();  // staged outputs -> visible to the TMA stores
+        }
+        if (tid == 0)
+            bulk_wait_read_all();  // the previous tile's stores have read their staging buffer
+        __syncthreads();           // stage s is consumed; staging buffer buf is complete
+        if (sm.err)
+            break;
+        const uint32_t ts = full ? a.ts_flags : 0u;
+        if (tid == 0) {
+            const uint32_t yb = smem_addr(sm.ycol[buf]);
+            if (a.y_col && (ts & SG_TS_Y)) {
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl)
+                    tma_store_box(&maps.y, yb + sl * SG_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
+            }
+            if (a.codes_col && (ts & SG_TS_CODES))
+                tma_store_box(&maps.codes, smem_addr(sm.ccol[buf]), col0 / 2, row0);
+            if (a.mask_col && (ts & SG_TS_MASK))
+                tma_store_box(&maps.mask, smem_addr(sm.mcol[buf]), col0 / 8, row0);
+            bulk_commit();
+            if (t_issue < t_end)
+                issue(s);
+        }
+        const bool cy = a.y_col && !(ts & SG_TS_Y), cc = a.codes_col && !(ts & SG_TS_CODES),
+                   cm = a.mask_col && !(ts & SG_TS_MASK);
+        if (cy || cc || cm)
+            copy_col_outputs(a, sm, buf, row0, nrows, col0, cy, cc, cm);
+        if (++s == SG_STAGES) {
+            s = 0;
+            phase ^= 1u;
         }
     }
 
-    // column-pass thread: warp w owns tile columns 32w..32w+31; lane = octet
-    // oc (8 columns) x row group g (rows 4g..4g+3)
-    const int oc = lane & 3, g = lane >> 2;
-    const int ccol = 32 * warp + 8 * oc;  // first tile column of the octet
-    const uint32_t cslab = (uint32_t)(warp >> 1) * SG_SLAB_BYTES;
-    const int cchunk = 4 * (warp & 1) + oc;
-    // row-pass thread: tile row rr, row-wise block bb (slab bb/2, half bb%2)
-    const int rr = 8 * (warp & 3) + (lane & 7);
-    const int bb = 2 * (lane >> 3) + (warp >> 2);
-
-    uint32_t j = 0;
-    for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++j) {
-        const int s = (int)(j % SG_STAGES);
-        int64_t row0, col0;
-        int nrows;
-        uint32_t rb;
-        staged_tile<GROUPS>(a, s_bpre, s_rst, t, row0, nrows, col0, rb);
-        const bool full = nrows == SG_ROWS && col0 + SG_COLS <= a.cols;  // the same for the whole CTA
-        if (!mbar_wait(smem_addr(&sm.full[s]), (j / SG_STAGES) & 1u)) {
+    if (tid == 0) {
+        if (sm.err) {
             if (a.status)
                 *a.status = MXFP4_ECUDA;
-            return;
+            // loads still in flight land in shared memory: wait for them
+            // (bounded) before the CTA releases it
+            for (int st = 0; st < SG_STAGES; ++st)
+                (void)mbar_wait(smem_addr(&sm.full[st]), phase ^ (st < s ? 1u : 0u));
         }
-        const uint32_t tile = smem_addr(sm.tiles[s]);
-
-        // ---- column pass: the thread's four rows; maxima down the 32 rows by
-        // shuffles across the eight row groups of the warp
-        {
-            uint4 cd[4];
-            uint32_t pm[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = 4 * g + i;
-                cd[i] = lds128(tile + cslab + swz(r, cchunk));
-                if (r < nrows) {
-                    pm[0] = vmax2(pm[0], cd[i].x & 0x7FFF7FFFu);
-                    pm[1] = vmax2(pm[1], cd[i].y & 0x7FFF7FFFu);
-                    pm[2] = vmax2(pm[2], cd[i].z & 0x7FFF7FFFu);
-                    pm[3] = vmax2(pm[3], cd[i].w & 0x7FFF7FFFu);
-                }
-            }
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-#pragma unroll
-                for (int h = 0; h < 4; ++h)
-                    pm[h] = vmax2(pm[h], __shfl_xor_sync(FULL, pm[h], off));
-            }
-            // lane g computes the parameters of column g of its octet; the
-            // octet's eight lanes share them by shuffles
-            const int gw = g >> 1;  // selects keep pm in registers
-            const uint32_t myw = gw == 0 ? pm[0] : (gw == 1 ? pm[1] : (gw == 2 ? pm[2] : pm[3]));
-            const uint32_t myA = (g & 1) ? (myw & 0xFFFF0000u) : (myw << 16);
-            const int myk = block_k(myA, a.mode, a.thr);
-            const QP myp = qp_of_k(myk);
-            const uint32_t mylim = lim16_of_k(myk);
-            uint32_t cflags = (k_fast16(myk) ? 0u : 1u) | ((myA >> 16) > mylim ? 2u : 0u);
-            {
-                const int64_t col = col0 + ccol + g;
-                if ((ALL && full) || (a.scales_col && col < a.cols))
-                    a.scales_col[(int64_t)rb * a.cols + col] = (uint8_t)e8_of(myA, myk);
-            }
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1)
-                cflags |= __shfl_xor_sync(FULL, cflags, off);
-            uint64_t inv2[4], scale2[4];
-            uint32_t limxc[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const int s0 = oc + 8 * h, s1 = oc + 8 * h + 4;  // lanes holding columns 2h and 2h+1
-                inv2[h] = pk2(__float_as_uint(__shfl_sync(FULL, myp.inv, s0)),
-                              __float_as_uint(__shfl_sync(FULL, myp.inv, s1)));
-                scale2[h] = pk2(__float_as_uint(__shfl_sync(FULL, myp.scale, s0)),
-                                __float_as_uint(__shfl_sync(FULL, myp.scale, s1)));
-                limxc[h] = (0x8000u + __shfl_sync(FULL, mylim, s0)) | ((0x8000u + __shfl_sync(FULL, mylim, s1)) << 16);
-            }
-            const int64_t col = col0 + ccol;
-            if (full && __all_sync(FULL, !(cflags & 1u))) {
-                // every octet of the warp is on the fast path and all 32 rows are real
-                const bool dosat = __any_sync(FULL, cflags & 2u);
-                char* yp = static_cast<char*>(a.y_col) + ((row0 + 4 * g) * a.ld_y + col) * 2;
-                uint8_t* cp = a.codes_col + (row0 + 4 * g) * cstride + col / 2;
-                uint8_t* mp = a.mask_col + (row0 + 4 * g) * mstride + col / 8;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w[4] = {cd[i].x, cd[i].y, cd[i].z, cd[i].w};
-                    uint32_t aw[4], wc[4], packed[4], nibs;
-#pragma unroll
-                    for (int h = 0; h < 4; ++h)
-                        prep16(w[h], aw[h], wc[h]);
-                    quant16x2<true>(aw, wc, inv2, scale2, lutb16, packed, nibs);
-                    const uint32_t sats = dosat ? sat8(aw, limxc) : 0u;
-                    if (ALL || a.y_col)
-                        st_stream(yp + i * a.ld_y * 2, make_uint4(packed[0], packed[1], packed[2], packed[3]));
-                    if (ALL || a.codes_col)
-                        *reinterpret_cast<uint32_t*>(cp + i * cstride) = nibs;
-                    if (ALL || a.mask_col)
-                        mp[i * mstride] = (uint8_t)sats;
-                }
-            } else if (col < a.cols) {
-                QP pc[8];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    pc[2 * h].inv = __uint_as_float(lo32(inv2[h]));
-                    pc[2 * h + 1].inv = __uint_as_float(hi32(inv2[h]));
-                    pc[2 * h].scale = __uint_as_float(lo32(scale2[h]));
-                    pc[2 * h + 1].scale = __uint_as_float(hi32(scale2[h]));
-                }
-                uint32_t Ac[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    Ac[e] = (e & 1) ? (pm[e / 2] & 0xFFFF0000u) : (pm[e / 2] << 16);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int r = 4 * g + i;
-                    if (r >= nrows)
-                        continue;
-                    const int64_t row = row0 + r;
-                    uint32_t packed[4], nibs, sats;
-                    if (!(cflags & 1u)) {
-                        const uint32_t w[4] = {cd[i].x, cd[i].y, cd[i].z, cd[i].w};
-                        uint32_t aw[4], wc[4];
-#pragma unroll
-                        for (int h = 0; h < 4; ++h)
-                            prep16(w[h], aw[h], wc[h]);
-                        quant16x2<true>(aw, wc, inv2, scale2, lutb16, packed, nibs);
-                        sats = sat8(aw, limxc);
-                    } else {
-                        const ChunkOut gch = general_chunk<8, true>(cd[i], Ac, a.mode, a.thr, lutb);
-                        packed[0] = gch.packed.x;
-                        packed[1] = gch.packed.y;
-                        packed[2] = gch.packed.z;
-                        packed[3] = gch.packed.w;
-                        nibs = gch.nibs;
-                        sats = gch.sats;
-                    }
-                    if (a.y_col)
-                        st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * 2,
-                                  make_uint4(packed[0], packed[1], packed[2], packed[3]));
-                    if (a.codes_col)
-                        *reinterpret_cast<uint32_t*>(a.codes_col + row * cstride + col / 2) = nibs;
-                    if (a.mask_col)
-                        a.mask_col[row * mstride + col / 8] = (uint8_t)sats;
-                }
-            }
-        }
-
-        // ---- row pass: one row-wise block per thread
-        if constexpr (ROW) {
-            const int64_t row = row0 + rr;
-            const int64_t col = col0 + 32 * bb;
-            const bool rok = rr < nrows && col < a.cols;
-            uint32_t aw[16], wc[16];
-            {
-                const uint32_t base = tile + (bb >> 1) * SG_SLAB_BYTES;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint4 c = lds128(base + swz(rr, 4 * (bb & 1) + jj));
-                    prep16(c.x, aw[4 * jj + 0], wc[4 * jj + 0]);
-                    prep16(c.y, aw[4 * jj + 1], wc[4 * jj + 1]);
-                    prep16(c.z, aw[4 * jj + 2], wc[4 * jj + 2]);
-                    prep16(c.w, aw[4 * jj + 3], wc[4 * jj + 3]);
-                }
-            }
-            uint32_t m2 = 0;
-#pragma unroll
-            for (int h = 0; h < 16; h += 2)
-                m2 = vmax2(m2, vmax2(aw[h], aw[h + 1]));
-            const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
-            const uint32_t A = am << 16;
-            const int k = block_k(A, a.mode, a.thr);
-            const bool fast = k_fast16(k);
-            uint32_t packed[16], nib[4], sats = 0;
-            if (full && __all_sync(FULL, fast)) {
-                const QP p = qp_of_k(k);
-                const uint64_t inv2 = pk2(__float_as_uint(p.inv), __float_as_uint(p.inv));
-                const uint64_t scale2 = pk2(__float_as_uint(p.scale), __float_as_uint(p.scale));
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-                    quant16x2<false>(aw + 4 * jj, wc + 4 * jj, &inv2, &scale2, lutb16, packed + 4 * jj, nib[jj]);
-                const uint32_t lim = lim16_of_k(k);
-                if (__any_sync(FULL, am > lim)) {
-                    const uint32_t lx = (0x8000u + lim) * 0x10001u;
-                    const uint32_t limx[4] = {lx, lx, lx, lx};
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const uint32_t a4w[4] = {aw[4 * jj], aw[4 * jj + 1], aw[4 * jj + 2], aw[4 * jj + 3]};
-                        sats |= sat8(a4w, limx) << (8 * jj);
-                    }
-                }
-                if (ALL && wide) {
-                    char* yp = static_cast<char*>(a.y_row) + (row * a.ld_y + col) * 2;
-                    st_global_v8(yp, packed);
-                    st_global_v8(yp + 32, packed + 8);
-                    *reinterpret_cast<uint4*>(a.codes_row + row * cstride + col / 2) =
-                        make_uint4(nib[0], nib[1], nib[2], nib[3]);
-                    *reinterpret_cast<uint32_t*>(a.mask_row + row * mstride + col / 8) = sats;
-                    a.scales_row[row * nblk + col / 32] = (uint8_t)e8_of(A, k);
-                } else {
-                    store_row_block(a, row, col, packed, nib, sats, e8_of(A, k), v8y, a16, a4, cstride, mstride,
-                                    nblk);
-                }
-            } else if (rok) {
-                if (fast) {
-                    const QP p = qp_of_k(k);
-                    const uint64_t inv2 = pk2(__float_as_uint(p.inv), __float_as_uint(p.inv));
-                    const uint64_t scale2 = pk2(__float_as_uint(p.scale), __float_as_uint(p.scale));
-                    const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
-                    const uint32_t limx[4] = {lx, lx, lx, lx};
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        quant16x2<false>(aw + 4 * jj, wc + 4 * jj, &inv2, &scale2, lutb16, packed + 4 * jj, nib[jj]);
-                        const uint32_t a4w[4] = {aw[4 * jj], aw[4 * jj + 1], aw[4 * jj + 2], aw[4 * jj + 3]};
-                        sats |= sat8(a4w, limx) << (8 * jj);
-                    }
-                } else {
-                    const uint32_t base = tile + (bb >> 1) * SG_SLAB_BYTES;
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const ChunkOut gch =
-                            general_chunk<8, false>(lds128(base + swz(rr, 4 * (bb & 1) + jj)), &A, a.mode, a.thr, lutb);
-                        packed[4 * jj + 0] = gch.packed.x;
-                        packed[4 * jj + 1] = gch.packed.y;
-                        packed[4 * jj + 2] = gch.packed.z;
-                        packed[4 * jj + 3] = gch.packed.w;
-                        nib[jj] = gch.nibs;
-                        sats |= gch.sats << (8 * jj);
-                    }
-                }
-                store_row_block(a, row, col, packed, nib, sats, e8_of(A, k), v8y, a16, a4, cstride, mstride, nblk);
-            }
-        }
-        __syncthreads();  // every warp is done with the stage
-        if (tid == 0) {
-            const uint32_t tn = t + SG_STAGES * gridDim.x;
-            if (tn < ntiles)
-                issue(tn, s);
-        }
+        bulk_wait_all();
     }
 }
 
