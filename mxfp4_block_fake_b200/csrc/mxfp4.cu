@@ -1311,10 +1311,10 @@ static bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, void* base, uint6
 
 // Maps of the staged kernel. x: bf16 [rows, cols] with row pitch ld * 2
 // bytes, 64 x 32 boxes with the 128-byte swizzle (out-of-range elements read
-// as zero). Column-wise outputs, each only where TMA can address it (16-byte
-// aligned base and row pitch) and the tensor holds at least one full tile:
-// y_col as x (pitch ld_y * 2), codes_col [rows, cols/2] bytes in 128 x 32
-// boxes with the 128-byte swizzle, mask_col [rows, cols/8] bytes in 32 x 32
+// as zero). Outputs of both directions, each only where TMA can address it
+// (16-byte aligned base and row pitch) and the tensor holds at least one
+// full tile: y as x (pitch ld_y * 2), codes [rows, cols/2] bytes in 128 x 32
+// boxes with the 128-byte swizzle, masks [rows, cols/8] bytes in 32 x 32
 // boxes. Returns false when the input map cannot be built.
 static bool make_staged_maps(StagedMaps* m, const KArgs& k, uint32_t* ts_flags)
 {
@@ -1337,6 +1337,18 @@ static bool make_staged_maps(StagedMaps* m, const KArgs& k, uint32_t* ts_flags)
         encode_2d(&m->mask, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.mask_col, (uint64_t)k.cols / 8, (uint64_t)k.rows,
                   (uint64_t)k.cols / 8, SG_COLS / 8, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
         *ts_flags |= SG_TS_MASK;
+    if (k.y_row && aligned(k.y_row, 16) && (k.ld_y * 2) % 16 == 0 &&
+        encode_2d(&m->yr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.y_row, (uint64_t)k.cols, (uint64_t)k.rows,
+                  (uint64_t)k.ld_y * 2, SG_SLAB_COLS, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        *ts_flags |= SG_TS_YR;
+    if (k.codes_row && aligned(k.codes_row, 16) && (k.cols / 2) % 16 == 0 &&
+        encode_2d(&m->codes_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.codes_row, (uint64_t)k.cols / 2, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 2, SG_COLS / 2, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        *ts_flags |= SG_TS_CODES_R;
+    if (k.mask_row && aligned(k.mask_row, 16) && (k.cols / 8) % 16 == 0 &&
+        encode_2d(&m->mask_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.mask_row, (uint64_t)k.cols / 8, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 8, SG_COLS / 8, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+        *ts_flags |= SG_TS_MASK_R;
     return true;
 }
 

@@ -44,14 +44,28 @@ constexpr int SG_MASK_WORDS = SG_ROWS * SG_COLS / 32;      // 256: saturation bi
 constexpr int SG_STAGES = 3;
 constexpr uint32_t SG_WAIT_LIMIT = 1u << 22;               // try_wait polls before giving up
 
-// which column-wise outputs leave through TMA stores on full tiles
-constexpr uint32_t SG_TS_Y = 1u, SG_TS_CODES = 2u, SG_TS_MASK = 4u;
+// which outputs leave through TMA stores on full tiles (the others, and every
+// output of a group-tail or ragged tile, are copied out by the threads)
+constexpr uint32_t SG_TS_Y = 1u, SG_TS_CODES = 2u, SG_TS_MASK = 4u;              // column-wise
+constexpr uint32_t SG_TS_YR = 8u, SG_TS_CODES_R = 16u, SG_TS_MASK_R = 32u;       // row-wise
+
+// Staged outputs of one tile. y tiles use the input's layout (four 4 KB
+// slabs of 64 columns with the 128-byte swizzle); codes are 32 rows of 128
+// bytes with the 128-byte swizzle; masks are 32 rows of 32 bytes; row-wise
+// scales are 32 rows of 8 bytes.
+// (Column-wise y is written over the tile's input in its stage instead.)
+struct __align__(1024) StagedOut {
+    uint8_t yrow[SG_TILE_BYTES];
+    uint8_t ccol[SG_CODE_BYTES];
+    uint8_t crow[SG_CODE_BYTES];
+    uint32_t mcol[SG_MASK_WORDS];
+    uint32_t mrow[SG_MASK_WORDS];
+    uint8_t srow[SG_ROWS * SG_COLS / 32];
+};
 
 struct __align__(1024) StagedSmem {
-    uint8_t tiles[SG_STAGES][SG_TILE_BYTES];  // input stages (1024-aligned swizzle atoms)
-    uint8_t ycol[2][SG_TILE_BYTES];           // column-wise y staging, input layout
-    uint8_t ccol[2][SG_CODE_BYTES];           // column-wise codes staging, 128-byte rows, swizzled
-    uint32_t mcol[2][SG_MASK_WORDS];          // column-wise saturation bits, 32-byte rows
+    uint8_t tiles[SG_STAGES][SG_TILE_BYTES];  // input stages (1024-aligned swizzle atoms); column-wise y
+    StagedOut out[2];                         // staged outputs, double-buffered by tile parity
     uint32_t limw[8][16];                     // per warp and column pair: 0x8000 + limit bits of each column
     int4 info[SG_STAGES];                     // row0, nrows, col0, row block of each stage's tile
     uint32_t lut[64];
@@ -59,10 +73,10 @@ struct __align__(1024) StagedSmem {
     int err;
 };
 
-// TMA descriptors: the input and the three column-wise outputs (the output
-// maps are only read when the matching SG_TS_* flag is set).
+// TMA descriptors: the input and the outputs (an output map is only read
+// when its SG_TS_* flag is set).
 struct StagedMaps {
-    CUtensorMap x, y, codes, mask;
+    CUtensorMap x, y, codes, mask, yr, codes_r, mask_r;
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -231,61 +245,6 @@ __device__ __forceinline__ void prep_bf(uint32_t w, uint32_t& aw, uint32_t& sg)
     sg = w & (aw + 0x7FFF7FFFu) & 0x80008000u;
 }
 
-__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v)
-{
-    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
-                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
-}
-
-// Stores of one row-wise block (32 elements): null outputs are skipped and a
-// row's last block may hold only 8, 16 or 24 real elements (cols is a
-// multiple of 8 here).
-__device__ __forceinline__ void store_row_block(const KArgs& a, int64_t row, int64_t col, const uint32_t* packed,
-                                                const uint32_t* nib, uint32_t sats, uint32_t e8, bool v8y, bool a16,
-                                                bool a4, int64_t cstride, int64_t mstride, int64_t nblk)
-{
-    const int64_t left = a.cols - col;
-    const int nchunk = left >= 32 ? 4 : (int)(left >> 3);
-    if (a.y_row) {
-        char* yp = static_cast<char*>(a.y_row) + (row * a.ld_y + col) * 2;
-        if (nchunk == 4 && v8y) {
-            st_global_v8(yp, packed);
-            st_global_v8(yp + 32, packed + 8);
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                if (jj < nchunk)
-                    st_stream(yp + 16 * jj,
-                              make_uint4(packed[4 * jj], packed[4 * jj + 1], packed[4 * jj + 2], packed[4 * jj + 3]));
-        }
-    }
-    if (a.codes_row) {
-        uint8_t* cp = a.codes_row + row * cstride + col / 2;
-        if (nchunk == 4 && a16) {
-            *reinterpret_cast<uint4*>(cp) = make_uint4(nib[0], nib[1], nib[2], nib[3]);
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                if (jj < nchunk)
-                    reinterpret_cast<uint32_t*>(cp)[jj] = nib[jj];
-        }
-    }
-    if (a.mask_row) {
-        uint8_t* mp = a.mask_row + row * mstride + col / 8;
-        if (nchunk == 4 && a4) {
-            *reinterpret_cast<uint32_t*>(mp) = sats;
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                if (jj < nchunk)
-                    mp[jj] = (uint8_t)(sats >> (8 * jj));
-        }
-    }
-    if (a.scales_row)
-        a.scales_row[row * nblk + col / 32] = (uint8_t)e8;
-}
-
 // Tile sequence of one CTA: row block rb and column tile ct, advanced in
 // order; g tracks the group that holds rb (largest g with s_bpre[g] <= rb,
 // which skips empty groups).
@@ -339,16 +298,14 @@ struct TileWalk {
     }
 };
 
-// Copy the staged column-wise outputs of a tile to global memory with the
-// threads (group tails, ragged tiles, outputs TMA cannot address).
-__device__ __forceinline__ void copy_col_outputs(const KArgs& a, const StagedSmem& sm, int buf, int row0, int nrows,
-                                                 int col0, bool cy, bool cc, bool cm)
+// Copy the staged outputs of a tile to global memory with the threads
+// (group tails, ragged tiles, outputs TMA cannot address). The flags select
+// the outputs; rows at or past nrows and columns at or past cols are skipped.
+__device__ __forceinline__ void copy_outputs(const KArgs& a, const uint8_t* ycol, const StagedOut& o, int row0,
+                                             int nrows, int col0, uint32_t which)
 {
     const int tid = threadIdx.x;
-    const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8;
-    const uint8_t* yb = sm.ycol[buf];
-    const uint8_t* cb = sm.ccol[buf];
-    const uint8_t* mb = reinterpret_cast<const uint8_t*>(sm.mcol[buf]);
+    const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8, nblk = (a.cols + 31) / 32;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         const int q = tid + NTHREADS * m;  // 0..1023
@@ -359,22 +316,44 @@ __device__ __forceinline__ void copy_col_outputs(const KArgs& a, const StagedSme
         const int col = col0 + 8 * u;  // y chunk u / codes word u / mask byte u: columns col..col+7
         if (col >= a.cols)
             continue;
-        if (cy) {
-            const uint4 v = sm_ld128(yb, (u >> 3) * SG_SLAB_BYTES + r * 128 + (((u & 7) ^ (r & 7)) << 4));
-            st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * 2, v);
-        }
-        if (cc) {
-            const uint32_t v = sm_ld32(cb, r * 128 + (((u >> 2) ^ (r & 7)) << 4) + 4 * (u & 3));
-            *reinterpret_cast<uint32_t*>(a.codes_col + row * cstride + col / 2) = v;
-        }
-        if (cm)
-            a.mask_col[row * mstride + col / 8] = mb[r * 32 + u];
+        const uint32_t yoff = (u >> 3) * SG_SLAB_BYTES + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+        const uint32_t coff = r * 128 + (((u >> 2) ^ (r & 7)) << 4) + 4 * (u & 3);
+        if (which & SG_TS_Y)
+            st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * 2, sm_ld128(ycol, yoff));
+        if (which & SG_TS_YR)
+            st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * 2, sm_ld128(o.yrow, yoff));
+        if (which & SG_TS_CODES)
+            *reinterpret_cast<uint32_t*>(a.codes_col + row * cstride + col / 2) = sm_ld32(o.ccol, coff);
+        if (which & SG_TS_CODES_R)
+            *reinterpret_cast<uint32_t*>(a.codes_row + row * cstride + col / 2) = sm_ld32(o.crow, coff);
+        if (which & SG_TS_MASK)
+            a.mask_col[row * mstride + col / 8] = reinterpret_cast<const uint8_t*>(o.mcol)[r * 32 + u];
+        if (which & SG_TS_MASK_R)
+            a.mask_row[row * mstride + col / 8] = reinterpret_cast<const uint8_t*>(o.mrow)[r * 32 + u];
+    }
+}
+
+// Row-wise scales of a tile (32 rows x 8 blocks) from staging: one row per
+// lane of warp 0.
+__device__ __forceinline__ void copy_row_scales(const KArgs& a, const StagedOut& o, int row0, int nrows, int col0)
+{
+    const int r = threadIdx.x;
+    if (r >= nrows)
+        return;
+    const int64_t nblk = (a.cols + 31) / 32;
+    uint8_t* dst = a.scales_row + (int64_t)(row0 + r) * nblk + col0 / 32;
+    const int nb = (int)min((int64_t)8, nblk - col0 / 32);
+    if (nb == 8 && ((uintptr_t)dst & 7) == 0) {
+        *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(o.srow + r * 8);
+    } else {
+        for (int b = 0; b < nb; ++b)
+            dst[b] = o.srow[r * 8 + b];
     }
 }
 
 // ORs a warp's column-pass saturation bits into the staged mask words (one
 // 32-bit word per tile row and warp, bit 2p + e for column pair p). Called
-// by the whole warp: the words were zeroed by other lanes.
+// by the whole warp, after the words were written by other lanes.
 __device__ __forceinline__ void col_sat_store(uint32_t* mwords, uint32_t bits, int h, int p, int warp)
 {
     __syncwarp();
@@ -424,10 +403,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
     const uint32_t t_end = (uint32_t)(((uint64_t)(blockIdx.x + 1) * ntiles) / gridDim.x);
     const uint32_t lutb = smem_addr(sm.lut) - 0x2C000000u;
     const uint32_t lutb16 = lutb + 0x04000000u;
-    const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8, nblk = (a.cols + 31) / 32;
-    const bool v8y = ((a.ld_y * 2) % 32 == 0) && ((uintptr_t)a.y_row % 32 == 0);
-    const bool a16 = (cstride % 16 == 0) && ((uintptr_t)a.codes_row % 16 == 0);
-    const bool a4 = (mstride % 4 == 0) && ((uintptr_t)a.mask_row % 4 == 0);
+    // outputs present (SG_TS_* bits); those not written by TMA are copied
+    const uint32_t present = (a.y_col ? SG_TS_Y : 0u) | (a.codes_col ? SG_TS_CODES : 0u) |
+                             (a.mask_col ? SG_TS_MASK : 0u) | (ROW && a.y_row ? SG_TS_YR : 0u) |
+                             (ROW && a.codes_row ? SG_TS_CODES_R : 0u) | (ROW && a.mask_row ? SG_TS_MASK_R : 0u);
 
     // producer state (thread 0): the next tile to load
     TileWalk<GROUPS> pw;
@@ -463,28 +442,29 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
         co[q] = rq * 128 + (((uint32_t)warp ^ rq) << 4) + p;
     }
     // row pass: warp w takes the row-wise blocks of columns 32w..32w+31 (the
-    // columns of its column pass), one tile row per lane; per-chunk byte
-    // offsets of the lane's block in a y tile
-    const int rr = lane, bb = warp;
+    // columns of its column pass), one tile row per lane. Byte offsets of the
+    // lane's block: chunks of a y tile, its 16 code bytes; word rr*8 + w of
+    // a mask tile; byte rr*8 + w of the scales.
+    const int rr = lane;
     uint32_t ro[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj)
-        ro[jj] = (uint32_t)(bb >> 1) * SG_SLAB_BYTES + rr * 128 + ((uint32_t)((4 * (bb & 1) + jj) ^ (rr & 7)) << 4);
-    // full tiles with every row-wise output present and wide-store aligned:
-    // the thread's outputs sit at fixed offsets from the tile's corner
-    const bool row_wide = ROW && a.y_row && a.codes_row && a.mask_row && a.scales_row && v8y && a16 && a4;
-    const int64_t ry = (int64_t)rr * a.ld_y * 2 + 64 * bb, rc = (int64_t)rr * cstride + 16 * bb,
-                  rm = (int64_t)rr * mstride + 4 * bb, rs = (int64_t)rr * nblk + bb;
+        ro[jj] = (uint32_t)(warp >> 1) * SG_SLAB_BYTES + rr * 128 +
+                 ((uint32_t)((4 * (warp & 1) + jj) ^ (rr & 7)) << 4);
+    const uint32_t rco = rr * 128 + (((uint32_t)warp ^ (uint32_t)(rr & 7)) << 4);
+    const int rw = rr * 8 + warp;
 
     int s = 0;
     uint32_t phase = 0;
     for (uint32_t t = t_begin, j = 0; t < t_end; ++t, ++j) {
-        const int buf = (int)(j & 1);
+        StagedOut& out = sm.out[j & 1];
         bool full = false;
         int row0 = 0, nrows = 0, col0 = 0;
         // the warp decides together, so that its shuffles and votes below
         // always see all 32 lanes
-        if (!__all_sync(FULL, mbar_wait(smem_addr(&sm.full[s]), phase))) {
+        const bool ok = __all_sync(FULL, mbar_wait(smem_addr(&sm.full[s]), phase));
+        uint8_t* tile = sm.tiles[s];
+        if (!ok) {
             sm.err = 1;
         } else {
             const int4 inf = sm.info[s];
@@ -493,26 +473,17 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
             col0 = inf.z;
             const uint32_t rb = (uint32_t)inf.w;
             full = nrows == SG_ROWS && col0 + SG_COLS <= a.cols;  // the same for the whole CTA
-            const uint8_t* tile = sm.tiles[s];
 
-            // ---- column pass: y and codes of this thread's column pair
-            uint32_t gsat = 0;  // saturation bits of general-path column pairs (bits 2i, 2i+1: word i)
+            // ---- column pass: the lane's column pair over its 16 rows. Its y
+            // words wait in registers until the warp's row pass has read the
+            // sub-tile, then replace the input in the stage.
+            uint32_t ycw[16];
+            uint32_t gsat = 0;  // saturation bits of a general-path column pair (bits 2i, 2i+1: word i)
             {
-                // per q (row mod 4 of the word): the word's address for i' = 0;
-                // word i = 4i' + q lies i' * 1024 bytes further
-                const uint32_t* tq[4];
-                uint32_t* yq[4];
-                uint8_t* cq[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    tq[q] = reinterpret_cast<const uint32_t*>(tile + yo[q]);
-                    yq[q] = reinterpret_cast<uint32_t*>(sm.ycol[buf] + yo[q]);
-                    cq[q] = sm.ccol[buf] + co[q];
-                }
                 uint32_t aw[16], sg[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    prep_bf(tq[i & 3][(i >> 2) * 256], aw[i], sg[i]);
+                    prep_bf(sm_ld32(tile, yo[i & 3] + (i >> 2) * 1024), aw[i], sg[i]);
                 if (!full) {
                     // rows past a group tail belong to the next group: neither
                     // their values nor their amax take part
@@ -542,6 +513,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
                             (uint16_t)e8p;
                     }
                 }
+                uint8_t* cq[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    cq[q] = out.ccol + co[q];
                 auto col_fast = [&]() {
                     const float inv_lo = __uint_as_float(0x3F800000u - ((uint32_t)k_lo << 23));
                     const float inv_hi = __uint_as_float(0x3F800000u - ((uint32_t)k_hi << 23));
@@ -549,8 +524,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         uint32_t P;
-                        const uint32_t o = qword(aw[i], sg[i], inv_lo, inv_hi, s2, lutb16, P);
-                        yq[i & 3][(i >> 2) * 256] = o;
+                        ycw[i] = qword(aw[i], sg[i], inv_lo, inv_hi, s2, lutb16, P);
                         cq[i & 3][(i >> 2) * 1024] = (uint8_t)e2m1_byte(P);
                     }
                 };
@@ -570,11 +544,13 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
                         dv.w = aw[i0 + 3] | sg[i0 + 3];
                         const ChunkOut gch = general_chunk<8, true>(dv, Ac, a.mode, a.thr, lutb);
                         gsat |= (gch.sats & 0xFFu) << (2 * i0);
-                        const uint32_t ov[4] = {gch.packed.x, gch.packed.y, gch.packed.z, gch.packed.w};
+                        ycw[i0] = gch.packed.x;
+                        ycw[i0 + 1] = gch.packed.y;
+                        ycw[i0 + 2] = gch.packed.z;
+                        ycw[i0 + 3] = gch.packed.w;
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const int i = i0 + u;
-                            yq[i & 3][(i >> 2) * 256] = ov[u];
                             cq[i & 3][(i >> 2) * 1024] = (uint8_t)(gch.nibs >> (8 * u));
                         }
                     }
@@ -586,14 +562,14 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
             // 32w..32w+31): row-wise outputs, and the column-wise saturation
             // word of the same 32 elements
             {
-                uint32_t aw[16], sg[16];
+                uint32_t bw[16], bs[16];
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
                     const uint4 c = sm_ld128(tile, ro[jj]);
-                    prep_bf(c.x, aw[4 * jj + 0], sg[4 * jj + 0]);
-                    prep_bf(c.y, aw[4 * jj + 1], sg[4 * jj + 1]);
-                    prep_bf(c.z, aw[4 * jj + 2], sg[4 * jj + 2]);
-                    prep_bf(c.w, aw[4 * jj + 3], sg[4 * jj + 3]);
+                    prep_bf(c.x, bw[4 * jj + 0], bs[4 * jj + 0]);
+                    prep_bf(c.y, bw[4 * jj + 1], bs[4 * jj + 1]);
+                    prep_bf(c.z, bw[4 * jj + 2], bs[4 * jj + 2]);
+                    prep_bf(c.w, bw[4 * jj + 3], bs[4 * jj + 3]);
                 }
                 if (a.mask_col) {
                     // rows past a group tail are not copied out; their word is don't-care
@@ -602,20 +578,20 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
                     for (int jj = 0; jj < 4; ++jj) {
                         const uint4 L = *reinterpret_cast<const uint4*>(&sm.limw[warp][4 * jj]);
                         const uint32_t lx[4] = {L.x, L.y, L.z, L.w};
-                        const uint32_t a4w[4] = {aw[4 * jj], aw[4 * jj + 1], aw[4 * jj + 2], aw[4 * jj + 3]};
+                        const uint32_t a4w[4] = {bw[4 * jj], bw[4 * jj + 1], bw[4 * jj + 2], bw[4 * jj + 3]};
                         cm |= sat8(a4w, lx) << (8 * jj);
                     }
-                    sm.mcol[buf][rr * 8 + warp] = cm;
+                    out.mcol[rw] = cm;
                 }
                 if constexpr (ROW) {
-                    uint32_t m2 = vmax2(vmax2(vmax2(aw[0], aw[1]), vmax2(aw[2], aw[3])),
-                                        vmax2(vmax2(aw[4], aw[5]), vmax2(aw[6], aw[7])));
-                    m2 = vmax2(m2, vmax2(vmax2(vmax2(aw[8], aw[9]), vmax2(aw[10], aw[11])),
-                                         vmax2(vmax2(aw[12], aw[13]), vmax2(aw[14], aw[15]))));
+                    uint32_t m2 = vmax2(vmax2(vmax2(bw[0], bw[1]), vmax2(bw[2], bw[3])),
+                                        vmax2(vmax2(bw[4], bw[5]), vmax2(bw[6], bw[7])));
+                    m2 = vmax2(m2, vmax2(vmax2(vmax2(bw[8], bw[9]), vmax2(bw[10], bw[11])),
+                                         vmax2(vmax2(bw[12], bw[13]), vmax2(bw[14], bw[15]))));
                     const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
                     const uint32_t A = am << 16;
                     const int k = block_kt<MODE>(A, a.thr);
-                    const bool fast = k_fast_bf(k);
+                    const bool rfast = k_fast_bf(k);
                     uint32_t packed[16], nib[4], sats = 0;
                     auto row_fast = [&]() {
                         const float inv = __uint_as_float(0x3F800000u - ((uint32_t)k << 23));
@@ -627,85 +603,92 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
                             uint32_t P[4];
 #pragma unroll
                             for (int u = 0; u < 4; ++u)
-                                packed[4 * jj + u] = qword(aw[4 * jj + u], sg[4 * jj + u], inv, inv, s2, lutb16, P[u]);
+                                packed[4 * jj + u] = qword(bw[4 * jj + u], bs[4 * jj + u], inv, inv, s2, lutb16, P[u]);
                             nib[jj] = e2m1_word(P);
-                            const uint32_t a4w[4] = {aw[4 * jj], aw[4 * jj + 1], aw[4 * jj + 2], aw[4 * jj + 3]};
+                            const uint32_t a4w[4] = {bw[4 * jj], bw[4 * jj + 1], bw[4 * jj + 2], bw[4 * jj + 3]};
                             sats |= sat8(a4w, limx) << (8 * jj);
                         }
                     };
-                    // the lane's block lies in the tile unless the tile is a
-                    // group tail or the row's ragged end
-                    if (full && __all_sync(FULL, fast)) {
+                    if (__all_sync(FULL, rfast)) {
+                        row_fast();  // the common case, straight-line
+                    } else if (rfast) {
                         row_fast();
-                        // fast-path blocks are finite with k <= 16: the byte is k + 127
-                        if (row_wide) {
-                            char* yp = static_cast<char*>(a.y_row) + ((int64_t)row0 * a.ld_y + col0) * 2 + ry;
-                            st_global_v8(yp, packed);
-                            st_global_v8(yp + 32, packed + 8);
-                            *reinterpret_cast<uint4*>(a.codes_row + (int64_t)row0 * cstride + col0 / 2 + rc) =
-                                make_uint4(nib[0], nib[1], nib[2], nib[3]);
-                            *reinterpret_cast<uint32_t*>(a.mask_row + (int64_t)row0 * mstride + col0 / 8 + rm) = sats;
-                            a.scales_row[(int64_t)row0 * nblk + col0 / 32 + rs] = (uint8_t)(k + 127);
-                        } else {
-                            store_row_block(a, (int64_t)row0 + rr, (int64_t)col0 + 32 * bb, packed, nib, sats,
-                                            (uint32_t)(k + 127), v8y, a16, a4, cstride, mstride, nblk);
-                        }
-                    } else if (rr < nrows && col0 + 32 * bb < a.cols) {
-                        if (fast) {
-                            row_fast();
-                        } else {
+                    } else {
 #pragma unroll
-                            for (int jj = 0; jj < 4; ++jj) {
-                                uint4 dv;
-                                dv.x = aw[4 * jj] | sg[4 * jj];
-                                dv.y = aw[4 * jj + 1] | sg[4 * jj + 1];
-                                dv.z = aw[4 * jj + 2] | sg[4 * jj + 2];
-                                dv.w = aw[4 * jj + 3] | sg[4 * jj + 3];
-                                const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
-                                packed[4 * jj + 0] = gch.packed.x;
-                                packed[4 * jj + 1] = gch.packed.y;
-                                packed[4 * jj + 2] = gch.packed.z;
-                                packed[4 * jj + 3] = gch.packed.w;
-                                nib[jj] = gch.nibs;
-                                sats |= gch.sats << (8 * jj);
-                            }
+                        for (int jj = 0; jj < 4; ++jj) {
+                            uint4 dv;
+                            dv.x = bw[4 * jj] | bs[4 * jj];
+                            dv.y = bw[4 * jj + 1] | bs[4 * jj + 1];
+                            dv.z = bw[4 * jj + 2] | bs[4 * jj + 2];
+                            dv.w = bw[4 * jj + 3] | bs[4 * jj + 3];
+                            const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
+                            packed[4 * jj + 0] = gch.packed.x;
+                            packed[4 * jj + 1] = gch.packed.y;
+                            packed[4 * jj + 2] = gch.packed.z;
+                            packed[4 * jj + 3] = gch.packed.w;
+                            nib[jj] = gch.nibs;
+                            sats |= gch.sats << (8 * jj);
                         }
-                        store_row_block(a, (int64_t)row0 + rr, (int64_t)col0 + 32 * bb, packed, nib, sats,
-                                        fast ? (uint32_t)(k + 127) : e8_of(A, k), v8y, a16, a4, cstride, mstride,
-                                        nblk);
                     }
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        *reinterpret_cast<uint4*>(out.yrow + ro[jj]) =
+                            make_uint4(packed[4 * jj], packed[4 * jj + 1], packed[4 * jj + 2], packed[4 * jj + 3]);
+                    *reinterpret_cast<uint4*>(out.crow + rco) = make_uint4(nib[0], nib[1], nib[2], nib[3]);
+                    out.mrow[rw] = sats;
+                    // fast-path blocks are finite with k <= 16: the byte is k + 127
+                    out.srow[rw] = (uint8_t)(rfast ? (uint32_t)(k + 127) : e8_of(A, k));
                 }
+            }
+            __syncwarp();  // every lane of the warp has read its row data from the sub-tile
+            {
+                uint32_t* yq[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    yq[q] = reinterpret_cast<uint32_t*>(tile + yo[q]);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    yq[i & 3][(i >> 2) * 256] = ycw[i];
             }
             // column pairs of the general path add their exact saturation bits
             if (__any_sync(FULL, gsat != 0u))
-                col_sat_store(sm.mcol[buf], gsat, h, p, warp);
+                col_sat_store(out.mcol, gsat, h, p, warp);
             fence_async_smem();  // staged outputs -> visible to the TMA stores
         }
         if (tid == 0)
-            bulk_wait_read_all();  // the previous tile's stores have read their staging buffer
-        __syncthreads();           // stage s is consumed; staging buffer buf is complete
+            bulk_wait_read_all();  // the previous tile's stores have read its stage and staging buffer
+        __syncthreads();           // this tile's outputs are complete; errors visible
         if (sm.err)
             break;
-        const uint32_t ts = full ? a.ts_flags : 0u;
+        const uint32_t tma = full ? (present & a.ts_flags) : 0u;
         if (tid == 0) {
-            const uint32_t yb = smem_addr(sm.ycol[buf]);
-            if (a.y_col && (ts & SG_TS_Y)) {
+            const uint32_t ybase_c = smem_addr(tile), ybase_r = smem_addr(out.yrow);
 #pragma unroll
-                for (int sl = 0; sl < 4; ++sl)
-                    tma_store_box(&maps.y, yb + sl * SG_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
+            for (int sl = 0; sl < 4; ++sl) {
+                if (tma & SG_TS_Y)
+                    tma_store_box(&maps.y, ybase_c + sl * SG_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
+                if (tma & SG_TS_YR)
+                    tma_store_box(&maps.yr, ybase_r + sl * SG_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
             }
-            if (a.codes_col && (ts & SG_TS_CODES))
-                tma_store_box(&maps.codes, smem_addr(sm.ccol[buf]), col0 / 2, row0);
-            if (a.mask_col && (ts & SG_TS_MASK))
-                tma_store_box(&maps.mask, smem_addr(sm.mcol[buf]), col0 / 8, row0);
+            if (tma & SG_TS_CODES)
+                tma_store_box(&maps.codes, smem_addr(out.ccol), col0 / 2, row0);
+            if (tma & SG_TS_CODES_R)
+                tma_store_box(&maps.codes_r, smem_addr(out.crow), col0 / 2, row0);
+            if (tma & SG_TS_MASK)
+                tma_store_box(&maps.mask, smem_addr(out.mcol), col0 / 8, row0);
+            if (tma & SG_TS_MASK_R)
+                tma_store_box(&maps.mask_r, smem_addr(out.mrow), col0 / 8, row0);
             bulk_commit();
-            if (t_issue < t_end)
-                issue(s);
+            // the previous tile's stage is free again (its stores have read
+            // it): load the tile SG_STAGES - 1 ahead of the next one into it
+            if (j > 0 && t_issue < t_end)
+                issue(s == 0 ? SG_STAGES - 1 : s - 1);
         }
-        const bool cy = a.y_col && !(ts & SG_TS_Y), cc = a.codes_col && !(ts & SG_TS_CODES),
-                   cm = a.mask_col && !(ts & SG_TS_MASK);
-        if (cy || cc || cm)
-            copy_col_outputs(a, sm, buf, row0, nrows, col0, cy, cc, cm);
+        const uint32_t copy = present & ~tma;
+        if (copy)
+            copy_outputs(a, tile, out, row0, nrows, col0, copy);
+        if (ROW && a.scales_row && warp == 0)
+            copy_row_scales(a, out, row0, nrows, col0);
         if (++s == SG_STAGES) {
             s = 0;
             phase ^= 1u;
