@@ -218,7 +218,7 @@ __device__ __forceinline__ void st_stream(void* p, const uint4& v)
 // Writes s_rst[g] = sum_{j<g} n_j and s_bpre[g] = sum_{j<g} ceil(n_j / BS) for
 // g = 0..G and returns S = s_bpre[G], or -1 when the list is not a partition
 // of [0, rows): a negative count, a decreasing offset, or a wrong total.
-// Every thread of the CTA must call it.
+// Every thread of the CTA must call it; the first NTHREADS hold the groups.
 template <int BS>
 __device__ int64_t build_plan(const KArgs& a, int32_t* s_bpre, int32_t* s_rst)
 {
@@ -256,7 +256,7 @@ __device__ int64_t build_plan(const KArgs& a, int32_t* s_bpre, int32_t* s_rst)
             ib += tb;
         }
     }
-    if (lane == 31) {
+    if (lane == 31 && warp < NTHREADS / 32) {  // a CTA may carry extra warps: they hold no groups
         s_wr[warp] = ir;
         s_wb[warp] = ib;
     }
@@ -1122,8 +1122,9 @@ static int device_sms()
     return info[dev].sms;
 }
 
-// Resident CTAs per SM of `fn`, cached per (device, kernel).
-static int occupancy(const void* fn, size_t smem)
+// Resident CTAs per SM of `fn` launched with `threads` per CTA, cached per
+// (device, kernel).
+static int occupancy(const void* fn, size_t smem, int threads = NTHREADS)
 {
     struct Entry {
         const void* fn;
@@ -1143,7 +1144,7 @@ static int occupancy(const void* fn, size_t smem)
                 return cache[i].occ;
     }
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NTHREADS, smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, smem) != cudaSuccess)
         return -1;
     if (occ < 1)
         occ = 1;
@@ -1372,13 +1373,13 @@ static mxfp4_status launch_staged(bool row, bool groups, const StagedMaps& maps,
     if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MXFP4_ECUDA;
     const int sms = device_sms();
-    const int occ = occupancy((const void*)fn, smem);
+    const int occ = occupancy((const void*)fn, smem, SG_THREADS);
     if (sms <= 0 || occ <= 0)
         return MXFP4_ECUDA;
     int64_t grid = (int64_t)sms * occ;
     if (tiles < grid)
         grid = tiles < 1 ? 1 : tiles;
-    fn<<<(unsigned)grid, NTHREADS, smem, s>>>(maps, k);
+    fn<<<(unsigned)grid, SG_THREADS, smem, s>>>(maps, k);
     return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
 }
 

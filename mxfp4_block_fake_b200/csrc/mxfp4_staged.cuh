@@ -42,7 +42,7 @@ constexpr int SG_TILE_BYTES = 4 * SG_SLAB_BYTES;           // 16384
 constexpr int SG_CODE_BYTES = SG_ROWS * SG_COLS / 2;       // 4096: e2m1 codes of a tile
 constexpr int SG_MASK_WORDS = SG_ROWS * SG_COLS / 32;      // 256: saturation bits of a tile
 constexpr int SG_STAGES = 3;
-constexpr uint32_t SG_WAIT_LIMIT = 1u << 22;               // try_wait polls before giving up
+constexpr uint64_t SG_WAIT_NS = 4000000000ull;             // an mbarrier wait gives up after 4 s
 
 // which outputs leave through TMA stores on full tiles (the others, and every
 // output of a group-tail or ragged tile, are copied out by the threads)
@@ -53,8 +53,8 @@ constexpr uint32_t SG_TS_YR = 8u, SG_TS_CODES_R = 16u, SG_TS_MASK_R = 32u;      
 // slabs of 64 columns with the 128-byte swizzle); codes are 32 rows of 128
 // bytes with the 128-byte swizzle; masks are 32 rows of 32 bytes; row-wise
 // scales are 32 rows of 8 bytes.
-// (Column-wise y is written over the tile's input in its stage instead.)
 struct __align__(1024) StagedOut {
+    uint8_t ycol[SG_TILE_BYTES];
     uint8_t yrow[SG_TILE_BYTES];
     uint8_t ccol[SG_CODE_BYTES];
     uint8_t crow[SG_CODE_BYTES];
@@ -64,14 +64,16 @@ struct __align__(1024) StagedOut {
 };
 
 struct __align__(1024) StagedSmem {
-    uint8_t tiles[SG_STAGES][SG_TILE_BYTES];  // input stages (1024-aligned swizzle atoms); column-wise y
-    StagedOut out[2];                         // staged outputs, double-buffered by tile parity
+    uint8_t tiles[SG_STAGES][SG_TILE_BYTES];  // input stages (1024-aligned swizzle atoms)
+    StagedOut out;                            // staged outputs of the tile in flight
     uint32_t limw[8][16];                     // per warp and column pair: 0x8000 + limit bits of each column
     int4 info[SG_STAGES];                     // row0, nrows, col0, row block of each stage's tile
     uint32_t lut[64];
-    unsigned long long full[SG_STAGES];       // mbarriers, one per stage
+    unsigned long long full[SG_STAGES];       // mbarriers: stage loaded (TMA transaction count)
     int err;
 };
+
+constexpr int SG_THREADS = NTHREADS;
 
 // TMA descriptors: the input and the outputs (an output map is only read
 // when its SG_TS_* flag is set).
@@ -92,21 +94,42 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of the given parity to complete; false after SG_WAIT_NS
+// of global time (the caller then records an error and stops).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
 {
-    for (uint32_t it = 0; it < SG_WAIT_LIMIT; ++it) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (done)
-            return true;
-    }
-    return false;
+    if (mbar_try(bar, parity))
+        return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try(bar, parity))
+        if (global_ns() - t0 > SG_WAIT_NS)
+            return false;
+    return true;
 }
 
 // One 64 x 32 box of bf16 from global memory into a 4 KB swizzled slab. The
@@ -298,14 +321,14 @@ struct TileWalk {
     }
 };
 
-// Copy the staged outputs of a tile to global memory with the threads
-// (group tails, ragged tiles, outputs TMA cannot address). The flags select
-// the outputs; rows at or past nrows and columns at or past cols are skipped.
-__device__ __forceinline__ void copy_outputs(const KArgs& a, const uint8_t* ycol, const StagedOut& o, int row0,
-                                             int nrows, int col0, uint32_t which)
+// Copy staged outputs of a tile to global memory with the threads of the CTA
+// (group tails, outputs TMA cannot address). The flags select the outputs;
+// rows at or past nrows and columns at or past cols are skipped.
+__device__ __forceinline__ void copy_outputs(const KArgs& a, const StagedOut& o, int row0, int nrows, int col0,
+                                             uint32_t which)
 {
     const int tid = threadIdx.x;
-    const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8, nblk = (a.cols + 31) / 32;
+    const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         const int q = tid + NTHREADS * m;  // 0..1023
@@ -319,7 +342,7 @@ __device__ __forceinline__ void copy_outputs(const KArgs& a, const uint8_t* ycol
         const uint32_t yoff = (u >> 3) * SG_SLAB_BYTES + r * 128 + (((u & 7) ^ (r & 7)) << 4);
         const uint32_t coff = r * 128 + (((u >> 2) ^ (r & 7)) << 4) + 4 * (u & 3);
         if (which & SG_TS_Y)
-            st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * 2, sm_ld128(ycol, yoff));
+            st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * 2, sm_ld128(o.ycol, yoff));
         if (which & SG_TS_YR)
             st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * 2, sm_ld128(o.yrow, yoff));
         if (which & SG_TS_CODES)
@@ -333,11 +356,11 @@ __device__ __forceinline__ void copy_outputs(const KArgs& a, const uint8_t* ycol
     }
 }
 
-// Row-wise scales of a tile (32 rows x 8 blocks) from staging: one row per
-// lane of warp 0.
-__device__ __forceinline__ void copy_row_scales(const KArgs& a, const StagedOut& o, int row0, int nrows, int col0)
+// Row-wise scales of a tile (32 rows x 8 blocks) from staging: one row per lane.
+__device__ __forceinline__ void copy_row_scales(const KArgs& a, const StagedOut& o, int row0, int nrows, int col0,
+                                                int lane)
 {
-    const int r = threadIdx.x;
+    const int r = lane;
     if (r >= nrows)
         return;
     const int64_t nblk = (a.cols + 31) / 32;
@@ -366,13 +389,14 @@ __device__ __forceinline__ void col_sat_store(uint32_t* mwords, uint32_t bits, i
 }
 
 template <bool ROW, bool GROUPS, int MODE>
-__global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_constant__ StagedMaps maps, const KArgs a)
+__global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_constant__ StagedMaps maps, const KArgs a)
 {
     extern __shared__ __align__(1024) uint8_t s_dyn[];
     // the swizzle pattern follows absolute shared-memory address bits, so the
     // slabs are placed on a 1024-byte boundary (1 KB of slack is requested)
     uint8_t* s_base = s_dyn + ((1024u - (smem_addr(s_dyn) & 1023u)) & 1023u);
     StagedSmem& sm = *reinterpret_cast<StagedSmem*>(s_base);
+    StagedOut& out = sm.out;
     int32_t* s_plan = reinterpret_cast<int32_t*>(s_base + sizeof(StagedSmem));
     int32_t* s_bpre = s_plan;
     int32_t* s_rst = s_plan + (GROUPS ? a.num_groups + 1 : 0);
@@ -403,10 +427,11 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
     const uint32_t t_end = (uint32_t)(((uint64_t)(blockIdx.x + 1) * ntiles) / gridDim.x);
     const uint32_t lutb = smem_addr(sm.lut) - 0x2C000000u;
     const uint32_t lutb16 = lutb + 0x04000000u;
-    // outputs present (SG_TS_* bits); those not written by TMA are copied
-    const uint32_t present = (a.y_col ? SG_TS_Y : 0u) | (a.codes_col ? SG_TS_CODES : 0u) |
-                             (a.mask_col ? SG_TS_MASK : 0u) | (ROW && a.y_row ? SG_TS_YR : 0u) |
-                             (ROW && a.codes_row ? SG_TS_CODES_R : 0u) | (ROW && a.mask_row ? SG_TS_MASK_R : 0u);
+    // outputs present, as SG_TS_* bits; those TMA cannot address are copied
+    const uint32_t col_out = (a.y_col ? SG_TS_Y : 0u) | (a.codes_col ? SG_TS_CODES : 0u) |
+                             (a.mask_col ? SG_TS_MASK : 0u);
+    const uint32_t row_out = (ROW && a.y_row ? SG_TS_YR : 0u) | (ROW && a.codes_row ? SG_TS_CODES_R : 0u) |
+                             (ROW && a.mask_row ? SG_TS_MASK_R : 0u);
 
     // producer state (thread 0): the next tile to load
     TileWalk<GROUPS> pw;
@@ -456,14 +481,16 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
 
     int s = 0;
     uint32_t phase = 0;
-    for (uint32_t t = t_begin, j = 0; t < t_end; ++t, ++j) {
-        StagedOut& out = sm.out[j & 1];
-        bool full = false;
+    for (uint32_t t = t_begin; t < t_end; ++t) {
         int row0 = 0, nrows = 0, col0 = 0;
         // the warp decides together, so that its shuffles and votes below
         // always see all 32 lanes
         const bool ok = __all_sync(FULL, mbar_wait(smem_addr(&sm.full[s]), phase));
-        uint8_t* tile = sm.tiles[s];
+        const uint8_t* tile = sm.tiles[s];
+        uint32_t cw[16];  // the column pass's raw words
+        int k_lo = 0, k_hi = 0;
+        uint32_t A_lo = 0, A_hi = 0;
+        bool fast = true;
         if (!ok) {
             sm.err = 1;
         } else {
@@ -472,223 +499,210 @@ __global__ void __launch_bounds__(NTHREADS, 2) qdq_staged_kernel(const __grid_co
             nrows = inf.y;
             col0 = inf.z;
             const uint32_t rb = (uint32_t)inf.w;
-            full = nrows == SG_ROWS && col0 + SG_COLS <= a.cols;  // the same for the whole CTA
+            const bool rows_full = nrows == SG_ROWS;
 
-            // ---- column pass: the lane's column pair over its 16 rows. Its y
-            // words wait in registers until the warp's row pass has read the
-            // sub-tile, then replace the input in the stage.
-            uint32_t ycw[16];
-            uint32_t gsat = 0;  // saturation bits of a general-path column pair (bits 2i, 2i+1: word i)
-            {
-                uint32_t aw[16], sg[16];
+            // ---- column pass, part 1: amax and parameters of the column pair
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                cw[i] = sm_ld32(tile, yo[i & 3] + (i >> 2) * 1024);
+            if (!rows_full) {
+                // rows past a group tail belong to the next group: neither
+                // their values nor their amax take part
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    prep_bf(sm_ld32(tile, yo[i & 3] + (i >> 2) * 1024), aw[i], sg[i]);
-                if (!full) {
-                    // rows past a group tail belong to the next group: neither
-                    // their values nor their amax take part
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (8 * (i >> 2) + 4 * h + (i & 3) >= nrows)
-                            aw[i] = sg[i] = 0u;
-                }
-                uint32_t m2 = vmax2(vmax2(vmax2(aw[0], aw[1]), vmax2(aw[2], aw[3])),
-                                    vmax2(vmax2(aw[4], aw[5]), vmax2(aw[6], aw[7])));
-                m2 = vmax2(m2, vmax2(vmax2(vmax2(aw[8], aw[9]), vmax2(aw[10], aw[11])),
-                                     vmax2(vmax2(aw[12], aw[13]), vmax2(aw[14], aw[15]))));
-                m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 16));
-                const uint32_t A_lo = m2 << 16, A_hi = m2 & 0xFFFF0000u;
-                const int k_lo = block_kt<MODE>(A_lo, a.thr), k_hi = block_kt<MODE>(A_hi, a.thr);
-                const bool fast = k_fast_bf(k_lo) && k_fast_bf(k_hi);
-                if (h == 0) {
-                    // the row pass of this warp tests its elements against these
-                    // limits (0xFFFF: never; the general path reports its own)
-                    sm.limw[warp][p] = fast ? (0x8000u + lim16_of_k(k_lo)) | ((0x8000u + lim16_of_k(k_hi)) << 16)
-                                            : 0xFFFFFFFFu;
-                    if (a.scales_col && (full || col0 + cpair < a.cols)) {
-                        // fast-path blocks are finite with k <= 16: the byte is k + 127
-                        const uint32_t e8p = fast ? (uint32_t)(k_lo + 127) | ((uint32_t)(k_hi + 127) << 8)
-                                                  : e8_of(A_lo, k_lo) | (e8_of(A_hi, k_hi) << 8);
-                        *reinterpret_cast<uint16_t*>(a.scales_col + (int64_t)rb * a.cols + col0 + cpair) =
-                            (uint16_t)e8p;
-                    }
-                }
-                uint8_t* cq[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    cq[q] = out.ccol + co[q];
-                auto col_fast = [&]() {
-                    const float inv_lo = __uint_as_float(0x3F800000u - ((uint32_t)k_lo << 23));
-                    const float inv_hi = __uint_as_float(0x3F800000u - ((uint32_t)k_hi << 23));
-                    const uint32_t s2 = bf16_pow2(k_lo) | (bf16_pow2(k_hi) << 16);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        uint32_t P;
-                        ycw[i] = qword(aw[i], sg[i], inv_lo, inv_hi, s2, lutb16, P);
-                        cq[i & 3][(i >> 2) * 1024] = (uint8_t)e2m1_byte(P);
-                    }
-                };
-                if (__all_sync(FULL, fast)) {
-                    col_fast();  // the common case, straight-line
-                } else if (fast) {
-                    col_fast();
-                } else {
-                    const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
-#pragma unroll
-                    for (int i0 = 0; i0 < 16; i0 += 4) {
-                        // the general path takes x itself; -0 halves may enter as +0
-                        uint4 dv;
-                        dv.x = aw[i0] | sg[i0];
-                        dv.y = aw[i0 + 1] | sg[i0 + 1];
-                        dv.z = aw[i0 + 2] | sg[i0 + 2];
-                        dv.w = aw[i0 + 3] | sg[i0 + 3];
-                        const ChunkOut gch = general_chunk<8, true>(dv, Ac, a.mode, a.thr, lutb);
-                        gsat |= (gch.sats & 0xFFu) << (2 * i0);
-                        ycw[i0] = gch.packed.x;
-                        ycw[i0 + 1] = gch.packed.y;
-                        ycw[i0 + 2] = gch.packed.z;
-                        ycw[i0 + 3] = gch.packed.w;
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int i = i0 + u;
-                            cq[i & 3][(i >> 2) * 1024] = (uint8_t)(gch.nibs >> (8 * u));
-                        }
-                    }
-                }
+                    if (8 * (i >> 2) + 4 * h + (i & 3) >= nrows)
+                        cw[i] = 0u;
             }
-            __syncwarp();  // limw of this warp
-
-            // ---- row pass: the lane's row-wise block (tile row rr, columns
-            // 32w..32w+31): row-wise outputs, and the column-wise saturation
-            // word of the same 32 elements
-            {
-                uint32_t bw[16], bs[16];
+            uint32_t m2 = 0;
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint4 c = sm_ld128(tile, ro[jj]);
-                    prep_bf(c.x, bw[4 * jj + 0], bs[4 * jj + 0]);
-                    prep_bf(c.y, bw[4 * jj + 1], bs[4 * jj + 1]);
-                    prep_bf(c.z, bw[4 * jj + 2], bs[4 * jj + 2]);
-                    prep_bf(c.w, bw[4 * jj + 3], bs[4 * jj + 3]);
-                }
-                if (a.mask_col) {
-                    // rows past a group tail are not copied out; their word is don't-care
-                    uint32_t cm = 0;
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const uint4 L = *reinterpret_cast<const uint4*>(&sm.limw[warp][4 * jj]);
-                        const uint32_t lx[4] = {L.x, L.y, L.z, L.w};
-                        const uint32_t a4w[4] = {bw[4 * jj], bw[4 * jj + 1], bw[4 * jj + 2], bw[4 * jj + 3]};
-                        cm |= sat8(a4w, lx) << (8 * jj);
-                    }
-                    out.mcol[rw] = cm;
-                }
-                if constexpr (ROW) {
-                    uint32_t m2 = vmax2(vmax2(vmax2(bw[0], bw[1]), vmax2(bw[2], bw[3])),
-                                        vmax2(vmax2(bw[4], bw[5]), vmax2(bw[6], bw[7])));
-                    m2 = vmax2(m2, vmax2(vmax2(vmax2(bw[8], bw[9]), vmax2(bw[10], bw[11])),
-                                         vmax2(vmax2(bw[12], bw[13]), vmax2(bw[14], bw[15]))));
-                    const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
-                    const uint32_t A = am << 16;
-                    const int k = block_kt<MODE>(A, a.thr);
-                    const bool rfast = k_fast_bf(k);
-                    uint32_t packed[16], nib[4], sats = 0;
-                    auto row_fast = [&]() {
-                        const float inv = __uint_as_float(0x3F800000u - ((uint32_t)k << 23));
-                        const uint32_t s2 = bf16_pow2(k) * 0x10001u;
-                        const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
-                        const uint32_t limx[4] = {lx, lx, lx, lx};
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            uint32_t P[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                packed[4 * jj + u] = qword(bw[4 * jj + u], bs[4 * jj + u], inv, inv, s2, lutb16, P[u]);
-                            nib[jj] = e2m1_word(P);
-                            const uint32_t a4w[4] = {bw[4 * jj], bw[4 * jj + 1], bw[4 * jj + 2], bw[4 * jj + 3]};
-                            sats |= sat8(a4w, limx) << (8 * jj);
-                        }
-                    };
-                    if (__all_sync(FULL, rfast)) {
-                        row_fast();  // the common case, straight-line
-                    } else if (rfast) {
-                        row_fast();
-                    } else {
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            uint4 dv;
-                            dv.x = bw[4 * jj] | bs[4 * jj];
-                            dv.y = bw[4 * jj + 1] | bs[4 * jj + 1];
-                            dv.z = bw[4 * jj + 2] | bs[4 * jj + 2];
-                            dv.w = bw[4 * jj + 3] | bs[4 * jj + 3];
-                            const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
-                            packed[4 * jj + 0] = gch.packed.x;
-                            packed[4 * jj + 1] = gch.packed.y;
-                            packed[4 * jj + 2] = gch.packed.z;
-                            packed[4 * jj + 3] = gch.packed.w;
-                            nib[jj] = gch.nibs;
-                            sats |= gch.sats << (8 * jj);
-                        }
-                    }
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        *reinterpret_cast<uint4*>(out.yrow + ro[jj]) =
-                            make_uint4(packed[4 * jj], packed[4 * jj + 1], packed[4 * jj + 2], packed[4 * jj + 3]);
-                    *reinterpret_cast<uint4*>(out.crow + rco) = make_uint4(nib[0], nib[1], nib[2], nib[3]);
-                    out.mrow[rw] = sats;
+            for (int i = 0; i < 16; ++i)
+                m2 = vmax2(m2, cw[i] & 0x7FFF7FFFu);
+            m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 16));
+            A_lo = m2 << 16;
+            A_hi = m2 & 0xFFFF0000u;
+            k_lo = block_kt<MODE>(A_lo, a.thr);
+            k_hi = block_kt<MODE>(A_hi, a.thr);
+            fast = k_fast_bf(k_lo) && k_fast_bf(k_hi);
+            if (h == 0) {
+                // the row pass of this warp tests its elements against these
+                // limits (0xFFFF: never; the general path reports its own)
+                sm.limw[warp][p] = fast ? (0x8000u + lim16_of_k(k_lo)) | ((0x8000u + lim16_of_k(k_hi)) << 16)
+                                        : 0xFFFFFFFFu;
+                if (a.scales_col && col0 + cpair < a.cols) {
                     // fast-path blocks are finite with k <= 16: the byte is k + 127
-                    out.srow[rw] = (uint8_t)(rfast ? (uint32_t)(k + 127) : e8_of(A, k));
+                    const uint32_t e8p = fast ? (uint32_t)(k_lo + 127) | ((uint32_t)(k_hi + 127) << 8)
+                                              : e8_of(A_lo, k_lo) | (e8_of(A_hi, k_hi) << 8);
+                    *reinterpret_cast<uint16_t*>(a.scales_col + (int64_t)rb * a.cols + col0 + cpair) =
+                        (uint16_t)e8p;
                 }
             }
-            __syncwarp();  // every lane of the warp has read its row data from the sub-tile
-            {
-                uint32_t* yq[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    yq[q] = reinterpret_cast<uint32_t*>(tile + yo[q]);
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    yq[i & 3][(i >> 2) * 256] = ycw[i];
-            }
-            // column pairs of the general path add their exact saturation bits
-            if (__any_sync(FULL, gsat != 0u))
-                col_sat_store(out.mcol, gsat, h, p, warp);
-            fence_async_smem();  // staged outputs -> visible to the TMA stores
         }
         if (tid == 0)
-            bulk_wait_read_all();  // the previous tile's stores have read its stage and staging buffer
-        __syncthreads();           // this tile's outputs are complete; errors visible
+            bulk_wait_read_all();  // the previous tile's stores have read the staging buffers
+        __syncthreads();           // staging free; limw complete; errors visible
         if (sm.err)
             break;
-        const uint32_t tma = full ? (present & a.ts_flags) : 0u;
+
+        // ---- column pass, part 2: y and codes of the column pair
+        uint32_t gsat = 0;  // saturation bits of a general-path column pair (bits 2i, 2i+1: word i)
+        {
+            uint32_t* yq[4];
+            uint8_t* cq[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                yq[q] = reinterpret_cast<uint32_t*>(out.ycol + yo[q]);
+                cq[q] = out.ccol + co[q];
+            }
+            auto col_fast = [&]() {
+                const float inv_lo = __uint_as_float(0x3F800000u - ((uint32_t)k_lo << 23));
+                const float inv_hi = __uint_as_float(0x3F800000u - ((uint32_t)k_hi << 23));
+                const uint32_t s2 = bf16_pow2(k_lo) | (bf16_pow2(k_hi) << 16);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    uint32_t aw, sg, P;
+                    prep_bf(cw[i], aw, sg);
+                    yq[i & 3][(i >> 2) * 256] = qword(aw, sg, inv_lo, inv_hi, s2, lutb16, P);
+                    cq[i & 3][(i >> 2) * 1024] = (uint8_t)e2m1_byte(P);
+                }
+            };
+            if (__all_sync(FULL, fast)) {
+                col_fast();  // the common case, straight-line
+            } else if (fast) {
+                col_fast();
+            } else {
+                const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
+#pragma unroll
+                for (int i0 = 0; i0 < 16; i0 += 4) {
+                    const uint4 dv = make_uint4(cw[i0], cw[i0 + 1], cw[i0 + 2], cw[i0 + 3]);
+                    const ChunkOut gch = general_chunk<8, true>(dv, Ac, a.mode, a.thr, lutb);
+                    gsat |= (gch.sats & 0xFFu) << (2 * i0);
+                    const uint32_t ov[4] = {gch.packed.x, gch.packed.y, gch.packed.z, gch.packed.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + u;
+                        yq[i & 3][(i >> 2) * 256] = ov[u];
+                        cq[i & 3][(i >> 2) * 1024] = (uint8_t)(gch.nibs >> (8 * u));
+                    }
+                }
+            }
+        }
+
+        // ---- row pass: the lane's row-wise block (tile row rr, columns
+        // 32w..32w+31): row-wise outputs, and the column-wise saturation word
+        // of the same 32 elements
+        {
+            uint32_t rw16[16];  // raw words of the lane's block
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const uint4 c = sm_ld128(tile, ro[jj]);
+                rw16[4 * jj + 0] = c.x;
+                rw16[4 * jj + 1] = c.y;
+                rw16[4 * jj + 2] = c.z;
+                rw16[4 * jj + 3] = c.w;
+            }
+            if (a.mask_col) {
+                // rows past a group tail are not copied out; their word is don't-care
+                uint32_t cm = 0;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint4 L = *reinterpret_cast<const uint4*>(&sm.limw[warp][4 * jj]);
+                    const uint32_t lx[4] = {L.x, L.y, L.z, L.w};
+                    const uint32_t a4w[4] = {rw16[4 * jj] & 0x7FFF7FFFu, rw16[4 * jj + 1] & 0x7FFF7FFFu,
+                                             rw16[4 * jj + 2] & 0x7FFF7FFFu, rw16[4 * jj + 3] & 0x7FFF7FFFu};
+                    cm |= sat8(a4w, lx) << (8 * jj);
+                }
+                out.mcol[rw] = cm;
+            }
+            if constexpr (ROW) {
+                // every row of the tile is computed, group tail or not: a
+                // row's row-wise outputs depend on that row alone
+                uint32_t m2 = 0;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    m2 = vmax2(m2, rw16[i] & 0x7FFF7FFFu);
+                const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
+                const uint32_t A = am << 16;
+                const int k = block_kt<MODE>(A, a.thr);
+                const bool rfast = k_fast_bf(k);
+                uint32_t nib[4], sats = 0;
+                auto row_fast = [&]() {
+                    const float inv = __uint_as_float(0x3F800000u - ((uint32_t)k << 23));
+                    const uint32_t s2 = bf16_pow2(k) * 0x10001u;
+                    const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
+                    const uint32_t limx[4] = {lx, lx, lx, lx};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        uint32_t P[4], o[4], a4w[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            uint32_t sg;
+                            prep_bf(rw16[4 * jj + u], a4w[u], sg);
+                            o[u] = qword(a4w[u], sg, inv, inv, s2, lutb16, P[u]);
+                        }
+                        *reinterpret_cast<uint4*>(out.yrow + ro[jj]) = make_uint4(o[0], o[1], o[2], o[3]);
+                        nib[jj] = e2m1_word(P);
+                        sats |= sat8(a4w, limx) << (8 * jj);
+                    }
+                };
+                if (__all_sync(FULL, rfast)) {
+                    row_fast();  // the common case, straight-line
+                } else if (rfast) {
+                    row_fast();
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const uint4 dv = make_uint4(rw16[4 * jj], rw16[4 * jj + 1], rw16[4 * jj + 2], rw16[4 * jj + 3]);
+                        const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
+                        *reinterpret_cast<uint4*>(out.yrow + ro[jj]) = gch.packed;
+                        nib[jj] = gch.nibs;
+                        sats |= gch.sats << (8 * jj);
+                    }
+                }
+                *reinterpret_cast<uint4*>(out.crow + rco) = make_uint4(nib[0], nib[1], nib[2], nib[3]);
+                out.mrow[rw] = sats;
+                // fast-path blocks are finite with k <= 16: the byte is k + 127
+                out.srow[rw] = (uint8_t)(rfast ? (uint32_t)(k + 127) : e8_of(A, k));
+            }
+        }
+        // column pairs of the general path add their exact saturation bits
+        if (__any_sync(FULL, gsat != 0u))
+            col_sat_store(out.mcol, gsat, h, p, warp);
+        fence_async_smem();  // staged outputs -> visible to the TMA stores
+        __syncthreads();     // stage s consumed; staged outputs complete
+
+        // Column-wise outputs of a group tail are copied (the rows past it
+        // belong to the next group); row-wise outputs always leave by TMA
+        // where it can address them, the rows past a group tail included:
+        // they equal what the tile that owns those rows writes. TMA clips
+        // rows and columns outside the tensor.
+        const uint32_t tma = (nrows == SG_ROWS ? col_out : 0u) | row_out;
+        const uint32_t copy = (col_out | row_out) & ~(tma & a.ts_flags);
         if (tid == 0) {
-            const uint32_t ybase_c = smem_addr(tile), ybase_r = smem_addr(out.yrow);
+            const uint32_t st = tma & a.ts_flags;
+            const uint32_t ybase_c = smem_addr(out.ycol), ybase_r = smem_addr(out.yrow);
 #pragma unroll
             for (int sl = 0; sl < 4; ++sl) {
-                if (tma & SG_TS_Y)
+                if ((st & SG_TS_Y) && col0 + sl * SG_SLAB_COLS < a.cols)
                     tma_store_box(&maps.y, ybase_c + sl * SG_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
-                if (tma & SG_TS_YR)
+                if ((st & SG_TS_YR) && col0 + sl * SG_SLAB_COLS < a.cols)
                     tma_store_box(&maps.yr, ybase_r + sl * SG_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
             }
-            if (tma & SG_TS_CODES)
+            if (st & SG_TS_CODES)
                 tma_store_box(&maps.codes, smem_addr(out.ccol), col0 / 2, row0);
-            if (tma & SG_TS_CODES_R)
+            if (st & SG_TS_CODES_R)
                 tma_store_box(&maps.codes_r, smem_addr(out.crow), col0 / 2, row0);
-            if (tma & SG_TS_MASK)
+            if (st & SG_TS_MASK)
                 tma_store_box(&maps.mask, smem_addr(out.mcol), col0 / 8, row0);
-            if (tma & SG_TS_MASK_R)
+            if (st & SG_TS_MASK_R)
                 tma_store_box(&maps.mask_r, smem_addr(out.mrow), col0 / 8, row0);
             bulk_commit();
-            // the previous tile's stage is free again (its stores have read
-            // it): load the tile SG_STAGES - 1 ahead of the next one into it
-            if (j > 0 && t_issue < t_end)
-                issue(s == 0 ? SG_STAGES - 1 : s - 1);
+            if (t_issue < t_end)
+                issue(s);
         }
-        const uint32_t copy = present & ~tma;
         if (copy)
-            copy_outputs(a, tile, out, row0, nrows, col0, copy);
+            copy_outputs(a, out, row0, nrows, col0, copy);
         if (ROW && a.scales_row && warp == 0)
-            copy_row_scales(a, out, row0, nrows, col0);
+            copy_row_scales(a, out, row0, nrows, col0, lane);
         if (++s == SG_STAGES) {
             s = 0;
             phase ^= 1u;
