@@ -181,14 +181,23 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
-def traffic_for(kernel_src: str, launch_bytes: int):
+def kernel_source_sha() -> str:
+    """sha256 over the CUDA sources of the library (the forward kernels)."""
+    h = hashlib.sha256()
+    for name in ("mxfp4.cu", "mxfp4_staged.cuh"):
+        with open(os.path.join(ROOT, "mxfp4_block_fake_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_for(launch_bytes: int):
     """DRAM traffic per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
+    on the current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
-        sha = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+        sha = kernel_source_sha()
         if t.get("source_sha256") != sha:
             return None
         scale = launch_bytes / t["algorithmic_bytes_per_launch"] if t.get("algorithmic_bytes_per_launch") else 1.0
@@ -351,7 +360,6 @@ def main():
             b = step_bytes(a.rows, a.cols, r["s_col"])
             value = weak_value(b["step"], a.steps, world, r["ms"])
             achieved = b["fwd"] / (r["fwd_ms"] / 1e3) / 1e9
-            src = os.path.join(ROOT, "mxfp4_block_fake_b200", "csrc", "mxfp4.cu")
             line = {
                 "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
                 "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(r["ms"] / a.steps, 4),
@@ -363,10 +371,10 @@ def main():
                 "elements_per_s": round(a.rows * a.cols * world * a.steps / (r["ms"] / 1e3), 1),
                 "parts_ms": {"qdq_fwd_dual": round(r["fwd_ms"], 4),
                              "ste_bwd": round(r["ms"] / a.steps - r["fwd_ms"], 4)},
-                "roofline": {"bound": "hbm", "kernel": "qdq_tile_kernel (dual, grouped, bf16, block 32)",
+                "roofline": {"bound": "hbm", "kernel": "qdq_staged_kernel (dual, grouped, bf16, block 32)",
                              "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                              "unit": "GB/s", "frac": round(achieved / peak, 4),
-                             "traffic": traffic_for(src, b["fwd"]),
+                             "traffic": traffic_for(b["fwd"]),
                              "algorithmic_bytes_per_launch": b["fwd"]},
                 "gpu_launches": 2 * a.steps,
                 "clocks": r["clocks"],
