@@ -70,10 +70,14 @@ struct __align__(1024) StagedSmem {
     int4 info[SG_STAGES];                     // row0, nrows, col0, row block of each stage's tile
     uint32_t lut[64];
     unsigned long long full[SG_STAGES];       // mbarriers: stage loaded (TMA transaction count)
+    unsigned long long sfree;                 // mbarrier: the previous tile's stores have read the staging
     int err;
 };
 
 constexpr int SG_THREADS = NTHREADS;
+// Thread 0 issues the TMA loads; thread SG_STORER (lane 0 of warp 1) issues
+// the TMA stores and waits for them, and its warp copies the row-wise scales.
+constexpr int SG_STORER = 32;
 
 // TMA descriptors: the input and the outputs (an output map is only read
 // when its SG_TS_* flag is set).
@@ -408,6 +412,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         sm.err = 0;
         for (int s = 0; s < SG_STAGES; ++s)
             mbar_init(smem_addr(&sm.full[s]), 1);
+        mbar_init(smem_addr(&sm.sfree), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     uint32_t S;
@@ -481,7 +486,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
 
     int s = 0;
     uint32_t phase = 0;
-    for (uint32_t t = t_begin; t < t_end; ++t) {
+    for (uint32_t t = t_begin, j = 0; t < t_end; ++t, ++j) {
         int row0 = 0, nrows = 0, col0 = 0;
         // the warp decides together, so that its shuffles and votes below
         // always see all 32 lanes
@@ -537,15 +542,20 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                 }
             }
         }
-        if (tid == 0)
-            bulk_wait_read_all();  // the previous tile's stores have read the staging buffers
-        __syncthreads();           // staging free; limw complete; errors visible
-        if (sm.err)
-            break;
+        // The staging buffers are free once the previous tile's stores have
+        // read them: the storer waits for that and signals; no CTA barrier.
+        if (tid == SG_STORER && j > 0) {
+            bulk_wait_read_all();
+            mbar_arrive(smem_addr(&sm.sfree));
+        }
+        const bool go = ok && (j == 0 || __all_sync(FULL, mbar_wait(smem_addr(&sm.sfree), (j - 1) & 1u)));
+        if (!go)
+            sm.err = 1;
+        __syncwarp();  // limw of this warp
 
         // ---- column pass, part 2: y and codes of the column pair
         uint32_t gsat = 0;  // saturation bits of a general-path column pair (bits 2i, 2i+1: word i)
-        {
+        if (go) {
             uint32_t* yq[4];
             uint8_t* cq[4];
 #pragma unroll
@@ -590,7 +600,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         // ---- row pass: the lane's row-wise block (tile row rr, columns
         // 32w..32w+31): row-wise outputs, and the column-wise saturation word
         // of the same 32 elements
-        {
+        if (go) {
             uint32_t rw16[16];  // raw words of the lane's block
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
@@ -665,10 +675,12 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             }
         }
         // column pairs of the general path add their exact saturation bits
-        if (__any_sync(FULL, gsat != 0u))
+        if (go && __any_sync(FULL, gsat != 0u))
             col_sat_store(out.mcol, gsat, h, p, warp);
         fence_async_smem();  // staged outputs -> visible to the TMA stores
-        __syncthreads();     // stage s consumed; staged outputs complete
+        __syncthreads();     // stage s consumed; staged outputs complete; errors visible
+        if (sm.err)
+            break;
 
         // Column-wise outputs of a group tail are copied (the rows past it
         // belong to the next group); row-wise outputs always leave by TMA
@@ -677,7 +689,9 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         // rows and columns outside the tensor.
         const uint32_t tma = (nrows == SG_ROWS ? col_out : 0u) | row_out;
         const uint32_t copy = (col_out | row_out) & ~(tma & a.ts_flags);
-        if (tid == 0) {
+        if (tid == 0 && t_issue < t_end)
+            issue(s);  // refill the consumed stage
+        if (tid == SG_STORER) {
             const uint32_t st = tma & a.ts_flags;
             const uint32_t ybase_c = smem_addr(out.ycol), ybase_r = smem_addr(out.yrow);
 #pragma unroll
@@ -696,30 +710,29 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             if (st & SG_TS_MASK_R)
                 tma_store_box(&maps.mask_r, smem_addr(out.mrow), col0 / 8, row0);
             bulk_commit();
-            if (t_issue < t_end)
-                issue(s);
         }
-        if (copy)
-            copy_outputs(a, out, row0, nrows, col0, copy);
-        if (ROW && a.scales_row && warp == 0)
+        if (ROW && a.scales_row && warp == SG_STORER / 32)
             copy_row_scales(a, out, row0, nrows, col0, lane);
+        if (copy) {
+            copy_outputs(a, out, row0, nrows, col0, copy);
+            __syncthreads();  // no warp writes the staging buffers before every copy is done
+        }
         if (++s == SG_STAGES) {
             s = 0;
             phase ^= 1u;
         }
     }
 
-    if (tid == 0) {
-        if (sm.err) {
-            if (a.status)
-                *a.status = MXFP4_ECUDA;
-            // loads still in flight land in shared memory: wait for them
-            // (bounded) before the CTA releases it
-            for (int st = 0; st < SG_STAGES; ++st)
-                (void)mbar_wait(smem_addr(&sm.full[st]), phase ^ (st < s ? 1u : 0u));
-        }
-        bulk_wait_all();
+    if (tid == 0 && sm.err) {
+        if (a.status)
+            *a.status = MXFP4_ECUDA;
+        // loads still in flight land in shared memory: wait for them
+        // (bounded) before the CTA releases it
+        for (int st = 0; st < SG_STAGES; ++st)
+            (void)mbar_wait(smem_addr(&sm.full[st]), phase ^ (st < s ? 1u : 0u));
     }
+    if (tid == SG_STORER)
+        bulk_wait_all();
 }
 
 }  // namespace mxfp4
