@@ -1355,20 +1355,21 @@ static bool make_staged_maps(StagedMaps* m, const KArgs& k, uint32_t* ts_flags)
 
 typedef void (*StagedFn)(const StagedMaps, const KArgs);
 
-static mxfp4_status launch_staged(bool row, bool groups, const StagedMaps& maps, const KArgs& k, int64_t tiles,
-                                  size_t plan_smem, cudaStream_t s)
+template <bool ROW, bool COL, bool GROUPS>
+static StagedFn pick_staged(int mode)
 {
-    StagedFn fn;
-    if (k.mode == MXFP4_SCALE_FLOOR)
-        fn = row ? (groups ? qdq_staged_kernel<true, true, MXFP4_SCALE_FLOOR>
-                           : qdq_staged_kernel<true, false, MXFP4_SCALE_FLOOR>)
-                 : (groups ? qdq_staged_kernel<false, true, MXFP4_SCALE_FLOOR>
-                           : qdq_staged_kernel<false, false, MXFP4_SCALE_FLOOR>);
-    else
-        fn = row ? (groups ? qdq_staged_kernel<true, true, MXFP4_SCALE_PAGE>
-                           : qdq_staged_kernel<true, false, MXFP4_SCALE_PAGE>)
-                 : (groups ? qdq_staged_kernel<false, true, MXFP4_SCALE_PAGE>
-                           : qdq_staged_kernel<false, false, MXFP4_SCALE_PAGE>);
+    return mode == MXFP4_SCALE_FLOOR ? qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_FLOOR>
+                                     : qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_PAGE>;
+}
+
+// row-only tiles never restart at groups (the caller routes row-only calls
+// with a group_list elsewhere)
+static mxfp4_status launch_staged(bool row, bool col, bool groups, const StagedMaps& maps, const KArgs& k,
+                                  int64_t tiles, size_t plan_smem, cudaStream_t s)
+{
+    StagedFn fn = !col ? pick_staged<true, false, false>(k.mode)
+                : row  ? (groups ? pick_staged<true, true, true>(k.mode) : pick_staged<true, true, false>(k.mode))
+                       : (groups ? pick_staged<false, true, true>(k.mode) : pick_staged<false, true, false>(k.mode));
     const size_t smem = sizeof(StagedSmem) + 1024 + plan_smem;
     if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MXFP4_ECUDA;
@@ -1500,7 +1501,7 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     const int64_t s_bound = groups ? A->rows / bs + A->num_groups : (A->rows + bs - 1) / bs;
 
     // TMA coordinates and the staged kernel's tile bookkeeping are 32-bit
-    if (fast && esz == 2 && bs == 32 && col && !grad && A->rows <= INT32_MAX - 2 * SG_ROWS &&
+    if (fast && esz == 2 && bs == 32 && (col || !groups) && !grad && A->rows <= INT32_MAX - 2 * SG_ROWS &&
         A->cols <= INT32_MAX - 2 * SG_COLS) {
         StagedMaps maps;
         if (make_staged_maps(&maps, k, &k.ts_flags)) {
@@ -1508,7 +1509,7 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
             if (s_bound * n_ct >= (int64_t)INT32_MAX)
                 return MXFP4_EUNSUPPORTED;
             k.n_ct = (uint32_t)n_ct;
-            return launch_staged(row, groups, maps, k, s_bound * n_ct, plan_smem, s);
+            return launch_staged(row, col, groups, maps, k, s_bound * n_ct, plan_smem, s);
         }
     }
     if (fast) {

@@ -392,7 +392,9 @@ __device__ __forceinline__ void col_sat_store(uint32_t* mwords, uint32_t bits, i
     }
 }
 
-template <bool ROW, bool GROUPS, int MODE>
+// ROW / COL: the directions computed (at least one); GROUPS: column-wise
+// blocks restart at group_list boundaries; MODE: the scale rule.
+template <bool ROW, bool COL, bool GROUPS, int MODE>
 __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_constant__ StagedMaps maps, const KArgs a)
 {
     extern __shared__ __align__(1024) uint8_t s_dyn[];
@@ -433,8 +435,9 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
     const uint32_t lutb = smem_addr(sm.lut) - 0x2C000000u;
     const uint32_t lutb16 = lutb + 0x04000000u;
     // outputs present, as SG_TS_* bits; those TMA cannot address are copied
-    const uint32_t col_out = (a.y_col ? SG_TS_Y : 0u) | (a.codes_col ? SG_TS_CODES : 0u) |
-                             (a.mask_col ? SG_TS_MASK : 0u);
+    const uint32_t col_out = COL ? (a.y_col ? SG_TS_Y : 0u) | (a.codes_col ? SG_TS_CODES : 0u) |
+                                       (a.mask_col ? SG_TS_MASK : 0u)
+                                 : 0u;
     const uint32_t row_out = (ROW && a.y_row ? SG_TS_YR : 0u) | (ROW && a.codes_row ? SG_TS_CODES_R : 0u) |
                              (ROW && a.mask_row ? SG_TS_MASK_R : 0u);
 
@@ -507,6 +510,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             const bool rows_full = nrows == SG_ROWS;
 
             // ---- column pass, part 1: amax and parameters of the column pair
+            if constexpr (COL) {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
                 cw[i] = sm_ld32(tile, yo[i & 3] + (i >> 2) * 1024);
@@ -541,6 +545,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                         (uint16_t)e8p;
                 }
             }
+            }  // COL
         }
         // The staging buffers are free once the previous tile's stores have
         // read them: the storer waits for that and signals; no CTA barrier.
@@ -555,7 +560,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
 
         // ---- column pass, part 2: y and codes of the column pair
         uint32_t gsat = 0;  // saturation bits of a general-path column pair (bits 2i, 2i+1: word i)
-        if (go) {
+        if (COL && go) {
             uint32_t* yq[4];
             uint8_t* cq[4];
 #pragma unroll
@@ -610,7 +615,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                 rw16[4 * jj + 2] = c.z;
                 rw16[4 * jj + 3] = c.w;
             }
-            if (a.mask_col) {
+            if (COL && a.mask_col) {
                 // rows past a group tail are not copied out; their word is don't-care
                 uint32_t cm = 0;
 #pragma unroll
@@ -675,7 +680,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             }
         }
         // column pairs of the general path add their exact saturation bits
-        if (go && __any_sync(FULL, gsat != 0u))
+        if (COL && go && __any_sync(FULL, gsat != 0u))
             col_sat_store(out.mcol, gsat, h, p, warp);
         fence_async_smem();  // staged outputs -> visible to the TMA stores
         __syncthreads();     // stage s consumed; staged outputs complete; errors visible
