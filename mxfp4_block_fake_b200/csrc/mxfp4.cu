@@ -1582,6 +1582,42 @@ mxfp4_status mxfp4_ste_bwd(const mxfp4_qdq_args* geom, const void* grad_out, voi
     const int esz = geom->dtype == MXFP4_BF16 ? 2 : 4;
     if (!grad_out || !grad_in || ld_grad < geom->cols || !aligned(grad_out, esz) || !aligned(grad_in, esz))
         return MXFP4_EINVAL;
+    if (clip_grad && !saved_mask && geom->dirs == MXFP4_ROWWISE && esz == 2 && geom->block == 32 &&
+        geom->cols % 32 == 0 && geom->x && geom->ld >= geom->cols && geom->ld % 16 == 0 && ld_grad % 16 == 0 &&
+        ((uintptr_t)geom->x | (uintptr_t)grad_out | (uintptr_t)grad_in) % 32 == 0 &&
+        geom->rows * (geom->cols / 32) < (int64_t)UINT32_MAX &&
+        (geom->scale_mode == MXFP4_SCALE_FLOOR ||
+         (geom->scale_mode == MXFP4_SCALE_PAGE && page_fast_ok(geom->scale_factor)))) {
+        // saved-free, row-wise, bf16 block 32: one streaming pass over x and grad_out
+        KArgs k;
+        memset(&k, 0, sizeof(k));
+        k.x = geom->x;
+        k.rows = geom->rows;
+        k.cols = geom->cols;
+        k.ld = geom->ld;
+        k.sf = geom->scale_factor;
+        k.mode = geom->scale_mode;
+        k.g_out = grad_out;
+        k.g_in = grad_in;
+        k.ld_g = ld_grad;
+        if (k.mode == MXFP4_SCALE_PAGE)
+            k.thr = page_threshold(geom->scale_factor);
+        const void* fn = k.mode == MXFP4_SCALE_FLOOR ? (const void*)ste_row_kernel<MXFP4_SCALE_FLOOR>
+                                                      : (const void*)ste_row_kernel<MXFP4_SCALE_PAGE>;
+        const int sms = device_sms();
+        const int occ = occupancy(fn, 0);
+        if (sms <= 0 || occ <= 0)
+            return MXFP4_ECUDA;
+        const int64_t blocks = geom->rows * (geom->cols / 32);
+        int64_t grid = (int64_t)sms * occ;
+        if ((blocks + NTHREADS - 1) / NTHREADS < grid)
+            grid = (blocks + NTHREADS - 1) / NTHREADS;
+        if (k.mode == MXFP4_SCALE_FLOOR)
+            ste_row_kernel<MXFP4_SCALE_FLOOR><<<(unsigned)grid, NTHREADS, 0, s>>>(k);
+        else
+            ste_row_kernel<MXFP4_SCALE_PAGE><<<(unsigned)grid, NTHREADS, 0, s>>>(k);
+        return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
+    }
     if (clip_grad && !saved_mask) {
         // saved-free: recompute the saturation of x in the same pass
         mxfp4_qdq_args g = *geom;

@@ -740,4 +740,81 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         bulk_wait_all();
 }
 
+// ---------------------------------------------------------------------------
+// Saved-free clipped STE backward, row-wise, bf16, block 32: grad_in =
+// grad_out with +0.0 where |x| exceeds its block's limit, the mask recomputed
+// from x in the same pass. One thread per block: two 32-byte loads of x and of
+// grad_out (one sector each, every sector used), the block amax and exponent,
+// a packed compare per word turned into a keep mask by a sign-replicating
+// byte permute, two 32-byte stores. Blocks off the fast range take the
+// general element path for their saturation bits. Requires cols % 32 == 0,
+// 32-byte aligned pointers and leading dimensions that are multiples of 16.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void ld_nc_v8(const void* p, uint32_t* v)
+{
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+                 : "l"(p));
+}
+
+__device__ __forceinline__ void st_cs_v8(void* p, const uint32_t* v)
+{
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(NTHREADS) ste_row_kernel(const KArgs a)
+{
+    const uint32_t nb = (uint32_t)(a.cols / 32);
+    const uint32_t total = (uint32_t)a.rows * nb;
+    __shared__ uint32_t s_lut[64];
+    if (threadIdx.x < 64)
+        s_lut[threadIdx.x] = lut_entry(threadIdx.x);
+    __syncthreads();
+    const uint32_t glutb = smem_addr(s_lut) - 0x2C000000u;
+    for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < total; u += gridDim.x * blockDim.x) {
+        const uint32_t row = u / nb, blk = u - row * nb;
+        const char* xp = static_cast<const char*>(a.x) + ((int64_t)row * a.ld + 32 * blk) * 2;
+        uint32_t w[16];
+        ld_nc_v8(xp, w);
+        ld_nc_v8(xp + 32, w + 8);
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            m2 = vmax2(m2, w[i] & 0x7FFF7FFFu);
+        const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
+        const uint32_t A = am << 16;
+        const int k = block_kt<MODE>(A, a.thr);
+        uint32_t keep[16];
+        if (k_fast_bf(k)) {
+            const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)  // bit 15 / 31 of lx - |x| set: that half does not saturate
+                keep[i] = prmt(lx - (w[i] & 0x7FFF7FFFu), 0u, 0xBB99u);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const ChunkOut gch = general_chunk<8, false>(
+                    make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]), &A, a.mode, a.thr, glutb);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    keep[4 * c + j] = ((gch.sats >> (2 * j)) & 1u ? 0u : 0xFFFFu) |
+                                      ((gch.sats >> (2 * j + 1)) & 1u ? 0u : 0xFFFF0000u);
+            }
+        }
+        const int64_t goff = ((int64_t)row * a.ld_g + 32 * blk) * 2;
+        uint32_t g[16];
+        ld_nc_v8(static_cast<const char*>(a.g_out) + goff, g);
+        ld_nc_v8(static_cast<const char*>(a.g_out) + goff + 32, g + 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            g[i] &= keep[i];
+        st_cs_v8(static_cast<char*>(a.g_in) + goff, g);
+        st_cs_v8(static_cast<char*>(a.g_in) + goff + 32, g + 8);
+    }
+}
+
 }  // namespace mxfp4

@@ -233,6 +233,20 @@ def test_ste_backward(dtype, direction, shape):
     assert np.array_equal(np_bits(gi), np_bits(g))
 
 
+@pytest.mark.parametrize("mode,sf", [("page", 6.0), ("page", 1.0), ("floor", 6.0)])
+@pytest.mark.parametrize("shape", [(96, 2048), (33, 4096)])
+def test_ste_recompute_rowwise_streaming(mode, sf, shape):
+    """Saved-free row-wise STE on the streaming path (bf16, block 32, cols % 32
+    == 0): special values, both scale rules, several scale factors."""
+    x = W.mixed(*shape, dtype=torch.bfloat16, seed=21)
+    g = W.mixed(*shape, dtype=torch.bfloat16, seed=22, specials=False)
+    ora = O.qdq_rowwise(oracle_in(x), 32, sf, O.SCALE_PAGE if mode == "page" else O.SCALE_FLOOR)
+    exp = ora_bits(O.ste_bwd(oracle_in(g), ora["mask"], True))
+    gi = ops.mxfp4_ste_bwd(g.cuda(), x=x.cuda(), clip_grad=True, direction="rowwise", scale_factor=sf,
+                           scale_mode=mode)
+    assert np.array_equal(np_bits(gi), exp)
+
+
 def test_invalid_group_list_writes_nothing_and_reports():
     x = W.mixed(100, 128, seed=13).cuda()
     for gl, t in (([50, 40, 60], 0), ([50, 60, 90], 0), ([50, -10, 60], 1), ([-1, 100], 0)):
