@@ -70,7 +70,8 @@ struct __align__(1024) StagedSmem {
     int4 info[SG_STAGES];                     // row0, nrows, col0, row block of each stage's tile
     uint32_t lut[64];
     unsigned long long full[SG_STAGES];       // mbarriers: stage loaded (TMA transaction count)
-    unsigned long long sfree;                 // mbarrier: the previous tile's stores have read the staging
+    unsigned long long sfree_c;               // mbarrier: the previous tile's column-wise stores have read their staging
+    unsigned long long sfree_r;               // mbarrier: the same for the row-wise stores
     int err;
 };
 
@@ -158,6 +159,7 @@ __device__ __forceinline__ void tma_store_box(const CUtensorMap* map, uint32_t s
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_but1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -414,7 +416,8 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         sm.err = 0;
         for (int s = 0; s < SG_STAGES; ++s)
             mbar_init(smem_addr(&sm.full[s]), 1);
-        mbar_init(smem_addr(&sm.sfree), 1);
+        mbar_init(smem_addr(&sm.sfree_c), 1);
+        mbar_init(smem_addr(&sm.sfree_r), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     uint32_t S;
@@ -549,18 +552,18 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         }
         // The staging buffers are free once the previous tile's stores have
         // read them: the storer waits for that and signals; no CTA barrier.
+        // The column-wise stores go first (their own bulk group), so the
+        // row-wise ones have the column pass's time to finish reading.
         if (tid == SG_STORER && j > 0) {
-            bulk_wait_read_all();
-            mbar_arrive(smem_addr(&sm.sfree));
+            bulk_wait_read_but1();
+            mbar_arrive(smem_addr(&sm.sfree_c));
         }
-        const bool go = ok && (j == 0 || __all_sync(FULL, mbar_wait(smem_addr(&sm.sfree), (j - 1) & 1u)));
-        if (!go)
-            sm.err = 1;
+        const bool go_c = ok && (j == 0 || __all_sync(FULL, mbar_wait(smem_addr(&sm.sfree_c), (j - 1) & 1u)));
         __syncwarp();  // limw of this warp
 
         // ---- column pass, part 2: y and codes of the column pair
         uint32_t gsat = 0;  // saturation bits of a general-path column pair (bits 2i, 2i+1: word i)
-        if (COL && go) {
+        if (COL && go_c) {
             uint32_t* yq[4];
             uint8_t* cq[4];
 #pragma unroll
@@ -601,6 +604,14 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                 }
             }
         }
+
+        if (tid == SG_STORER && j > 0) {
+            bulk_wait_read_all();
+            mbar_arrive(smem_addr(&sm.sfree_r));
+        }
+        const bool go = go_c && (j == 0 || __all_sync(FULL, mbar_wait(smem_addr(&sm.sfree_r), (j - 1) & 1u)));
+        if (!go)
+            sm.err = 1;
 
         // ---- row pass: the lane's row-wise block (tile row rr, columns
         // 32w..32w+31): row-wise outputs, and the column-wise saturation word
@@ -700,21 +711,23 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             const uint32_t st = tma & a.ts_flags;
             const uint32_t ybase_c = smem_addr(out.ycol), ybase_r = smem_addr(out.yrow);
 #pragma unroll
-            for (int sl = 0; sl < 4; ++sl) {
+            for (int sl = 0; sl < 4; ++sl)
                 if ((st & SG_TS_Y) && col0 + sl * SG_SLAB_COLS < a.cols)
                     tma_store_box(&maps.y, ybase_c + sl * SG_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
-                if ((st & SG_TS_YR) && col0 + sl * SG_SLAB_COLS < a.cols)
-                    tma_store_box(&maps.yr, ybase_r + sl * SG_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
-            }
             if (st & SG_TS_CODES)
                 tma_store_box(&maps.codes, smem_addr(out.ccol), col0 / 2, row0);
-            if (st & SG_TS_CODES_R)
-                tma_store_box(&maps.codes_r, smem_addr(out.crow), col0 / 2, row0);
             if (st & SG_TS_MASK)
                 tma_store_box(&maps.mask, smem_addr(out.mcol), col0 / 8, row0);
+            bulk_commit();  // column-wise group
+#pragma unroll
+            for (int sl = 0; sl < 4; ++sl)
+                if ((st & SG_TS_YR) && col0 + sl * SG_SLAB_COLS < a.cols)
+                    tma_store_box(&maps.yr, ybase_r + sl * SG_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
+            if (st & SG_TS_CODES_R)
+                tma_store_box(&maps.codes_r, smem_addr(out.crow), col0 / 2, row0);
             if (st & SG_TS_MASK_R)
                 tma_store_box(&maps.mask_r, smem_addr(out.mrow), col0 / 8, row0);
-            bulk_commit();
+            bulk_commit();  // row-wise group
         }
         if (ROW && a.scales_row && warp == SG_STORER / 32)
             copy_row_scales(a, out, row0, nrows, col0, lane);
