@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--groups", type=int, default=256)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-modes", action="store_true",
+                   help="skip the extra single-GPU timings of the row-wise and training-step modes")
     return p.parse_args()
 
 
@@ -308,8 +310,65 @@ def run_ours(a, rank: int, world: int):
         barrier()
         e2e = (reduce_max([s0.elapsed_time(s1)], world, "cuda")[0], h2d, d2h)
 
-    return dict(ms=ms, fwd_ms=fwd_ms, s_col=s_col, clocks=sampler.summary(), e2e=e2e,
+    modes = None
+    if world == 1 and not a.no_modes:
+        modes = time_modes(a, xd, gd, res, gi, stream)
+
+    return dict(ms=ms, fwd_ms=fwd_ms, s_col=s_col, clocks=sampler.summary(), e2e=e2e, modes=modes,
                 x_h=x_h, g_h=g_h, offsets=offsets, np=np)
+
+
+def time_modes(a, xd, gd, res, gi, stream, steps: int = 20):
+    """Other modes of the hot path on the same tensors (device-resident, CUDA
+    events): row-wise fwd with all outputs + STE from the saved mask, and the
+    training step of the pages' recipe (row-wise fwd, saved-free STE)."""
+    import torch
+
+    from mxfp4_block_fake_b200 import _abi, ops
+
+    n = a.rows * a.cols
+    sp = stream.cuda_stream
+    rargs = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode=a.scale_mode, dirs=_abi.ROWWISE)
+    rargs.y_row, rargs.codes_row = res.y_row.data_ptr(), res.codes_row.data_ptr()
+    rargs.scales_row, rargs.mask_row = res.scales_row.data_ptr(), res.mask_row.data_ptr()
+    rargs.ld_y = a.cols
+    vargs = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode=a.scale_mode, dirs=_abi.ROWWISE)
+    vargs.y_row, vargs.ld_y = res.y_row.data_ptr(), a.cols
+    bargs = ops.make_args(gd, block=32, scale_factor=6.0, scale_mode=a.scale_mode, dirs=_abi.ROWWISE)
+    bargs.x = None
+    rargs_x = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode=a.scale_mode, dirs=_abi.ROWWISE)
+    g_ptr, gi_ptr, m_ptr = gd.data_ptr(), gi.data_ptr(), res.mask_row.data_ptr()
+
+    def call(st, name):
+        if st:
+            _abi.check(st, name)
+
+    def row_step():
+        call(_abi.mxfp4_qdq_fwd(rargs, sp), "mxfp4_qdq_fwd")
+        call(_abi.mxfp4_ste_bwd(bargs, g_ptr, gi_ptr, a.cols, m_ptr, 1, sp), "mxfp4_ste_bwd")
+
+    def train_step():
+        call(_abi.mxfp4_qdq_fwd(vargs, sp), "mxfp4_qdq_fwd")
+        call(_abi.mxfp4_ste_bwd(rargs_x, g_ptr, gi_ptr, a.cols, None, 1, sp), "mxfp4_ste_bwd")
+
+    peak, _ = measured_peaks()
+    out = {}
+    for name, fn, bpe in (("rowwise_fwd_all_outputs_ste_mask", row_step, 4 + 0.5 + 1 / 32 + 0.125 + 4.125),
+                          ("training_step_rowwise_fwd_ste_recompute", train_step, 4 + 6)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        gbs = n * bpe / (ms / 1e3) / 1e9
+        out[name] = {"ms_per_step": round(ms, 4), "bytes_per_element": round(bpe, 4), "GB/s": round(gbs, 1),
+                     "frac_of_measured_peak": round(gbs / peak, 4)}
+    return out
 
 
 def cpu_baseline(a, x_h, g_h, offsets, rows: int):
@@ -379,6 +438,8 @@ def main():
                 "gpu_launches": 2 * a.steps,
                 "clocks": r["clocks"],
             }
+            if r["modes"] is not None:
+                line["modes"] = r["modes"]
             if r["e2e"] is not None:
                 ms_e, h2d, d2h = r["e2e"]
                 line["e2e"] = {"value": round(weak_value(b["step"], a.steps, world, ms_e), 2),
