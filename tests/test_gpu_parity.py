@@ -154,6 +154,42 @@ def test_strided_and_unaligned_inputs(dtype, dirs):
             check_dir(res, ora["col"], "col", x.shape[1], label="strided")
 
 
+@pytest.mark.parametrize("offsets", [(0, 0), (4, 1), (4, 0), (0, 3)])
+@pytest.mark.parametrize("rows,cols,counts", [(96, 512, None), (70, 768, [20, 0, 37, 13]), (64, 256, [64])])
+def test_padded_and_offset_outputs(offsets, rows, cols, counts):
+    """Outputs in padded rows (ld_y > cols) and code/mask buffers starting at
+    byte offsets: tensor-map stores where they can address the output,
+    thread copies where they cannot; both must give the oracle's bytes."""
+    co, mo = offsets
+    x = W.mixed(rows, cols, dtype=torch.bfloat16, seed=31)
+    xd = x.cuda()
+    dev = xd.device
+    u8 = dict(dtype=torch.uint8, device=dev)
+
+    def flat(n, off):
+        return torch.full((n + off,), 0xA5, **u8)[off:]
+
+    ng = 0 if counts is None else len(counts)
+    r = ops.QDQResult()
+    r.y_row = torch.empty((rows, cols + 8), dtype=torch.bfloat16, device=dev)[:, :cols]
+    r.y_col = torch.empty((rows, cols + 8), dtype=torch.bfloat16, device=dev)[:, :cols]
+    r.codes_row = flat(rows * cols // 2, co).view(rows, cols // 2)
+    r.codes_col = flat(rows * cols // 2, co).view(rows, cols // 2)
+    r.mask_row = flat(rows * cols // 8, mo).view(rows, cols // 8)
+    r.mask_col = flat(rows * cols // 8, mo).view(rows, cols // 8)
+    r.scales_row = torch.empty((rows, cols // 32), **u8)
+    r.scales_col = torch.empty((ops.colwise_scale_rows_bound(rows, ng, 32), cols), **u8)
+    r.status = torch.empty((1,), dtype=torch.int32, device=dev)
+    gl = None if counts is None else torch.tensor(counts, dtype=torch.int64, device=dev)
+    ops.mxfp4_qdq_fwd(xd, rowwise=True, colwise=True, group_list=gl, group_list_type=1, emit_codes=True,
+                      emit_mask=True, out=r, check=True)
+    torch.cuda.synchronize()
+    xo = oracle_in(x)
+    ends = None if counts is None else np.cumsum(np.asarray(counts, np.int64))
+    check_dir(r, O.qdq_rowwise(xo, 32, 6.0, O.SCALE_PAGE), "row", cols, label="padded/offset")
+    check_dir(r, O.qdq_colwise(xo, 32, 6.0, O.SCALE_PAGE, ends=ends), "col", cols, label="padded/offset")
+
+
 @pytest.mark.parametrize("sf", [1.0, 4.0, 7.5, 0.75, 3.0e-38, 1.0e30])
 def test_scale_factors_page_mode(sf):
     x = W.mixed(64, 512, seed=6)
