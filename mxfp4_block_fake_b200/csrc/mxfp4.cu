@@ -1353,6 +1353,46 @@ static bool make_staged_maps(StagedMaps* m, const KArgs& k, uint32_t* ts_flags)
     return true;
 }
 
+// Maps of the block-128 staged kernel: the same tensors in 64 x 128 boxes
+// (x and y, 128-byte swizzle), codes in 64-byte x 128 boxes with the 64-byte
+// swizzle, masks in 16-byte x 128 boxes.
+static bool make_staged128_maps(StagedMaps* m, const KArgs& k, uint32_t* ts_flags)
+{
+    memset(m, 0, sizeof(*m));
+    *ts_flags = 0;
+    if (!encode_2d(&m->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(k.x), (uint64_t)k.cols,
+                   (uint64_t)k.rows, (uint64_t)k.ld * 2, SG_SLAB_COLS, SB_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        return false;
+    if (k.cols < SB_COLS || k.rows < SB_ROWS)
+        return true;
+    const bool ypitch = (k.ld_y * 2) % 16 == 0, cpitch = (k.cols / 2) % 16 == 0, mpitch = (k.cols / 8) % 16 == 0;
+    if (k.y_col && aligned(k.y_col, 16) && ypitch &&
+        encode_2d(&m->y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.y_col, (uint64_t)k.cols, (uint64_t)k.rows,
+                  (uint64_t)k.ld_y * 2, SG_SLAB_COLS, SB_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        *ts_flags |= SG_TS_Y;
+    if (k.y_row && aligned(k.y_row, 16) && ypitch &&
+        encode_2d(&m->yr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.y_row, (uint64_t)k.cols, (uint64_t)k.rows,
+                  (uint64_t)k.ld_y * 2, SG_SLAB_COLS, SB_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        *ts_flags |= SG_TS_YR;
+    if (k.codes_col && aligned(k.codes_col, 16) && cpitch &&
+        encode_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.codes_col, (uint64_t)k.cols / 2, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 2, SB_COLS / 2, SB_ROWS, CU_TENSOR_MAP_SWIZZLE_64B))
+        *ts_flags |= SG_TS_CODES;
+    if (k.codes_row && aligned(k.codes_row, 16) && cpitch &&
+        encode_2d(&m->codes_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.codes_row, (uint64_t)k.cols / 2, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 2, SB_COLS / 2, SB_ROWS, CU_TENSOR_MAP_SWIZZLE_64B))
+        *ts_flags |= SG_TS_CODES_R;
+    if (k.mask_col && aligned(k.mask_col, 16) && mpitch &&
+        encode_2d(&m->mask, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.mask_col, (uint64_t)k.cols / 8, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 8, SB_COLS / 8, SB_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+        *ts_flags |= SG_TS_MASK;
+    if (k.mask_row && aligned(k.mask_row, 16) && mpitch &&
+        encode_2d(&m->mask_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.mask_row, (uint64_t)k.cols / 8, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 8, SB_COLS / 8, SB_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+        *ts_flags |= SG_TS_MASK_R;
+    return true;
+}
+
 typedef void (*StagedFn)(const StagedMaps, const KArgs);
 
 template <bool ROW, bool COL, bool GROUPS>
@@ -1360,6 +1400,33 @@ static StagedFn pick_staged(int mode)
 {
     return mode == MXFP4_SCALE_FLOOR ? qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_FLOOR>
                                      : qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_PAGE>;
+}
+
+template <bool ROW, bool COL, bool GROUPS>
+static StagedFn pick_staged128(int mode)
+{
+    return mode == MXFP4_SCALE_FLOOR ? qdq_staged128_kernel<ROW, COL, GROUPS, MXFP4_SCALE_FLOOR>
+                                     : qdq_staged128_kernel<ROW, COL, GROUPS, MXFP4_SCALE_PAGE>;
+}
+
+static mxfp4_status launch_staged128(bool row, bool col, bool groups, const StagedMaps& maps, const KArgs& k,
+                                     int64_t tiles, size_t plan_smem, cudaStream_t s)
+{
+    StagedFn fn = !col ? pick_staged128<true, false, false>(k.mode)
+                : row  ? (groups ? pick_staged128<true, true, true>(k.mode) : pick_staged128<true, true, false>(k.mode))
+                       : (groups ? pick_staged128<false, true, true>(k.mode) : pick_staged128<false, true, false>(k.mode));
+    const size_t smem = sizeof(Staged128Smem) + 1024 + plan_smem;
+    if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MXFP4_ECUDA;
+    const int sms = device_sms();
+    const int occ = occupancy((const void*)fn, smem, SB_THREADS);
+    if (sms <= 0 || occ <= 0)
+        return MXFP4_ECUDA;
+    int64_t grid = (int64_t)sms * occ;
+    if (tiles < grid)
+        grid = tiles < 1 ? 1 : tiles;
+    fn<<<(unsigned)grid, SB_THREADS, smem, s>>>(maps, k);
+    return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
 }
 
 // row-only tiles never restart at groups (the caller routes row-only calls
@@ -1510,6 +1577,17 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
                 return MXFP4_EUNSUPPORTED;
             k.n_ct = (uint32_t)n_ct;
             return launch_staged(row, col, groups, maps, k, s_bound * n_ct, plan_smem, s);
+        }
+    }
+    if (fast && esz == 2 && bs == 128 && (col || !groups) && !grad && A->rows <= INT32_MAX - 2 * SB_ROWS &&
+        A->cols <= INT32_MAX - 2 * SB_COLS) {
+        StagedMaps maps;
+        if (make_staged128_maps(&maps, k, &k.ts_flags)) {
+            const int64_t n_ct = (A->cols + SB_COLS - 1) / SB_COLS;
+            if (s_bound * n_ct >= (int64_t)INT32_MAX)
+                return MXFP4_EUNSUPPORTED;
+            k.n_ct = (uint32_t)n_ct;
+            return launch_staged128(row, col, groups, maps, k, s_bound * n_ct, plan_smem, s);
         }
     }
     if (fast) {
