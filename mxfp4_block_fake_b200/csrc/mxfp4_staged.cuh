@@ -776,7 +776,7 @@ constexpr int SB_SLAB_BYTES = SG_SLAB_COLS * 2 * SB_ROWS;  // 16384
 constexpr int SB_TILE_BYTES = 2 * SB_SLAB_BYTES;           // 32768
 constexpr int SB_CODE_BYTES = SB_ROWS * SB_COLS / 2;       // 8192: 64-byte rows
 constexpr int SB_MASK_WORDS = SB_ROWS * SB_COLS / 32;      // 512: 16-byte rows
-constexpr int SB_STAGES = 2;
+constexpr int SB_STAGES = 3;
 constexpr int SB_THREADS = 512;
 
 struct __align__(1024) StagedOut128 {
