@@ -395,6 +395,94 @@ def cpu_baseline(a, x_h, g_h, offsets, rows: int):
     return dict(value=b / dt / 1e9, seconds=dt, rows=rows, s_col=s_col)
 
 
+def _oracle_warm(_):
+    """Pool warm-up: import the oracle (loads its C library) in the worker."""
+    import oracle  # noqa: F401
+
+    return os.getpid()
+
+
+def _oracle_chunk(job):
+    """One worker of the all-cores baseline: the oracle on rows [r0, r1) of
+    the batch (whole groups), read from memory-mapped files."""
+    import numpy as np
+
+    import oracle as O
+
+    path_x, path_g, shape, r0, r1, ends, mode = job
+    xs = np.ascontiguousarray(np.memmap(path_x, np.uint16, "r", shape=shape)[r0:r1])
+    gs = np.ascontiguousarray(np.memmap(path_g, np.uint16, "r", shape=shape)[r0:r1])
+    t0 = time.perf_counter()
+    r = O.qdq_rowwise(xs, 32, 6.0, mode)
+    O.qdq_colwise(xs, 32, 6.0, mode, ends=np.asarray(ends, np.int64))
+    O.ste_bwd(gs, r["mask"], True)
+    return time.perf_counter() - t0
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline_all_cores(a, x_h, g_h, offsets, max_procs: int = 64):
+    """The oracle, as it stands, on the whole batch, the groups split into
+    contiguous chunks over one process per host core (spawned; the oracle
+    itself is single-threaded). Wall time of the chunks (each reads its rows
+    from a memory-mapped copy of the batch), pool warm-up excluded."""
+    import multiprocessing as mp
+    import shutil
+    import tempfile
+
+    import numpy as np
+    import torch
+
+    import oracle as O
+
+    procs = max(1, min(os.cpu_count() or 1, max_procs))
+    ends = offsets.numpy().astype(np.int64)
+    rows = a.rows
+    # split at group ends nearest to equal row counts
+    cuts = [0]
+    for k in range(1, procs):
+        target = k * rows // procs
+        e = int(ends[int(np.argmin(np.abs(ends - target)))])
+        if e > cuts[-1]:
+            cuts.append(e)
+    if cuts[-1] != rows:
+        cuts.append(rows)
+    mode = O.SCALE_PAGE if a.scale_mode == "page" else O.SCALE_FLOOR
+    xs = x_h.contiguous().view(torch.int16).numpy().view(np.uint16)
+    gs = g_h.contiguous().view(torch.int16).numpy().view(np.uint16)
+    tmp = tempfile.mkdtemp(prefix="mxfp4_cpu_baseline_")
+    try:
+        path_x, path_g = os.path.join(tmp, "x.u16"), os.path.join(tmp, "g.u16")
+        xs.tofile(path_x)
+        gs.tofile(path_g)
+        jobs = []
+        for r0, r1 in zip(cuts[:-1], cuts[1:]):
+            local = ends[(ends > r0) & (ends <= r1)] - r0
+            if len(local) == 0 or local[-1] != r1 - r0:
+                local = np.append(local, r1 - r0)
+            jobs.append((path_x, path_g, xs.shape, r0, r1, local.tolist(), mode))
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(len(jobs)) as pool:
+            pool.map(_oracle_warm, range(len(jobs)))
+            t0 = time.perf_counter()
+            pool.map(_oracle_chunk, jobs, chunksize=1)
+            wall = time.perf_counter() - t0
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+    s_col = O.colwise_scale_rows(ends, 32)
+    b = step_bytes(rows, a.cols, s_col)["step"]
+    return dict(value=b / wall / 1e9, seconds=wall, cores=len(jobs))
+
+
 def main():
     a = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -451,6 +539,16 @@ def main():
                     "value": round(cb["value"], 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                     "sample": f"first {cb['rows']} of {a.rows} rows x {a.cols} cols of the same batch "
                               f"(groups cut at the sample end), one full step, {cb['seconds']:.1f} s"}
+                try:
+                    cp = cpu_baseline_all_cores(a, r["x_h"], r["g_h"], r["offsets"])
+                    line["cpu_baseline_all_cores"] = {
+                        "value": round(cp["value"], 4), "unit": "GB/s", "cores": cp["cores"], "kind": "oracle",
+                        "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+                        "sample": f"the whole batch ({a.rows} x {a.cols}), one full step, groups split into "
+                                  f"{cp['cores']} contiguous chunks, one spawned process each, "
+                                  f"{cp['seconds']:.1f} s wall"}
+                except Exception as e:  # noqa: BLE001 - a baseline, not the measurement
+                    line["cpu_baseline_all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

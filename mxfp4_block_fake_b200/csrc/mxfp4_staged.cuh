@@ -183,10 +183,6 @@ __device__ __forceinline__ uint4 sm_ld128(const uint8_t* base, uint32_t off)
 {
     return *reinterpret_cast<const uint4*>(base + off);
 }
-__device__ __forceinline__ void sm_st32(uint8_t* base, uint32_t off, uint32_t v)
-{
-    *reinterpret_cast<uint32_t*>(base + off) = v;
-}
 
 __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b)
 {

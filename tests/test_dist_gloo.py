@@ -84,3 +84,21 @@ def test_reference_arm_under_torchrun_prints_once():
     j = json.loads(lines[0])
     assert j["impl"] == "reference" and j["unit"] == "GB/s" and j["value"] > 0
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_all_cores_cpu_baseline_matches_single_process_work():
+    """The all-cores oracle baseline (spawned processes over whole groups)
+    covers every row and group exactly once: the chunk boundaries fall on
+    group ends and the bytes are those of one full step."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from mxfp4_block_fake_b200 import workloads as W
+
+    class A:
+        rows, cols, groups, scale_mode = 1024, 256, 12, "page"
+
+    x_h, _, offsets = W.moe_grouped(A.rows, A.cols, A.groups, seed=4)
+    g_h = W.train_step_grad(A.rows, A.cols, seed=5)
+    r = bench.cpu_baseline_all_cores(A, x_h, g_h, offsets, max_procs=3)
+    assert 1 <= r["cores"] <= 3
+    assert r["value"] > 0 and r["seconds"] > 0
