@@ -270,6 +270,86 @@ __device__ __forceinline__ void prep_bf(uint32_t w, uint32_t& aw, uint32_t& sg)
     sg = w & (aw + 0x7FFF7FFFu) & 0x80008000u;
 }
 
+// ---- E2M1 rounding by the hardware convert ---------------------------------
+// The convert rounds to nearest with ties to even; the codebook's rule sends
+// ties up (away from zero). Multiplying y by (1 + 2^-20) first moves exact
+// midpoints above themselves and nothing else across one: y is a bf16 value
+// times 2^-k (8 significant bits), so a y below a midpoint lies at least one
+// bf16 ulp (2^-8 relative) below it, and the one rounding of the product
+// changes it by at most 2^-24 relative. The product is formed as
+// x * (2^-k (1 + 2^-20)) + 0 in one fma: adding +0 turns -0 into +0 (the
+// codebook's sign rule for zero inputs) and keeps the sign of every nonzero
+// product, however small. Codes above 6 saturate to 6 in the convert, as in
+// the codebook. Checked against the table path for every finite bf16 value
+// and every fast-path k.
+
+// 2^-k (1 + 2^-20) for a fast-path k (mantissa bit 3 set).
+__device__ __forceinline__ float inv_nudged(int k) { return __uint_as_float((0x3F800000u - ((uint32_t)k << 23)) | 8u); }
+
+// 2^k for a fast-path k.
+__device__ __forceinline__ float pow2f_k(int k) { return __uint_as_float(0x3F800000u + ((uint32_t)k << 23)); }
+
+// Nudged scaled values of both halves of a bf16 word.
+__device__ __forceinline__ void nudged_pair(uint32_t w, float invn_lo, float invn_hi, float& ylo, float& yhi)
+{
+    asm("fma.rn.f32 %0, %1, %2, 0f00000000;" : "=f"(ylo) : "f"(__uint_as_float(w << 16)), "f"(invn_lo));
+    asm("fma.rn.f32 %0, %1, %2, 0f00000000;" : "=f"(yhi) : "f"(__uint_as_float(w & 0xFFFF0000u)), "f"(invn_hi));
+}
+
+// code * 2^k of both halves from the f16x2 codes, as packed bf16 (exact).
+__device__ __forceinline__ uint32_t dequant_pair(uint32_t h, float sc_lo, float sc_hi)
+{
+    float clo, chi;
+    asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+        : "=f"(clo), "=f"(chi)
+        : "r"(h));
+    return __byte_perm(__float_as_uint(clo * sc_lo), __float_as_uint(chi * sc_hi), 0x7632);
+}
+
+// One word: its E2M1 byte (low element in the low nibble) and its
+// dequantised packed bf16 pair.
+__device__ __forceinline__ uint32_t qword_cvt(uint32_t w, float invn_lo, float invn_hi, float sc_lo, float sc_hi,
+                                              uint32_t& byte)
+{
+    float ylo, yhi;
+    nudged_pair(w, invn_lo, invn_hi, ylo, yhi);
+    uint32_t h;
+    asm("{\n\t.reg .b8 q;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q, %2, %3;\n\t"
+        "cvt.u32.u8 %0, q;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, q;\n\t}"
+        : "=r"(byte), "=r"(h)
+        : "f"(yhi), "f"(ylo));
+    return dequant_pair(h, sc_lo, sc_hi);
+}
+
+// Four words with one scale: the 32-bit E2M1 nibble word and four
+// dequantised packed bf16 pairs.
+__device__ __forceinline__ uint32_t qword4_cvt(const uint32_t* w, float invn, float sc, uint32_t* o)
+{
+    float y[8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        nudged_pair(w[u], invn, invn, y[2 * u], y[2 * u + 1]);
+    uint32_t nibs, h[4];
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %8, %7;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %10, %9;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %12, %11;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, q0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, q1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, q2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %4, q3;\n\t}"
+        : "=r"(nibs), "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        o[u] = dequant_pair(h[u], sc, sc);
+    return nibs;
+}
+
 // Tile sequence of one CTA: row block rb and column tile ct, advanced in
 // order; g tracks the group that holds rb (largest g with s_bpre[g] <= rb,
 // which skips empty groups). Tiles are TR rows (one column-wise block) by TC
@@ -985,15 +1065,14 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
 
         if constexpr (COL) {
             auto col_fast = [&]() {
-                const float inv_lo = __uint_as_float(0x3F800000u - ((uint32_t)k_lo << 23));
-                const float inv_hi = __uint_as_float(0x3F800000u - ((uint32_t)k_hi << 23));
-                const uint32_t s2 = bf16_pow2(k_lo) | (bf16_pow2(k_hi) << 16);
+                const float invn_lo = inv_nudged(k_lo), invn_hi = inv_nudged(k_hi);
+                const float sc_lo = pow2f_k(k_lo), sc_hi = pow2f_k(k_hi);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    uint32_t aw, sg, P;
-                    prep_bf(cw[i], aw, sg);
-                    *reinterpret_cast<uint32_t*>(out.ycol + yo + i * 1024) = qword(aw, sg, inv_lo, inv_hi, s2, lutb16, P);
-                    out.ccol[co + i * 512] = (uint8_t)e2m1_byte(P);
+                    uint32_t byte;
+                    *reinterpret_cast<uint32_t*>(out.ycol + yo + i * 1024) =
+                        qword_cvt(cw[i], invn_lo, invn_hi, sc_lo, sc_hi, byte);
+                    out.ccol[co + i * 512] = (uint8_t)byte;
                 }
             };
             if (__all_sync(FULL, fast)) {
@@ -1054,21 +1133,16 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
                 const bool rfast = k_fast_bf(k);
                 uint32_t nib[4], sats = 0;
                 auto row_fast = [&]() {
-                    const float inv = __uint_as_float(0x3F800000u - ((uint32_t)k << 23));
-                    const uint32_t s2 = bf16_pow2(k) * 0x10001u;
+                    const float invn = inv_nudged(k), sc = pow2f_k(k);
                     const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
                     const uint32_t limx[4] = {lx, lx, lx, lx};
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
-                        uint32_t P[4], o[4], a4w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            uint32_t sg;
-                            prep_bf(rw16[4 * jj + u], a4w[u], sg);
-                            o[u] = qword(a4w[u], sg, inv, inv, s2, lutb16, P[u]);
-                        }
+                        uint32_t o[4];
+                        nib[jj] = qword4_cvt(rw16 + 4 * jj, invn, sc, o);
                         *reinterpret_cast<uint4*>(out.yrow + ro[jj]) = make_uint4(o[0], o[1], o[2], o[3]);
-                        nib[jj] = e2m1_word(P);
+                        const uint32_t a4w[4] = {rw16[4 * jj] & 0x7FFF7FFFu, rw16[4 * jj + 1] & 0x7FFF7FFFu,
+                                                 rw16[4 * jj + 2] & 0x7FFF7FFFu, rw16[4 * jj + 3] & 0x7FFF7FFFu};
                         sats |= sat8(a4w, limx) << (8 * jj);
                     }
                 };
