@@ -222,6 +222,36 @@ def test_every_bf16_value_as_element_and_as_block_max(mode):
     check_dir(res, ora["row"], "row", 32, label="bf16 sweep")
 
 
+@pytest.mark.parametrize("mode", ["page", "floor"])
+def test_every_bf16_value_block128_both_directions(mode):
+    """Every finite bf16 value, in the low and the high half of a 32-bit word
+    and with both signs, as element under fixed block maxima and as block
+    maximum, through the dual kernel with blocks of 128: once with the
+    sweep laid along rows, once along columns (the transpose)."""
+    allv = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    rows = []
+    for shift in (0, 2):
+        blk = np.zeros((65536, 128), np.uint16)
+        blk[:, 0] = allv
+        blk[:, 33] = np.where((allv & 0x7F80) >= (shift << 7), allv - (shift << 7), allv)
+        blk[:, 98] = allv ^ 0x8000
+        blk[:, 5] = 0x3F80
+        rows.append(blk)
+    for mx in (0x40C0, 0x4090, 0x3F80, 0x40F8, 0x0010, 0x7F7F):
+        blk = np.zeros((65536, 128), np.uint16)
+        blk[:, 127] = mx
+        blk[:, 7] = allv
+        blk[:, 64] = allv ^ 0x8000
+        rows.append(blk)
+    xb = np.concatenate(rows)
+    for arr in (xb, np.ascontiguousarray(xb.T)):
+        x = torch.from_numpy(arr.view(np.int16).copy()).view(torch.bfloat16)
+        res, ora = run_both(x, block=128, mode=mode, rowwise=True, colwise=True)
+        check_dir(res, ora["row"], "row", arr.shape[1], label="bf16 sweep b128")
+        check_dir(res, ora["col"], "col", arr.shape[1], label="bf16 sweep b128")
+        del res, ora, x
+
+
 def test_fp32_random_patterns():
     rng = np.random.default_rng(7)
     bits = rng.integers(0, 2 ** 32, (4096, 256), dtype=np.uint64).astype(np.uint32)
