@@ -320,8 +320,10 @@ def run_ours(a, rank: int, world: int):
 
 def time_modes(a, xd, gd, res, gi, stream, steps: int = 20):
     """Other modes of the hot path on the same tensors (device-resident, CUDA
-    events): row-wise fwd with all outputs + STE from the saved mask, and the
-    training step of the pages' recipe (row-wise fwd, saved-free STE)."""
+    events): row-wise fwd with all outputs + STE from the saved mask, the
+    training step of the pages' recipe (row-wise fwd, saved-free STE), and the
+    real-quantisation producer (row-wise E2M1 codes + E8M0 scales in the
+    block-scaled MMA layout, no dequantised values)."""
     import torch
 
     from mxfp4_block_fake_b200 import _abi, ops
@@ -338,6 +340,11 @@ def time_modes(a, xd, gd, res, gi, stream, steps: int = 20):
     bargs.x = None
     rargs_x = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode=a.scale_mode, dirs=_abi.ROWWISE)
     g_ptr, gi_ptr, m_ptr = gd.data_ptr(), gi.data_ptr(), res.mask_row.data_ptr()
+    mma_scales = torch.zeros((ops.scales_row_bytes(a.rows, a.cols, 32, "mma"),), dtype=torch.uint8,
+                             device=xd.device)
+    margs = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode=a.scale_mode, dirs=_abi.ROWWISE)
+    margs.codes_row, margs.scales_row = res.codes_row.data_ptr(), mma_scales.data_ptr()
+    margs.scales_row_layout, margs.ld_y = _abi.SCALES_MMA, a.cols
 
     def call(st, name):
         if st:
@@ -351,10 +358,14 @@ def time_modes(a, xd, gd, res, gi, stream, steps: int = 20):
         call(_abi.mxfp4_qdq_fwd(vargs, sp), "mxfp4_qdq_fwd")
         call(_abi.mxfp4_ste_bwd(rargs_x, g_ptr, gi_ptr, a.cols, None, 1, sp), "mxfp4_ste_bwd")
 
+    def mma_operand():
+        call(_abi.mxfp4_qdq_fwd(margs, sp), "mxfp4_qdq_fwd")
+
     peak, _ = measured_peaks()
     out = {}
     for name, fn, bpe in (("rowwise_fwd_all_outputs_ste_mask", row_step, 4 + 0.5 + 1 / 32 + 0.125 + 4.125),
-                          ("training_step_rowwise_fwd_ste_recompute", train_step, 4 + 6)):
+                          ("training_step_rowwise_fwd_ste_recompute", train_step, 4 + 6),
+                          ("mxfp4_mma_operand_rowwise_codes_scales", mma_operand, 2 + 0.5 + 1 / 32)):
         for _ in range(3):
             fn()
         torch.cuda.synchronize()

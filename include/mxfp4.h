@@ -36,7 +36,20 @@
  *                               nibble of element c is the low nibble of byte
  *                               c/2 when c is even, the high one when odd;
  *                               nibble = sign << 3 | code index (E2M1 bits).
- *   scales_row                  [rows][ceil(cols/block)] E8M0 bytes (k + 127).
+ *   scales_row                  [rows][ceil(cols/block)] E8M0 bytes (k + 127),
+ *                               row-major, or (scales_row_layout =
+ *                               MXFP4_SCALES_MMA) in the scale-factor layout
+ *                               that block-scaled tensor-core GEMMs read
+ *                               (cuBLAS documentation, "1D block scaling
+ *                               factors layout"): the [rows][nblk] matrix is
+ *                               cut into atoms of 128 rows x 4 block columns,
+ *                               512 bytes each, stored atom row by atom row
+ *                               (atom (i, j) at byte 512 * (i * ceil(nblk/4)
+ *                               + j)); inside an atom, entry (r, c) sits at
+ *                               byte 16 * (r % 32) + 4 * (r / 32) + c. The
+ *                               buffer holds mxfp4_scales_row_bytes() bytes;
+ *                               entries past rows or nblk (the padding of the
+ *                               last atoms) are not written.
  *   scales_col                  [S][cols] E8M0 bytes, S = sum over groups of
  *                               ceil(group rows / block), groups in order.
  *                               mxfp4_colwise_scale_rows() gives S from a host
@@ -95,7 +108,11 @@ typedef enum {
 /* Largest num_groups a call accepts. */
 #define MXFP4_MAX_GROUPS 4096
 
-#define MXFP4_ABI_VERSION 1
+/* Layouts of scales_row (mxfp4_qdq_args.scales_row_layout). */
+#define MXFP4_SCALES_ROWMAJOR 0
+#define MXFP4_SCALES_MMA 1
+
+#define MXFP4_ABI_VERSION 2
 
 /*
  * Arguments of one QDQ call. Zero-initialise and fill what is used; every
@@ -115,6 +132,10 @@ typedef enum {
  *   group_list_type 0 = cumulative end offsets, 1 = counts.
  *   status         optional device int32 that receives the group_list check.
  *   y_row, y_col   dequantised outputs, x's dtype, leading dimension ld_y.
+ *   scales_row_layout MXFP4_SCALES_ROWMAJOR (0) or MXFP4_SCALES_MMA: the
+ *                  latter, with block 32, gives the E8M0 operand scales of an
+ *                  MXFP4 block-scaled GEMM whose K dimension is `cols`
+ *                  (codes_row is then its K-major E2M1 operand as is).
  */
 typedef struct mxfp4_qdq_args {
     const void* x;
@@ -139,6 +160,7 @@ typedef struct mxfp4_qdq_args {
     uint8_t* codes_col;
     uint8_t* scales_col;
     uint8_t* mask_col;
+    int32_t scales_row_layout;
 } mxfp4_qdq_args;
 
 /*
@@ -190,6 +212,11 @@ int64_t mxfp4_colwise_scale_rows(const int64_t* host_group_list, int64_t num_gro
 /* Upper bound on S that needs no group sizes: floor(rows/block) + num_groups
  * (ceil(rows/block) without groups). */
 int64_t mxfp4_colwise_scale_rows_bound(int64_t rows, int64_t num_groups, int32_t block);
+
+/* Bytes of a scales_row buffer for `rows` x `cols` with blocks of `block` in
+ * `layout` (MXFP4_SCALES_ROWMAJOR: rows * ceil(cols/block); MXFP4_SCALES_MMA:
+ * 512 * ceil(rows/128) * ceil(ceil(cols/block)/4)); -1 for invalid arguments. */
+int64_t mxfp4_scales_row_bytes(int64_t rows, int64_t cols, int32_t block, int32_t layout);
 
 /* Static English text of a status; never NULL. */
 const char* mxfp4_status_string(mxfp4_status status);

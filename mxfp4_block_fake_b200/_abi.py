@@ -17,8 +17,9 @@ OK, EINVAL, EUNSUPPORTED, ECUDA = 0, 1, 2, 3
 F32, BF16 = 0, 1
 SCALE_PAGE, SCALE_FLOOR = 0, 1
 ROWWISE, COLWISE = 1, 2
+SCALES_ROWMAJOR, SCALES_MMA = 0, 1
 MAX_GROUPS = 4096
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 # Every symbol include/mxfp4.h declares.
 EXPORTS = (
@@ -27,6 +28,7 @@ EXPORTS = (
     "mxfp4_qdq_fwd_bwd",
     "mxfp4_colwise_scale_rows",
     "mxfp4_colwise_scale_rows_bound",
+    "mxfp4_scales_row_bytes",
     "mxfp4_status_string",
     "mxfp4_abi_version",
 )
@@ -56,6 +58,7 @@ class QdqArgs(ctypes.Structure):
         ("codes_col", ctypes.c_void_p),
         ("scales_col", ctypes.c_void_p),
         ("mask_col", ctypes.c_void_p),
+        ("scales_row_layout", ctypes.c_int32),
     ]
 
 
@@ -96,6 +99,8 @@ def lib() -> ctypes.CDLL:
     L.mxfp4_colwise_scale_rows.restype = i64
     L.mxfp4_colwise_scale_rows_bound.argtypes = [i64, i64, i32]
     L.mxfp4_colwise_scale_rows_bound.restype = i64
+    L.mxfp4_scales_row_bytes.argtypes = [i64, i64, i32, i32]
+    L.mxfp4_scales_row_bytes.restype = i64
     L.mxfp4_status_string.argtypes = [i32]
     L.mxfp4_status_string.restype = ctypes.c_char_p
     L.mxfp4_abi_version.argtypes = []

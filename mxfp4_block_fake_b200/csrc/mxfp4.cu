@@ -67,7 +67,20 @@ struct KArgs {
     uint32_t n_ct;  // column tiles of the tile kernel
     uint32_t thr;   // PAGE mode: fp32 bits of T0 (see qparams)
     uint32_t ts_flags;  // staged kernel: column-wise outputs written by TMA stores (SG_TS_*)
+    int32_t srow_mma;   // scales_row in the MMA scale-factor layout (MXFP4_SCALES_MMA)
 };
+
+// Byte offset of row-wise scale (row, b) of a [rows][nblk] scale matrix:
+// row-major, or the block-scaled MMA layout (atoms of 128 rows x 4 block
+// columns, 512 bytes, atom rows in order; entry (r, c) of an atom at
+// 16 (r mod 32) + 4 floor(r / 32) + c).
+__device__ __forceinline__ int64_t srow_off(const KArgs& a, int64_t row, int64_t b, int64_t nblk)
+{
+    if (!a.srow_mma)
+        return row * nblk + b;
+    const int64_t ncb = (nblk + 3) >> 2;
+    return ((((row >> 7) * ncb + (b >> 2))) << 9) + ((row & 31) << 4) + (((row >> 5) & 3) << 2) + (b & 3);
+}
 
 // ---------------------------------------------------------------------------
 // Per-block parameters
@@ -846,7 +859,7 @@ __global__ void __launch_bounds__(NTHREADS, COL ? 2 : 1) qdq_tile_kernel(const K
                     if (a.mask_row && (VEC == 8 || !(lc & 1)))
                         a.mask_row[row * mstride + col / 8] = (uint8_t)sats;
                     if (a.scales_row && (lc % BL) == 0)
-                        a.scales_row[row * nblk + col / BS] = (uint8_t)e8_of(A, k);
+                        a.scales_row[srow_off(a, row, col / BS, nblk)] = (uint8_t)e8_of(A, k);
                 }
             }
             if constexpr (COL) {
@@ -966,7 +979,7 @@ __global__ void __launch_bounds__(NTHREADS) generic_row_kernel(const KArgs a)
             }
         }
         if (a.scales_row)
-            a.scales_row[row * nblk + b] = (uint8_t)p.e8;
+            a.scales_row[srow_off(a, row, b, nblk)] = (uint8_t)p.e8;
     }
 }
 
@@ -1471,6 +1484,8 @@ static mxfp4_status check_geometry(const mxfp4_qdq_args* a)
         return MXFP4_EUNSUPPORTED;
     if (a->dirs == 0 || (a->dirs & ~(MXFP4_ROWWISE | MXFP4_COLWISE)))
         return MXFP4_EINVAL;
+    if (a->scales_row_layout != MXFP4_SCALES_ROWMAJOR && a->scales_row_layout != MXFP4_SCALES_MMA)
+        return MXFP4_EINVAL;
     if (a->group_list) {
         if (a->num_groups < 1)
             return MXFP4_EINVAL;
@@ -1522,6 +1537,7 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
         k.y_row = A->y_row;
         k.codes_row = A->codes_row;
         k.scales_row = A->scales_row;
+        k.srow_mma = A->scales_row_layout == MXFP4_SCALES_MMA;
         k.mask_row = A->mask_row;
     }
     if (col) {
@@ -1770,6 +1786,18 @@ const char* mxfp4_status_string(mxfp4_status status)
     case MXFP4_ECUDA: return "CUDA error";
     }
     return "unknown status";
+}
+
+int64_t mxfp4_scales_row_bytes(int64_t rows, int64_t cols, int32_t block, int32_t layout)
+{
+    if (rows < 0 || cols < 0 || block <= 0)
+        return -1;
+    const int64_t nblk = (cols + block - 1) / block;
+    if (layout == MXFP4_SCALES_ROWMAJOR)
+        return rows * nblk;
+    if (layout == MXFP4_SCALES_MMA)
+        return 512 * ((rows + 127) / 128) * ((nblk + 3) / 4);
+    return -1;
 }
 
 int32_t mxfp4_abi_version(void) { return MXFP4_ABI_VERSION; }

@@ -439,16 +439,29 @@ __device__ __forceinline__ void copy_outputs(const KArgs& a, const StagedOut& o,
     }
 }
 
-// Row-wise scales of a tile (32 rows x 8 blocks) from staging: one row per lane.
+// Row-wise scales of a tile (32 rows x 8 blocks) from staging: one row per
+// lane. In the MMA layout a tile's row holds two 4-byte atom entries (its
+// first block is a multiple of 8).
 __device__ __forceinline__ void copy_row_scales(const KArgs& a, const StagedOut& o, int row0, int nrows, int col0,
                                                 int lane)
 {
     const int r = lane;
     if (r >= nrows)
         return;
-    const int64_t nblk = (a.cols + 31) / 32;
-    uint8_t* dst = a.scales_row + (int64_t)(row0 + r) * nblk + col0 / 32;
-    const int nb = (int)min((int64_t)8, nblk - col0 / 32);
+    const int64_t nblk = (a.cols + 31) / 32, b0 = col0 / 32, row = (int64_t)row0 + r;
+    const int nb = (int)min((int64_t)8, nblk - b0);
+    if (a.srow_mma) {
+        if (nb == 8 && ((uintptr_t)a.scales_row & 3) == 0) {
+            const uint2 v = *reinterpret_cast<const uint2*>(o.srow + r * 8);
+            *reinterpret_cast<uint32_t*>(a.scales_row + srow_off(a, row, b0, nblk)) = v.x;
+            *reinterpret_cast<uint32_t*>(a.scales_row + srow_off(a, row, b0 + 4, nblk)) = v.y;
+        } else {
+            for (int b = 0; b < nb; ++b)
+                a.scales_row[srow_off(a, row, b0 + b, nblk)] = o.srow[r * 8 + b];
+        }
+        return;
+    }
+    uint8_t* dst = a.scales_row + row * nblk + b0;
     if (nb == 8 && ((uintptr_t)dst & 7) == 0) {
         *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(o.srow + r * 8);
     } else {
@@ -946,7 +959,6 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
     const uint32_t t_begin = (uint32_t)(((uint64_t)blockIdx.x * ntiles) / gridDim.x);
     const uint32_t t_end = (uint32_t)(((uint64_t)(blockIdx.x + 1) * ntiles) / gridDim.x);
     const uint32_t lutb = smem_addr(sm.lut) - 0x2C000000u;
-    const uint32_t lutb16 = lutb + 0x04000000u;
     const uint32_t col_out = COL ? (a.y_col ? SG_TS_Y : 0u) | (a.codes_col ? SG_TS_CODES : 0u) |
                                        (a.mask_col ? SG_TS_MASK : 0u)
                                  : 0u;
@@ -1196,7 +1208,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
             copy_outputs128(a, out, row0, nrows, col0, copy);
         if (ROW && a.scales_row && tid < SB_ROWS && tid < nrows) {
             const int64_t nblk = (a.cols + 127) / 128;
-            a.scales_row[(int64_t)(row0 + tid) * nblk + col0 / 128] = sm.srow[tid];
+            a.scales_row[srow_off(a, (int64_t)row0 + tid, col0 / 128, nblk)] = sm.srow[tid];
         }
         if (++s == SB_STAGES) {
             s = 0;

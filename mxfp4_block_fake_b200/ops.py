@@ -7,7 +7,9 @@ CUDA tensors: there is no CPU path.
 Tensor conventions follow include/mxfp4.h: x is 2-D [rows, cols] with unit
 stride along cols (a 1-D tensor is one row); outputs are contiguous; masks are
 bit-packed [rows, ceil(cols/8)] uint8; codes are nibble pairs
-[rows, ceil(cols/2)] uint8; row-wise scales [rows, ceil(cols/block)] uint8;
+[rows, ceil(cols/2)] uint8; row-wise scales [rows, ceil(cols/block)] uint8,
+or, with scales_layout="mma", a flat zero-initialised uint8 buffer in the
+block-scaled MMA scale-factor layout (128 x 4 atoms; include/mxfp4.h);
 column-wise scales [S_bound, cols] uint8 (only the first S rows are written,
 S = mxfp4_colwise_scale_rows(...)).
 """
@@ -22,6 +24,7 @@ from . import _abi
 _DTYPES = {torch.float32: _abi.F32, torch.bfloat16: _abi.BF16}
 _MODES = {"page": _abi.SCALE_PAGE, "floor": _abi.SCALE_FLOOR}
 _DIRS = {"rowwise": _abi.ROWWISE, "colwise": _abi.COLWISE}
+_SCALE_LAYOUTS = {"rowmajor": _abi.SCALES_ROWMAJOR, "mma": _abi.SCALES_MMA}
 
 
 @dataclasses.dataclass
@@ -35,6 +38,7 @@ class QDQResult:
     scales_col: torch.Tensor | None = None
     mask_col: torch.Tensor | None = None
     status: torch.Tensor | None = None
+    scales_layout: str = "rowmajor"  # layout of scales_row
 
 
 def _ptr(t: torch.Tensor | None):
@@ -108,19 +112,32 @@ def mxfp4_colwise_scale_rows(group_list, group_list_type: int, rows: int, block:
     return _abi.mxfp4_colwise_scale_rows(group_list, group_list_type, rows, block)
 
 
+def scales_row_bytes(rows: int, cols: int, block: int, scales_layout: str = "rowmajor") -> int:
+    if scales_layout not in _SCALE_LAYOUTS:
+        raise ValueError(f"scales_layout must be one of {tuple(_SCALE_LAYOUTS)}, got {scales_layout!r}")
+    n = _abi.lib().mxfp4_scales_row_bytes(rows, cols, block, _SCALE_LAYOUTS[scales_layout])
+    if n < 0:
+        raise ValueError("invalid geometry")
+    return n
+
+
 def alloc_outputs(x: torch.Tensor, *, block: int, rowwise: bool, colwise: bool, num_groups: int,
                   emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
-                  with_status: bool = False) -> QDQResult:
+                  with_status: bool = False, scales_layout: str = "rowmajor") -> QDQResult:
     rows, cols = x.shape
     dev = x.device
-    r = QDQResult()
+    r = QDQResult(scales_layout=scales_layout)
     u8 = dict(dtype=torch.uint8, device=dev)
     if rowwise:
         if emit_values:
             r.y_row = torch.empty((rows, cols), dtype=x.dtype, device=dev)
         if emit_codes:
             r.codes_row = torch.empty((rows, (cols + 1) // 2), **u8)
-            r.scales_row = torch.empty((rows, (cols + block - 1) // block), **u8)
+            if scales_layout == "mma":
+                # the padding of the last atoms is never written: zeros
+                r.scales_row = torch.zeros((scales_row_bytes(rows, cols, block, "mma"),), **u8)
+            else:
+                r.scales_row = torch.empty((rows, (cols + block - 1) // block), **u8)
         if emit_mask:
             r.mask_row = torch.empty((rows, (cols + 7) // 8), **u8)
     if colwise:
@@ -142,6 +159,9 @@ def _fill_outputs(a: _abi.QdqArgs, r: QDQResult) -> None:
     a.ld_y = _ld(ys[0]) if ys else a.cols
     a.codes_row, a.scales_row, a.mask_row = _ptr(r.codes_row), _ptr(r.scales_row), _ptr(r.mask_row)
     a.codes_col, a.scales_col, a.mask_col = _ptr(r.codes_col), _ptr(r.scales_col), _ptr(r.mask_col)
+    if r.scales_layout not in _SCALE_LAYOUTS:
+        raise ValueError(f"scales_layout must be one of {tuple(_SCALE_LAYOUTS)}, got {r.scales_layout!r}")
+    a.scales_row_layout = _SCALE_LAYOUTS[r.scales_layout]
 
 
 def _check_status(r: QDQResult, where: str) -> None:
@@ -153,9 +173,10 @@ def _check_status(r: QDQResult, where: str) -> None:
 def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0, scale_mode: str = "page",
                   rowwise: bool = True, colwise: bool = False, group_list=None, group_list_type: int = 0,
                   emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
-                  check: bool = False, out: QDQResult | None = None) -> QDQResult:
+                  check: bool = False, out: QDQResult | None = None, scales_layout: str = "rowmajor") -> QDQResult:
     """QDQ forward; returns the requested outputs. check=True synchronises and
-    raises on an invalid group_list."""
+    raises on an invalid group_list. scales_layout="mma" writes the row-wise
+    scales in the block-scaled MMA scale-factor layout."""
     x = _as_2d(x)
     gl, ng = _group_args(group_list, group_list_type, x.device)
     dirs = (_abi.ROWWISE if rowwise else 0) | (_abi.COLWISE if colwise else 0)
@@ -163,7 +184,8 @@ def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0
         raise ValueError("at least one of rowwise / colwise must be set")
     r = out if out is not None else alloc_outputs(
         x, block=block, rowwise=rowwise, colwise=colwise, num_groups=ng, emit_values=emit_values,
-        emit_codes=emit_codes, emit_mask=emit_mask, with_status=check or gl is not None)
+        emit_codes=emit_codes, emit_mask=emit_mask, with_status=check or gl is not None,
+        scales_layout=scales_layout)
     a = make_args(x, block=block, scale_factor=scale_factor, scale_mode=scale_mode, dirs=dirs,
                   group_list=gl, group_list_type=group_list_type, status=r.status)
     _fill_outputs(a, r)
@@ -227,3 +249,19 @@ def mxfp4_qdq_fwd_bwd(x: torch.Tensor, grad_out: torch.Tensor, *, grad_direction
                                 _stream(x.device))
     _abi.check(st, "mxfp4_qdq_fwd_bwd")
     return r, gi
+
+
+def mxfp4_mma_operand(x: torch.Tensor, *, scale_mode: str = "page", scale_factor: float = 6.0,
+                      out: QDQResult | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Real MXFP4 operand of a block-scaled GEMM that contracts over x's last
+    dimension: (codes [rows, cols/2] as torch.float4_e2m1fn_x2, first element
+    in the low nibble; E8M0 scales as torch.float8_e8m0fnu in the 128 x 4 atom
+    layout). Block 32 along the contraction; one pass of the row-wise kernel
+    writing codes and scales only. Decoding code * 2^(scale - 127) gives the
+    fake-quantised values the same call would return as y_row."""
+    x2 = _as_2d(x)
+    if x2.shape[1] % 2:
+        raise ValueError("the contraction dimension must be even (two E2M1 codes per byte)")
+    r = mxfp4_qdq_fwd(x2, block=32, scale_factor=scale_factor, scale_mode=scale_mode, rowwise=True,
+                      emit_values=False, emit_codes=True, out=out, scales_layout="mma")
+    return r.codes_row.view(torch.float4_e2m1fn_x2), r.scales_row.view(torch.float8_e8m0fnu)

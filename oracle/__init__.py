@@ -157,6 +157,25 @@ def unpack_bits(mask: np.ndarray, cols: int) -> np.ndarray:
     return np.unpackbits(mask, axis=1, bitorder="little")[:, :cols].astype(bool)
 
 
+def mma_scale_layout(scales: np.ndarray) -> np.ndarray:
+    """Row-wise scales [R, C] (one byte per block) -> the flat byte buffer of
+    the block-scaled MMA scale-factor layout, as the cuBLAS documentation
+    defines it ("1D block scaling factors layout"): the matrix is padded to
+    multiples of 128 rows and 4 columns and cut into 128 x 4 atoms of 512
+    bytes, atom (i, j) at byte 512 * (i * ceil(C / 4) + j); inside an atom,
+    entry (r, c) is at byte 16 * (r % 32) + 4 * (r // 32) + c. Padding is 0."""
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    R, C = s.shape
+    n_rb, n_cb = -(-R // 128), -(-C // 4)
+    out = np.zeros(512 * n_rb * n_cb, np.uint8)
+    r = np.arange(R, dtype=np.int64)[:, None]
+    c = np.arange(C, dtype=np.int64)[None, :]
+    i, rr = r // 128, r % 128
+    j, cc = c // 4, c % 4
+    out[512 * (i * n_cb + j) + 16 * (rr % 32) + 4 * (rr // 32) + cc] = s
+    return out
+
+
 def unpack_nibbles(codes: np.ndarray, cols: int) -> np.ndarray:
     """Packed [rows, ceil(cols/2)] codes -> uint8 [rows, cols] nibbles (low nibble first)."""
     lo = codes & 0x0F
@@ -170,5 +189,5 @@ def unpack_nibbles(codes: np.ndarray, cols: int) -> np.ndarray:
 __all__ = [
     "F32", "BF16", "SCALE_PAGE", "SCALE_FLOOR", "lib", "build", "bf16_to_f32", "f32_to_bf16",
     "scale_page", "scale_floor", "qdq_block", "group_ends", "colwise_scale_rows", "qdq_rowwise",
-    "qdq_colwise", "ste_bwd", "unpack_bits", "unpack_nibbles",
+    "qdq_colwise", "ste_bwd", "unpack_bits", "unpack_nibbles", "mma_scale_layout",
 ]

@@ -190,6 +190,82 @@ def test_padded_and_offset_outputs(offsets, rows, cols, counts):
     check_dir(r, O.qdq_colwise(xo, 32, 6.0, O.SCALE_PAGE, ends=ends), "col", cols, label="padded/offset")
 
 
+MMA_CASES = [
+    # (dtype, block, rows, cols, colwise, counts, scales byte offset)
+    (torch.bfloat16, 32, 300, 1024, False, None, 0),       # staged, row-wise only
+    (torch.bfloat16, 32, 300, 1024, True, None, 0),        # staged, dual
+    (torch.bfloat16, 32, 261, 1000, True, [100, 0, 61, 100], 0),  # staged, grouped, ragged
+    (torch.bfloat16, 32, 300, 200, True, None, 0),         # staged, 7 blocks per row
+    (torch.bfloat16, 32, 300, 1024, True, None, 1),        # staged, unaligned scales buffer
+    (torch.bfloat16, 128, 300, 1024, True, None, 0),       # staged block 128
+    (torch.bfloat16, 128, 130, 640, False, None, 0),       # block 128 row-wise
+    (torch.float32, 32, 129, 136, True, None, 0),          # register-tile kernel
+    (torch.float32, 128, 260, 512, False, None, 0),        # register-tile kernel, block 128
+    (torch.bfloat16, 32, 5, 999, True, None, 0),           # scalar kernels (odd cols)
+]
+
+
+@pytest.mark.parametrize("case", MMA_CASES)
+def test_mma_scale_layout(case):
+    """Row-wise scales written straight into the block-scaled MMA layout
+    (128 x 4 atoms) equal the oracle's row-major scales placed by the
+    oracle's layout; padding bytes stay untouched; the other outputs are the
+    same as with the row-major layout."""
+    dtype, block, rows, cols, colwise, counts, soff = case
+    x = W.mixed(rows, cols, dtype=dtype, seed=41 + rows)
+    xd = x.cuda()
+    ng = 0 if counts is None else len(counts)
+    r = ops.alloc_outputs(xd, block=block, rowwise=True, colwise=colwise, num_groups=ng, emit_codes=True,
+                          emit_mask=True, with_status=True, scales_layout="mma")
+    n = r.scales_row.numel()
+    r.scales_row = torch.zeros((n + soff,), dtype=torch.uint8, device=xd.device)[soff:]
+    gl = None if counts is None else torch.tensor(counts, dtype=torch.int64, device=xd.device)
+    ops.mxfp4_qdq_fwd(xd, block=block, rowwise=True, colwise=colwise, group_list=gl, group_list_type=1,
+                      emit_codes=True, emit_mask=True, out=r, check=True)
+    torch.cuda.synchronize()
+    xo = oracle_in(x)
+    ora = O.qdq_rowwise(xo, block, 6.0, O.SCALE_PAGE)
+    got = r.scales_row.cpu().numpy()
+    exp = O.mma_scale_layout(ora["scales"])
+    assert got.size == exp.size
+    bad = np.flatnonzero(got != exp)
+    assert bad.size == 0, f"{bad.size} scale bytes differ, first at {bad[:4].tolist()}"
+    r.scales_row = None
+    check_dir(r, ora, "row", cols, label="mma layout")
+    if colwise:
+        ends = None if counts is None else np.cumsum(np.asarray(counts, np.int64))
+        check_dir(r, O.qdq_colwise(xo, block, 6.0, O.SCALE_PAGE, ends=ends), "col", cols, label="mma layout")
+
+
+@pytest.mark.parametrize("mode", ["page", "floor"])
+@pytest.mark.parametrize("mnk", [(256, 384, 2048), (192, 256, 1024)])
+def test_mma_operands_in_a_real_fp4_gemm(mode, mnk):
+    """The packed codes and MMA-layout scales, fed to a block-scaled FP4
+    tensor-core GEMM (torch's scaled_mm, MXFP4: E2M1 data, E8M0 scales per 32
+    along K, 128 x 4 scale atoms), give the product of the fake-quantised
+    matrices: real quantisation equals fake quantisation. Reference: the
+    oracle's dequantised values multiplied in float64. Bound: the bf16 output
+    rounding (2^-8 relative) plus fp32 accumulation over K terms
+    (K 2^-23 of the sum of |products|)."""
+    from torch.nn.functional import ScalingType, SwizzleType, scaled_mm
+    M, N, K = mnk
+    x = torch.randn(M, K, generator=torch.Generator().manual_seed(M)).to(torch.bfloat16)
+    w = torch.randn(N, K, generator=torch.Generator().manual_seed(N + 1)).to(torch.bfloat16)
+    cx, sx = ops.mxfp4_mma_operand(x.cuda(), scale_mode=mode)
+    cw, sw = ops.mxfp4_mma_operand(w.cuda(), scale_mode=mode)
+    out = scaled_mm(cx, cw.t(), sx, ScalingType.BlockWise1x32, sw, ScalingType.BlockWise1x32,
+                    swizzle_a=SwizzleType.SWIZZLE_32_4_4, swizzle_b=SwizzleType.SWIZZLE_32_4_4,
+                    output_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    yx = O.bf16_to_f32(O.qdq_rowwise(oracle_in(x), 32, 6.0, MODES[mode])["y"]).astype(np.float64)
+    yw = O.bf16_to_f32(O.qdq_rowwise(oracle_in(w), 32, 6.0, MODES[mode])["y"]).astype(np.float64)
+    ref = yx @ yw.T
+    mag = np.abs(yx) @ np.abs(yw).T
+    err = np.abs(out.float().cpu().numpy().astype(np.float64) - ref)
+    bound = 2.0 ** -8 * np.abs(ref) + K * 2.0 ** -23 * mag
+    assert np.all(err <= bound), f"max err/bound {float((err / bound).max()):.3f}"
+
+
 @pytest.mark.parametrize("sf", [1.0, 4.0, 7.5, 0.75, 3.0e-38, 1.0e30])
 def test_scale_factors_page_mode(sf):
     x = W.mixed(64, 512, seed=6)

@@ -408,3 +408,50 @@ def test_torch_page_formula_agrees_on_bf16(oracle_mod):
     ref = (q * scale).reshape(512, 256).to(torch.bfloat16)
     res = O.qdq_rowwise(xb.view(torch.int16).numpy().view(np.uint16), 32, 6.0, 0)
     assert np.array_equal(res["y"], ref.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_mma_scale_layout_hand_offsets(oracle_mod):
+    """Offsets worked out by hand from the cuBLAS "1D block scaling factors
+    layout" rule (128 x 4 atoms, atom rows in order, entry (r, c) of an atom
+    at 16 (r mod 32) + 4 floor(r / 32) + c) for a 130 x 5 scale matrix: two
+    atom rows by two atom columns, 2048 bytes."""
+    O = oracle_mod
+    s = np.zeros((130, 5), np.uint8)
+    expect = {(0, 0): 0, (1, 0): 16, (31, 0): 496, (32, 0): 4, (33, 1): 21, (127, 3): 511,
+              (0, 4): 512, (127, 4): 512 + 511 - 3, (128, 0): 1024, (129, 4): 1552}
+    for n, (rc, _) in enumerate(expect.items()):
+        s[rc] = n + 1
+    out = O.mma_scale_layout(s)
+    assert out.size == 2048
+    for n, (rc, off) in enumerate(expect.items()):
+        assert out[off] == n + 1, (rc, off)
+    assert np.count_nonzero(out) == len(expect)
+
+
+@pytest.mark.parametrize("shape", [(128, 4), (130, 5), (256, 56), (1, 1), (300, 7), (513, 224)])
+def test_mma_scale_layout_by_reshapes(oracle_mod, shape):
+    """The same layout derived by tensor reshapes instead of an index formula:
+    pad, cut into 128 x 4 tiles taken tile row by tile row, view each tile as
+    4 row-quarters x 32 rows x 4 columns and swap the first two axes."""
+    R, C = shape
+    rng = np.random.default_rng(R * 1000 + C)
+    s = rng.integers(1, 256, shape, dtype=np.uint16).astype(np.uint8)
+    n_rb, n_cb = -(-R // 128), -(-C // 4)
+    padded = np.zeros((128 * n_rb, 4 * n_cb), np.uint8)
+    padded[:R, :C] = s
+    tiles = padded.reshape(n_rb, 128, n_cb, 4).transpose(0, 2, 1, 3).reshape(-1, 4, 32, 4)
+    ref = tiles.transpose(0, 2, 1, 3).reshape(-1)
+    assert np.array_equal(oracle_mod.mma_scale_layout(s), ref)
+
+
+def test_mma_scale_layout_is_a_placement(oracle_mod):
+    """Every entry lands on its own byte; the rest (padding) stays 0."""
+    O = oracle_mod
+    R, C = 300, 7
+    idx = np.arange(R * C, dtype=np.int64).reshape(R, C)
+    lo, hi = (idx & 0xFF).astype(np.uint8), (idx >> 8).astype(np.uint8)
+    a, b = O.mma_scale_layout(lo), O.mma_scale_layout(hi)
+    placed = a.astype(np.int64) | (b.astype(np.int64) << 8)
+    nz = O.mma_scale_layout(np.ones((R, C), np.uint8)) == 1
+    assert nz.sum() == R * C and placed.size == 512 * 3 * 2
+    assert np.array_equal(np.sort(placed[nz]), np.arange(R * C))
