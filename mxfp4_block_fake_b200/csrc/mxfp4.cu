@@ -74,12 +74,15 @@ struct KArgs {
 // row-major, or the block-scaled MMA layout (atoms of 128 rows x 4 block
 // columns, 512 bytes, atom rows in order; entry (r, c) of an atom at
 // 16 (r mod 32) + 4 floor(r / 32) + c).
+__device__ __forceinline__ int64_t srow_off_mma(int64_t row, int64_t b, int64_t nblk)
+{
+    const int64_t ncb = (nblk + 3) >> 2;
+    return (((row >> 7) * ncb + (b >> 2)) << 9) + ((row & 31) << 4) + (((row >> 5) & 3) << 2) + (b & 3);
+}
+
 __device__ __forceinline__ int64_t srow_off(const KArgs& a, int64_t row, int64_t b, int64_t nblk)
 {
-    if (!a.srow_mma)
-        return row * nblk + b;
-    const int64_t ncb = (nblk + 3) >> 2;
-    return ((((row >> 7) * ncb + (b >> 2))) << 9) + ((row & 31) << 4) + (((row >> 5) & 3) << 2) + (b & 3);
+    return a.srow_mma ? srow_off_mma(row, b, nblk) : row * nblk + b;
 }
 
 // ---------------------------------------------------------------------------
@@ -1408,11 +1411,16 @@ static bool make_staged128_maps(StagedMaps* m, const KArgs& k, uint32_t* ts_flag
 
 typedef void (*StagedFn)(const StagedMaps, const KArgs);
 
+// SMMA (row-wise scales in the MMA layout) is its own instantiation, so the
+// row-major kernels carry no code for it
 template <bool ROW, bool COL, bool GROUPS>
-static StagedFn pick_staged(int mode)
+static StagedFn pick_staged(int mode, bool smma)
 {
-    return mode == MXFP4_SCALE_FLOOR ? qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_FLOOR>
-                                     : qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_PAGE>;
+    if (ROW && smma)
+        return mode == MXFP4_SCALE_FLOOR ? qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_FLOOR, ROW>
+                                         : qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_PAGE, ROW>;
+    return mode == MXFP4_SCALE_FLOOR ? qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_FLOOR, false>
+                                     : qdq_staged_kernel<ROW, COL, GROUPS, MXFP4_SCALE_PAGE, false>;
 }
 
 template <bool ROW, bool COL, bool GROUPS>
@@ -1447,9 +1455,10 @@ static mxfp4_status launch_staged128(bool row, bool col, bool groups, const Stag
 static mxfp4_status launch_staged(bool row, bool col, bool groups, const StagedMaps& maps, const KArgs& k,
                                   int64_t tiles, size_t plan_smem, cudaStream_t s)
 {
-    StagedFn fn = !col ? pick_staged<true, false, false>(k.mode)
-                : row  ? (groups ? pick_staged<true, true, true>(k.mode) : pick_staged<true, true, false>(k.mode))
-                       : (groups ? pick_staged<false, true, true>(k.mode) : pick_staged<false, true, false>(k.mode));
+    const bool sm = k.srow_mma && k.scales_row;
+    StagedFn fn = !col ? pick_staged<true, false, false>(k.mode, sm)
+                : row  ? (groups ? pick_staged<true, true, true>(k.mode, sm) : pick_staged<true, true, false>(k.mode, sm))
+                       : (groups ? pick_staged<false, true, true>(k.mode, sm) : pick_staged<false, true, false>(k.mode, sm));
     const size_t smem = sizeof(StagedSmem) + 1024 + plan_smem;
     if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MXFP4_ECUDA;
@@ -1462,6 +1471,25 @@ static mxfp4_status launch_staged(bool row, bool col, bool groups, const StagedM
         grid = tiles < 1 ? 1 : tiles;
     fn<<<(unsigned)grid, SG_THREADS, smem, s>>>(maps, k);
     return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
+}
+
+static mxfp4_status launch_codes_row(const KArgs& k, int64_t blocks, cudaStream_t s)
+{
+    const bool floor = k.mode == MXFP4_SCALE_FLOOR, sm = k.srow_mma && k.scales_row;
+    const void* fn = floor ? (sm ? (const void*)codes_row_kernel<MXFP4_SCALE_FLOOR, true>
+                                 : (const void*)codes_row_kernel<MXFP4_SCALE_FLOOR, false>)
+                           : (sm ? (const void*)codes_row_kernel<MXFP4_SCALE_PAGE, true>
+                                 : (const void*)codes_row_kernel<MXFP4_SCALE_PAGE, false>);
+    const int sms = device_sms();
+    const int occ = occupancy(fn, 0);
+    if (sms <= 0 || occ <= 0)
+        return MXFP4_ECUDA;
+    int64_t grid = (int64_t)sms * occ;
+    if ((blocks + NTHREADS - 1) / NTHREADS < grid)
+        grid = (blocks + NTHREADS - 1) / NTHREADS;
+    void* args[] = {const_cast<KArgs*>(&k)};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(NTHREADS), args, 0, s) == cudaSuccess ? MXFP4_OK
+                                                                                               : MXFP4_ECUDA;
 }
 
 static mxfp4_status check_geometry(const mxfp4_qdq_args* a)
@@ -1582,6 +1610,14 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     const int bs = A->block;
     const size_t plan_smem = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
     const int64_t s_bound = groups ? A->rows / bs + A->num_groups : (A->rows + bs - 1) / bs;
+
+    // row-wise codes / scales / masks without values (real quantisation):
+    // one streaming pass, one thread per block
+    if (fast && row && !col && esz == 2 && bs == 32 && !grad && !k.y_row &&
+        (k.codes_row || k.scales_row || k.mask_row) && A->cols % 32 == 0 && A->ld % 16 == 0 &&
+        aligned(A->x, 32) && (!k.codes_row || aligned(k.codes_row, 16)) && (!k.mask_row || aligned(k.mask_row, 4)) &&
+        A->rows * (A->cols / 32) < (int64_t)UINT32_MAX)
+        return launch_codes_row(k, A->rows * (A->cols / 32), s);
 
     // TMA coordinates and the staged kernel's tile bookkeeping are 32-bit
     if (fast && esz == 2 && bs == 32 && (col || !groups) && !grad && A->rows <= INT32_MAX - 2 * SG_ROWS &&

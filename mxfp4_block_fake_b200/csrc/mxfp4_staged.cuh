@@ -440,28 +440,31 @@ __device__ __forceinline__ void copy_outputs(const KArgs& a, const StagedOut& o,
 }
 
 // Row-wise scales of a tile (32 rows x 8 blocks) from staging: one row per
-// lane. In the MMA layout a tile's row holds two 4-byte atom entries (its
-// first block is a multiple of 8).
+// lane. SMMA: the MMA layout, where a tile's row holds two 4-byte atom
+// entries (its first block is a multiple of 8).
+template <bool SMMA>
 __device__ __forceinline__ void copy_row_scales(const KArgs& a, const StagedOut& o, int row0, int nrows, int col0,
                                                 int lane)
 {
     const int r = lane;
     if (r >= nrows)
         return;
-    const int64_t nblk = (a.cols + 31) / 32, b0 = col0 / 32, row = (int64_t)row0 + r;
-    const int nb = (int)min((int64_t)8, nblk - b0);
-    if (a.srow_mma) {
+    const int64_t nblk = (a.cols + 31) / 32;
+    if constexpr (SMMA) {
+        const int64_t b0 = col0 / 32, row = (int64_t)row0 + r;
+        const int nb = (int)min((int64_t)8, nblk - b0);
         if (nb == 8 && ((uintptr_t)a.scales_row & 3) == 0) {
             const uint2 v = *reinterpret_cast<const uint2*>(o.srow + r * 8);
-            *reinterpret_cast<uint32_t*>(a.scales_row + srow_off(a, row, b0, nblk)) = v.x;
-            *reinterpret_cast<uint32_t*>(a.scales_row + srow_off(a, row, b0 + 4, nblk)) = v.y;
+            *reinterpret_cast<uint32_t*>(a.scales_row + srow_off_mma(row, b0, nblk)) = v.x;
+            *reinterpret_cast<uint32_t*>(a.scales_row + srow_off_mma(row, b0 + 4, nblk)) = v.y;
         } else {
             for (int b = 0; b < nb; ++b)
-                a.scales_row[srow_off(a, row, b0 + b, nblk)] = o.srow[r * 8 + b];
+                a.scales_row[srow_off_mma(row, b0 + b, nblk)] = o.srow[r * 8 + b];
         }
         return;
     }
-    uint8_t* dst = a.scales_row + row * nblk + b0;
+    uint8_t* dst = a.scales_row + (int64_t)(row0 + r) * nblk + col0 / 32;
+    const int nb = (int)min((int64_t)8, nblk - col0 / 32);
     if (nb == 8 && ((uintptr_t)dst & 7) == 0) {
         *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(o.srow + r * 8);
     } else {
@@ -485,8 +488,9 @@ __device__ __forceinline__ void col_sat_store(uint32_t* mwords, uint32_t bits, i
 }
 
 // ROW / COL: the directions computed (at least one); GROUPS: column-wise
-// blocks restart at group_list boundaries; MODE: the scale rule.
-template <bool ROW, bool COL, bool GROUPS, int MODE>
+// blocks restart at group_list boundaries; MODE: the scale rule; SMMA:
+// row-wise scales in the MMA layout.
+template <bool ROW, bool COL, bool GROUPS, int MODE, bool SMMA>
 __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_constant__ StagedMaps maps, const KArgs a)
 {
     extern __shared__ __align__(1024) uint8_t s_dyn[];
@@ -820,7 +824,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             bulk_commit();  // row-wise group
         }
         if (ROW && a.scales_row && warp == SG_STORER / 32)
-            copy_row_scales(a, out, row0, nrows, col0, lane);
+            copy_row_scales<SMMA>(a, out, row0, nrows, col0, lane);
         if (copy) {
             copy_outputs(a, out, row0, nrows, col0, copy);
             __syncthreads();  // no warp writes the staging buffers before every copy is done
@@ -1301,6 +1305,89 @@ __global__ void __launch_bounds__(NTHREADS) ste_row_kernel(const KArgs a)
             g[i] &= keep[i];
         st_cs_v8(static_cast<char*>(a.g_in) + goff, g);
         st_cs_v8(static_cast<char*>(a.g_in) + goff + 32, g + 8);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Row-wise bf16 block 32 without dequantised values: the real-quantisation
+// producer (packed E2M1 codes, E8M0 scales, saturation bits). One thread per
+// block: two 32-byte streaming loads, amax, k, the codes by the nudged
+// hardware convert (no dequantisation needed), one 16-byte code store, one
+// 4-byte mask word and one scale byte (SMMA: in the MMA layout). Blocks off
+// the fast k range take the general element path.
+// ---------------------------------------------------------------------------
+
+// E2M1 bytes of four words sharing one scale, as one 32-bit nibble word.
+__device__ __forceinline__ uint32_t nibs4_cvt(const uint32_t* w, float invn)
+{
+    float y[8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        nudged_pair(w[u], invn, invn, y[2 * u], y[2 * u + 1]);
+    uint32_t nibs;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(nibs)
+        : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+    return nibs;
+}
+
+template <int MODE, bool SMMA>
+__global__ void __launch_bounds__(NTHREADS) codes_row_kernel(const KArgs a)
+{
+    const uint32_t nb = (uint32_t)(a.cols / 32);
+    const uint32_t total = (uint32_t)a.rows * nb;
+    __shared__ uint32_t s_lut[64];
+    if (threadIdx.x < 64)
+        s_lut[threadIdx.x] = lut_entry(threadIdx.x);
+    __syncthreads();
+    const uint32_t glutb = smem_addr(s_lut) - 0x2C000000u;
+    for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < total; u += gridDim.x * blockDim.x) {
+        const uint32_t row = u / nb, blk = u - row * nb;
+        const char* xp = static_cast<const char*>(a.x) + ((int64_t)row * a.ld + 32 * blk) * 2;
+        uint32_t w[16];
+        ld_nc_v8(xp, w);
+        ld_nc_v8(xp + 32, w + 8);
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            m2 = vmax2(m2, w[i] & 0x7FFF7FFFu);
+        const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
+        const uint32_t A = am << 16;
+        const int k = block_kt<MODE>(A, a.thr);
+        uint32_t nib[4], sats = 0, e8;
+        if (k_fast_bf(k)) {
+            const float invn = inv_nudged(k);
+            const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
+            const uint32_t limx[4] = {lx, lx, lx, lx};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                nib[c] = nibs4_cvt(w + 4 * c, invn);
+                const uint32_t a4w[4] = {w[4 * c] & 0x7FFF7FFFu, w[4 * c + 1] & 0x7FFF7FFFu,
+                                         w[4 * c + 2] & 0x7FFF7FFFu, w[4 * c + 3] & 0x7FFF7FFFu};
+                sats |= sat8(a4w, limx) << (8 * c);
+            }
+            e8 = (uint32_t)(k + 127);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const ChunkOut gch = general_chunk<8, false>(
+                    make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]), &A, a.mode, a.thr, glutb);
+                nib[c] = gch.nibs;
+                sats |= gch.sats << (8 * c);
+            }
+            e8 = e8_of(A, k);
+        }
+        if (a.codes_row)
+            st_stream(a.codes_row + (int64_t)row * (a.cols / 2) + 16 * blk, make_uint4(nib[0], nib[1], nib[2], nib[3]));
+        if (a.mask_row)
+            *reinterpret_cast<uint32_t*>(a.mask_row + (int64_t)row * (a.cols / 8) + 4 * blk) = sats;
+        if (a.scales_row)
+            a.scales_row[SMMA ? srow_off_mma(row, blk, nb) : (int64_t)row * nb + blk] = (uint8_t)e8;
     }
 }
 

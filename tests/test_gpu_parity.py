@@ -274,10 +274,10 @@ def test_scale_factors_page_mode(sf):
     check_dir(res, ora["col"], "col", 512)
 
 
-@pytest.mark.parametrize("mode", ["page", "floor"])
-def test_every_bf16_value_as_element_and_as_block_max(mode):
+def bf16_sweep_block32() -> np.ndarray:
+    """Rows of 32-element blocks: every bf16 value as block maximum (with a
+    neighbour and its negation), and as element under fixed maxima."""
     allv = np.arange(65536, dtype=np.uint32).astype(np.uint16)
-    # as block maximum: row = [v, v/2-ish neighbours...] -> every amax pattern incl. inf / NaN
     rows = []
     for shift in (0, 1, 3):
         blk = np.zeros((65536, 32), np.uint16)
@@ -286,16 +286,57 @@ def test_every_bf16_value_as_element_and_as_block_max(mode):
         blk[:, 2] = allv ^ 0x8000
         blk[:, 5] = 0x3F80
         rows.append(blk)
-    # as element under fixed maxima
     for mx in (0x40C0, 0x4090, 0x3F80, 0x40F8, 0x0010, 0x7F7F):
         blk = np.zeros((65536, 32), np.uint16)
         blk[:, 0] = mx
         blk[:, 7] = allv
         rows.append(blk)
-    xb = np.concatenate(rows)
+    return np.concatenate(rows)
+
+
+@pytest.mark.parametrize("mode", ["page", "floor"])
+def test_every_bf16_value_as_element_and_as_block_max(mode):
+    xb = bf16_sweep_block32()
     x = torch.from_numpy(xb.view(np.int16).copy()).view(torch.bfloat16)
     res, ora = run_both(x, block=32, mode=mode, rowwise=True, colwise=False)
     check_dir(res, ora["row"], "row", 32, label="bf16 sweep")
+
+
+def codes_only(x: torch.Tensor, mode: str, layout: str):
+    res = ops.mxfp4_qdq_fwd(x.cuda(), block=32, scale_mode=mode, rowwise=True, emit_values=False,
+                            emit_codes=True, emit_mask=True, scales_layout=layout, check=True)
+    torch.cuda.synchronize()
+    ora = O.qdq_rowwise(oracle_in(x), 32, 6.0, MODES[mode])
+    exp_s = O.mma_scale_layout(ora["scales"]).reshape(-1) if layout == "mma" else ora["scales"]
+    return res, ora, exp_s
+
+
+@pytest.mark.parametrize("mode", ["page", "floor"])
+@pytest.mark.parametrize("layout", ["rowmajor", "mma"])
+def test_every_bf16_value_codes_without_values(mode, layout):
+    """The same sweep through the codes-only producer (no dequantised
+    values: packed codes, scales, masks)."""
+    xb = bf16_sweep_block32().reshape(-1, 256)  # 8 blocks per row
+    x = torch.from_numpy(xb.view(np.int16).copy()).view(torch.bfloat16)
+    res, ora, exp_s = codes_only(x, mode, layout)
+    assert res.y_row is None
+    assert np.array_equal(np_bits(res.codes_row), ora["codes"]), "codes"
+    assert np.array_equal(np_bits(res.mask_row), ora["mask"]), "mask"
+    assert np.array_equal(np_bits(res.scales_row).reshape(exp_s.shape), exp_s), "scales"
+
+
+@pytest.mark.parametrize("mode", ["page", "floor"])
+@pytest.mark.parametrize("layout", ["rowmajor", "mma"])
+@pytest.mark.parametrize("shape", [(300, 1024), (37, 4096), (1, 32), (129, 96), (64, 1000), (5, 999)])
+def test_rowwise_codes_without_values(mode, layout, shape):
+    """Codes, scales and masks without dequantised values on mixed inputs
+    (specials included): the streaming producer where cols % 32 == 0, the
+    staged and scalar kernels elsewhere."""
+    x = W.mixed(*shape, seed=57 + shape[0])
+    res, ora, exp_s = codes_only(x, mode, layout)
+    assert np.array_equal(np_bits(res.codes_row), ora["codes"]), "codes"
+    assert np.array_equal(np_bits(res.mask_row), ora["mask"]), "mask"
+    assert np.array_equal(np_bits(res.scales_row).reshape(exp_s.shape), exp_s), "scales"
 
 
 @pytest.mark.parametrize("mode", ["page", "floor"])
