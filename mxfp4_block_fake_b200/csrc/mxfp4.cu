@@ -1473,13 +1473,18 @@ static mxfp4_status launch_staged(bool row, bool col, bool groups, const StagedM
     return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
 }
 
-static mxfp4_status launch_codes_row(const KArgs& k, int64_t blocks, cudaStream_t s)
+template <bool SMMA, bool VALS>
+static const void* pick_row_stream(int mode)
 {
-    const bool floor = k.mode == MXFP4_SCALE_FLOOR, sm = k.srow_mma && k.scales_row;
-    const void* fn = floor ? (sm ? (const void*)codes_row_kernel<MXFP4_SCALE_FLOOR, true>
-                                 : (const void*)codes_row_kernel<MXFP4_SCALE_FLOOR, false>)
-                           : (sm ? (const void*)codes_row_kernel<MXFP4_SCALE_PAGE, true>
-                                 : (const void*)codes_row_kernel<MXFP4_SCALE_PAGE, false>);
+    return mode == MXFP4_SCALE_FLOOR ? (const void*)row_stream_kernel<MXFP4_SCALE_FLOOR, SMMA, VALS>
+                                     : (const void*)row_stream_kernel<MXFP4_SCALE_PAGE, SMMA, VALS>;
+}
+
+static mxfp4_status launch_row_stream(const KArgs& k, int64_t blocks, cudaStream_t s)
+{
+    const bool sm = k.srow_mma && k.scales_row;
+    const void* fn = k.y_row ? (sm ? pick_row_stream<true, true>(k.mode) : pick_row_stream<false, true>(k.mode))
+                             : (sm ? pick_row_stream<true, false>(k.mode) : pick_row_stream<false, false>(k.mode));
     const int sms = device_sms();
     const int occ = occupancy(fn, 0);
     if (sms <= 0 || occ <= 0)
@@ -1611,13 +1616,15 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     const size_t plan_smem = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
     const int64_t s_bound = groups ? A->rows / bs + A->num_groups : (A->rows + bs - 1) / bs;
 
-    // row-wise codes / scales / masks without values (real quantisation):
-    // one streaming pass, one thread per block
-    if (fast && row && !col && esz == 2 && bs == 32 && !grad && !k.y_row &&
-        (k.codes_row || k.scales_row || k.mask_row) && A->cols % 32 == 0 && A->ld % 16 == 0 &&
-        aligned(A->x, 32) && (!k.codes_row || aligned(k.codes_row, 16)) && (!k.mask_row || aligned(k.mask_row, 4)) &&
+    // row-wise only, bf16 block 32, with codes or masks (or without values):
+    // one streaming pass, one thread per block. Values alone go to the staged
+    // kernel, whose tiled stores measured faster for that traffic mix.
+    if (fast && row && !col && esz == 2 && bs == 32 && !grad && (!k.y_row || k.codes_row || k.mask_row) &&
+        A->cols % 32 == 0 && A->ld % 16 == 0 &&
+        aligned(A->x, 32) && (!k.y_row || (aligned(k.y_row, 32) && A->ld_y % 16 == 0)) &&
+        (!k.codes_row || aligned(k.codes_row, 16)) && (!k.mask_row || aligned(k.mask_row, 4)) &&
         A->rows * (A->cols / 32) < (int64_t)UINT32_MAX)
-        return launch_codes_row(k, A->rows * (A->cols / 32), s);
+        return launch_row_stream(k, A->rows * (A->cols / 32), s);
 
     // TMA coordinates and the staged kernel's tile bookkeeping are 32-bit
     if (fast && esz == 2 && bs == 32 && (col || !groups) && !grad && A->rows <= INT32_MAX - 2 * SG_ROWS &&

@@ -1309,12 +1309,12 @@ __global__ void __launch_bounds__(NTHREADS) ste_row_kernel(const KArgs a)
 }
 
 // ---------------------------------------------------------------------------
-// Row-wise bf16 block 32 without dequantised values: the real-quantisation
-// producer (packed E2M1 codes, E8M0 scales, saturation bits). One thread per
-// block: two 32-byte streaming loads, amax, k, the codes by the nudged
-// hardware convert (no dequantisation needed), one 16-byte code store, one
-// 4-byte mask word and one scale byte (SMMA: in the MMA layout). Blocks off
-// the fast k range take the general element path.
+// Row-wise bf16 block 32, one streaming pass: one thread per block, two
+// 32-byte loads, amax, k, the codes by the nudged hardware convert, then the
+// outputs asked for: dequantised values (VALS: two 32-byte streaming
+// stores), one 16-byte code store, one 4-byte mask word and one scale byte
+// (SMMA: in the MMA layout). Without values this is the real-quantisation
+// producer. Blocks off the fast k range take the general element path.
 // ---------------------------------------------------------------------------
 
 // E2M1 bytes of four words sharing one scale, as one 32-bit nibble word.
@@ -1336,8 +1336,8 @@ __device__ __forceinline__ uint32_t nibs4_cvt(const uint32_t* w, float invn)
     return nibs;
 }
 
-template <int MODE, bool SMMA>
-__global__ void __launch_bounds__(NTHREADS) codes_row_kernel(const KArgs a)
+template <int MODE, bool SMMA, bool VALS>
+__global__ void __launch_bounds__(NTHREADS) row_stream_kernel(const KArgs a)
 {
     const uint32_t nb = (uint32_t)(a.cols / 32);
     const uint32_t total = (uint32_t)a.rows * nb;
@@ -1359,14 +1359,17 @@ __global__ void __launch_bounds__(NTHREADS) codes_row_kernel(const KArgs a)
         const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
         const uint32_t A = am << 16;
         const int k = block_kt<MODE>(A, a.thr);
-        uint32_t nib[4], sats = 0, e8;
+        uint32_t nib[4], sats = 0, e8, yv[VALS ? 16 : 1];
         if (k_fast_bf(k)) {
             const float invn = inv_nudged(k);
             const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
             const uint32_t limx[4] = {lx, lx, lx, lx};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                nib[c] = nibs4_cvt(w + 4 * c, invn);
+                if constexpr (VALS)
+                    nib[c] = qword4_cvt(w + 4 * c, invn, pow2f_k(k), yv + 4 * c);
+                else
+                    nib[c] = nibs4_cvt(w + 4 * c, invn);
                 const uint32_t a4w[4] = {w[4 * c] & 0x7FFF7FFFu, w[4 * c + 1] & 0x7FFF7FFFu,
                                          w[4 * c + 2] & 0x7FFF7FFFu, w[4 * c + 3] & 0x7FFF7FFFu};
                 sats |= sat8(a4w, limx) << (8 * c);
@@ -1379,8 +1382,19 @@ __global__ void __launch_bounds__(NTHREADS) codes_row_kernel(const KArgs a)
                     make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]), &A, a.mode, a.thr, glutb);
                 nib[c] = gch.nibs;
                 sats |= gch.sats << (8 * c);
+                if constexpr (VALS) {
+                    yv[4 * c] = gch.packed.x;
+                    yv[4 * c + 1] = gch.packed.y;
+                    yv[4 * c + 2] = gch.packed.z;
+                    yv[4 * c + 3] = gch.packed.w;
+                }
             }
             e8 = e8_of(A, k);
+        }
+        if constexpr (VALS) {
+            char* yp = static_cast<char*>(a.y_row) + ((int64_t)row * a.ld_y + 32 * blk) * 2;
+            st_cs_v8(yp, yv);
+            st_cs_v8(yp + 32, yv + 8);
         }
         if (a.codes_row)
             st_stream(a.codes_row + (int64_t)row * (a.cols / 2) + 16 * blk, make_uint4(nib[0], nib[1], nib[2], nib[3]));

@@ -302,6 +302,24 @@ def test_every_bf16_value_as_element_and_as_block_max(mode):
     check_dir(res, ora["row"], "row", 32, label="bf16 sweep")
 
 
+@pytest.mark.parametrize("mode", ["page", "floor"])
+@pytest.mark.parametrize("scales", [False, True])
+def test_every_bf16_value_values_only(mode, scales):
+    """The sweep with dequantised values alone (and with scales): the row-wise
+    kernel for that output mix differs from the one with codes and masks."""
+    xb = bf16_sweep_block32().reshape(-1, 256)
+    x = torch.from_numpy(xb.view(np.int16).copy()).view(torch.bfloat16)
+    xd = x.cuda()
+    r = ops.QDQResult()
+    r.y_row = torch.empty_like(xd)
+    if scales:
+        r.scales_row = torch.empty((xd.shape[0], 8), dtype=torch.uint8, device=xd.device)
+    ops.mxfp4_qdq_fwd(xd, block=32, scale_mode=mode, rowwise=True, out=r)
+    torch.cuda.synchronize()
+    ora = O.qdq_rowwise(oracle_in(x), 32, 6.0, MODES[mode])
+    check_dir(r, ora, "row", 256, label="values only")
+
+
 def codes_only(x: torch.Tensor, mode: str, layout: str):
     res = ops.mxfp4_qdq_fwd(x.cuda(), block=32, scale_mode=mode, rowwise=True, emit_values=False,
                             emit_codes=True, emit_mask=True, scales_layout=layout, check=True)
@@ -550,3 +568,49 @@ def test_full_size_sampled(name):
                                     emit_codes=True, emit_mask=True, check=True)
             _sample_full(x, xd, res, True, True, mode, 32, ends=offsets.numpy(), seed=3)
     torch.cuda.synchronize()
+
+
+def test_cuda_graph_capture_and_replay():
+    """The forward (dual, grouped, all outputs) and the STE backward capture
+    into one CUDA graph: no host synchronisation or allocation on the path.
+    Replays on new inputs copied into the captured buffers give the same
+    bytes as eager calls."""
+    rows, cols, counts = 640, 768, [100, 0, 37, 250, 253]
+    gl = torch.tensor(np.cumsum(counts), dtype=torch.int64, device="cuda")
+    xs = [W.mixed(rows, cols, seed=71 + i, specials=False) for i in range(3)]
+    gs = [torch.randn(rows, cols, generator=torch.Generator().manual_seed(81 + i)).to(torch.bfloat16)
+          for i in range(3)]
+    xd, gd = xs[0].cuda(), gs[0].cuda()
+    r = ops.alloc_outputs(xd, block=32, rowwise=True, colwise=True, num_groups=len(counts), emit_codes=True,
+                          emit_mask=True, with_status=True)
+    gi = torch.empty_like(gd)
+
+    def step():
+        ops.mxfp4_qdq_fwd(xd, rowwise=True, colwise=True, group_list=gl, emit_codes=True, emit_mask=True, out=r)
+        ops.mxfp4_ste_bwd(gd, saved_mask=r.mask_row, clip_grad=True, out=gi)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()  # warm-up outside the capture (kernel attributes, tensor maps)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    names = ("y_row", "y_col", "codes_row", "scales_row", "mask_row", "codes_col", "scales_col", "mask_col")
+    for i in (1, 2, 0):
+        xd.copy_(xs[i].cuda())
+        gd.copy_(gs[i].cuda())
+        graph.replay()
+        torch.cuda.synchronize()
+        got = {n: getattr(r, n).clone() for n in names}
+        got_g = gi.clone()
+        step()
+        torch.cuda.synchronize()
+        for n in names:
+            assert torch.equal(got[n], getattr(r, n)), f"replay {i}: {n}"
+        assert torch.equal(got_g.view(torch.int16), gi.view(torch.int16)), f"replay {i}: grad_in"
+        assert int(r.status.item()) == 0
+    ora = O.qdq_rowwise(oracle_in(xs[0]), 32, 6.0, O.SCALE_PAGE)
+    check_dir(r, ora, "row", cols, label="graph replay")
+    del graph
