@@ -351,7 +351,8 @@ def time_modes(a, xd, gd, res, gi, stream, steps: int = 20):
     events): row-wise fwd with all outputs + STE from the saved mask, the
     training step of the pages' recipe (row-wise fwd, saved-free STE), and the
     real-quantisation producer (row-wise E2M1 codes + E8M0 scales in the
-    block-scaled MMA layout, no dequantised values)."""
+    block-scaled MMA layout, no dequantised values), and blocks of 128 in
+    both directions with every output (ungrouped)."""
     import torch
 
     from mxfp4_block_fake_b200 import _abi, ops
@@ -389,11 +390,21 @@ def time_modes(a, xd, gd, res, gi, stream, steps: int = 20):
     def mma_operand():
         call(_abi.mxfp4_qdq_fwd(margs, sp), "mxfp4_qdq_fwd")
 
+    r128 = ops.alloc_outputs(xd, block=128, rowwise=True, colwise=True, num_groups=0, emit_codes=True,
+                             emit_mask=True)
+    dargs = ops.make_args(xd, block=128, scale_factor=6.0, scale_mode=a.scale_mode,
+                          dirs=_abi.ROWWISE | _abi.COLWISE)
+    ops._fill_outputs(dargs, r128)
+
+    def dual128():
+        call(_abi.mxfp4_qdq_fwd(dargs, sp), "mxfp4_qdq_fwd")
+
     peak, _ = measured_peaks()
     out = {}
     for name, fn, bpe in (("rowwise_fwd_all_outputs_ste_mask", row_step, 4 + 0.5 + 1 / 32 + 0.125 + 4.125),
                           ("training_step_rowwise_fwd_ste_recompute", train_step, 4 + 6),
-                          ("mxfp4_mma_operand_rowwise_codes_scales", mma_operand, 2 + 0.5 + 1 / 32)):
+                          ("mxfp4_mma_operand_rowwise_codes_scales", mma_operand, 2 + 0.5 + 1 / 32),
+                          ("dual_block128_all_outputs", dual128, 2 + 4 + 1 + 2 / 128 + 0.25)):
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
