@@ -47,6 +47,14 @@ def lib() -> ctypes.CDLL:
         L.oracle_qdq_colwise.restype = i32
         L.oracle_ste_bwd.argtypes = [P, i32, i64, i64, P, i32, P]
         L.oracle_ste_bwd.restype = None
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e4m3_encode.argtypes = [f32]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_qdq8_rowwise.argtypes = [P, i32, i64, i64, i64, P, P, P, P]
+        L.oracle_qdq8_rowwise.restype = i32
+        L.oracle_qdq8_colwise.argtypes = [P, i32, i64, i64, i64, P, i64, P, P, P, P]
+        L.oracle_qdq8_colwise.restype = i32
         _lib = L
     return _lib
 
@@ -141,6 +149,44 @@ def qdq_colwise(x: np.ndarray, block: int = 32, scale_factor: float = 6.0, mode:
     return dict(y=y, codes=codes, scales=scales, mask=mask)
 
 
+def qdq8_rowwise(x: np.ndarray):
+    """Row-wise MXFP8 QDQ (E4M3 elements, E8M0 scale per 32): dict(y, codes
+    [rows, cols] bytes, scales [rows, ceil(cols/32)], mask)."""
+    x = np.ascontiguousarray(x)
+    dt = _dtype_code(x)
+    rows, cols = x.shape
+    y = np.empty_like(x)
+    codes = np.zeros((rows, cols), np.uint8)
+    scales = np.zeros((rows, (cols + 31) // 32), np.uint8)
+    mask = np.zeros((rows, (cols + 7) // 8), np.uint8)
+    lib().oracle_qdq8_rowwise(_ptr(x), dt, rows, cols, cols, _ptr(y), _ptr(codes), _ptr(scales), _ptr(mask))
+    return dict(y=y, codes=codes, scales=scales, mask=mask)
+
+
+def qdq8_colwise(x: np.ndarray, ends=None):
+    """Column-wise MXFP8 QDQ (blocks of 32 rows restarting at group ends)."""
+    x = np.ascontiguousarray(x)
+    dt = _dtype_code(x)
+    rows, cols = x.shape
+    e = None if ends is None else np.ascontiguousarray(ends, dtype=np.int64)
+    s = colwise_scale_rows(e if e is not None else np.array([rows], np.int64), 32)
+    y = np.empty_like(x)
+    codes = np.zeros((rows, cols), np.uint8)
+    scales = np.zeros((s, cols), np.uint8)
+    mask = np.zeros((rows, (cols + 7) // 8), np.uint8)
+    lib().oracle_qdq8_colwise(_ptr(x), dt, rows, cols, cols, _ptr(e), 0 if e is None else e.size,
+                              _ptr(y), _ptr(codes), _ptr(scales), _ptr(mask))
+    return dict(y=y, codes=codes, scales=scales, mask=mask)
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().oracle_e4m3_value(code & 0x7F)) * (-1.0 if code & 0x80 else 1.0)
+
+
+def e4m3_encode(y: float) -> int:
+    return int(lib().oracle_e4m3_encode(y))
+
+
 def ste_bwd(grad_out: np.ndarray, mask: np.ndarray, clip_grad: bool = True) -> np.ndarray:
     g = np.ascontiguousarray(grad_out)
     dt = _dtype_code(g)
@@ -189,5 +235,6 @@ def unpack_nibbles(codes: np.ndarray, cols: int) -> np.ndarray:
 __all__ = [
     "F32", "BF16", "SCALE_PAGE", "SCALE_FLOOR", "lib", "build", "bf16_to_f32", "f32_to_bf16",
     "scale_page", "scale_floor", "qdq_block", "group_ends", "colwise_scale_rows", "qdq_rowwise",
-    "qdq_colwise", "ste_bwd", "unpack_bits", "unpack_nibbles", "mma_scale_layout",
+    "qdq_colwise", "ste_bwd", "unpack_bits", "unpack_nibbles", "mma_scale_layout", "qdq8_rowwise",
+    "qdq8_colwise", "e4m3_value", "e4m3_encode",
 ]

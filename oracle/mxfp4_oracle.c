@@ -388,6 +388,157 @@ int oracle_qdq_colwise(const void* x, int dtype, int64_t rows, int64_t cols, int
     return 0;
 }
 
+/* ---- MXFP8: E4M3 elements with E8M0 block scales ------------------------- */
+/*
+ * [GMM] FakeW4A8GroupedLinear quantises activations and gradients to MXFP8
+ * (E4M3 elements, one E8M0 scale per 32 elements) but the page only names the
+ * NPU operators. Reading: the OCP Microscaling format rule, the same rule as
+ * scale_mode FLOOR above with the element type's largest exponent:
+ *   scale  = 2^(floor(log2 amax) - 8), saturated below at 2^-127
+ *            (E4M3's largest normal is 1.75 * 2^8 = 448);
+ *   code   = the E4M3 value nearest to x / scale, ties to the even code,
+ *            magnitudes above 448 saturating to 448, the sign kept (so -0 and
+ *            negative values that round to zero give the code 0x80);
+ *   out    = decode(code) * scale, cast to the input dtype;
+ *   sat    = |x| > 448 * scale.
+ * Non-finite blocks follow the MXFP4 convention: NaN outputs, code 0, E8M0
+ * 0xFF, no saturation.
+ */
+
+/* E4M3 (OCP "E4M3FN"): sign, 4 exponent bits (bias 7), 3 mantissa bits; no
+ * infinities; S.1111.111 is NaN. Value of a code without its sign bit. */
+double oracle_e4m3_value(uint8_t c)
+{
+    int e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        return ldexp((double)m, -9);      /* subnormal: m * 2^-9 */
+    return ldexp(1.0 + m / 8.0, e - 7);   /* normal: (1 + m/8) * 2^(e-7) */
+}
+
+/* Nearest E4M3 code to a finite y: search of the 127 finite magnitudes, ties
+ * to the even code, saturation at 448, sign bit from y. */
+uint8_t oracle_e4m3_encode(float y)
+{
+    double a = fabs((double)y);
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double d = fabs(a - oracle_e4m3_value((uint8_t)c));
+        if (d < bd || (d == bd && (c & 1) == 0 && (best & 1) != 0)) {
+            bd = d;
+            best = c;
+        }
+    }
+    if (a > 448.0)
+        best = 0x7E;
+    return (uint8_t)(best | (signbit(y) ? 0x80 : 0));
+}
+
+void oracle_qdq8_block(const float* v, int n, float* out, uint8_t* code, uint8_t* sat, uint8_t* e8m0)
+{
+    float amax = block_amax(v, n);
+    double e = floor(log2((double)amax)) - 8.0; /* -inf at 0, NaN at NaN, +inf at inf */
+    if (e < -127.0)
+        e = -127.0;
+    float scale = (float)exp2(e);
+    float limit = 448.0f * scale;
+    for (int i = 0; i < n; ++i) {
+        if (!isfinite(scale)) {
+            out[i] = canonical_nan();
+            code[i] = 0;
+            sat[i] = 0;
+            continue;
+        }
+        float y = v[i] / scale; /* exact scaling by a power of two, rounded once */
+        uint8_t c = oracle_e4m3_encode(y);
+        double q = oracle_e4m3_value((uint8_t)(c & 0x7F));
+        out[i] = (float)((c & 0x80 ? -q : q) * (double)scale); /* exact in fp32 */
+        code[i] = c;
+        sat[i] = fabsf(v[i]) > limit ? 1 : 0;
+    }
+    *e8m0 = e8m0_of(scale);
+}
+
+/* Row-wise MXFP8 QDQ, blocks of 32 along a row; codes [rows][cols] bytes,
+ * the other outputs as in oracle_qdq_rowwise. */
+int oracle_qdq8_rowwise(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                        void* y, uint8_t* codes, uint8_t* scales, uint8_t* mask)
+{
+    const int block = 32;
+    float v[32], o[32];
+    uint8_t cd[32], st[32];
+    int64_t nblk = (cols + block - 1) / block, mstride = (cols + 7) / 8;
+    if (mask)
+        memset(mask, 0, (size_t)(rows * mstride));
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nblk; ++b) {
+            int64_t c0 = b * block;
+            int n = (int)((cols - c0) < block ? (cols - c0) : block);
+            for (int i = 0; i < n; ++i)
+                v[i] = load_elem(x, dtype, r * ld + c0 + i);
+            uint8_t e8;
+            oracle_qdq8_block(v, n, o, cd, st, &e8);
+            for (int i = 0; i < n; ++i) {
+                if (y)
+                    store_elem(y, dtype, r * cols + c0 + i, o[i]);
+                if (codes)
+                    codes[r * cols + c0 + i] = cd[i];
+                if (mask)
+                    put_bit(mask + r * mstride, c0 + i, st[i]);
+            }
+            if (scales)
+                scales[r * nblk + b] = e8;
+        }
+    }
+    return 0;
+}
+
+/* Column-wise MXFP8 QDQ, blocks of 32 rows restarting at group starts; codes
+ * [rows][cols] bytes, the other outputs as in oracle_qdq_colwise. */
+int oracle_qdq8_colwise(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                        const int64_t* ends, int64_t num_groups,
+                        void* y, uint8_t* codes, uint8_t* scales, uint8_t* mask)
+{
+    const int block = 32;
+    float v[32], o[32];
+    uint8_t cd[32], st[32];
+    int64_t one_end = rows;
+    if (!ends) {
+        ends = &one_end;
+        num_groups = 1;
+    }
+    int64_t mstride = (cols + 7) / 8;
+    if (mask)
+        memset(mask, 0, (size_t)(rows * mstride));
+    int64_t srow = 0, start = 0;
+    for (int64_t g = 0; g < num_groups; ++g) {
+        for (int64_t r0 = start; r0 < ends[g]; r0 += block, ++srow) {
+            int n = (int)((ends[g] - r0) < block ? (ends[g] - r0) : block);
+            for (int64_t c = 0; c < cols; ++c) {
+                for (int i = 0; i < n; ++i)
+                    v[i] = load_elem(x, dtype, (r0 + i) * ld + c);
+                uint8_t e8;
+                oracle_qdq8_block(v, n, o, cd, st, &e8);
+                for (int i = 0; i < n; ++i) {
+                    int64_t r = r0 + i;
+                    if (y)
+                        store_elem(y, dtype, r * cols + c, o[i]);
+                    if (codes)
+                        codes[r * cols + c] = cd[i];
+                    if (mask)
+                        put_bit(mask + r * mstride, c, st[i]);
+                }
+                if (scales)
+                    scales[srow * cols + c] = e8;
+            }
+        }
+        start = ends[g];
+    }
+    return 0;
+}
+
 /*
  * [QAT] _MXFP4FakeQuantSTE.backward: plain STE returns grad_out unchanged;
  * clipped STE writes 0.0 where the saturation mask is set
