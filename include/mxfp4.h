@@ -108,11 +108,26 @@ typedef enum {
 /* Largest num_groups a call accepts. */
 #define MXFP4_MAX_GROUPS 4096
 
+/* Element formats (mxfp4_qdq_args.elem_format). E4M3 is the MXFP8 element of
+ * the W4A8 path (MindSpore hyper-parallel fake_w4a8_gmm_func.py,
+ * FakeW4A8GroupedLinear, which quantises activations and gradients to MXFP8;
+ * the page names the operators only). Its reading is the OCP Microscaling
+ * rule: scale 2^(floor(log2 amax) - 8) saturated below at 2^-127 (E4M3's
+ * largest normal is 1.75 * 2^8 = 448), each x / scale rounded to the nearest
+ * E4M3 value with ties to the even code and magnitudes above 448 saturating
+ * to 448, the sign kept (-0 and negative values rounding to zero give code
+ * 0x80); output decode(code) * scale in x's dtype; saturation |x| > 448 *
+ * scale. E4M3 requires block 32 and MXFP4_SCALE_FLOOR (else
+ * MXFP4_EUNSUPPORTED); its codes are one byte per element, [rows][cols] for
+ * both directions. Non-finite blocks as for E2M1. */
+#define MXFP4_ELEM_E2M1 0
+#define MXFP4_ELEM_E4M3 1
+
 /* Layouts of scales_row (mxfp4_qdq_args.scales_row_layout). */
 #define MXFP4_SCALES_ROWMAJOR 0
 #define MXFP4_SCALES_MMA 1
 
-#define MXFP4_ABI_VERSION 2
+#define MXFP4_ABI_VERSION 3
 
 /*
  * Arguments of one QDQ call. Zero-initialise and fill what is used; every
@@ -136,6 +151,7 @@ typedef enum {
  *                  latter, with block 32, gives the E8M0 operand scales of an
  *                  MXFP4 block-scaled GEMM whose K dimension is `cols`
  *                  (codes_row is then its K-major E2M1 operand as is).
+ *   elem_format    MXFP4_ELEM_E2M1 (0, MXFP4) or MXFP4_ELEM_E4M3 (MXFP8).
  */
 typedef struct mxfp4_qdq_args {
     const void* x;
@@ -161,6 +177,7 @@ typedef struct mxfp4_qdq_args {
     uint8_t* scales_col;
     uint8_t* mask_col;
     int32_t scales_row_layout;
+    int32_t elem_format;
 } mxfp4_qdq_args;
 
 /*

@@ -18,8 +18,9 @@ F32, BF16 = 0, 1
 SCALE_PAGE, SCALE_FLOOR = 0, 1
 ROWWISE, COLWISE = 1, 2
 SCALES_ROWMAJOR, SCALES_MMA = 0, 1
+ELEM_E2M1, ELEM_E4M3 = 0, 1
 MAX_GROUPS = 4096
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 # Every symbol include/mxfp4.h declares.
 EXPORTS = (
@@ -59,6 +60,7 @@ class QdqArgs(ctypes.Structure):
         ("scales_col", ctypes.c_void_p),
         ("mask_col", ctypes.c_void_p),
         ("scales_row_layout", ctypes.c_int32),
+        ("elem_format", ctypes.c_int32),
     ]
 
 

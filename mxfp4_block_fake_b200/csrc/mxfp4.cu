@@ -68,6 +68,7 @@ struct KArgs {
     uint32_t thr;   // PAGE mode: fp32 bits of T0 (see qparams)
     uint32_t ts_flags;  // staged kernel: column-wise outputs written by TMA stores (SG_TS_*)
     int32_t srow_mma;   // scales_row in the MMA scale-factor layout (MXFP4_SCALES_MMA)
+    int32_t fmt;        // MXFP4_ELEM_E2M1 or MXFP4_ELEM_E4M3
 };
 
 // Byte offset of row-wise scale (row, b) of a [rows][nblk] scale matrix:
@@ -151,6 +152,52 @@ __device__ __forceinline__ uint32_t qdq_elem(uint32_t xb, const BP& p, uint32_t&
     nib = (neg >> 28) | i;
     sat = (xb & 0x7FFFFFFFu) > p.lim ? 1u : 0u;
     return __float_as_uint(o);
+}
+
+// ---------------------------------------------------------------------------
+// MXFP8: E4M3 elements (scale mode FLOOR, block 32)
+// ---------------------------------------------------------------------------
+
+// k = floor(log2 amax) - 8 from the biased exponent (E4M3's largest normal is
+// 1.75 * 2^8 = 448), saturated at -127 (subnormal and zero amax included).
+__device__ __forceinline__ int k_e4m3(uint32_t A) { return max((int)(A >> 23) - 135, -127); }
+
+__device__ __forceinline__ BP block_params8(uint32_t A)
+{
+    const bool special = A >= 0x7F800000u;
+    const int k = special ? 0 : k_e4m3(A);
+    BP p;
+    p.inv = __uint_as_float(pow2_bits(-k));
+    p.scale = __uint_as_float(pow2_bits(k));
+    p.lim = ((uint32_t)(k + 135) << 23) | 0x00600000u;  // fp32 bits of 448 * 2^k = 1.75 * 2^(k + 8)
+    p.nanm = special ? 0xFFFFFFFFu : 0u;
+    p.e8 = special ? 0xFFu : (uint32_t)(k + 127);
+    return p;
+}
+
+// One element: fp32 bits of decode(code) * 2^k (exact: codes have four
+// significant bits and 2^k >= 2^-127), the E4M3 code of y = x * 2^-k by the
+// hardware convert (nearest even, saturating at 448, sign kept) and the
+// saturation flag.
+__device__ __forceinline__ uint32_t qdq8_elem(uint32_t xb, const BP& p, uint32_t& code, uint32_t& sat)
+{
+    const float y = __fmul_rn(__uint_as_float(xb), p.inv);
+    uint16_t q;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(q) : "f"(0.0f), "f"(y));
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(q));
+    float c;
+    asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %1;\n\tcvt.f32.f16 %0, l;\n\t}" : "=f"(c) : "r"(h));
+    code = q & 0xFFu;
+    sat = (xb & 0x7FFFFFFFu) > p.lim ? 1u : 0u;
+    return __float_as_uint(__fmul_rn(c, p.scale));
+}
+
+// fp32 bits -> the same bits rounded to bf16 (nearest even) in the top half;
+// finite values only.
+__device__ __forceinline__ uint32_t round_bf16_bits(uint32_t b)
+{
+    return (b + 0x7FFFu + ((b >> 16) & 1u)) & 0xFFFF0000u;
 }
 
 // ---------------------------------------------------------------------------
@@ -938,8 +985,8 @@ __device__ __forceinline__ void store_bits(void* base, int64_t i, uint32_t v)
         static_cast<uint32_t*>(base)[i] = v;
 }
 
-// One thread per (row, row-wise block).
-template <int ESZ, int BS, bool GRAD>
+// One thread per (row, row-wise block). FMT: MXFP4_ELEM_E2M1 or _E4M3.
+template <int ESZ, int BS, bool GRAD, int FMT>
 __global__ void __launch_bounds__(NTHREADS) generic_row_kernel(const KArgs a)
 {
     const int64_t nblk = (a.cols + BS - 1) / BS;
@@ -954,11 +1001,14 @@ __global__ void __launch_bounds__(NTHREADS) generic_row_kernel(const KArgs a)
         uint32_t am = 0;
         for (int j = 0; j < n; ++j)
             am = max(am, load_bits<ESZ>(a.x, xo + j) & 0x7FFFFFFFu);
-        const BP p = block_params(am, a.mode, a.sf);
+        const BP p = FMT == MXFP4_ELEM_E4M3 ? block_params8(am) : block_params(am, a.mode, a.sf);
         uint32_t nacc = 0, sacc = 0;
         for (int j = 0; j < n; ++j) {
             uint32_t nb, st;
-            uint32_t ob = qdq_elem(load_bits<ESZ>(a.x, xo + j), p, nb, st);
+            uint32_t ob = FMT == MXFP4_ELEM_E4M3 ? qdq8_elem(load_bits<ESZ>(a.x, xo + j), p, nb, st)
+                                                : qdq_elem(load_bits<ESZ>(a.x, xo + j), p, nb, st);
+            if (FMT == MXFP4_ELEM_E4M3 && ESZ == 2)
+                ob = round_bf16_bits(ob);
             if (p.nanm) {
                 ob = QNAN32;
                 nb = 0;
@@ -966,9 +1016,11 @@ __global__ void __launch_bounds__(NTHREADS) generic_row_kernel(const KArgs a)
             }
             if (a.y_row)
                 store_bits<ESZ>(a.y_row, row * a.ld_y + c0 + j, ob);
+            if (FMT == MXFP4_ELEM_E4M3 && a.codes_row)
+                a.codes_row[row * a.cols + c0 + j] = (uint8_t)nb;
             nacc |= nb << (4 * (j & 1));
             sacc |= st << (j & 7);
-            if (a.codes_row && ((j & 1) || j == n - 1))
+            if (FMT == MXFP4_ELEM_E2M1 && a.codes_row && ((j & 1) || j == n - 1))
                 a.codes_row[row * cstride + (c0 + j) / 2] = (uint8_t)nacc;
             if ((j & 1) || j == n - 1)
                 nacc = 0;
@@ -988,7 +1040,7 @@ __global__ void __launch_bounds__(NTHREADS) generic_row_kernel(const KArgs a)
 
 // One thread per (column-wise block, 8 adjacent columns): whole code and mask
 // bytes are owned by one thread.
-template <int ESZ, int BS, bool GROUPS, bool GRAD>
+template <int ESZ, int BS, bool GROUPS, bool GRAD, int FMT>
 __global__ void __launch_bounds__(NTHREADS) generic_col_kernel(const KArgs a)
 {
     extern __shared__ int32_t s_plan[];
@@ -1033,7 +1085,7 @@ __global__ void __launch_bounds__(NTHREADS) generic_col_kernel(const KArgs a)
         BP p[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-            p[c] = block_params(am[c], a.mode, a.sf);
+            p[c] = FMT == MXFP4_ELEM_E4M3 ? block_params8(am[c]) : block_params(am[c], a.mode, a.sf);
         for (int r = 0; r < nrows; ++r) {
             const int64_t row = row0 + r;
             uint32_t nibs = 0, sats = 0;
@@ -1042,7 +1094,10 @@ __global__ void __launch_bounds__(NTHREADS) generic_col_kernel(const KArgs a)
                 if (c >= nc)
                     continue;
                 uint32_t nb, st;
-                uint32_t ob = qdq_elem(load_bits<ESZ>(a.x, row * a.ld + c0 + c), p[c], nb, st);
+                uint32_t ob = FMT == MXFP4_ELEM_E4M3 ? qdq8_elem(load_bits<ESZ>(a.x, row * a.ld + c0 + c), p[c], nb, st)
+                                                    : qdq_elem(load_bits<ESZ>(a.x, row * a.ld + c0 + c), p[c], nb, st);
+                if (FMT == MXFP4_ELEM_E4M3 && ESZ == 2)
+                    ob = round_bf16_bits(ob);
                 if (p[c].nanm) {
                     ob = QNAN32;
                     nb = 0;
@@ -1050,6 +1105,8 @@ __global__ void __launch_bounds__(NTHREADS) generic_col_kernel(const KArgs a)
                 }
                 if (a.y_col)
                     store_bits<ESZ>(a.y_col, row * a.ld_y + c0 + c, ob);
+                if (FMT == MXFP4_ELEM_E4M3 && a.codes_col)
+                    a.codes_col[row * a.cols + c0 + c] = (uint8_t)nb;
                 nibs |= nb << (4 * c);
                 sats |= st << c;
                 if (GRAD && a.grad_dir == MXFP4_COLWISE) {
@@ -1057,7 +1114,7 @@ __global__ void __launch_bounds__(NTHREADS) generic_col_kernel(const KArgs a)
                     store_bits<ESZ>(a.g_in, gi, st ? 0u : load_bits<ESZ>(a.g_out, gi));
                 }
             }
-            if (a.codes_col) {
+            if (FMT == MXFP4_ELEM_E2M1 && a.codes_col) {
                 for (int j = 0; j < (nc + 1) / 2; ++j)
                     a.codes_col[row * cstride + c0 / 2 + j] = (uint8_t)(nibs >> (8 * j));
             }
@@ -1247,28 +1304,43 @@ static KernelFn pick_tile_shape(bool row, bool col, bool groups, bool grad, int&
                 : pick_tile<ESZ, BS, TS::LC, TS::RPT, TS::WR, false>(row, col, groups);
 }
 
-static KernelFn pick_generic_row(int esz, int bs, bool grad)
+template <int FMT>
+static KernelFn pick_generic_row_f(int esz, int bs, bool grad)
 {
+    if (FMT == MXFP4_ELEM_E4M3)  // block 32 only
+        return esz == 2 ? (grad ? generic_row_kernel<2, 32, true, FMT> : generic_row_kernel<2, 32, false, FMT>)
+                        : (grad ? generic_row_kernel<4, 32, true, FMT> : generic_row_kernel<4, 32, false, FMT>);
     if (esz == 2)
-        return bs == 32 ? (grad ? generic_row_kernel<2, 32, true> : generic_row_kernel<2, 32, false>)
-                        : (grad ? generic_row_kernel<2, 128, true> : generic_row_kernel<2, 128, false>);
-    return bs == 32 ? (grad ? generic_row_kernel<4, 32, true> : generic_row_kernel<4, 32, false>)
-                    : (grad ? generic_row_kernel<4, 128, true> : generic_row_kernel<4, 128, false>);
+        return bs == 32 ? (grad ? generic_row_kernel<2, 32, true, FMT> : generic_row_kernel<2, 32, false, FMT>)
+                        : (grad ? generic_row_kernel<2, 128, true, FMT> : generic_row_kernel<2, 128, false, FMT>);
+    return bs == 32 ? (grad ? generic_row_kernel<4, 32, true, FMT> : generic_row_kernel<4, 32, false, FMT>)
+                    : (grad ? generic_row_kernel<4, 128, true, FMT> : generic_row_kernel<4, 128, false, FMT>);
 }
 
-template <int ESZ, int BS>
+static KernelFn pick_generic_row(int esz, int bs, bool grad, int fmt)
+{
+    return fmt == MXFP4_ELEM_E4M3 ? pick_generic_row_f<MXFP4_ELEM_E4M3>(esz, bs, grad)
+                                  : pick_generic_row_f<MXFP4_ELEM_E2M1>(esz, bs, grad);
+}
+
+template <int ESZ, int BS, int FMT>
 static KernelFn pick_generic_col_bs(bool groups, bool grad)
 {
     if (groups)
-        return grad ? generic_col_kernel<ESZ, BS, true, true> : generic_col_kernel<ESZ, BS, true, false>;
-    return grad ? generic_col_kernel<ESZ, BS, false, true> : generic_col_kernel<ESZ, BS, false, false>;
+        return grad ? generic_col_kernel<ESZ, BS, true, true, FMT> : generic_col_kernel<ESZ, BS, true, false, FMT>;
+    return grad ? generic_col_kernel<ESZ, BS, false, true, FMT> : generic_col_kernel<ESZ, BS, false, false, FMT>;
 }
 
-static KernelFn pick_generic_col(int esz, int bs, bool groups, bool grad)
+static KernelFn pick_generic_col(int esz, int bs, bool groups, bool grad, int fmt)
 {
+    if (fmt == MXFP4_ELEM_E4M3)  // block 32 only
+        return esz == 2 ? pick_generic_col_bs<2, 32, MXFP4_ELEM_E4M3>(groups, grad)
+                        : pick_generic_col_bs<4, 32, MXFP4_ELEM_E4M3>(groups, grad);
     if (esz == 2)
-        return bs == 32 ? pick_generic_col_bs<2, 32>(groups, grad) : pick_generic_col_bs<2, 128>(groups, grad);
-    return bs == 32 ? pick_generic_col_bs<4, 32>(groups, grad) : pick_generic_col_bs<4, 128>(groups, grad);
+        return bs == 32 ? pick_generic_col_bs<2, 32, MXFP4_ELEM_E2M1>(groups, grad)
+                        : pick_generic_col_bs<2, 128, MXFP4_ELEM_E2M1>(groups, grad);
+    return bs == 32 ? pick_generic_col_bs<4, 32, MXFP4_ELEM_E2M1>(groups, grad)
+                    : pick_generic_col_bs<4, 128, MXFP4_ELEM_E2M1>(groups, grad);
 }
 
 static mxfp4_status launch(KernelFn fn, int64_t work_units, size_t smem, const KArgs& k, cudaStream_t s)
@@ -1497,6 +1569,22 @@ static mxfp4_status launch_row_stream(const KArgs& k, int64_t blocks, cudaStream
                                                                                                : MXFP4_ECUDA;
 }
 
+static mxfp4_status launch_row_stream8(const KArgs& k, int64_t blocks, cudaStream_t s)
+{
+    const void* fn = k.srow_mma && k.scales_row ? (const void*)row_stream8_kernel<true>
+                                                : (const void*)row_stream8_kernel<false>;
+    const int sms = device_sms();
+    const int occ = occupancy(fn, 0);
+    if (sms <= 0 || occ <= 0)
+        return MXFP4_ECUDA;
+    int64_t grid = (int64_t)sms * occ;
+    if ((blocks + NTHREADS - 1) / NTHREADS < grid)
+        grid = (blocks + NTHREADS - 1) / NTHREADS;
+    void* args[] = {const_cast<KArgs*>(&k)};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(NTHREADS), args, 0, s) == cudaSuccess ? MXFP4_OK
+                                                                                               : MXFP4_ECUDA;
+}
+
 static mxfp4_status check_geometry(const mxfp4_qdq_args* a)
 {
     if (!a)
@@ -1519,6 +1607,10 @@ static mxfp4_status check_geometry(const mxfp4_qdq_args* a)
         return MXFP4_EINVAL;
     if (a->scales_row_layout != MXFP4_SCALES_ROWMAJOR && a->scales_row_layout != MXFP4_SCALES_MMA)
         return MXFP4_EINVAL;
+    if (a->elem_format != MXFP4_ELEM_E2M1 && a->elem_format != MXFP4_ELEM_E4M3)
+        return MXFP4_EINVAL;
+    if (a->elem_format == MXFP4_ELEM_E4M3 && (a->block != 32 || a->scale_mode != MXFP4_SCALE_FLOOR))
+        return MXFP4_EUNSUPPORTED;
     if (a->group_list) {
         if (a->num_groups < 1)
             return MXFP4_EINVAL;
@@ -1580,6 +1672,7 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
         k.mask_col = A->mask_col;
     }
     k.ld_y = A->ld_y;
+    k.fmt = A->elem_format;
     if ((k.y_row || k.y_col) && A->ld_y < A->cols)
         return MXFP4_EINVAL;
     if ((k.y_row && !aligned(k.y_row, esz)) || (k.y_col && !aligned(k.y_col, esz)))
@@ -1615,6 +1708,42 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     const int bs = A->block;
     const size_t plan_smem = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
     const int64_t s_bound = groups ? A->rows / bs + A->num_groups : (A->rows + bs - 1) / bs;
+
+    if (k.fmt == MXFP4_ELEM_E4M3 && esz == 2 && !grad) {
+        // MXFP8, bf16: the row-wise part on the streaming kernel, the
+        // column-wise part on the column-pair kernel, where their layout
+        // conditions hold; the rest on the generic kernels
+        const bool row8 = row && fast && A->cols % 32 == 0 && A->ld % 16 == 0 && aligned(A->x, 32) &&
+                          (!k.y_row || (aligned(k.y_row, 32) && A->ld_y % 16 == 0)) &&
+                          (!k.codes_row || aligned(k.codes_row, 32)) && (!k.mask_row || aligned(k.mask_row, 4)) &&
+                          A->rows * (A->cols / 32) < (int64_t)UINT32_MAX;
+        const bool col8 = col && A->cols % 8 == 0 && A->ld % 2 == 0 && aligned(A->x, 4) &&
+                          (!k.y_col || (aligned(k.y_col, 4) && A->ld_y % 2 == 0)) &&
+                          (!k.codes_col || aligned(k.codes_col, 2)) && (!k.scales_col || aligned(k.scales_col, 2));
+        if (row8 || col8) {
+            if (row) {
+                KArgs kr = k;
+                kr.y_col = nullptr;
+                kr.codes_col = kr.scales_col = kr.mask_col = nullptr;
+                st = row8 ? launch_row_stream8(kr, A->rows * (A->cols / 32), s)
+                          : launch(pick_generic_row(esz, bs, false, k.fmt),
+                                   (A->rows * ((A->cols + bs - 1) / bs) + NTHREADS - 1) / NTHREADS, 0, kr, s);
+                if (st != MXFP4_OK)
+                    return st;
+            }
+            if (col) {
+                const int64_t units = s_bound * ((A->cols + 7) / 8);
+                if (col8)
+                    return launch(groups ? col_pair8_kernel<true> : col_pair8_kernel<false>,
+                                  (s_bound * (A->cols / 2) + NTHREADS - 1) / NTHREADS, plan_smem, k, s);
+                return launch(pick_generic_col(esz, bs, groups, false, k.fmt), (units + NTHREADS - 1) / NTHREADS,
+                              plan_smem, k, s);
+            }
+            return st;
+        }
+    }
+    if (k.fmt == MXFP4_ELEM_E4M3)
+        fast = false;  // MXFP8 otherwise: the generic kernels below
 
     // row-wise only, bf16 block 32, with codes or masks (or without values):
     // one streaming pass, one thread per block. Values alone go to the staged
@@ -1669,14 +1798,14 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     if (row) {
         KArgs kr = k;
         kr.y_col = nullptr;
-        st = launch(pick_generic_row(esz, bs, grad && grad_dir == MXFP4_ROWWISE),
+        st = launch(pick_generic_row(esz, bs, grad && grad_dir == MXFP4_ROWWISE, k.fmt),
                     (A->rows * ((A->cols + bs - 1) / bs) + NTHREADS - 1) / NTHREADS, 0, kr, s);
         if (st != MXFP4_OK)
             return st;
     }
     if (col) {
         const int64_t units = s_bound * ((A->cols + 7) / 8);
-        st = launch(pick_generic_col(esz, bs, groups, grad && grad_dir == MXFP4_COLWISE),
+        st = launch(pick_generic_col(esz, bs, groups, grad && grad_dir == MXFP4_COLWISE, k.fmt),
                     (units + NTHREADS - 1) / NTHREADS, plan_smem, k, s);
     }
     return st;
@@ -1720,6 +1849,7 @@ mxfp4_status mxfp4_ste_bwd(const mxfp4_qdq_args* geom, const void* grad_out, voi
     if (!grad_out || !grad_in || ld_grad < geom->cols || !aligned(grad_out, esz) || !aligned(grad_in, esz))
         return MXFP4_EINVAL;
     if (clip_grad && !saved_mask && geom->dirs == MXFP4_ROWWISE && esz == 2 && geom->block == 32 &&
+        geom->elem_format == MXFP4_ELEM_E2M1 &&
         geom->cols % 32 == 0 && geom->x && geom->ld >= geom->cols && geom->ld % 16 == 0 && ld_grad % 16 == 0 &&
         ((uintptr_t)geom->x | (uintptr_t)grad_out | (uintptr_t)grad_in) % 32 == 0 &&
         geom->rows * (geom->cols / 32) < (int64_t)UINT32_MAX &&

@@ -1405,4 +1405,200 @@ __global__ void __launch_bounds__(NTHREADS) row_stream_kernel(const KArgs a)
     }
 }
 
+// ---------------------------------------------------------------------------
+// MXFP8 row-wise, bf16, block 32, one streaming pass: one thread per block,
+// two 32-byte loads, amax and k (floor(log2 amax) - 8, at least -127), per
+// pair of elements one E4M3 convert (nearest even, saturating at 448) and one
+// back to exact f16 codes, widened and multiplied by 2^k (exact), then the
+// outputs asked for: two 32-byte stores of values, one 32-byte store of codes,
+// a 4-byte mask word, a scale byte (SMMA: MMA layout). Non-finite blocks:
+// NaN values, codes 0, no saturation, E8M0 0xFF.
+// ---------------------------------------------------------------------------
+
+template <bool SMMA>
+__global__ void __launch_bounds__(NTHREADS) row_stream8_kernel(const KArgs a)
+{
+    const uint32_t nb = (uint32_t)(a.cols / 32);
+    const uint32_t total = (uint32_t)a.rows * nb;
+    for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < total; u += gridDim.x * blockDim.x) {
+        const uint32_t row = u / nb, blk = u - row * nb;
+        const char* xp = static_cast<const char*>(a.x) + ((int64_t)row * a.ld + 32 * blk) * 2;
+        uint32_t w[16];
+        ld_nc_v8(xp, w);
+        ld_nc_v8(xp + 32, w + 8);
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            m2 = vmax2(m2, w[i] & 0x7FFF7FFFu);
+        const uint32_t A = max(m2 & 0xFFFFu, m2 >> 16) << 16;
+        uint32_t yv[16], cw[8], sats = 0, e8;
+        if (A < 0x7F800000u) {
+            const int k = k_e4m3(A);
+            const float inv = __uint_as_float(pow2_bits(-k)), sc = __uint_as_float(pow2_bits(k));
+            uint32_t q[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float ylo = __fmul_rn(__uint_as_float(w[i] << 16), inv);
+                const float yhi = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
+                uint16_t qq;
+                asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(qq) : "f"(yhi), "f"(ylo));
+                uint32_t h;
+                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(qq));
+                float clo, chi;
+                asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+                    : "=f"(clo), "=f"(chi)
+                    : "r"(h));
+                // exact products with at most four significant bits: bf16 keeps them
+                yv[i] = __byte_perm(__float_as_uint(__fmul_rn(clo, sc)), __float_as_uint(__fmul_rn(chi, sc)), 0x7632);
+                q[i] = qq;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                cw[j] = q[2 * j] | (q[2 * j + 1] << 16);
+            // bf16 bits of 448 * 2^k = 1.75 * 2^(k + 8)
+            const uint32_t lx = (0x8000u + (((uint32_t)(k + 135) << 7) | 0x60u)) * 0x10001u;
+            const uint32_t limx[4] = {lx, lx, lx, lx};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint32_t a4w[4] = {w[4 * c] & 0x7FFF7FFFu, w[4 * c + 1] & 0x7FFF7FFFu,
+                                         w[4 * c + 2] & 0x7FFF7FFFu, w[4 * c + 3] & 0x7FFF7FFFu};
+                sats |= sat8(a4w, limx) << (8 * c);
+            }
+            e8 = (uint32_t)(k + 127);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                yv[i] = 0x7FC07FC0u;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                cw[j] = 0u;
+            e8 = 0xFFu;
+        }
+        if (a.y_row) {
+            char* yp = static_cast<char*>(a.y_row) + ((int64_t)row * a.ld_y + 32 * blk) * 2;
+            st_cs_v8(yp, yv);
+            st_cs_v8(yp + 32, yv + 8);
+        }
+        if (a.codes_row)
+            st_cs_v8(a.codes_row + (int64_t)row * a.cols + 32 * blk, cw);
+        if (a.mask_row)
+            *reinterpret_cast<uint32_t*>(a.mask_row + (int64_t)row * (a.cols / 8) + 4 * blk) = sats;
+        if (a.scales_row)
+            a.scales_row[SMMA ? srow_off_mma(row, blk, nb) : (int64_t)row * nb + blk] = (uint8_t)e8;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// MXFP8 column-wise, bf16, block 32 with group restarts: one thread per
+// (column-wise block, column pair). Consecutive lanes take consecutive column
+// pairs of the same block, so every load and store of a warp is one
+// contiguous row segment (128 bytes of x or y). A lane keeps its 32 words in
+// registers: amax of both columns, k, then per row the E4M3 pair convert, the
+// exact dequantisation, the 2-byte code store; the saturation bits of four
+// lanes (8 columns) are OR-ed by two shuffles into the mask byte of each row.
+// Requires cols % 8 == 0 (a mask byte's four lanes share a block), 4-byte
+// aligned x / y rows and 2-byte aligned codes and scales.
+// ---------------------------------------------------------------------------
+
+template <bool GROUPS>
+__global__ void __launch_bounds__(NTHREADS) col_pair8_kernel(const KArgs a)
+{
+    extern __shared__ int32_t s_plan8[];
+    int32_t* s_bpre = s_plan8;
+    int32_t* s_rst = s_plan8 + (GROUPS ? a.num_groups + 1 : 0);
+    int64_t S;
+    if constexpr (GROUPS) {
+        S = build_plan<32>(a, s_bpre, s_rst);  // contains __syncthreads
+        if (blockIdx.x == 0 && threadIdx.x == 0 && a.status)
+            *a.status = S < 0 ? MXFP4_EINVAL : MXFP4_OK;
+        if (S < 0)
+            return;
+    } else {
+        S = (a.rows + 31) / 32;
+    }
+    const int lane = threadIdx.x & 31;
+    const int64_t npairs = a.cols / 2, mstride = a.cols / 8;
+    const int64_t total = S * npairs;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    // the loop runs per warp, so that all lanes take part in the shuffles
+    for (int64_t base = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) & ~31ll; base < total; base += stride) {
+        const int64_t idx = base + lane;
+        const bool on = idx < total;
+        const int64_t rb = on ? idx / npairs : 0, pr = on ? idx - rb * npairs : 0;
+        int64_t row0 = 0;
+        int nrows = 0;
+        if (on) {
+            if constexpr (GROUPS) {
+                plan_lookup(s_bpre, s_rst, a.num_groups, (uint32_t)rb, 32, row0, nrows);
+            } else {
+                row0 = rb * 32;
+                nrows = (int)min((int64_t)32, a.rows - row0);
+            }
+        }
+        const int64_t c = 2 * pr;
+        uint32_t w[32];
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+            w[r] = r < nrows ? *reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(a.x) +
+                                                                   (row0 + r) * a.ld + c)
+                             : 0u;
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+            m2 = vmax2(m2, w[r] & 0x7FFF7FFFu);
+        const uint32_t A_lo = m2 << 16, A_hi = m2 & 0xFFFF0000u;
+        const bool sp_lo = A_lo >= 0x7F800000u, sp_hi = A_hi >= 0x7F800000u;
+        const int k_lo = sp_lo ? 0 : k_e4m3(A_lo), k_hi = sp_hi ? 0 : k_e4m3(A_hi);
+        const float inv_lo = __uint_as_float(pow2_bits(-k_lo)), inv_hi = __uint_as_float(pow2_bits(-k_hi));
+        const float sc_lo = __uint_as_float(pow2_bits(k_lo)), sc_hi = __uint_as_float(pow2_bits(k_hi));
+        // 0x8000 + bf16 bits of 448 * 2^k per half; 0xFFFF: never (non-finite block)
+        const uint32_t lx = (sp_lo ? 0xFFFFu : 0x8000u + (((uint32_t)(k_lo + 135) << 7) | 0x60u)) |
+                            ((sp_hi ? 0xFFFFu : 0x8000u + (((uint32_t)(k_hi + 135) << 7) | 0x60u)) << 16);
+        const uint32_t nanw = (sp_lo ? 0x0000FFFFu : 0u) | (sp_hi ? 0xFFFF0000u : 0u);
+        const int sh = 2 * (int)(pr & 3);
+        uint32_t satw = 0;  // 4 rows at a time: byte j = row 4m + j's bits of the 8 columns
+#pragma unroll
+        for (int r = 0; r < 32; ++r) {
+            const float ylo = __fmul_rn(__uint_as_float(w[r] << 16), inv_lo);
+            const float yhi = __fmul_rn(__uint_as_float(w[r] & 0xFFFF0000u), inv_hi);
+            uint16_t qq;
+            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(qq) : "f"(yhi), "f"(ylo));
+            uint32_t h;
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(qq));
+            float clo, chi;
+            asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+                : "=f"(clo), "=f"(chi)
+                : "r"(h));
+            uint32_t yw = __byte_perm(__float_as_uint(__fmul_rn(clo, sc_lo)), __float_as_uint(__fmul_rn(chi, sc_hi)),
+                                      0x7632);
+            yw = (yw & ~nanw) | (0x7FC07FC0u & nanw);
+            const uint32_t qw = (uint32_t)qq & ~(nanw & 0x00FF00FFu) & ~((nanw >> 8) & 0x0000FF00u);
+            const uint32_t keep = lx - (w[r] & 0x7FFF7FFFu);  // bit 15 / 31 set: that half does not saturate
+            const uint32_t two = ((~keep >> 15) & 1u) | ((~keep >> 30) & 2u);
+            satw |= two << (sh + 8 * (r & 3));
+            if (r < nrows) {
+                const int64_t row = row0 + r;
+                if (a.y_col)
+                    *reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(a.y_col) + row * a.ld_y + c) = yw;
+                if (a.codes_col)
+                    *reinterpret_cast<uint16_t*>(a.codes_col + row * a.cols + c) = (uint16_t)qw;
+            }
+            if ((r & 3) == 3) {
+                satw |= __shfl_xor_sync(FULL, satw, 1);
+                satw |= __shfl_xor_sync(FULL, satw, 2);
+                if (a.mask_col && on && (pr & 3) == 0) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (r - 3 + j < nrows)
+                            a.mask_col[(row0 + r - 3 + j) * mstride + c / 8] = (uint8_t)(satw >> (8 * j));
+                }
+                satw = 0;
+            }
+        }
+        if (a.scales_col && on)
+            *reinterpret_cast<uint16_t*>(a.scales_col + rb * a.cols + c) =
+                (uint16_t)((sp_lo ? 0xFFu : (uint32_t)(k_lo + 127)) | ((sp_hi ? 0xFFu : (uint32_t)(k_hi + 127)) << 8));
+    }
+}
+
 }  // namespace mxfp4

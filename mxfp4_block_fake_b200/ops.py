@@ -25,6 +25,15 @@ _DTYPES = {torch.float32: _abi.F32, torch.bfloat16: _abi.BF16}
 _MODES = {"page": _abi.SCALE_PAGE, "floor": _abi.SCALE_FLOOR}
 _DIRS = {"rowwise": _abi.ROWWISE, "colwise": _abi.COLWISE}
 _SCALE_LAYOUTS = {"rowmajor": _abi.SCALES_ROWMAJOR, "mma": _abi.SCALES_MMA}
+# element formats: E2M1 (MXFP4) and E4M3 (MXFP8: block 32, scale_mode "floor",
+# one code byte per element)
+_ELEM_FORMATS = {"e2m1": _abi.ELEM_E2M1, "e4m3": _abi.ELEM_E4M3}
+
+
+def _elem_format(name: str) -> int:
+    if name not in _ELEM_FORMATS:
+        raise ValueError(f"elem_format must be one of {tuple(_ELEM_FORMATS)}, got {name!r}")
+    return _ELEM_FORMATS[name]
 
 
 @dataclasses.dataclass
@@ -39,6 +48,7 @@ class QDQResult:
     mask_col: torch.Tensor | None = None
     status: torch.Tensor | None = None
     scales_layout: str = "rowmajor"  # layout of scales_row
+    elem_format: str = "e2m1"
 
 
 def _ptr(t: torch.Tensor | None):
@@ -81,7 +91,8 @@ def _group_args(group_list, group_list_type: int, device):
 
 
 def make_args(x: torch.Tensor, *, block: int, scale_factor: float, scale_mode: str, dirs: int,
-              group_list=None, group_list_type: int = 0, status: torch.Tensor | None = None) -> _abi.QdqArgs:
+              group_list=None, group_list_type: int = 0, status: torch.Tensor | None = None,
+              elem_format: str = "e2m1") -> _abi.QdqArgs:
     a = _abi.QdqArgs()
     a.x = x.data_ptr()
     a.dtype = _DTYPES[x.dtype]
@@ -98,6 +109,7 @@ def make_args(x: torch.Tensor, *, block: int, scale_factor: float, scale_mode: s
         a.num_groups = group_list.numel()
         a.group_list_type = int(group_list_type)
     a.status = _ptr(status)
+    a.elem_format = _elem_format(elem_format)
     return a
 
 
@@ -123,16 +135,18 @@ def scales_row_bytes(rows: int, cols: int, block: int, scales_layout: str = "row
 
 def alloc_outputs(x: torch.Tensor, *, block: int, rowwise: bool, colwise: bool, num_groups: int,
                   emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
-                  with_status: bool = False, scales_layout: str = "rowmajor") -> QDQResult:
+                  with_status: bool = False, scales_layout: str = "rowmajor",
+                  elem_format: str = "e2m1") -> QDQResult:
     rows, cols = x.shape
     dev = x.device
-    r = QDQResult(scales_layout=scales_layout)
+    r = QDQResult(scales_layout=scales_layout, elem_format=elem_format)
+    ccols = cols if _elem_format(elem_format) == _abi.ELEM_E4M3 else (cols + 1) // 2
     u8 = dict(dtype=torch.uint8, device=dev)
     if rowwise:
         if emit_values:
             r.y_row = torch.empty((rows, cols), dtype=x.dtype, device=dev)
         if emit_codes:
-            r.codes_row = torch.empty((rows, (cols + 1) // 2), **u8)
+            r.codes_row = torch.empty((rows, ccols), **u8)
             if scales_layout == "mma":
                 # the padding of the last atoms is never written: zeros
                 r.scales_row = torch.zeros((scales_row_bytes(rows, cols, block, "mma"),), **u8)
@@ -144,7 +158,7 @@ def alloc_outputs(x: torch.Tensor, *, block: int, rowwise: bool, colwise: bool, 
         if emit_values:
             r.y_col = torch.empty((rows, cols), dtype=x.dtype, device=dev)
         if emit_codes:
-            r.codes_col = torch.empty((rows, (cols + 1) // 2), **u8)
+            r.codes_col = torch.empty((rows, ccols), **u8)
             r.scales_col = torch.empty((colwise_scale_rows_bound(rows, num_groups, block), cols), **u8)
         if emit_mask:
             r.mask_col = torch.empty((rows, (cols + 7) // 8), **u8)
@@ -173,10 +187,12 @@ def _check_status(r: QDQResult, where: str) -> None:
 def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0, scale_mode: str = "page",
                   rowwise: bool = True, colwise: bool = False, group_list=None, group_list_type: int = 0,
                   emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
-                  check: bool = False, out: QDQResult | None = None, scales_layout: str = "rowmajor") -> QDQResult:
+                  check: bool = False, out: QDQResult | None = None, scales_layout: str = "rowmajor",
+                  elem_format: str = "e2m1") -> QDQResult:
     """QDQ forward; returns the requested outputs. check=True synchronises and
     raises on an invalid group_list. scales_layout="mma" writes the row-wise
-    scales in the block-scaled MMA scale-factor layout."""
+    scales in the block-scaled MMA scale-factor layout. elem_format="e4m3"
+    quantises to MXFP8 (block 32, scale_mode "floor")."""
     x = _as_2d(x)
     gl, ng = _group_args(group_list, group_list_type, x.device)
     dirs = (_abi.ROWWISE if rowwise else 0) | (_abi.COLWISE if colwise else 0)
@@ -185,9 +201,9 @@ def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0
     r = out if out is not None else alloc_outputs(
         x, block=block, rowwise=rowwise, colwise=colwise, num_groups=ng, emit_values=emit_values,
         emit_codes=emit_codes, emit_mask=emit_mask, with_status=check or gl is not None,
-        scales_layout=scales_layout)
+        scales_layout=scales_layout, elem_format=elem_format)
     a = make_args(x, block=block, scale_factor=scale_factor, scale_mode=scale_mode, dirs=dirs,
-                  group_list=gl, group_list_type=group_list_type, status=r.status)
+                  group_list=gl, group_list_type=group_list_type, status=r.status, elem_format=r.elem_format)
     _fill_outputs(a, r)
     _abi.check(_abi.mxfp4_qdq_fwd(a, _stream(x.device)), "mxfp4_qdq_fwd")
     if check:
@@ -198,9 +214,10 @@ def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0
 def mxfp4_ste_bwd(grad_out: torch.Tensor, *, saved_mask: torch.Tensor | None = None,
                   x: torch.Tensor | None = None, clip_grad: bool = True, block: int = 32,
                   scale_factor: float = 6.0, scale_mode: str = "page", direction: str = "rowwise",
-                  group_list=None, group_list_type: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
+                  group_list=None, group_list_type: int = 0, out: torch.Tensor | None = None,
+                  elem_format: str = "e2m1") -> torch.Tensor:
     """Plain / clipped STE backward. With clip_grad and no saved_mask the mask
-    is recomputed from x in the same pass."""
+    is recomputed from x in the same pass (for elem_format's saturation)."""
     shape = grad_out.shape
     g = _as_2d(grad_out, "grad_out")
     if not g.is_contiguous():
@@ -217,7 +234,7 @@ def mxfp4_ste_bwd(grad_out: torch.Tensor, *, saved_mask: torch.Tensor | None = N
             raise ValueError("clip_grad without saved_mask needs x to recompute the mask")
     gl, _ = _group_args(group_list, group_list_type, g.device)
     a = make_args(x2, block=block, scale_factor=scale_factor, scale_mode=scale_mode,
-                  dirs=_DIRS[direction], group_list=gl, group_list_type=group_list_type)
+                  dirs=_DIRS[direction], group_list=gl, group_list_type=group_list_type, elem_format=elem_format)
     if x is None:
         a.x = None
     st = _abi.mxfp4_ste_bwd(a, g.data_ptr(), gi2.data_ptr(), g.shape[1], _ptr(saved_mask),
@@ -230,7 +247,8 @@ def mxfp4_qdq_fwd_bwd(x: torch.Tensor, grad_out: torch.Tensor, *, grad_direction
                       block: int = 32, scale_factor: float = 6.0, scale_mode: str = "page",
                       rowwise: bool = True, colwise: bool = False, group_list=None, group_list_type: int = 0,
                       emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
-                      out: QDQResult | None = None, grad_in: torch.Tensor | None = None):
+                      out: QDQResult | None = None, grad_in: torch.Tensor | None = None,
+                      elem_format: str = "e2m1"):
     """Fused forward + clipped-STE backward; returns (QDQResult, grad_in)."""
     x = _as_2d(x)
     g = _as_2d(grad_out, "grad_out").contiguous()
@@ -240,10 +258,10 @@ def mxfp4_qdq_fwd_bwd(x: torch.Tensor, grad_out: torch.Tensor, *, grad_direction
     dirs = (_abi.ROWWISE if rowwise else 0) | (_abi.COLWISE if colwise else 0)
     r = out if out is not None else alloc_outputs(
         x, block=block, rowwise=rowwise, colwise=colwise, num_groups=ng, emit_values=emit_values,
-        emit_codes=emit_codes, emit_mask=emit_mask, with_status=gl is not None)
+        emit_codes=emit_codes, emit_mask=emit_mask, with_status=gl is not None, elem_format=elem_format)
     gi = grad_in if grad_in is not None else torch.empty_like(g)
     a = make_args(x, block=block, scale_factor=scale_factor, scale_mode=scale_mode, dirs=dirs,
-                  group_list=gl, group_list_type=group_list_type, status=r.status)
+                  group_list=gl, group_list_type=group_list_type, status=r.status, elem_format=r.elem_format)
     _fill_outputs(a, r)
     st = _abi.mxfp4_qdq_fwd_bwd(a, g.data_ptr(), gi.data_ptr(), g.shape[1], _DIRS[grad_direction],
                                 _stream(x.device))
