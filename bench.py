@@ -340,19 +340,21 @@ def run_ours(a, rank: int, world: int):
 
     modes = None
     if world == 1 and not a.no_modes:
-        modes = time_modes(a, xd, gd, res, gi, stream)
+        modes = time_modes(a, xd, gd, res, gi, stream, gl)
 
     return dict(ms=ms, fwd_ms=fwd_ms, s_col=s_col, clocks=sampler.summary(), e2e=e2e, modes=modes,
                 x_h=x_h, g_h=g_h, offsets=offsets, np=np)
 
 
-def time_modes(a, xd, gd, res, gi, stream, steps: int = 20):
+def time_modes(a, xd, gd, res, gi, stream, gl, steps: int = 20):
     """Other modes of the hot path on the same tensors (device-resident, CUDA
     events): row-wise fwd with all outputs + STE from the saved mask, the
     training step of the pages' recipe (row-wise fwd, saved-free STE), and the
     real-quantisation producer (row-wise E2M1 codes + E8M0 scales in the
-    block-scaled MMA layout, no dequantised values), and blocks of 128 in
-    both directions with every output (ungrouped)."""
+    block-scaled MMA layout, no dequantised values), blocks of 128 in both
+    directions with every output (ungrouped), and the MXFP8 element format
+    (E4M3, the OCP scale rule) row-wise and in both directions with the
+    groups."""
     import torch
 
     from mxfp4_block_fake_b200 import _abi, ops
@@ -399,12 +401,29 @@ def time_modes(a, xd, gd, res, gi, stream, steps: int = 20):
     def dual128():
         call(_abi.mxfp4_qdq_fwd(dargs, sp), "mxfp4_qdq_fwd")
 
+    r8 = ops.alloc_outputs(xd, block=32, rowwise=True, colwise=True, num_groups=a.groups, emit_codes=True,
+                           emit_mask=True, with_status=True, elem_format="e4m3")
+    row8 = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode="floor", dirs=_abi.ROWWISE, elem_format="e4m3")
+    ops._fill_outputs(row8, r8)
+    row8.y_col = row8.codes_col = row8.scales_col = row8.mask_col = None
+    dual8 = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode="floor", dirs=_abi.ROWWISE | _abi.COLWISE,
+                          group_list=gl, group_list_type=0, status=r8.status, elem_format="e4m3")
+    ops._fill_outputs(dual8, r8)
+
+    def mxfp8_row():
+        call(_abi.mxfp4_qdq_fwd(row8, sp), "mxfp4_qdq_fwd")
+
+    def mxfp8_dual():
+        call(_abi.mxfp4_qdq_fwd(dual8, sp), "mxfp4_qdq_fwd")
+
     peak, _ = measured_peaks()
     out = {}
     for name, fn, bpe in (("rowwise_fwd_all_outputs_ste_mask", row_step, 4 + 0.5 + 1 / 32 + 0.125 + 4.125),
                           ("training_step_rowwise_fwd_ste_recompute", train_step, 4 + 6),
                           ("mxfp4_mma_operand_rowwise_codes_scales", mma_operand, 2 + 0.5 + 1 / 32),
-                          ("dual_block128_all_outputs", dual128, 2 + 4 + 1 + 2 / 128 + 0.25)):
+                          ("dual_block128_all_outputs", dual128, 2 + 4 + 1 + 2 / 128 + 0.25),
+                          ("mxfp8_rowwise_all_outputs", mxfp8_row, 2 + 2 + 1 + 1 / 32 + 0.125),
+                          ("mxfp8_dual_grouped_all_outputs", mxfp8_dual, 2 + 4 + 2 + 2 / 32 + 0.25)):
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
