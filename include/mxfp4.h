@@ -32,10 +32,12 @@
  * Data layout (all row-major, element strides in elements):
  *   x, y_row, y_col, grads      [rows][cols], leading dimensions ld / ld_y /
  *                               ld_grad (>= cols); dtype fp32 or bf16.
- *   codes_row, codes_col        [rows][ceil(cols/2)] bytes, contiguous; the
- *                               nibble of element c is the low nibble of byte
- *                               c/2 when c is even, the high one when odd;
- *                               nibble = sign << 3 | code index (E2M1 bits).
+ *   codes_row, codes_col        E2M1: [rows][ceil(cols/2)] bytes, contiguous;
+ *                               the nibble of element c is the low nibble of
+ *                               byte c/2 when c is even, the high one when
+ *                               odd; nibble = sign << 3 | code index (E2M1
+ *                               bits). E4M3 (elem_format): [rows][cols]
+ *                               bytes, one E4M3 code per element.
  *   scales_row                  [rows][ceil(cols/block)] E8M0 bytes (k + 127),
  *                               row-major, or (scales_row_layout =
  *                               MXFP4_SCALES_MMA) in the scale-factor layout
