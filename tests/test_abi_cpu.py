@@ -126,9 +126,24 @@ def _args(abi, **kw):
     (dict(dirs=2, group_list=4096, num_groups=5000), 2),
     (dict(dirs=2, group_list=4096, num_groups=3, group_list_type=2), 1),
     (dict(dirs=2, group_list=4097, num_groups=3), 1),
+    (dict(scales_row_layout=2), 1), (dict(elem_format=2), 1), (dict(elem_format=-1), 1),
+    (dict(elem_format=1), 2),                               # MXFP8 in PAGE mode
+    (dict(elem_format=1, scale_mode=1, block=128), 2),      # MXFP8 with blocks of 128
 ])
 def test_fwd_rejects_bad_arguments_on_host(abi, kw, expected):
     assert abi.mxfp4_qdq_fwd(_args(abi, **kw), None) == expected
+
+
+@pytest.mark.parametrize("rows,cols,block", [(130, 160, 32), (128, 128, 32), (1, 1, 32), (300, 7168, 32),
+                                             (257, 1000, 128), (0, 64, 32)])
+def test_scales_row_bytes(abi, oracle_mod, rows, cols, block):
+    L = abi.lib()
+    nblk = -(-cols // block)
+    assert L.mxfp4_scales_row_bytes(rows, cols, block, abi.SCALES_ROWMAJOR) == rows * nblk
+    mma = oracle_mod.mma_scale_layout(np.zeros((rows, nblk), np.uint8)).size if rows else 0
+    assert L.mxfp4_scales_row_bytes(rows, cols, block, abi.SCALES_MMA) == mma
+    assert L.mxfp4_scales_row_bytes(rows, cols, block, 7) == -1
+    assert L.mxfp4_scales_row_bytes(-1, cols, block, abi.SCALES_ROWMAJOR) == -1
 
 
 def test_null_args_and_bad_bwd_arguments(abi):
