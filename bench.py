@@ -340,21 +340,21 @@ def run_ours(a, rank: int, world: int):
 
     modes = None
     if world == 1 and not a.no_modes:
-        modes = time_modes(a, xd, gd, res, gi, stream, gl)
+        modes = time_modes(a, xd, gd, res, gi, stream, gl, s_col)
 
     return dict(ms=ms, fwd_ms=fwd_ms, s_col=s_col, clocks=sampler.summary(), e2e=e2e, modes=modes,
                 x_h=x_h, g_h=g_h, offsets=offsets, np=np)
 
 
-def time_modes(a, xd, gd, res, gi, stream, gl, steps: int = 20):
+def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
     """Other modes of the hot path on the same tensors (device-resident, CUDA
     events): row-wise fwd with all outputs + STE from the saved mask, the
     training step of the pages' recipe (row-wise fwd, saved-free STE), and the
     real-quantisation producer (row-wise E2M1 codes + E8M0 scales in the
     block-scaled MMA layout, no dequantised values), blocks of 128 in both
-    directions with every output (ungrouped), and the MXFP8 element format
+    directions with every output (ungrouped), the MXFP8 element format
     (E4M3, the OCP scale rule) row-wise and in both directions with the
-    groups."""
+    groups, and the bench step itself with the other scale rule."""
     import torch
 
     from mxfp4_block_fake_b200 import _abi, ops
@@ -410,6 +410,17 @@ def time_modes(a, xd, gd, res, gi, stream, gl, steps: int = 20):
                           group_list=gl, group_list_type=0, status=r8.status, elem_format="e4m3")
     ops._fill_outputs(dual8, r8)
 
+    other = "floor" if a.scale_mode == "page" else "page"
+    fo_args = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode=other, dirs=_abi.ROWWISE | _abi.COLWISE,
+                            group_list=gl, group_list_type=0, status=res.status)
+    ops._fill_outputs(fo_args, res)
+    bo_args = ops.make_args(gd, block=32, scale_factor=6.0, scale_mode=other, dirs=_abi.ROWWISE)
+    bo_args.x = None
+
+    def step_other_mode():
+        call(_abi.mxfp4_qdq_fwd(fo_args, sp), "mxfp4_qdq_fwd")
+        call(_abi.mxfp4_ste_bwd(bo_args, g_ptr, gi_ptr, a.cols, m_ptr, 1, sp), "mxfp4_ste_bwd")
+
     def mxfp8_row():
         call(_abi.mxfp4_qdq_fwd(row8, sp), "mxfp4_qdq_fwd")
 
@@ -423,7 +434,8 @@ def time_modes(a, xd, gd, res, gi, stream, gl, steps: int = 20):
                           ("mxfp4_mma_operand_rowwise_codes_scales", mma_operand, 2 + 0.5 + 1 / 32),
                           ("dual_block128_all_outputs", dual128, 2 + 4 + 1 + 2 / 128 + 0.25),
                           ("mxfp8_rowwise_all_outputs", mxfp8_row, 2 + 2 + 1 + 1 / 32 + 0.125),
-                          ("mxfp8_dual_grouped_all_outputs", mxfp8_dual, 2 + 4 + 2 + 2 / 32 + 0.25)):
+                          ("mxfp8_dual_grouped_all_outputs", mxfp8_dual, 2 + 4 + 2 + 2 / 32 + 0.25),
+                          (f"bench_step_{other}_scale", step_other_mode, step_bytes(a.rows, a.cols, s_col)["step"] / n)):
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
