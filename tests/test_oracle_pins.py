@@ -391,8 +391,10 @@ def test_ste_bwd_is_masked_fill(oracle_mod, dtype):
 
 def test_torch_page_formula_agrees_on_bf16(oracle_mod):
     """Cross-check against torch CPU ops evaluating the page's fp32 steps
-    (log2 / round / exp2 / bucketize). The survey of all bf16 amax values found
-    fp32 log2 rounding agrees with the exact reading for bf16 inputs."""
+    (log2 / round / exp2 / bucketize). For bf16 inputs fp32 log2 followed by
+    round() agrees with the exact nearest integer of log2 for every amax (no
+    bf16 amax / 6 lies within fp32 rounding of a half-integer power of two),
+    so the two readings give the same bytes here."""
     torch = pytest.importorskip("torch")
     O = oracle_mod
     g = torch.Generator().manual_seed(21)
@@ -408,6 +410,11 @@ def test_torch_page_formula_agrees_on_bf16(oracle_mod):
     ref = (q * scale).reshape(512, 256).to(torch.bfloat16)
     res = O.qdq_rowwise(xb.view(torch.int16).numpy().view(np.uint16), 32, 6.0, 0)
     assert np.array_equal(res["y"], ref.view(torch.int16).numpy().view(np.uint16))
+    # every finite positive bf16 amax: torch's fp32 scale equals the oracle's
+    allb = torch.arange(1, 0x7F80, dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float()
+    t_scale = torch.exp2(torch.round(torch.log2(torch.clamp(allb / 6.0, min=2.0 ** -30))))
+    o_scale = np.array([O.scale_page(float(v), 6.0) for v in allb.tolist()], np.float32)
+    assert np.array_equal(t_scale.numpy(), o_scale)
 
 
 def test_mma_scale_layout_hand_offsets(oracle_mod):
