@@ -614,3 +614,51 @@ def test_cuda_graph_capture_and_replay():
     ora = O.qdq_rowwise(oracle_in(xs[0]), 32, 6.0, O.SCALE_PAGE)
     check_dir(r, ora, "row", cols, label="graph replay")
     del graph
+
+
+def test_full_size_bench_modes_sampled():
+    """The other calls the benchmark times, at its full size (MoE activation
+    65536 x 7168), checked on sampled rows and columns: the real-quantisation
+    producer (codes + MMA-layout scales, no values) and MXFP8 in both
+    directions with the groups."""
+    torch.cuda.empty_cache()
+    x, counts, offsets = W.moe_grouped()
+    xd = x.cuda()
+    gl = offsets.cuda()
+    rows, cols = x.shape
+    rng = np.random.default_rng(11)
+    ri = np.sort(rng.choice(rows, size=256, replace=False))
+    rit = torch.from_numpy(ri).cuda()
+    # producer: codes of sampled rows; scale bytes at the positions the
+    # oracle's layout gives the sampled rows
+    codes, scales = ops.mxfp4_mma_operand(xd)
+    torch.cuda.synchronize()
+    ora = O.qdq_rowwise(oracle_in(x[torch.from_numpy(ri)]), 32, 6.0, O.SCALE_PAGE)
+    assert np.array_equal(np_bits(codes.view(torch.uint8)[rit]), ora["codes"])
+    nblk = cols // 32
+    full = np.zeros((rows, nblk), np.uint8)
+    full[ri] = ora["scales"]
+    sel = np.zeros((rows, nblk), np.uint8)
+    sel[ri] = 1
+    pos = O.mma_scale_layout(sel) == 1
+    got = np_bits(scales.view(torch.uint8))
+    assert np.array_equal(got[pos], O.mma_scale_layout(full)[pos])
+    del codes, scales
+    # MXFP8, both directions, grouped
+    res = ops.mxfp4_qdq_fwd(xd, block=32, scale_mode="floor", rowwise=True, colwise=True, group_list=gl,
+                            emit_codes=True, emit_mask=True, check=True, elem_format="e4m3")
+    torch.cuda.synchronize()
+    o8 = O.qdq8_rowwise(oracle_in(x[torch.from_numpy(ri)]))
+    assert np.array_equal(np_bits(res.y_row[rit]), o8["y"])
+    assert np.array_equal(np_bits(res.codes_row[rit]), o8["codes"])
+    assert np.array_equal(np_bits(res.scales_row[rit]), o8["scales"])
+    assert np.array_equal(np_bits(res.mask_row[rit]), o8["mask"])
+    oc = np.sort(rng.choice(cols // 8, size=16, replace=False))
+    ci = (oc[:, None] * 8 + np.arange(8)).reshape(-1)
+    cit = torch.from_numpy(ci).cuda()
+    c8 = O.qdq8_colwise(oracle_in(x[:, torch.from_numpy(ci)]), offsets.numpy())
+    s = c8["scales"].shape[0]
+    assert np.array_equal(np_bits(res.y_col[:, cit]), c8["y"])
+    assert np.array_equal(np_bits(res.codes_col[:, cit]), c8["codes"])
+    assert np.array_equal(np_bits(res.scales_col[:s][:, cit]), c8["scales"])
+    assert np.array_equal(np_bits(res.mask_col[:, torch.from_numpy(oc).cuda()]), c8["mask"])
