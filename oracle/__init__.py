@@ -3,6 +3,11 @@
 TEST INFRASTRUCTURE: only tests/, __graft_entry__.smoke() and bench.py's CPU
 baseline leg import this package. The CUDA library and its binding never do.
 
+mma_scale_layout restates the scale-factor layout of block-scaled tensor-core
+GEMMs as the cuBLAS documentation defines it; the pages fix no such layout
+(parity against them unpinned), and the tests pin it to hand-computed offsets
+and to a derivation by reshapes.
+
 bf16 data is passed as numpy uint16 arrays holding the raw bf16 bit patterns;
 fp32 data as numpy float32 arrays. All arrays are 2-D [rows, cols] row-major.
 """

@@ -39,6 +39,18 @@
  *     of byte j is element 8j+b of the row.
  *   - Column-wise blocks run down a column, restart at each group start and
  *     end early at a group end; scale rows are stored group after group.
+ *
+ * Parity status (what pins each function; the tests hold the pins):
+ *   - scales, rounding, outputs, masks, STE: pinned by hand-worked blocks
+ *     (tests/golden), closed forms, exhaustive bf16 sweeps, a brute-force
+ *     nearest-code search and algebraic invariants;
+ *   - packed layouts: the nibble values and the decode identity are pinned;
+ *     the nibble order within a byte and the order of column-wise scale rows
+ *     are conventions the pages do not fix: parity unpinned;
+ *   - MXFP8 (oracle_qdq8_*, oracle_e4m3_*): the pages give no MXFP8
+ *     arithmetic, so parity against them is unpinned; the functions are
+ *     pinned against the E4M3 / OCP definitions (bit-field value set,
+ *     nearest-even search over every bf16 value, torch's float8_e4m3fn cast).
  */
 #include <math.h>
 #include <stdint.h>
