@@ -1501,7 +1501,7 @@ __global__ void __launch_bounds__(NTHREADS) row_stream8_kernel(const KArgs a)
 // ---------------------------------------------------------------------------
 
 template <bool GROUPS>
-__global__ void __launch_bounds__(NTHREADS) col_pair8_kernel(const KArgs a)
+__global__ void __launch_bounds__(NTHREADS, 2) col_pair8_kernel(const KArgs a)
 {
     extern __shared__ int32_t s_plan8[];
     int32_t* s_bpre = s_plan8;
@@ -1520,13 +1520,14 @@ __global__ void __launch_bounds__(NTHREADS) col_pair8_kernel(const KArgs a)
     const int64_t npairs = a.cols / 2, mstride = a.cols / 8;
     const int64_t total = S * npairs;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    // the loop runs per warp, so that all lanes take part in the shuffles
-    for (int64_t base = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) & ~31ll; base < total; base += stride) {
+    // tile of a warp iteration: this lane's column pair and block rows
+    auto locate = [&](int64_t base, int64_t& rb, int64_t& pr, int64_t& row0, int& nrows) {
         const int64_t idx = base + lane;
         const bool on = idx < total;
-        const int64_t rb = on ? idx / npairs : 0, pr = on ? idx - rb * npairs : 0;
-        int64_t row0 = 0;
-        int nrows = 0;
+        rb = on ? idx / npairs : 0;
+        pr = on ? idx - rb * npairs : 0;
+        row0 = 0;
+        nrows = 0;
         if (on) {
             if constexpr (GROUPS) {
                 plan_lookup(s_bpre, s_rst, a.num_groups, (uint32_t)rb, 32, row0, nrows);
@@ -1535,13 +1536,31 @@ __global__ void __launch_bounds__(NTHREADS) col_pair8_kernel(const KArgs a)
                 nrows = (int)min((int64_t)32, a.rows - row0);
             }
         }
-        const int64_t c = 2 * pr;
-        uint32_t w[32];
+        return on;
+    };
+    auto load = [&](int64_t row0, int nrows, int64_t pr, uint32_t (&w)[32]) {
 #pragma unroll
         for (int r = 0; r < 32; ++r)
             w[r] = r < nrows ? *reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(a.x) +
-                                                                   (row0 + r) * a.ld + c)
+                                                                   (row0 + r) * a.ld + 2 * pr)
                              : 0u;
+    };
+    // the loop runs per warp, so that all lanes take part in the shuffles; the
+    // next tile's words are loaded before this tile's are converted
+    int64_t base = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) & ~31ll;
+    int64_t rb, pr, row0;
+    int nrows;
+    bool on = locate(base, rb, pr, row0, nrows);
+    uint32_t w[32];
+    load(row0, nrows, pr, w);
+    for (; base < total; base += stride) {
+        int64_t rb_n, pr_n, row0_n;
+        int nrows_n;
+        const bool on_n = locate(base + stride, rb_n, pr_n, row0_n, nrows_n);
+        uint32_t wn[32];
+        load(row0_n, nrows_n, pr_n, wn);
+
+        const int64_t c = 2 * pr;
         uint32_t m2 = 0;
 #pragma unroll
         for (int r = 0; r < 32; ++r)
@@ -1598,6 +1617,14 @@ __global__ void __launch_bounds__(NTHREADS) col_pair8_kernel(const KArgs a)
         if (a.scales_col && on)
             *reinterpret_cast<uint16_t*>(a.scales_col + rb * a.cols + c) =
                 (uint16_t)((sp_lo ? 0xFFu : (uint32_t)(k_lo + 127)) | ((sp_hi ? 0xFFu : (uint32_t)(k_hi + 127)) << 8));
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+            w[r] = wn[r];
+        rb = rb_n;
+        pr = pr_n;
+        row0 = row0_n;
+        nrows = nrows_n;
+        on = on_n;
     }
 }
 
