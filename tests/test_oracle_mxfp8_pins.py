@@ -127,3 +127,26 @@ def test_mxfp8_colwise_is_rowwise_of_transpose(oracle_mod):
     assert np.array_equal(c["y"], r["y"].T)
     assert np.array_equal(c["codes"], r["codes"].T)
     assert np.array_equal(c["scales"], r["scales"].T)
+
+
+def test_mxfp8_colwise_groups_equal_per_group_slices(oracle_mod):
+    """Group restarts: the grouped column-wise result equals the column-wise
+    result of each group's rows on their own, scale rows stacked group after
+    group; empty groups add no rows."""
+    O = oracle_mod
+    rng = np.random.default_rng(8)
+    counts = [0, 45, 32, 0, 1, 70, 0]
+    rows, cols = sum(counts), 24
+    x = (rng.standard_normal((rows, cols)) * 2.0 ** rng.integers(-20, 20, (rows, 1))).astype(np.float32)
+    ends = np.cumsum(counts)
+    g = O.qdq8_colwise(x, ends)
+    start, srows = 0, []
+    for e in ends:
+        if e > start:
+            part = O.qdq8_colwise(np.ascontiguousarray(x[start:e]))
+            assert np.array_equal(g["y"][start:e], part["y"])
+            assert np.array_equal(g["codes"][start:e], part["codes"])
+            assert np.array_equal(g["mask"][start:e], part["mask"])
+            srows.append(part["scales"])
+        start = e
+    assert np.array_equal(g["scales"], np.concatenate(srows))
