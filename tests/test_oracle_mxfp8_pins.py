@@ -150,3 +150,21 @@ def test_mxfp8_colwise_groups_equal_per_group_slices(oracle_mod):
             srows.append(part["scales"])
         start = e
     assert np.array_equal(g["scales"], np.concatenate(srows))
+
+
+def test_mxfp8_outputs_of_bf16_inputs_are_bf16_values():
+    """decode(code) * 2^k is a bf16 value for every bf16 x (|x| below the
+    block bound 2^(k+9)), so narrowing it to bf16 is exact; checked at the
+    scales where bf16's subnormal range or its top could break it, and
+    around 2^0."""
+    b = np.arange(65536, dtype=np.uint32)
+    f = (b << 16).view(np.float32)
+    x = f[np.isfinite(f)].astype(np.float64)
+    g = e4m3_grid()
+    for k in list(range(-127, -117)) + list(range(-20, 21)) + list(range(110, 120)):
+        xs = x[np.abs(x) < 2.0 ** (k + 9)]
+        codes = nearest_even_codes((xs * 2.0 ** -k).astype(np.float32))
+        out = np.where(codes & 0x80, -1.0, 1.0) * g[codes & 0x7F] * 2.0 ** k
+        o32 = out.astype(np.float32)
+        assert np.array_equal(o32.astype(np.float64), out), k
+        assert np.all((o32.view(np.uint32) & 0xFFFF) == 0), k
