@@ -72,9 +72,12 @@
  * Errors: argument errors are found on the host before any launch and
  * returned as a status (nothing is written). A group_list lives in device
  * memory, so its validity (non-negative counts, non-decreasing offsets, last
- * offset == rows) is checked by the kernels: an invalid list makes every
- * kernel of the call write nothing and, when `status` is non-NULL, store
- * MXFP4_EINVAL there (MXFP4_OK otherwise). No kernel traps or asserts.
+ * offset == rows) is checked by the kernels: with an invalid list no
+ * column-wise output and no gradient is written (row-wise outputs, which do
+ * not depend on the groups, may be) and, when `status` is non-NULL, the
+ * kernels store MXFP4_EINVAL there (MXFP4_OK otherwise), so that a caller
+ * that passes a group_list must read `status` before using any output. No
+ * kernel traps or asserts.
  */
 #ifndef MXFP4_H
 #define MXFP4_H

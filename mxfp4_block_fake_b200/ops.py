@@ -56,6 +56,11 @@ def _ptr(t: torch.Tensor | None):
 
 
 def _as_2d(x: torch.Tensor, name: str = "x") -> torch.Tensor:
+    """2-D view of x that the library can address as [rows][ld] with unit
+    stride along the columns and ld >= cols. Anything else (a transposed or
+    sliced last dimension, rows that overlap such as an expanded tensor with
+    row stride 0) is copied first, so that the library never reads outside
+    x's storage or with a wrong pitch."""
     if x.ndim == 0:
         raise ValueError(f"{name} must have at least 1 dimension")
     if not x.is_cuda:
@@ -66,13 +71,24 @@ def _as_2d(x: torch.Tensor, name: str = "x") -> torch.Tensor:
         x = x.unsqueeze(0)
     elif x.ndim > 2:
         x = x.reshape(-1, x.shape[-1])
-    if x.shape[-1] > 1 and x.stride(-1) != 1:
+    if not rows_addressable(tuple(x.shape), tuple(x.stride())):
         x = x.contiguous()
     return x
 
 
+def rows_addressable(shape: tuple, stride: tuple) -> bool:
+    """True when a 2-D tensor of this shape and stride is the [rows][ld]
+    layout of the C ABI: unit stride along the columns (unless there is only
+    one column) and rows that do not overlap (row stride >= cols, unless
+    there is only one row)."""
+    rows, cols = shape
+    return not ((cols > 1 and stride[1] != 1) or (rows > 1 and stride[0] < cols))
+
+
 def _ld(t: torch.Tensor) -> int:
-    return max(t.stride(0), t.shape[1]) if t.shape[0] > 1 else t.shape[1]
+    """Leading dimension (elements between rows) of a 2-D tensor laid out as
+    _as_2d requires; a single row has no pitch and reports its width."""
+    return t.stride(0) if t.shape[0] > 1 else t.shape[1]
 
 
 def _stream(device: torch.device) -> int:
@@ -167,34 +183,110 @@ def alloc_outputs(x: torch.Tensor, *, block: int, rowwise: bool, colwise: bool, 
     return r
 
 
-def _fill_outputs(a: _abi.QdqArgs, r: QDQResult) -> None:
-    a.y_row, a.y_col = _ptr(r.y_row), _ptr(r.y_col)
+def _need(t: torch.Tensor, name: str, shape, dtype, device, min_rows: int | None = None) -> None:
+    """An output buffer must be a contiguous CUDA tensor of the given shape
+    and dtype on x's device (min_rows: at least that many rows instead of
+    exactly shape[0])."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    ok = (t.dim() == len(shape) and tuple(t.shape[1:]) == tuple(shape[1:]) and
+          (t.shape[0] >= min_rows if min_rows is not None else t.shape[0] == shape[0]))
+    if not ok:
+        want = f"[>= {min_rows}, {', '.join(map(str, shape[1:]))}]" if min_rows is not None else list(shape)
+        raise ValueError(f"{name} has shape {list(t.shape)}, expected {want}")
+
+
+def _fill_outputs(a: _abi.QdqArgs, r: QDQResult, x: torch.Tensor | None = None) -> None:
+    """Copies the output pointers of r into a. With x given, every buffer is
+    first checked against the geometry in a (shape, dtype, device, layout), so
+    that no kernel can write outside a caller-supplied tensor."""
+    if r.scales_layout not in _SCALE_LAYOUTS:
+        raise ValueError(f"scales_layout must be one of {tuple(_SCALE_LAYOUTS)}, got {r.scales_layout!r}")
     ys = [t for t in (r.y_row, r.y_col) if t is not None]
+    if x is not None:
+        rows, cols, blk, dev = a.rows, a.cols, a.block, x.device
+        e4m3 = a.elem_format == _abi.ELEM_E4M3
+        ccols = cols if e4m3 else (cols + 1) // 2
+        nblk = (cols + blk - 1) // blk
+        for name in ("y_row", "y_col"):
+            t = getattr(r, name)
+            if t is None:
+                continue
+            if not t.is_cuda or t.device != dev or t.dtype != x.dtype or tuple(t.shape) != (rows, cols):
+                raise ValueError(f"{name} must be a {x.dtype} CUDA tensor of shape {[rows, cols]} on {dev}")
+            if not rows_addressable(tuple(t.shape), tuple(t.stride())):
+                raise ValueError(f"{name} must have unit column stride and non-overlapping rows")
+        if len(ys) == 2 and _ld(ys[0]) != _ld(ys[1]):
+            raise ValueError("y_row and y_col must have the same row stride (one ld_y is passed)")
+        u8 = torch.uint8
+        for name in ("codes_row", "codes_col"):
+            if getattr(r, name) is not None:
+                _need(getattr(r, name), name, (rows, ccols), u8, dev)
+        for name in ("mask_row", "mask_col"):
+            if getattr(r, name) is not None:
+                _need(getattr(r, name), name, (rows, (cols + 7) // 8), u8, dev)
+        if r.scales_row is not None:
+            if r.scales_layout == "mma":
+                t = r.scales_row
+                if not t.is_cuda or t.device != dev or t.dtype != u8 or not t.is_contiguous():
+                    raise ValueError("scales_row (mma layout) must be a contiguous uint8 CUDA tensor")
+                if t.numel() < scales_row_bytes(rows, cols, blk, "mma"):
+                    raise ValueError("scales_row (mma layout) is smaller than mxfp4_scales_row_bytes()")
+            else:
+                _need(r.scales_row, "scales_row", (rows, nblk), u8, dev)
+        if r.scales_col is not None:
+            _need(r.scales_col, "scales_col", (0, cols), u8, dev,
+                  min_rows=colwise_scale_rows_bound(rows, int(a.num_groups) if a.group_list else 0, blk))
+        if r.status is not None:
+            _need(r.status, "status", (1,), torch.int32, dev)
+    a.y_row, a.y_col = _ptr(r.y_row), _ptr(r.y_col)
     a.ld_y = _ld(ys[0]) if ys else a.cols
     a.codes_row, a.scales_row, a.mask_row = _ptr(r.codes_row), _ptr(r.scales_row), _ptr(r.mask_row)
     a.codes_col, a.scales_col, a.mask_col = _ptr(r.codes_col), _ptr(r.scales_col), _ptr(r.mask_col)
-    if r.scales_layout not in _SCALE_LAYOUTS:
-        raise ValueError(f"scales_layout must be one of {tuple(_SCALE_LAYOUTS)}, got {r.scales_layout!r}")
     a.scales_row_layout = _SCALE_LAYOUTS[r.scales_layout]
 
 
-def _check_status(r: QDQResult, where: str) -> None:
-    if r.status is not None:
-        st = int(r.status.item())
-        _abi.check(st, where + " (group_list)")
+def _check_status(status: torch.Tensor | None, where: str) -> None:
+    if status is not None:
+        _abi.check(int(status.item()), where + " (group_list)")
+
+
+def _grad_buffer(out: torch.Tensor | None, g: torch.Tensor, shape, name: str) -> torch.Tensor:
+    """The gradient output: a new tensor, or a caller's contiguous tensor of
+    grad_out's shape and dtype (the library writes it with grad_out's pitch)."""
+    if out is None:
+        return torch.empty_like(g)
+    if not out.is_cuda or out.device != g.device or out.dtype != g.dtype or not out.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {g.dtype} CUDA tensor on {g.device}")
+    if out.numel() != g.numel() or tuple(out.shape) not in (tuple(shape), tuple(g.shape)):
+        raise ValueError(f"{name} has shape {list(out.shape)}, expected {list(shape)}")
+    return out.view(g.shape)
 
 
 def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0, scale_mode: str = "page",
                   rowwise: bool = True, colwise: bool = False, group_list=None, group_list_type: int = 0,
                   emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
-                  check: bool = False, out: QDQResult | None = None, scales_layout: str = "rowmajor",
+                  check: bool | None = None, out: QDQResult | None = None, scales_layout: str = "rowmajor",
                   elem_format: str = "e2m1") -> QDQResult:
-    """QDQ forward; returns the requested outputs. check=True synchronises and
-    raises on an invalid group_list. scales_layout="mma" writes the row-wise
-    scales in the block-scaled MMA scale-factor layout. elem_format="e4m3"
-    quantises to MXFP8 (block 32, scale_mode "floor")."""
+    """QDQ forward; returns the requested outputs.
+
+    A group_list lives in device memory and is validated by the kernels,
+    which write nothing when it is not a partition of the rows. check (the
+    default when a group_list is given) synchronises and raises
+    MXFP4ArgumentError for such a list. With check=False the call stays
+    asynchronous (CUDA-graph capturable) and the outputs are undefined unless
+    the returned status tensor reads 0 (MXFP4_OK) once the stream reaches it.
+    scales_layout="mma" writes the row-wise scales in the block-scaled MMA
+    scale-factor layout. elem_format="e4m3" quantises to MXFP8 (block 32,
+    scale_mode "floor")."""
     x = _as_2d(x)
     gl, ng = _group_args(group_list, group_list_type, x.device)
+    if check is None:
+        check = gl is not None and colwise
     dirs = (_abi.ROWWISE if rowwise else 0) | (_abi.COLWISE if colwise else 0)
     if dirs == 0:
         raise ValueError("at least one of rowwise / colwise must be set")
@@ -202,12 +294,14 @@ def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0
         x, block=block, rowwise=rowwise, colwise=colwise, num_groups=ng, emit_values=emit_values,
         emit_codes=emit_codes, emit_mask=emit_mask, with_status=check or gl is not None,
         scales_layout=scales_layout, elem_format=elem_format)
+    if check and r.status is None:
+        r.status = torch.empty((1,), dtype=torch.int32, device=x.device)
     a = make_args(x, block=block, scale_factor=scale_factor, scale_mode=scale_mode, dirs=dirs,
                   group_list=gl, group_list_type=group_list_type, status=r.status, elem_format=r.elem_format)
-    _fill_outputs(a, r)
+    _fill_outputs(a, r, x)
     _abi.check(_abi.mxfp4_qdq_fwd(a, _stream(x.device)), "mxfp4_qdq_fwd")
     if check:
-        _check_status(r, "mxfp4_qdq_fwd")
+        _check_status(r.status, "mxfp4_qdq_fwd")
     return r
 
 
@@ -215,15 +309,21 @@ def mxfp4_ste_bwd(grad_out: torch.Tensor, *, saved_mask: torch.Tensor | None = N
                   x: torch.Tensor | None = None, clip_grad: bool = True, block: int = 32,
                   scale_factor: float = 6.0, scale_mode: str = "page", direction: str = "rowwise",
                   group_list=None, group_list_type: int = 0, out: torch.Tensor | None = None,
-                  elem_format: str = "e2m1") -> torch.Tensor:
+                  elem_format: str = "e2m1", check: bool | None = None,
+                  status: torch.Tensor | None = None) -> torch.Tensor:
     """Plain / clipped STE backward. With clip_grad and no saved_mask the mask
-    is recomputed from x in the same pass (for elem_format's saturation)."""
+    is recomputed from x in the same pass (for elem_format's saturation).
+
+    A group_list only matters when the column-wise mask is recomputed; it is
+    then validated by the kernel. check (the default in that case)
+    synchronises and raises MXFP4ArgumentError for an invalid list; with
+    check=False pass a 1-element int32 CUDA `status` tensor and read it: the
+    gradient is undefined unless it holds 0."""
     shape = grad_out.shape
     g = _as_2d(grad_out, "grad_out")
     if not g.is_contiguous():
         g = g.contiguous()
-    gi = out if out is not None else torch.empty_like(g)
-    gi2 = gi.view(g.shape)
+    gi2 = _grad_buffer(out, g, shape, "out")
     if x is not None:
         x2 = _as_2d(x)
         if x2.shape != g.shape or x2.dtype != g.dtype:
@@ -232,15 +332,27 @@ def mxfp4_ste_bwd(grad_out: torch.Tensor, *, saved_mask: torch.Tensor | None = N
         x2 = g  # geometry only; x is not read when the mask is saved
         if clip_grad and saved_mask is None:
             raise ValueError("clip_grad without saved_mask needs x to recompute the mask")
+    if saved_mask is not None and clip_grad:
+        _need(saved_mask, "saved_mask", (g.shape[0], (g.shape[1] + 7) // 8), torch.uint8, g.device)
     gl, _ = _group_args(group_list, group_list_type, g.device)
+    validates = gl is not None and clip_grad and saved_mask is None and direction == "colwise"
+    if check is None:
+        check = validates
+    if validates and status is None:
+        if not check:
+            raise ValueError("check=False with a group_list needs a status tensor to report the list check")
+        status = torch.empty((1,), dtype=torch.int32, device=g.device)
     a = make_args(x2, block=block, scale_factor=scale_factor, scale_mode=scale_mode,
-                  dirs=_DIRS[direction], group_list=gl, group_list_type=group_list_type, elem_format=elem_format)
+                  dirs=_DIRS[direction], group_list=gl, group_list_type=group_list_type,
+                  status=status if validates else None, elem_format=elem_format)
     if x is None:
         a.x = None
     st = _abi.mxfp4_ste_bwd(a, g.data_ptr(), gi2.data_ptr(), g.shape[1], _ptr(saved_mask),
                             int(bool(clip_grad)), _stream(g.device))
     _abi.check(st, "mxfp4_ste_bwd")
-    return gi.view(shape)
+    if check and validates:
+        _check_status(status, "mxfp4_ste_bwd")
+    return gi2.view(shape)
 
 
 def mxfp4_qdq_fwd_bwd(x: torch.Tensor, grad_out: torch.Tensor, *, grad_direction: str = "rowwise",
@@ -248,24 +360,32 @@ def mxfp4_qdq_fwd_bwd(x: torch.Tensor, grad_out: torch.Tensor, *, grad_direction
                       rowwise: bool = True, colwise: bool = False, group_list=None, group_list_type: int = 0,
                       emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
                       out: QDQResult | None = None, grad_in: torch.Tensor | None = None,
-                      elem_format: str = "e2m1"):
-    """Fused forward + clipped-STE backward; returns (QDQResult, grad_in)."""
+                      elem_format: str = "e2m1", check: bool | None = None):
+    """Fused forward + clipped-STE backward; returns (QDQResult, grad_in).
+    A group_list is checked as in mxfp4_qdq_fwd (check defaults to True with
+    one; with check=False read the returned status before using anything)."""
     x = _as_2d(x)
     g = _as_2d(grad_out, "grad_out").contiguous()
     if g.shape != x.shape or g.dtype != x.dtype:
         raise ValueError("x and grad_out must have the same shape and dtype")
     gl, ng = _group_args(group_list, group_list_type, x.device)
+    if check is None:
+        check = gl is not None and colwise
     dirs = (_abi.ROWWISE if rowwise else 0) | (_abi.COLWISE if colwise else 0)
     r = out if out is not None else alloc_outputs(
         x, block=block, rowwise=rowwise, colwise=colwise, num_groups=ng, emit_values=emit_values,
-        emit_codes=emit_codes, emit_mask=emit_mask, with_status=gl is not None, elem_format=elem_format)
-    gi = grad_in if grad_in is not None else torch.empty_like(g)
+        emit_codes=emit_codes, emit_mask=emit_mask, with_status=check or gl is not None, elem_format=elem_format)
+    if check and r.status is None:
+        r.status = torch.empty((1,), dtype=torch.int32, device=x.device)
+    gi = _grad_buffer(grad_in, g, g.shape, "grad_in")
     a = make_args(x, block=block, scale_factor=scale_factor, scale_mode=scale_mode, dirs=dirs,
                   group_list=gl, group_list_type=group_list_type, status=r.status, elem_format=r.elem_format)
-    _fill_outputs(a, r)
+    _fill_outputs(a, r, x)
     st = _abi.mxfp4_qdq_fwd_bwd(a, g.data_ptr(), gi.data_ptr(), g.shape[1], _DIRS[grad_direction],
                                 _stream(x.device))
     _abi.check(st, "mxfp4_qdq_fwd_bwd")
+    if check:
+        _check_status(r.status, "mxfp4_qdq_fwd_bwd")
     return r, gi
 
 

@@ -1,12 +1,26 @@
-"""Page-level API over the CUDA library: differentiable MXFP4 fake quantisation
-and a quantisation-aware-training Linear.
+"""Quantisation-aware training over the CUDA library.
 
-Mirrors the public surface of amct pull request 264, mxfp4_qat/fake_quant.py
-and linear.py (mxfp4_quant_dequant, mxfp4_saturation_mask, mxfp4_fake_quant,
-MXFP4FakeQuantizer, MXFP4QATConfig, MXFP4QATLinear, convert_to_mxfp4_qat),
-with the backend switch replaced by the one CUDA path and a scale_mode
-argument added ("page": 2^round(log2(amax/scale_factor)), "floor":
-2^(floor(log2 amax) - 2)). Blocks run along the last dimension.
+Public surface (names and signatures as in amct pull request 264,
+mxfp4_qat/fake_quant.py and mxfp4_qat/linear.py, so that code written
+against that page runs unchanged):
+
+  mxfp4_quant_dequant(x, ...)      fake-quantised copy of x, no autograd
+  mxfp4_saturation_mask(x, ...)    bool tensor, True where |x| > 6 * 2^k
+  mxfp4_fake_quant(x, ...)         differentiable QDQ, plain or clipped STE
+  MXFP4FakeQuantizer               module form of mxfp4_fake_quant
+  MXFP4QATConfig                   what a converted layer quantises, and how
+  MXFP4QATLinear                   nn.Linear computing linear(Q(x), Q(W), b)
+  convert_to_mxfp4_qat(model, ..)  swaps the model's nn.Linear layers in place
+
+Blocks run along the last dimension. Every quantisation is one call of the
+library (values and, for the clipped STE, the bit-packed saturation mask in
+the same pass); the backward is one masking kernel over the saved mask. The
+page's backend switch is not offered: there is one CUDA path. scale_mode
+selects the scale rule ("page": 2^round(log2(amax / scale_factor)) with the
+2^-30 floor; "floor": 2^max(floor(log2 amax) - 2, -127)).
+
+Nothing here holds a parameter or a buffer of its own: a converted model has
+the same state_dict keys and tensors as the float model.
 """
 from __future__ import annotations
 
@@ -22,101 +36,123 @@ BLOCK_SIZE = 32
 SCALE_FACTOR = 6.0
 MXFP4_E2M1_MAX = 6.0
 
+_BLOCKS = (32, 128)
+_RULES = ("page", "floor")
 
-def _validate(block_size: int, scale_factor: float, scale_mode: str = "page") -> None:
-    # fake_quant.py _validate: non-positive block_size / scale_factor are errors
-    if block_size <= 0:
-        raise ValueError(f"block_size must be positive, got {block_size}")
-    if scale_factor <= 0:
-        raise ValueError(f"scale_factor must be positive, got {scale_factor}")
-    if block_size not in (32, 128):
-        raise ValueError(f"block_size must be 32 or 128 on this path, got {block_size}")
-    if scale_mode not in ("page", "floor"):
-        raise ValueError(f"scale_mode must be 'page' or 'floor', got {scale_mode!r}")
+
+@dataclasses.dataclass(frozen=True)
+class _Spec:
+    """One validated quantisation setting (block length, scale divisor, rule)."""
+
+    block: int
+    divisor: float
+    rule: str
+
+    @staticmethod
+    def of(block_size, scale_factor, scale_mode) -> "_Spec":
+        if isinstance(block_size, bool) or int(block_size) != block_size or block_size not in _BLOCKS:
+            raise ValueError(f"MXFP4 blocks hold 32 or 128 elements here; block_size={block_size!r}")
+        sf = float(scale_factor)
+        if not sf > 0.0 or sf == float("inf"):
+            raise ValueError(f"the scale divisor must be a finite positive number; scale_factor={scale_factor!r}")
+        if scale_mode not in _RULES:
+            raise ValueError(f"scale_mode selects the scale rule and is 'page' or 'floor'; got {scale_mode!r}")
+        return _Spec(int(block_size), sf, scale_mode)
+
+    def qdq(self, x: torch.Tensor, *, values: bool = True, mask: bool = False) -> ops.QDQResult:
+        if x.ndim == 0:
+            raise ValueError("a 0-dim tensor has no last dimension to block")
+        return ops.mxfp4_qdq_fwd(x, block=self.block, scale_factor=self.divisor, scale_mode=self.rule,
+                                 emit_values=values, emit_mask=mask)
+
+
+def unpack_mask(packed: torch.Tensor, cols: int) -> torch.Tensor:
+    """Bit-packed saturation mask [rows, ceil(cols/8)] (bit b of byte j is
+    column 8j + b) -> bool [rows, cols]."""
+    weights = torch.tensor([1 << b for b in range(8)], dtype=torch.uint8, device=packed.device)
+    spread = torch.bitwise_and(packed.unsqueeze(-1), weights) != 0
+    return spread.flatten(-2)[..., :cols]
 
 
 def mxfp4_quant_dequant(x: torch.Tensor, block_size: int = BLOCK_SIZE, scale_factor: float = SCALE_FACTOR,
                         scale_mode: str = "page") -> torch.Tensor:
-    """QDQ without autograd; same shape, dtype and device as x."""
-    _validate(block_size, scale_factor, scale_mode)
-    if x.ndim == 0:
-        raise ValueError("x must have at least 1 dimension")
-    r = ops.mxfp4_qdq_fwd(x, block=block_size, scale_factor=scale_factor, scale_mode=scale_mode)
-    return r.y_row.view(x.shape)
-
-
-def unpack_mask(packed: torch.Tensor, cols: int) -> torch.Tensor:
-    """Bit-packed [rows, ceil(cols/8)] -> bool [rows, cols]."""
-    shifts = torch.arange(8, device=packed.device, dtype=torch.uint8)
-    bits = (packed.unsqueeze(-1) >> shifts) & 1
-    return bits.reshape(packed.shape[0], -1)[:, :cols].bool()
+    """x fake-quantised to MXFP4 (same shape, dtype and device); no graph is
+    recorded."""
+    return _Spec.of(block_size, scale_factor, scale_mode).qdq(x).y_row.view(x.shape)
 
 
 def mxfp4_saturation_mask(x: torch.Tensor, block_size: int = BLOCK_SIZE, scale_factor: float = SCALE_FACTOR,
                           scale_mode: str = "page") -> torch.Tensor:
-    """bool mask, True where |x| > 6 * block scale (the clipped elements)."""
-    _validate(block_size, scale_factor, scale_mode)
-    r = ops.mxfp4_qdq_fwd(x, block=block_size, scale_factor=scale_factor, scale_mode=scale_mode,
-                          emit_values=False, emit_mask=True)
+    """Where x was clipped: True for |x| > 6 * 2^k of its block (those are the
+    elements whose gradient the clipped STE drops)."""
+    r = _Spec.of(block_size, scale_factor, scale_mode).qdq(x, values=False, mask=True)
     return unpack_mask(r.mask_row, x.shape[-1]).view(x.shape)
 
 
 class _MXFP4FakeQuantSTE(torch.autograd.Function):
-    """Forward: one kernel writes the QDQ values (and, for the clipped STE, the
-    bit-packed saturation mask). Backward: one kernel masks the gradient."""
+    """QDQ forward with a straight-through backward. The clipped variant keeps
+    the forward's bit-packed saturation mask (one bit per element) and zeroes
+    the gradient there; the plain variant passes the gradient unchanged."""
 
     @staticmethod
     def forward(ctx, x, block_size, scale_factor, clip_grad, scale_mode):
-        ctx.clip_grad = clip_grad
-        ctx.meta = (block_size, scale_factor, scale_mode)
-        r = ops.mxfp4_qdq_fwd(x, block=block_size, scale_factor=scale_factor, scale_mode=scale_mode,
-                              emit_mask=clip_grad)
-        if clip_grad:
+        spec = _Spec.of(block_size, scale_factor, scale_mode)
+        r = spec.qdq(x, mask=bool(clip_grad))
+        ctx.spec = spec
+        ctx.clip = bool(clip_grad)
+        if ctx.clip:
             ctx.save_for_backward(r.mask_row)
         return r.y_row.view(x.shape)
 
     @staticmethod
     def backward(ctx, grad_output):
-        if not ctx.clip_grad:
-            return grad_output, None, None, None, None
-        (mask,) = ctx.saved_tensors
-        block_size, scale_factor, scale_mode = ctx.meta
-        g = ops.mxfp4_ste_bwd(grad_output.contiguous(), saved_mask=mask, clip_grad=True, block=block_size,
-                              scale_factor=scale_factor, scale_mode=scale_mode)
+        g = grad_output
+        if ctx.clip:
+            (mask,) = ctx.saved_tensors
+            s = ctx.spec
+            g = ops.mxfp4_ste_bwd(grad_output, saved_mask=mask, clip_grad=True, block=s.block,
+                                  scale_factor=s.divisor, scale_mode=s.rule)
         return g, None, None, None, None
 
 
 def mxfp4_fake_quant(x: torch.Tensor, block_size: int = BLOCK_SIZE, scale_factor: float = SCALE_FACTOR,
                      clip_grad: bool = False, scale_mode: str = "page") -> torch.Tensor:
-    """Differentiable MXFP4 fake quantisation with a plain or clipped STE."""
-    _validate(block_size, scale_factor, scale_mode)
+    """Differentiable MXFP4 fake quantisation: the forward is
+    mxfp4_quant_dequant, the backward a straight-through estimator (clip_grad:
+    saturated elements get a zero gradient)."""
+    _Spec.of(block_size, scale_factor, scale_mode)
     return _MXFP4FakeQuantSTE.apply(x, block_size, scale_factor, clip_grad, scale_mode)
 
 
 class MXFP4FakeQuantizer(nn.Module):
-    """Stateless module form of mxfp4_fake_quant (no parameters or buffers, so a
-    model's state_dict is unchanged by inserting it)."""
+    """mxfp4_fake_quant as a module. It registers no parameter and no buffer,
+    so inserting it leaves a model's state_dict as it was."""
 
     def __init__(self, block_size: int = BLOCK_SIZE, scale_factor: float = SCALE_FACTOR,
                  clip_grad: bool = False, scale_mode: str = "page") -> None:
         super().__init__()
-        _validate(block_size, scale_factor, scale_mode)
-        self.block_size = block_size
-        self.scale_factor = scale_factor
-        self.clip_grad = clip_grad
-        self.scale_mode = scale_mode
+        self._spec = _Spec.of(block_size, scale_factor, scale_mode)
+        self.clip_grad = bool(clip_grad)
+
+    block_size = property(lambda self: self._spec.block)
+    scale_factor = property(lambda self: self._spec.divisor)
+    scale_mode = property(lambda self: self._spec.rule)
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
-        return mxfp4_fake_quant(x, self.block_size, self.scale_factor, self.clip_grad, self.scale_mode)
+        s = self._spec
+        return _MXFP4FakeQuantSTE.apply(x, s.block, s.divisor, self.clip_grad, s.rule)
 
     def extra_repr(self) -> str:
-        return (f"block_size={self.block_size}, scale_factor={self.scale_factor}, "
-                f"clip_grad={self.clip_grad}, scale_mode={self.scale_mode!r}")
+        s = self._spec
+        ste = "clipped" if self.clip_grad else "plain"
+        return f"E2M1 x {s.block}, rule={s.rule}, divisor={s.divisor:g}, STE {ste}"
 
 
 @dataclasses.dataclass
 class MXFP4QATConfig:
-    """Settings shared by converted layers (quantize_input=False is W4A16)."""
+    """What a converted layer fake-quantises and with which settings. The
+    defaults quantise the weight only (W4A16); quantize_input adds the layer
+    input (W4A4)."""
 
     quantize_weight: bool = True
     quantize_input: bool = False
@@ -126,55 +162,77 @@ class MXFP4QATConfig:
     scale_mode: str = "page"
 
     def __post_init__(self) -> None:
-        _validate(self.block_size, self.scale_factor, self.scale_mode)
+        _Spec.of(self.block_size, self.scale_factor, self.scale_mode)
 
     def make_quantizer(self) -> MXFP4FakeQuantizer:
         return MXFP4FakeQuantizer(self.block_size, self.scale_factor, self.clip_grad, self.scale_mode)
 
 
 class MXFP4QATLinear(nn.Linear):
-    """nn.Linear computing F.linear(Q(x), Q(W), b); the bias is not quantised and
-    the master weight stays in its own precision (the STE routes its gradient)."""
+    """nn.Linear whose forward is linear(Q(x), Q(W), b): Q fake-quantises
+    (MXFP4, blocks along the input features), the bias stays as it is. The
+    optimiser updates the unquantised master weight; the STE carries the
+    gradient of Q(W) back to it. As an nn.Linear with stateless quantizers it
+    has exactly the float layer's state_dict."""
 
     def __init__(self, in_features: int, out_features: int, bias: bool = True, device=None, dtype=None,
                  config: MXFP4QATConfig | None = None) -> None:
         super().__init__(in_features, out_features, bias, device=device, dtype=dtype)
-        self.config = config if config is not None else MXFP4QATConfig()
-        self.weight_quantizer = self.config.make_quantizer() if self.config.quantize_weight else None
-        self.input_quantizer = self.config.make_quantizer() if self.config.quantize_input else None
+        self._attach(config)
+
+    def _attach(self, config: MXFP4QATConfig | None) -> None:
+        self.config = MXFP4QATConfig() if config is None else config
+        c = self.config
+        self.weight_quantizer = c.make_quantizer() if c.quantize_weight else None
+        self.input_quantizer = c.make_quantizer() if c.quantize_input else None
 
     @classmethod
     def from_linear(cls, linear: nn.Linear, config: MXFP4QATConfig | None = None) -> "MXFP4QATLinear":
-        """Adopt an existing layer's Parameter objects (no copy, optimiser state stays valid)."""
-        layer = cls(linear.in_features, linear.out_features, bias=linear.bias is not None, device="meta",
-                    dtype=linear.weight.dtype, config=config)
+        """A QAT layer that takes over linear's own Parameter objects: nothing
+        is allocated or copied, and an optimiser that already holds those
+        parameters keeps training them."""
+        layer = cls.__new__(cls)
+        nn.Module.__init__(layer)
+        layer.in_features, layer.out_features = linear.in_features, linear.out_features
         layer.weight = linear.weight
-        if linear.bias is not None:
-            layer.bias = linear.bias
+        layer.register_parameter("bias", linear.bias)
+        layer._attach(config)
+        layer.train(linear.training)
         return layer
 
     def forward(self, input: torch.Tensor) -> torch.Tensor:
-        if self.input_quantizer is not None:
-            input = self.input_quantizer(input)
         w = self.weight if self.weight_quantizer is None else self.weight_quantizer(self.weight)
-        return F.linear(input, w, self.bias)
+        x = input if self.input_quantizer is None else self.input_quantizer(input)
+        return F.linear(x, w, self.bias)
 
 
 def convert_to_mxfp4_qat(module: nn.Module, config: MXFP4QATConfig | None = None,
                          skip_names: tuple[str, ...] = ()) -> nn.Module:
-    """Replace every nn.Linear (subclasses included) under module in place;
-    dotted paths containing any of skip_names are left alone; converting twice
-    is a no-op. Returns module."""
+    """Swap, in place, every nn.Linear below `module` (subclasses included)
+    for an MXFP4QATLinear that adopts its parameters, and return `module`.
 
-    def walk(m: nn.Module, prefix: str) -> None:
-        for name, child in list(m.named_children()):
-            path = prefix + name
-            if any(s in path for s in skip_names) or isinstance(child, MXFP4QATLinear):
-                continue
-            if isinstance(child, nn.Linear):
-                setattr(m, name, MXFP4QATLinear.from_linear(child, config))
-            else:
-                walk(child, path + ".")
-
-    walk(module, "")
+    skip_names are substrings of dotted module paths ("encoder.layers.0.fc");
+    a module whose path contains one is left as it is, with everything below
+    it. Layers that are already MXFP4QATLinear stay untouched, so a second
+    call changes nothing. A layer reachable under several paths (tied or
+    shared) becomes one QAT layer at all of them. `module` itself is never
+    replaced, even when it is an nn.Linear."""
+    swaps: list[tuple[str, nn.Linear]] = []
+    inside: list[str] = []  # paths of Linear layers: their own children are theirs
+    for path, sub in module.named_modules(remove_duplicate=False):
+        if not path or any(path.startswith(p + ".") for p in inside):
+            continue
+        if any(s in path for s in skip_names):
+            continue
+        if isinstance(sub, nn.Linear):
+            inside.append(path)
+            if not isinstance(sub, MXFP4QATLinear):
+                swaps.append((path, sub))
+    made: dict[int, MXFP4QATLinear] = {}
+    for path, lin in swaps:
+        parent_path, _, name = path.rpartition(".")
+        parent = module.get_submodule(parent_path) if parent_path else module
+        if id(lin) not in made:
+            made[id(lin)] = MXFP4QATLinear.from_linear(lin, config)
+        setattr(parent, name, made[id(lin)])
     return module

@@ -178,3 +178,29 @@ def test_product_code_never_imports_the_oracle():
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
                 assert "liboracle" not in text and "mxfp4_oracle" not in text, f
     _ = sys
+
+
+def test_layout_predicate_copies_expanded_and_overlapping_inputs():
+    """The binding passes a tensor's own pitch to the library only when its
+    rows are [rows][ld] with ld >= cols and unit column stride; expanded
+    (row stride 0), overlapping (0 < row stride < cols) and transposed
+    inputs are copied first."""
+    import torch
+
+    from mxfp4_block_fake_b200.ops import rows_addressable
+
+    base = torch.zeros(8, 64)
+    assert rows_addressable(tuple(base.shape), tuple(base.stride()))
+    padded = torch.zeros(8, 80)[:, :64]
+    assert rows_addressable(tuple(padded.shape), tuple(padded.stride()))
+    expanded = torch.zeros(1, 64).expand(8, 64)
+    assert expanded.stride(0) == 0
+    assert not rows_addressable(tuple(expanded.shape), tuple(expanded.stride()))
+    overlap = torch.zeros(200).as_strided((8, 64), (16, 1))
+    assert not rows_addressable(tuple(overlap.shape), tuple(overlap.stride()))
+    transposed = torch.zeros(64, 8).t()
+    assert not rows_addressable(tuple(transposed.shape), tuple(transposed.stride()))
+    one_row = torch.zeros(1, 64).expand(1, 64)
+    assert rows_addressable(tuple(one_row.shape), tuple(one_row.stride()))
+    one_col = torch.zeros(8, 5)[:, 2:3]
+    assert rows_addressable(tuple(one_col.shape), tuple(one_col.stride()))

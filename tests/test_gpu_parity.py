@@ -8,9 +8,8 @@ Shapes span several tiles plus ragged tails (rows not a multiple of the block,
 cols not a multiple of the block, of 8, or of the tile width), strided and
 unaligned inputs (the generic kernels), empty tensors, group lists with empty
 groups and partial tail blocks, every finite bf16 value as element and as
-block maximum, and (test_full_size_sampled) the full sizes of the workloads
-in the launch configuration the benchmark times, checked on sampled rows and
-columns.
+block maximum. The workloads at their full sizes, compared in full, are in
+test_gpu_full_size.py.
 """
 from __future__ import annotations
 
@@ -320,6 +319,22 @@ def test_every_bf16_value_values_only(mode, scales):
     check_dir(r, ora, "row", 256, label="values only")
 
 
+@pytest.mark.parametrize("mode", ["page", "floor"])
+@pytest.mark.parametrize("counts", [None, [32], [16, 0, 16]])
+def test_every_bf16_value_block32_along_columns(mode, counts):
+    """The block-32 sweep laid along columns (the transpose: 32 rows, one
+    column per sweep block) through the staged dual kernel, every output of
+    both directions: every finite bf16 value as element and as column-block
+    maximum, in the low and the high half of a 32-bit word. Ungrouped, with
+    one group, and with groups that cut every column block into two tails
+    (the group-tail path of the kernel)."""
+    xb = np.ascontiguousarray(bf16_sweep_block32().T)  # [32, 589824]
+    x = torch.from_numpy(xb.view(np.int16).copy()).view(torch.bfloat16)
+    res, ora = run_both(x, block=32, mode=mode, rowwise=True, colwise=True, counts=counts)
+    check_dir(res, ora["row"], "row", xb.shape[1], label="bf16 sweep along columns")
+    check_dir(res, ora["col"], "col", xb.shape[1], label="bf16 sweep along columns")
+
+
 def codes_only(x: torch.Tensor, mode: str, layout: str):
     res = ops.mxfp4_qdq_fwd(x.cuda(), block=32, scale_mode=mode, rowwise=True, emit_values=False,
                             emit_codes=True, emit_mask=True, scales_layout=layout, check=True)
@@ -472,104 +487,6 @@ def test_empty_inputs():
         ops.mxfp4_qdq_fwd(torch.tensor(1.0, device="cuda"))
 
 
-def test_qat_linear_tiny_fwd_bwd():
-    """Tiny QAT linear, fp32 x [4,64] and W [32,64], block 32 along the last dim:
-    forward y = Q(x) Q(W)^T, clipped-STE grads for grad_out = ones."""
-    from mxfp4_block_fake_b200 import MXFP4QATConfig, MXFP4QATLinear
-    torch.backends.cuda.matmul.allow_tf32 = False
-    x, w = W.qat_linear_tiny()
-    for clip in (False, True):
-        lin = MXFP4QATLinear(64, 32, bias=False, config=MXFP4QATConfig(quantize_input=True, clip_grad=clip))
-        with torch.no_grad():
-            lin.weight.copy_(w)
-        lin = lin.cuda()
-        xd = x.cuda().requires_grad_(True)
-        y = lin(xd)
-        y.backward(torch.ones_like(y))
-        qx = O.qdq_rowwise(x.numpy(), 32, 6.0, O.SCALE_PAGE)
-        qw = O.qdq_rowwise(w.numpy(), 32, 6.0, O.SCALE_PAGE)
-        # products of <=2-significant-bit values summed over 64 terms: exact in float64
-        y_exp = qx["y"].astype(np.float64) @ qw["y"].astype(np.float64).T
-        np.testing.assert_allclose(y.detach().cpu().numpy(), y_exp, rtol=2e-7, atol=0)
-        ones = np.ones((4, 32))
-        dx = ones @ qw["y"].astype(np.float64)
-        dw = ones.T @ qx["y"].astype(np.float64)
-        if clip:
-            dx = np.where(O.unpack_bits(qx["mask"], 64), 0.0, dx)
-            dw = np.where(O.unpack_bits(qw["mask"], 64), 0.0, dw)
-        np.testing.assert_allclose(xd.grad.cpu().numpy(), dx, rtol=2e-7, atol=0)
-        np.testing.assert_allclose(lin.weight.grad.cpu().numpy(), dw, rtol=2e-7, atol=0)
-
-
-def _sample_full(x: torch.Tensor, xd: torch.Tensor, res: ops.QDQResult, rowwise: bool, colwise: bool,
-                 mode: str, block: int, ends=None, nsamp: int = 256, seed: int = 0):
-    """Compare sampled rows (row-wise) and sampled columns (column-wise, all
-    row-blocks) of full-size outputs with the oracle run on those slices."""
-    rng = np.random.default_rng(seed)
-    rows, cols = x.shape
-    if rowwise:
-        ri = np.sort(rng.choice(rows, size=min(nsamp, rows), replace=False))
-        rit = torch.from_numpy(ri).cuda()
-        ora = O.qdq_rowwise(oracle_in(x[torch.from_numpy(ri)]), block, 6.0, MODES[mode])
-        sub = ops.QDQResult(y_row=res.y_row[rit], codes_row=None if res.codes_row is None else res.codes_row[rit],
-                            scales_row=None if res.scales_row is None else res.scales_row[rit],
-                            mask_row=None if res.mask_row is None else res.mask_row[rit])
-        check_dir(sub, ora, "row", cols, label="full-size rows")
-    if colwise:
-        # whole aligned octets of columns so that mask and code bytes compare directly
-        oc = np.sort(rng.choice(cols // 8, size=min(nsamp // 8, cols // 8), replace=False))
-        ci = (oc[:, None] * 8 + np.arange(8)).reshape(-1)
-        cit = torch.from_numpy(ci).cuda()
-        ora = O.qdq_colwise(oracle_in(x[:, torch.from_numpy(ci)]), block, 6.0, MODES[mode], ends=ends)
-        s = ora["scales"].shape[0]
-        assert np.array_equal(np_bits(res.y_col[:, cit]), ora_bits(ora["y"]))
-        if res.codes_col is not None:
-            bc = torch.from_numpy((oc[:, None] * 4 + np.arange(4)).reshape(-1)).cuda()
-            assert np.array_equal(np_bits(res.codes_col[:, bc]), ora["codes"])
-            assert np.array_equal(np_bits(res.scales_col[:s][:, cit]), ora["scales"])
-        if res.mask_col is not None:
-            assert np.array_equal(np_bits(res.mask_col[:, torch.from_numpy(oc).cuda()]), ora["mask"])
-
-
-@pytest.mark.parametrize("name", ["act_rowwise", "weight_dual", "train_step", "moe_grouped"])
-def test_full_size_sampled(name):
-    """Full workload sizes, launched exactly as the benchmark launches them."""
-    torch.cuda.empty_cache()
-    if name == "act_rowwise":
-        x = W.act_rowwise()
-        xd = x.cuda()
-        res = ops.mxfp4_qdq_fwd(xd, emit_codes=True)
-        _sample_full(x, xd, res, True, False, "page", 32)
-    elif name == "weight_dual":
-        x = W.weight_dual()
-        xd = x.cuda()
-        for block in (32, 128):
-            res = ops.mxfp4_qdq_fwd(xd, block=block, rowwise=True, colwise=True, emit_codes=True)
-            _sample_full(x, xd, res, True, True, "page", block)
-    elif name == "train_step":
-        x, g = W.train_step()
-        xd, gd = x.cuda(), g.cuda()
-        res = ops.mxfp4_qdq_fwd(xd, emit_mask=True)
-        gi = ops.mxfp4_ste_bwd(gd, x=xd, clip_grad=True)
-        gi2 = ops.mxfp4_ste_bwd(gd, saved_mask=res.mask_row, clip_grad=True)
-        _sample_full(x, xd, res, True, False, "page", 32)
-        assert torch.equal(gi.view(torch.int16), gi2.view(torch.int16))
-        rng = np.random.default_rng(1)
-        ri = torch.from_numpy(np.sort(rng.choice(x.shape[0], 256, replace=False)))
-        ora = O.qdq_rowwise(oracle_in(x[ri]), 32, 6.0, O.SCALE_PAGE)
-        exp = O.ste_bwd(oracle_in(g[ri]), ora["mask"], True)
-        assert np.array_equal(np_bits(gi[ri.cuda()]), exp)
-    else:
-        x, counts, offsets = W.moe_grouped()
-        xd = x.cuda()
-        gl = offsets.cuda()
-        for mode in ("page", "floor"):
-            res = ops.mxfp4_qdq_fwd(xd, scale_mode=mode, rowwise=True, colwise=True, group_list=gl,
-                                    emit_codes=True, emit_mask=True, check=True)
-            _sample_full(x, xd, res, True, True, mode, 32, ends=offsets.numpy(), seed=3)
-    torch.cuda.synchronize()
-
-
 def test_cuda_graph_capture_and_replay():
     """The forward (dual, grouped, all outputs) and the STE backward capture
     into one CUDA graph: no host synchronisation or allocation on the path.
@@ -586,7 +503,8 @@ def test_cuda_graph_capture_and_replay():
     gi = torch.empty_like(gd)
 
     def step():
-        ops.mxfp4_qdq_fwd(xd, rowwise=True, colwise=True, group_list=gl, emit_codes=True, emit_mask=True, out=r)
+        ops.mxfp4_qdq_fwd(xd, rowwise=True, colwise=True, group_list=gl, emit_codes=True, emit_mask=True, out=r,
+                          check=False)
         ops.mxfp4_ste_bwd(gd, saved_mask=r.mask_row, clip_grad=True, out=gi)
 
     s = torch.cuda.Stream()
@@ -614,51 +532,3 @@ def test_cuda_graph_capture_and_replay():
     ora = O.qdq_rowwise(oracle_in(xs[0]), 32, 6.0, O.SCALE_PAGE)
     check_dir(r, ora, "row", cols, label="graph replay")
     del graph
-
-
-def test_full_size_bench_modes_sampled():
-    """The other calls the benchmark times, at its full size (MoE activation
-    65536 x 7168), checked on sampled rows and columns: the real-quantisation
-    producer (codes + MMA-layout scales, no values) and MXFP8 in both
-    directions with the groups."""
-    torch.cuda.empty_cache()
-    x, counts, offsets = W.moe_grouped()
-    xd = x.cuda()
-    gl = offsets.cuda()
-    rows, cols = x.shape
-    rng = np.random.default_rng(11)
-    ri = np.sort(rng.choice(rows, size=256, replace=False))
-    rit = torch.from_numpy(ri).cuda()
-    # producer: codes of sampled rows; scale bytes at the positions the
-    # oracle's layout gives the sampled rows
-    codes, scales = ops.mxfp4_mma_operand(xd)
-    torch.cuda.synchronize()
-    ora = O.qdq_rowwise(oracle_in(x[torch.from_numpy(ri)]), 32, 6.0, O.SCALE_PAGE)
-    assert np.array_equal(np_bits(codes.view(torch.uint8)[rit]), ora["codes"])
-    nblk = cols // 32
-    full = np.zeros((rows, nblk), np.uint8)
-    full[ri] = ora["scales"]
-    sel = np.zeros((rows, nblk), np.uint8)
-    sel[ri] = 1
-    pos = O.mma_scale_layout(sel) == 1
-    got = np_bits(scales.view(torch.uint8))
-    assert np.array_equal(got[pos], O.mma_scale_layout(full)[pos])
-    del codes, scales
-    # MXFP8, both directions, grouped
-    res = ops.mxfp4_qdq_fwd(xd, block=32, scale_mode="floor", rowwise=True, colwise=True, group_list=gl,
-                            emit_codes=True, emit_mask=True, check=True, elem_format="e4m3")
-    torch.cuda.synchronize()
-    o8 = O.qdq8_rowwise(oracle_in(x[torch.from_numpy(ri)]))
-    assert np.array_equal(np_bits(res.y_row[rit]), o8["y"])
-    assert np.array_equal(np_bits(res.codes_row[rit]), o8["codes"])
-    assert np.array_equal(np_bits(res.scales_row[rit]), o8["scales"])
-    assert np.array_equal(np_bits(res.mask_row[rit]), o8["mask"])
-    oc = np.sort(rng.choice(cols // 8, size=16, replace=False))
-    ci = (oc[:, None] * 8 + np.arange(8)).reshape(-1)
-    cit = torch.from_numpy(ci).cuda()
-    c8 = O.qdq8_colwise(oracle_in(x[:, torch.from_numpy(ci)]), offsets.numpy())
-    s = c8["scales"].shape[0]
-    assert np.array_equal(np_bits(res.y_col[:, cit]), c8["y"])
-    assert np.array_equal(np_bits(res.codes_col[:, cit]), c8["codes"])
-    assert np.array_equal(np_bits(res.scales_col[:s][:, cit]), c8["scales"])
-    assert np.array_equal(np_bits(res.mask_col[:, torch.from_numpy(oc).cuda()]), c8["mask"])

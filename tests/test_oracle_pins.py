@@ -462,3 +462,33 @@ def test_mma_scale_layout_is_a_placement(oracle_mod):
     nz = O.mma_scale_layout(np.ones((R, C), np.uint8)) == 1
     assert nz.sum() == R * C and placed.size == 512 * 3 * 2
     assert np.array_equal(np.sort(placed[nz]), np.arange(R * C))
+
+
+def test_threaded_oracle_equals_single_calls():
+    """The chunked, threaded runner used by the full-size GPU tests returns
+    exactly what one oracle call over the whole array returns (ragged row and
+    column counts, groups with empty members and tails, both formats)."""
+    import oracle as O
+    from tests import oracle_par as OP
+
+    rng = np.random.default_rng(5)
+    for rows, cols in ((301, 1000), (64, 4104), (7, 37)):
+        xb = rng.integers(0, 1 << 16, (rows, cols), dtype=np.uint64).astype(np.uint16)
+        xb[:, ::7] &= 0x3FFF  # plenty of finite values next to the random patterns
+        ends = np.cumsum([0, rows // 3, 0, rows - rows // 3]).astype(np.int64)[1:]
+        for mode in (O.SCALE_PAGE, O.SCALE_FLOOR):
+            for block in (32, 128):
+                a, b = OP.qdq_rowwise(xb, block, 6.0, mode), O.qdq_rowwise(xb, block, 6.0, mode)
+                for k in a:
+                    assert np.array_equal(a[k], b[k]), (rows, cols, k)
+                a, b = OP.qdq_colwise(xb, block, 6.0, mode, ends), O.qdq_colwise(xb, block, 6.0, mode, ends)
+                for k in a:
+                    assert np.array_equal(a[k], b[k]), (rows, cols, k)
+        a, b = OP.qdq8_rowwise(xb), O.qdq8_rowwise(xb)
+        for k in a:
+            assert np.array_equal(a[k], b[k])
+        a, b = OP.qdq8_colwise(xb, ends), O.qdq8_colwise(xb, ends)
+        for k in a:
+            assert np.array_equal(a[k], b[k])
+        m = O.qdq_rowwise(xb, 32, 6.0, O.SCALE_PAGE)["mask"]
+        assert np.array_equal(OP.ste_bwd(xb, m, True), O.ste_bwd(xb, m, True))
