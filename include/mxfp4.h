@@ -132,7 +132,43 @@ typedef enum {
 #define MXFP4_SCALES_ROWMAJOR 0
 #define MXFP4_SCALES_MMA 1
 
-#define MXFP4_ABI_VERSION 3
+/* Layouts of codes_col and scales_col (mxfp4_qdq_args.col_layout).
+ *
+ * MXFP4_COLS_ROWMAJOR (0): as described at the top of this file.
+ *
+ * MXFP4_COLS_MMA: the column-wise result as the operand of a block-scaled
+ * tensor-core GEMM that contracts over the rows, group by group -- the
+ * weight-gradient GEMM of a grouped linear layer, which multiplies the
+ * column-wise views of activations and gradients transposed (MindSpore
+ * hyper-parallel fake_w4a8_gmm_func.py, FakeW4A8GroupedLinear._select_operands,
+ * layout "TN"; the page fixes no byte layout, this is the library's). Each
+ * group's K range is its rows padded to a multiple of 128 (four blocks of 32,
+ * one column of scale atoms); group g starts at K slot
+ * K0_g = sum_{j<g} 128 * ceil(n_j / 128), and k_alloc (a multiple of 128, at
+ * least the sum over all groups; mxfp4_colwise_operand_k) is the K extent of
+ * the buffers:
+ *   codes_col   [cols][k_alloc / 2] bytes, 16-byte aligned: the E2M1 nibble of
+ *               x[first row of g + t][c] is in byte c * k_alloc/2 + (K0_g + t)/2,
+ *               the low nibble for even t; slots t >= n_g of the group's padded
+ *               range hold 0. Row c is K-major: the operand as it stands.
+ *   scales_col  the [cols][k_alloc / 32] E8M0 matrix whose entry
+ *               (c, K0_g/32 + b) is the scale of block b of group g in column c
+ *               (127 for the padding blocks of a group), in the 128 x 4 atom
+ *               layout of MXFP4_SCALES_MMA; 2-byte aligned;
+ *               mxfp4_colwise_operand_scale_bytes() bytes. Atom rows past cols
+ *               and K slots past the last group are not written.
+ * Group g's operand is then the [cols][128 ceil(n_g/128)] sub-matrix at K0_g
+ * (row stride k_alloc/2 bytes) with the atom columns from K0_g/128 on.
+ * Requires bf16 x (4-byte aligned, even ld), block 32, E2M1, and in PAGE mode
+ * a scale_factor in [2^-64, 11] (else MXFP4_EUNSUPPORTED); no fused backward.
+ * y_col and mask_col, when also given, keep their row-major layout. An
+ * invalid group_list, or groups whose padded K exceeds k_alloc, write no
+ * operand byte and set status to MXFP4_EINVAL.
+ */
+#define MXFP4_COLS_ROWMAJOR 0
+#define MXFP4_COLS_MMA 1
+
+#define MXFP4_ABI_VERSION 4
 
 /*
  * Arguments of one QDQ call. Zero-initialise and fill what is used; every
@@ -157,6 +193,10 @@ typedef enum {
  *                  MXFP4 block-scaled GEMM whose K dimension is `cols`
  *                  (codes_row is then its K-major E2M1 operand as is).
  *   elem_format    MXFP4_ELEM_E2M1 (0, MXFP4) or MXFP4_ELEM_E4M3 (MXFP8).
+ *   col_layout     MXFP4_COLS_ROWMAJOR (0) or MXFP4_COLS_MMA (the K-major
+ *                  GEMM operand layout of codes_col / scales_col).
+ *   k_alloc        MXFP4_COLS_MMA only: K slots per codes_col row (a multiple
+ *                  of 128, >= mxfp4_colwise_operand_k()).
  */
 typedef struct mxfp4_qdq_args {
     const void* x;
@@ -183,6 +223,8 @@ typedef struct mxfp4_qdq_args {
     uint8_t* mask_col;
     int32_t scales_row_layout;
     int32_t elem_format;
+    int32_t col_layout;
+    int64_t k_alloc;
 } mxfp4_qdq_args;
 
 /*
@@ -239,6 +281,21 @@ int64_t mxfp4_colwise_scale_rows_bound(int64_t rows, int64_t num_groups, int32_t
  * `layout` (MXFP4_SCALES_ROWMAJOR: rows * ceil(cols/block); MXFP4_SCALES_MMA:
  * 512 * ceil(rows/128) * ceil(ceil(cols/block)/4)); -1 for invalid arguments. */
 int64_t mxfp4_scales_row_bytes(int64_t rows, int64_t cols, int32_t block, int32_t layout);
+
+/* MXFP4_COLS_MMA: the K extent sum_g 128 * ceil(n_g / 128) of a group_list
+ * held in HOST memory (128 * ceil(rows / 128) for a NULL list); -1 when the
+ * list is not a valid partition of [0, rows). */
+int64_t mxfp4_colwise_operand_k(const int64_t* host_group_list, int64_t num_groups, int32_t group_list_type,
+                                int64_t rows);
+
+/* An upper bound on mxfp4_colwise_operand_k that needs no group sizes:
+ * 128 * (floor(rows / 128) + num_groups), or 128 * ceil(rows / 128) without
+ * groups; -1 for rows < 0. */
+int64_t mxfp4_colwise_operand_k_bound(int64_t rows, int64_t num_groups);
+
+/* Bytes of a MXFP4_COLS_MMA scales_col buffer: 512 * ceil(cols / 128) *
+ * (k_alloc / 128); -1 for invalid arguments. */
+int64_t mxfp4_colwise_operand_scale_bytes(int64_t cols, int64_t k_alloc);
 
 /* Static English text of a status; never NULL. */
 const char* mxfp4_status_string(mxfp4_status status);

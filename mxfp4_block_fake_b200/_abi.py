@@ -18,9 +18,10 @@ F32, BF16 = 0, 1
 SCALE_PAGE, SCALE_FLOOR = 0, 1
 ROWWISE, COLWISE = 1, 2
 SCALES_ROWMAJOR, SCALES_MMA = 0, 1
+COLS_ROWMAJOR, COLS_MMA = 0, 1
 ELEM_E2M1, ELEM_E4M3 = 0, 1
 MAX_GROUPS = 4096
-ABI_VERSION = 3
+ABI_VERSION = 4
 
 # Every symbol include/mxfp4.h declares.
 EXPORTS = (
@@ -30,6 +31,9 @@ EXPORTS = (
     "mxfp4_colwise_scale_rows",
     "mxfp4_colwise_scale_rows_bound",
     "mxfp4_scales_row_bytes",
+    "mxfp4_colwise_operand_k",
+    "mxfp4_colwise_operand_k_bound",
+    "mxfp4_colwise_operand_scale_bytes",
     "mxfp4_status_string",
     "mxfp4_abi_version",
 )
@@ -61,6 +65,8 @@ class QdqArgs(ctypes.Structure):
         ("mask_col", ctypes.c_void_p),
         ("scales_row_layout", ctypes.c_int32),
         ("elem_format", ctypes.c_int32),
+        ("col_layout", ctypes.c_int32),
+        ("k_alloc", ctypes.c_int64),
     ]
 
 
@@ -103,6 +109,12 @@ def lib() -> ctypes.CDLL:
     L.mxfp4_colwise_scale_rows_bound.restype = i64
     L.mxfp4_scales_row_bytes.argtypes = [i64, i64, i32, i32]
     L.mxfp4_scales_row_bytes.restype = i64
+    L.mxfp4_colwise_operand_k.argtypes = [P, i64, i32, i64]
+    L.mxfp4_colwise_operand_k.restype = i64
+    L.mxfp4_colwise_operand_k_bound.argtypes = [i64, i64]
+    L.mxfp4_colwise_operand_k_bound.restype = i64
+    L.mxfp4_colwise_operand_scale_bytes.argtypes = [i64, i64]
+    L.mxfp4_colwise_operand_scale_bytes.restype = i64
     L.mxfp4_status_string.argtypes = [i32]
     L.mxfp4_status_string.restype = ctypes.c_char_p
     L.mxfp4_abi_version.argtypes = []
@@ -152,3 +164,12 @@ def mxfp4_colwise_scale_rows(host_group_list, group_list_type: int, rows: int, b
 
 def mxfp4_colwise_scale_rows_bound(rows: int, num_groups: int, block: int) -> int:
     return lib().mxfp4_colwise_scale_rows_bound(rows, num_groups, block)
+
+
+def mxfp4_colwise_operand_k(host_group_list, group_list_type: int, rows: int) -> int:
+    """host_group_list: a sequence of ints (host memory), or None for one group."""
+    if host_group_list is None:
+        return lib().mxfp4_colwise_operand_k(None, 0, group_list_type, rows)
+    n = len(host_group_list)
+    arr = (ctypes.c_int64 * n)(*[int(v) for v in host_group_list])
+    return lib().mxfp4_colwise_operand_k(arr, n, group_list_type, rows)

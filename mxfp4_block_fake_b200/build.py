@@ -32,7 +32,8 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = (SRC, HDR, __file__, os.path.join(PKG, "csrc", "mxfp4_staged.cuh"))
+    csrc = os.path.join(PKG, "csrc")
+    deps = (HDR, __file__, *(os.path.join(csrc, f) for f in os.listdir(csrc)))
     return any(os.path.getmtime(p) > t for p in deps)
 
 

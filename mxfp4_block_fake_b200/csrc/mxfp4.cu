@@ -69,6 +69,7 @@ struct KArgs {
     uint32_t ts_flags;  // staged kernel: column-wise outputs written by TMA stores (SG_TS_*)
     int32_t srow_mma;   // scales_row in the MMA scale-factor layout (MXFP4_SCALES_MMA)
     int32_t fmt;        // MXFP4_ELEM_E2M1 or MXFP4_ELEM_E4M3
+    int64_t k_alloc;    // column-wise operand layout: K slots per codes row (MXFP4_COLS_MMA)
 };
 
 // Byte offset of row-wise scale (row, b) of a [rows][nblk] scale matrix:
@@ -1164,6 +1165,7 @@ __global__ void __launch_bounds__(NTHREADS)
 }  // namespace mxfp4
 
 #include "mxfp4_staged.cuh"
+#include "mxfp4_operand.cuh"
 
 namespace mxfp4 {
 
@@ -1611,6 +1613,8 @@ static mxfp4_status check_geometry(const mxfp4_qdq_args* a)
         return MXFP4_EINVAL;
     if (a->elem_format == MXFP4_ELEM_E4M3 && (a->block != 32 || a->scale_mode != MXFP4_SCALE_FLOOR))
         return MXFP4_EUNSUPPORTED;
+    if (a->col_layout != MXFP4_COLS_ROWMAJOR && a->col_layout != MXFP4_COLS_MMA)
+        return MXFP4_EINVAL;
     if (a->group_list) {
         if (a->num_groups < 1)
             return MXFP4_EINVAL;
@@ -1622,6 +1626,66 @@ static mxfp4_status check_geometry(const mxfp4_qdq_args* a)
             return MXFP4_EINVAL;
     }
     return MXFP4_OK;
+}
+
+// Column-wise codes and scales in the GEMM operand layout (MXFP4_COLS_MMA):
+// host checks, then one launch of col_operand_kernel.
+static mxfp4_status launch_col_operand(const mxfp4_qdq_args* A, cudaStream_t s)
+{
+    if (A->block != 32 || A->elem_format != MXFP4_ELEM_E2M1 || A->dtype != MXFP4_BF16)
+        return MXFP4_EUNSUPPORTED;
+    if (A->scale_mode == MXFP4_SCALE_PAGE && !page_fast_ok(A->scale_factor))
+        return MXFP4_EUNSUPPORTED;
+    const bool groups = A->group_list != nullptr;
+    if (A->k_alloc <= 0 || A->k_alloc % OP_KPAD != 0 || A->k_alloc > (int64_t)INT32_MAX * OP_KPAD)
+        return MXFP4_EINVAL;
+    if (!groups && A->k_alloc < OP_KPAD * ((A->rows + OP_KPAD - 1) / OP_KPAD))
+        return MXFP4_EINVAL;
+    if (!A->x || A->ld < A->cols || !aligned(A->x, 4) || A->ld % 2 != 0)
+        return MXFP4_EINVAL;
+    if ((A->codes_col && !aligned(A->codes_col, 16)) || (A->scales_col && !aligned(A->scales_col, 2)))
+        return MXFP4_EINVAL;
+    KArgs k;
+    memset(&k, 0, sizeof(k));
+    k.x = A->x;
+    k.rows = A->rows;
+    k.cols = A->cols;
+    k.ld = A->ld;
+    k.sf = A->scale_factor;
+    k.mode = A->scale_mode;
+    k.codes_col = A->codes_col;
+    k.scales_col = A->scales_col;
+    k.group_list = groups ? A->group_list : nullptr;
+    k.num_groups = groups ? (int32_t)A->num_groups : 0;
+    k.gl_type = A->group_list_type;
+    k.status = A->status;
+    k.k_alloc = A->k_alloc;
+    if (A->scale_mode == MXFP4_SCALE_PAGE)
+        k.thr = page_threshold(A->scale_factor);
+    if (A->status && !groups && cudaMemsetAsync(A->status, 0, sizeof(int32_t), s) != cudaSuccess)
+        return MXFP4_ECUDA;
+    const void* fn;
+    if (A->scale_mode == MXFP4_SCALE_FLOOR)
+        fn = groups ? (const void*)col_operand_kernel<MXFP4_SCALE_FLOOR, true>
+                    : (const void*)col_operand_kernel<MXFP4_SCALE_FLOOR, false>;
+    else
+        fn = groups ? (const void*)col_operand_kernel<MXFP4_SCALE_PAGE, true>
+                    : (const void*)col_operand_kernel<MXFP4_SCALE_PAGE, false>;
+    const size_t plan_smem = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
+    // the grid covers the K units the caller allocated: units past the real
+    // groups' end exit at once
+    const int64_t units = (A->k_alloc / 64) * ((A->cols + 1) / 2);
+    const int sms = device_sms();
+    const int occ = occupancy(fn, plan_smem);
+    if (sms <= 0 || occ <= 0)
+        return MXFP4_ECUDA;
+    int64_t grid = (int64_t)sms * occ;
+    if ((units + NTHREADS - 1) / NTHREADS < grid)
+        grid = (units + NTHREADS - 1) / NTHREADS;
+    void* args[] = {&k};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(NTHREADS), args, plan_smem, s) == cudaSuccess
+               ? MXFP4_OK
+               : MXFP4_ECUDA;
 }
 
 // Validates, then queues the forward (and the fused backward when g_in is set).
@@ -1645,6 +1709,31 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
         if (A->status && cudaMemsetAsync(A->status, 0, sizeof(int32_t), s) != cudaSuccess)
             return MXFP4_ECUDA;
         return MXFP4_OK;
+    }
+    if (col && A->col_layout == MXFP4_COLS_MMA && (A->codes_col || A->scales_col)) {
+        // The operand kernel runs last, so that its group_list check (which
+        // also covers k_alloc) is the last word written to status; the other
+        // outputs of the call go through the usual paths first.
+        if (grad)
+            return MXFP4_EUNSUPPORTED;
+        mxfp4_qdq_args R = *A;
+        R.codes_col = R.scales_col = nullptr;
+        R.col_layout = MXFP4_COLS_ROWMAJOR;
+        const bool rows_out = row && (R.y_row || R.codes_row || R.scales_row || R.mask_row);
+        const bool cols_out = R.y_col || R.mask_col;
+        if (!cols_out)
+            R.dirs &= ~MXFP4_COLWISE;
+        if (!rows_out)
+            R.dirs &= ~MXFP4_ROWWISE;
+        if (R.dirs != 0) {
+            // host checks of the operand first: nothing is queued for an invalid call
+            if (A->k_alloc <= 0 || A->k_alloc % OP_KPAD != 0)
+                return MXFP4_EINVAL;
+            st = run_qdq(&R, nullptr, nullptr, 0, 0, s);
+            if (st != MXFP4_OK)
+                return st;
+        }
+        return launch_col_operand(A, s);
     }
     if (!A->x || A->ld < A->cols || !aligned(A->x, esz))
         return MXFP4_EINVAL;
@@ -1971,6 +2060,44 @@ int64_t mxfp4_scales_row_bytes(int64_t rows, int64_t cols, int32_t block, int32_
     if (layout == MXFP4_SCALES_MMA)
         return 512 * ((rows + 127) / 128) * ((nblk + 3) / 4);
     return -1;
+}
+
+int64_t mxfp4_colwise_operand_k(const int64_t* host_group_list, int64_t num_groups, int32_t group_list_type,
+                                int64_t rows)
+{
+    if (rows < 0)
+        return -1;
+    if (!host_group_list)
+        return OP_KPAD * ((rows + OP_KPAD - 1) / OP_KPAD);
+    if (num_groups < 1 || (group_list_type != 0 && group_list_type != 1))
+        return -1;
+    int64_t total = 0, prev = 0, k = 0;
+    for (int64_t g = 0; g < num_groups; ++g) {
+        const int64_t v = host_group_list[g];
+        const int64_t n = group_list_type == 1 ? v : v - prev;
+        prev = v;
+        if (n < 0 || n > rows)
+            return -1;
+        total += n;
+        k += OP_KPAD * ((n + OP_KPAD - 1) / OP_KPAD);
+    }
+    return total == rows ? k : -1;
+}
+
+int64_t mxfp4_colwise_operand_k_bound(int64_t rows, int64_t num_groups)
+{
+    if (rows < 0)
+        return -1;
+    if (num_groups <= 0)
+        return OP_KPAD * ((rows + OP_KPAD - 1) / OP_KPAD);
+    return OP_KPAD * (rows / OP_KPAD + num_groups);
+}
+
+int64_t mxfp4_colwise_operand_scale_bytes(int64_t cols, int64_t k_alloc)
+{
+    if (cols < 0 || k_alloc < 0 || k_alloc % OP_KPAD != 0)
+        return -1;
+    return 512 * ((cols + 127) / 128) * (k_alloc / OP_KPAD);
 }
 
 int32_t mxfp4_abi_version(void) { return MXFP4_ABI_VERSION; }

@@ -28,6 +28,7 @@ _SCALE_LAYOUTS = {"rowmajor": _abi.SCALES_ROWMAJOR, "mma": _abi.SCALES_MMA}
 # element formats: E2M1 (MXFP4) and E4M3 (MXFP8: block 32, scale_mode "floor",
 # one code byte per element)
 _ELEM_FORMATS = {"e2m1": _abi.ELEM_E2M1, "e4m3": _abi.ELEM_E4M3}
+_COL_LAYOUTS = {"rowmajor": _abi.COLS_ROWMAJOR, "mma": _abi.COLS_MMA}
 
 
 def _elem_format(name: str) -> int:
@@ -49,6 +50,8 @@ class QDQResult:
     status: torch.Tensor | None = None
     scales_layout: str = "rowmajor"  # layout of scales_row
     elem_format: str = "e2m1"
+    col_layout: str = "rowmajor"  # layout of codes_col / scales_col ("mma": K-major GEMM operand)
+    k_alloc: int = 0  # col_layout "mma": K slots per codes_col row
 
 
 def _ptr(t: torch.Tensor | None):
@@ -149,13 +152,26 @@ def scales_row_bytes(rows: int, cols: int, block: int, scales_layout: str = "row
     return n
 
 
+def colwise_operand_k(group_list, group_list_type: int, rows: int) -> int:
+    """K extent of the column-wise GEMM operand (col_layout "mma"): exact for
+    a host group list (or none), the size-free bound for a device tensor."""
+    if isinstance(group_list, torch.Tensor):
+        return _abi.lib().mxfp4_colwise_operand_k_bound(rows, group_list.numel())
+    k = _abi.mxfp4_colwise_operand_k(None if group_list is None else list(group_list), group_list_type, rows)
+    if k < 0:
+        raise ValueError("group_list is not a partition of the rows")
+    return k
+
+
 def alloc_outputs(x: torch.Tensor, *, block: int, rowwise: bool, colwise: bool, num_groups: int,
                   emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
                   with_status: bool = False, scales_layout: str = "rowmajor",
-                  elem_format: str = "e2m1") -> QDQResult:
+                  elem_format: str = "e2m1", col_layout: str = "rowmajor", k_alloc: int | None = None) -> QDQResult:
     rows, cols = x.shape
     dev = x.device
-    r = QDQResult(scales_layout=scales_layout, elem_format=elem_format)
+    if col_layout not in _COL_LAYOUTS:
+        raise ValueError(f"col_layout must be one of {tuple(_COL_LAYOUTS)}, got {col_layout!r}")
+    r = QDQResult(scales_layout=scales_layout, elem_format=elem_format, col_layout=col_layout)
     ccols = cols if _elem_format(elem_format) == _abi.ELEM_E4M3 else (cols + 1) // 2
     u8 = dict(dtype=torch.uint8, device=dev)
     if rowwise:
@@ -173,7 +189,13 @@ def alloc_outputs(x: torch.Tensor, *, block: int, rowwise: bool, colwise: bool, 
     if colwise:
         if emit_values:
             r.y_col = torch.empty((rows, cols), dtype=x.dtype, device=dev)
-        if emit_codes:
+        if emit_codes and col_layout == "mma":
+            # K slots past the groups and atom rows past cols are not written: zeros
+            k = int(k_alloc) if k_alloc is not None else _abi.lib().mxfp4_colwise_operand_k_bound(rows, num_groups)
+            r.k_alloc = k
+            r.codes_col = torch.zeros((cols, k // 2), **u8)
+            r.scales_col = torch.zeros((max(0, _abi.lib().mxfp4_colwise_operand_scale_bytes(cols, k)),), **u8)
+        elif emit_codes:
             r.codes_col = torch.empty((rows, ccols), **u8)
             r.scales_col = torch.empty((colwise_scale_rows_bound(rows, num_groups, block), cols), **u8)
         if emit_mask:
@@ -223,9 +245,13 @@ def _fill_outputs(a: _abi.QdqArgs, r: QDQResult, x: torch.Tensor | None = None) 
         if len(ys) == 2 and _ld(ys[0]) != _ld(ys[1]):
             raise ValueError("y_row and y_col must have the same row stride (one ld_y is passed)")
         u8 = torch.uint8
-        for name in ("codes_row", "codes_col"):
-            if getattr(r, name) is not None:
-                _need(getattr(r, name), name, (rows, ccols), u8, dev)
+        if r.col_layout not in _COL_LAYOUTS:
+            raise ValueError(f"col_layout must be one of {tuple(_COL_LAYOUTS)}, got {r.col_layout!r}")
+        col_mma = r.col_layout == "mma"
+        if r.codes_row is not None:
+            _need(r.codes_row, "codes_row", (rows, ccols), u8, dev)
+        if r.codes_col is not None:
+            _need(r.codes_col, "codes_col", (cols, r.k_alloc // 2) if col_mma else (rows, ccols), u8, dev)
         for name in ("mask_row", "mask_col"):
             if getattr(r, name) is not None:
                 _need(getattr(r, name), name, (rows, (cols + 7) // 8), u8, dev)
@@ -238,7 +264,13 @@ def _fill_outputs(a: _abi.QdqArgs, r: QDQResult, x: torch.Tensor | None = None) 
                     raise ValueError("scales_row (mma layout) is smaller than mxfp4_scales_row_bytes()")
             else:
                 _need(r.scales_row, "scales_row", (rows, nblk), u8, dev)
-        if r.scales_col is not None:
+        if r.scales_col is not None and col_mma:
+            t = r.scales_col
+            if not t.is_cuda or t.device != dev or t.dtype != u8 or not t.is_contiguous():
+                raise ValueError("scales_col (mma layout) must be a contiguous uint8 CUDA tensor")
+            if t.numel() < _abi.lib().mxfp4_colwise_operand_scale_bytes(cols, r.k_alloc):
+                raise ValueError("scales_col (mma layout) is smaller than mxfp4_colwise_operand_scale_bytes()")
+        elif r.scales_col is not None:
             _need(r.scales_col, "scales_col", (0, cols), u8, dev,
                   min_rows=colwise_scale_rows_bound(rows, int(a.num_groups) if a.group_list else 0, blk))
         if r.status is not None:
@@ -248,6 +280,8 @@ def _fill_outputs(a: _abi.QdqArgs, r: QDQResult, x: torch.Tensor | None = None) 
     a.codes_row, a.scales_row, a.mask_row = _ptr(r.codes_row), _ptr(r.scales_row), _ptr(r.mask_row)
     a.codes_col, a.scales_col, a.mask_col = _ptr(r.codes_col), _ptr(r.scales_col), _ptr(r.mask_col)
     a.scales_row_layout = _SCALE_LAYOUTS[r.scales_layout]
+    a.col_layout = _COL_LAYOUTS[r.col_layout]
+    a.k_alloc = int(r.k_alloc)
 
 
 def _check_status(status: torch.Tensor | None, where: str) -> None:
@@ -271,7 +305,7 @@ def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0
                   rowwise: bool = True, colwise: bool = False, group_list=None, group_list_type: int = 0,
                   emit_values: bool = True, emit_codes: bool = False, emit_mask: bool = False,
                   check: bool | None = None, out: QDQResult | None = None, scales_layout: str = "rowmajor",
-                  elem_format: str = "e2m1") -> QDQResult:
+                  elem_format: str = "e2m1", col_layout: str = "rowmajor", k_alloc: int | None = None) -> QDQResult:
     """QDQ forward; returns the requested outputs.
 
     A group_list lives in device memory and is validated by the kernels,
@@ -282,7 +316,10 @@ def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0
     the returned status tensor reads 0 (MXFP4_OK) once the stream reaches it.
     scales_layout="mma" writes the row-wise scales in the block-scaled MMA
     scale-factor layout. elem_format="e4m3" quantises to MXFP8 (block 32,
-    scale_mode "floor")."""
+    scale_mode "floor"). col_layout="mma" writes the column-wise codes and
+    scales as the K-major operand of a GEMM contracting over the rows (each
+    group padded to 128 rows; include/mxfp4.h, MXFP4_COLS_MMA); k_alloc
+    defaults to the exact K of a host group list, else to the bound."""
     x = _as_2d(x)
     gl, ng = _group_args(group_list, group_list_type, x.device)
     if check is None:
@@ -293,7 +330,9 @@ def mxfp4_qdq_fwd(x: torch.Tensor, *, block: int = 32, scale_factor: float = 6.0
     r = out if out is not None else alloc_outputs(
         x, block=block, rowwise=rowwise, colwise=colwise, num_groups=ng, emit_values=emit_values,
         emit_codes=emit_codes, emit_mask=emit_mask, with_status=check or gl is not None,
-        scales_layout=scales_layout, elem_format=elem_format)
+        scales_layout=scales_layout, elem_format=elem_format, col_layout=col_layout,
+        k_alloc=(k_alloc if k_alloc is not None or col_layout != "mma"
+                 else colwise_operand_k(group_list, group_list_type, x.shape[0])))
     if check and r.status is None:
         r.status = torch.empty((1,), dtype=torch.int32, device=x.device)
     a = make_args(x, block=block, scale_factor=scale_factor, scale_mode=scale_mode, dirs=dirs,
@@ -403,3 +442,21 @@ def mxfp4_mma_operand(x: torch.Tensor, *, scale_mode: str = "page", scale_factor
     r = mxfp4_qdq_fwd(x2, block=32, scale_factor=scale_factor, scale_mode=scale_mode, rowwise=True,
                       emit_values=False, emit_codes=True, out=out, scales_layout="mma")
     return r.codes_row.view(torch.float4_e2m1fn_x2), r.scales_row.view(torch.float8_e8m0fnu)
+
+
+def mxfp4_colwise_mma_operand(x: torch.Tensor, *, group_list=None, group_list_type: int = 0,
+                              scale_mode: str = "page", scale_factor: float = 6.0, k_alloc: int | None = None,
+                              check: bool | None = None):
+    """Real MXFP4 operand of a block-scaled GEMM that contracts over x's rows,
+    per group (the weight-gradient direction): returns (codes [cols,
+    k_alloc/2] as torch.float4_e2m1fn_x2, K-major, first row in the low
+    nibble; E8M0 scales as torch.float8_e8m0fnu in the 128 x 4 atom layout of
+    the [cols][k_alloc/32] scale matrix; k_alloc). Group g occupies K slots
+    [K0_g, K0_g + 128 ceil(n_g/128)) with K0_g the sum of the earlier groups'
+    padded sizes; the padding codes are 0. A group_list given as a host
+    sequence fixes k_alloc exactly; a device tensor uses the bound."""
+    x2 = _as_2d(x)
+    r = mxfp4_qdq_fwd(x2, block=32, scale_factor=scale_factor, scale_mode=scale_mode, rowwise=False,
+                      colwise=True, group_list=group_list, group_list_type=group_list_type, emit_values=False,
+                      emit_codes=True, col_layout="mma", k_alloc=k_alloc, check=check)
+    return r.codes_col.view(torch.float4_e2m1fn_x2), r.scales_col.view(torch.float8_e8m0fnu), r.k_alloc

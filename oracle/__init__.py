@@ -227,6 +227,53 @@ def mma_scale_layout(scales: np.ndarray) -> np.ndarray:
     return out
 
 
+def colwise_operand_k(ends) -> int:
+    """K extent of the column-wise operand: every group padded to a multiple
+    of 128 rows (four blocks of 32, one scale-atom column)."""
+    e = np.asarray(ends, np.int64)
+    n = np.diff(np.concatenate([[0], e]))
+    return int(np.sum(-(-n // 128)) * 128)
+
+
+def colwise_operand_layout(codes: np.ndarray, scales: np.ndarray, ends, cols: int, k_alloc: int | None = None):
+    """Column-wise E2M1 codes and E8M0 scales (the layout qdq_colwise returns)
+    -> the operand of a block-scaled GEMM that contracts over the rows, group
+    by group. The pages fix no such layout (parity unpinned); it is this
+    library's layout, pinned by hand-computed offsets in the tests:
+
+      K0_g   = sum over j < g of 128 * ceil(n_j / 128)   (group g's first K slot)
+      codesT [cols][k_alloc / 2]: the nibble of x[start_g + t, c] is nibble
+             (t & 1) of byte c * k_alloc/2 + (K0_g + t) / 2; slots t >= n_g
+             up to the group's padded end hold nibble 0
+      scales the [cols][k_alloc / 32] E8M0 matrix whose entry (c, K0_g/32 + b)
+             is block b of group g in column c (127 for the padding blocks of
+             the group), stored in the 128 x 4 atom layout of mma_scale_layout
+
+    Slots past sum of the padded groups (up to k_alloc) are left 0."""
+    e = np.asarray(ends, np.int64)
+    starts = np.concatenate([[0], e[:-1]])
+    n = e - starts
+    kpad = -(-n // 128) * 128
+    k0 = np.concatenate([[0], np.cumsum(kpad)[:-1]])
+    ktot = int(kpad.sum())
+    k_alloc = ktot if k_alloc is None else int(k_alloc)
+    assert k_alloc >= ktot and k_alloc % 128 == 0
+    nib = unpack_nibbles(codes, cols)  # [rows][cols]
+    kmat = np.zeros((cols, k_alloc), np.uint8)  # nibble per (column, K slot)
+    smat = np.zeros((cols, k_alloc // 32), np.uint8)
+    srow = 0
+    for g in range(len(e)):
+        if n[g] == 0:
+            continue
+        kmat[:, k0[g]:k0[g] + n[g]] = nib[starts[g]:e[g]].T
+        nb = -(-int(n[g]) // 32)
+        smat[:, k0[g] // 32:k0[g] // 32 + kpad[g] // 32] = 127
+        smat[:, k0[g] // 32:k0[g] // 32 + nb] = scales[srow:srow + nb].T
+        srow += nb
+    codesT = (kmat[:, 0::2] | (kmat[:, 1::2] << 4)).astype(np.uint8)
+    return codesT, mma_scale_layout(smat)
+
+
 def unpack_nibbles(codes: np.ndarray, cols: int) -> np.ndarray:
     """Packed [rows, ceil(cols/2)] codes -> uint8 [rows, cols] nibbles (low nibble first)."""
     lo = codes & 0x0F
@@ -241,5 +288,5 @@ __all__ = [
     "F32", "BF16", "SCALE_PAGE", "SCALE_FLOOR", "lib", "build", "bf16_to_f32", "f32_to_bf16",
     "scale_page", "scale_floor", "qdq_block", "group_ends", "colwise_scale_rows", "qdq_rowwise",
     "qdq_colwise", "ste_bwd", "unpack_bits", "unpack_nibbles", "mma_scale_layout", "qdq8_rowwise",
-    "qdq8_colwise", "e4m3_value", "e4m3_encode",
+    "qdq8_colwise", "e4m3_value", "e4m3_encode", "colwise_operand_k", "colwise_operand_layout",
 ]

@@ -106,6 +106,29 @@ def test_colwise_scale_rows_matches_oracle(abi, oracle_mod, block):
     assert abi.mxfp4_colwise_scale_rows(None, 0, 100, 32) == 4
 
 
+def test_colwise_operand_k_matches_oracle(abi, oracle_mod):
+    rng = np.random.default_rng(4)
+    L = abi.lib()
+    for trial in range(200):
+        g = int(rng.integers(1, 40))
+        counts = rng.integers(0, 400, g)
+        counts[rng.random(g) < 0.3] = 0
+        rows = int(counts.sum())
+        ends = np.cumsum(counts)
+        exp = oracle_mod.colwise_operand_k(ends)
+        assert abi.mxfp4_colwise_operand_k(counts.tolist(), 1, rows) == exp
+        assert abi.mxfp4_colwise_operand_k(ends.tolist(), 0, rows) == exp
+        assert L.mxfp4_colwise_operand_k_bound(rows, g) >= exp
+    assert abi.mxfp4_colwise_operand_k(None, 0, 300) == 384
+    assert abi.mxfp4_colwise_operand_k([3, 2, 8], 0, 8) == -1
+    assert abi.mxfp4_colwise_operand_k([3, -1, 6], 1, 8) == -1
+    assert L.mxfp4_colwise_operand_k_bound(300, 0) == 384 and L.mxfp4_colwise_operand_k_bound(-1, 2) == -1
+    for cols, k in ((3, 384), (256, 128), (130, 1024), (0, 128)):
+        exp = oracle_mod.mma_scale_layout(np.zeros((cols, k // 32), np.uint8)).size if cols else 0
+        assert L.mxfp4_colwise_operand_scale_bytes(cols, k) == exp
+    assert L.mxfp4_colwise_operand_scale_bytes(10, 100) == -1
+
+
 def _args(abi, **kw):
     a = abi.QdqArgs()
     a.dtype, a.block, a.rows, a.cols, a.ld = abi.BF16, 32, 4, 64, 64
@@ -129,6 +152,17 @@ def _args(abi, **kw):
     (dict(scales_row_layout=2), 1), (dict(elem_format=2), 1), (dict(elem_format=-1), 1),
     (dict(elem_format=1), 2),                               # MXFP8 in PAGE mode
     (dict(elem_format=1, scale_mode=1, block=128), 2),      # MXFP8 with blocks of 128
+    (dict(col_layout=2), 1), (dict(col_layout=-1), 1),
+    # column-wise GEMM operand layout: k_alloc, dtype and alignment are checked on the host
+    (dict(dirs=2, codes_col=8192, col_layout=1, k_alloc=100), 1),
+    (dict(dirs=2, codes_col=8192, col_layout=1, k_alloc=0), 1),
+    (dict(dirs=2, codes_col=8192, col_layout=1, k_alloc=128, rows=200), 1),
+    (dict(dirs=2, codes_col=8200, col_layout=1, k_alloc=128), 1),
+    (dict(dirs=2, scales_col=8193, col_layout=1, k_alloc=128), 1),
+    (dict(dirs=2, codes_col=8192, col_layout=1, k_alloc=128, dtype=0), 2),
+    (dict(dirs=2, codes_col=8192, col_layout=1, k_alloc=128, block=128), 2),
+    (dict(dirs=2, codes_col=8192, col_layout=1, k_alloc=128, scale_factor=100.0), 2),
+    (dict(dirs=3, codes_col=8192, col_layout=1, k_alloc=100, y_row=8192), 1),
 ])
 def test_fwd_rejects_bad_arguments_on_host(abi, kw, expected):
     assert abi.mxfp4_qdq_fwd(_args(abi, **kw), None) == expected

@@ -492,3 +492,40 @@ def test_threaded_oracle_equals_single_calls():
             assert np.array_equal(a[k], b[k])
         m = O.qdq_rowwise(xb, 32, 6.0, O.SCALE_PAGE)["mask"]
         assert np.array_equal(OP.ste_bwd(xb, m, True), O.ste_bwd(xb, m, True))
+
+
+def test_colwise_operand_layout_hand_offsets():
+    """The column-wise real-quantisation operand layout, against offsets
+    worked out by hand: groups [40, 0, 130] over 3 columns pad to K slots
+    [0, 128) and [128, 384); nibble of x[r, c] = (3r + c) mod 16, column-wise
+    scale byte (s, c) = 10s + c."""
+    import oracle as O
+
+    rows, cols = 170, 3
+    r = np.arange(rows)[:, None]
+    c = np.arange(cols)[None, :]
+    nib = ((3 * r + c) % 16).astype(np.uint8)
+    codes = np.zeros((rows, 2), np.uint8)
+    codes[:, 0] = nib[:, 0] | (nib[:, 1] << 4)
+    codes[:, 1] = nib[:, 2]
+    scales = (10 * np.arange(7)[:, None] + np.arange(3)[None, :]).astype(np.uint8)
+    ends = np.array([40, 40, 170])
+    assert O.colwise_operand_k(ends) == 384
+    codesT, sc = O.colwise_operand_layout(codes, scales, ends, cols)
+    flat = codesT.reshape(-1)
+    assert codesT.shape == (3, 192)
+    assert flat[0] == 0x30                 # rows 0, 1 of column 0
+    assert flat[192 + 19] == 0x63          # rows 38, 39 of column 1
+    assert flat[192 + 20] == 0             # padding of group 0 in column 1
+    assert flat[2 * 192 + 64] == 0xDA      # rows 40, 41 (group 2's first slots) of column 2
+    assert flat[2 * 192 + 64 + 65] == 0    # slot 130 of group 2: padding
+    assert sc.size == 512 * 3
+    assert sc[529] == 31                   # column 1, scale column 5 = group 2 block 1 = row 3
+    assert sc[34] == 127                   # column 2, scale column 2: padding block of group 0
+    assert sc[1024] == 60                  # column 0, scale column 8 = group 2 block 4 = row 6
+    assert sc[1024 + 32 + 3] == 127        # column 2, scale column 11: padding
+    assert sc[0] == 0 and sc[16 + 1] == 11  # column 0 block 0; column 1 block 1
+    # k_alloc wider than needed: the rows get longer, the extra slots stay 0
+    codesW, scW = O.colwise_operand_layout(codes, scales, ends, cols, k_alloc=512)
+    assert codesW.shape == (3, 256) and np.array_equal(codesW[:, :192], codesT) and not codesW[:, 192:].any()
+    assert scW.size == 512 * 4
