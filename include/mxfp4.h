@@ -159,7 +159,7 @@ typedef enum {
  *               and K slots past the last group are not written.
  * Group g's operand is then the [cols][128 ceil(n_g/128)] sub-matrix at K0_g
  * (row stride k_alloc/2 bytes) with the atom columns from K0_g/128 on.
- * Requires bf16 x (4-byte aligned, even ld), block 32, E2M1, and in PAGE mode
+ * Requires bf16 x, block 32, E2M1, and in PAGE mode
  * a scale_factor in [2^-64, 11] (else MXFP4_EUNSUPPORTED); no fused backward.
  * y_col and mask_col, when also given, keep their row-major layout. An
  * invalid group_list, or groups whose padded K exceeds k_alloc, write no

@@ -1641,7 +1641,7 @@ static mxfp4_status launch_col_operand(const mxfp4_qdq_args* A, cudaStream_t s)
         return MXFP4_EINVAL;
     if (!groups && A->k_alloc < OP_KPAD * ((A->rows + OP_KPAD - 1) / OP_KPAD))
         return MXFP4_EINVAL;
-    if (!A->x || A->ld < A->cols || !aligned(A->x, 4) || A->ld % 2 != 0)
+    if (!A->x || A->ld < A->cols || !aligned(A->x, 2))
         return MXFP4_EINVAL;
     if ((A->codes_col && !aligned(A->codes_col, 16)) || (A->scales_col && !aligned(A->scales_col, 2)))
         return MXFP4_EINVAL;

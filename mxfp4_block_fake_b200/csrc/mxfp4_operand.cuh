@@ -20,8 +20,9 @@
 // row stride of k_alloc / 2 bytes.
 //
 // One thread per (block pair, column pair): 64 rows of one 32-bit word (two
-// bf16 columns); a warp covers 64 adjacent columns, so every load
-// instruction of the warp reads one 128-byte row segment. Per column and
+// bf16 columns; two 16-bit loads when x's rows are not 4-byte aligned); a
+// warp covers 64 adjacent columns, so every load instruction of the warp
+// reads one 128-byte row segment. Per column and
 // block: the amax, the scale exponent, the codes of 32 rows by the nudged
 // hardware convert (the same argument as the row-wise producer: the nudge
 // turns the convert's ties-to-even into the codebook's ties-up for bf16
@@ -72,6 +73,9 @@ __global__ void __launch_bounds__(NTHREADS) col_operand_kernel(const KArgs a)
     const int64_t kbytes = a.k_alloc / 2;   // bytes per codes row
     const int64_t nsc = a.k_alloc / 32;     // scale columns
     const uint16_t* xb = static_cast<const uint16_t*>(a.x);
+    // a column pair is one aligned 32-bit word when x is 4-byte aligned and ld
+    // even; otherwise it is read as two 16-bit elements
+    const bool words = ((uintptr_t)a.x & 3u) == 0 && (a.ld & 1) == 0;
     for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
         const int64_t bp = u / npairs, cp = u - bp * npairs;
         const int64_t c = 2 * cp;
@@ -110,7 +114,10 @@ __global__ void __launch_bounds__(NTHREADS) col_operand_kernel(const KArgs a)
 #pragma unroll
             for (int r = 0; r < 32; ++r) {
                 const uint16_t* p = xb + (r0 + r) * a.ld + c;
-                w[r] = r < n ? (two ? __ldcs(reinterpret_cast<const unsigned int*>(p)) : (uint32_t)__ldcs(p)) : 0u;
+                w[r] = r >= n ? 0u
+                       : !two ? (uint32_t)__ldcs(p)
+                       : words ? __ldcs(reinterpret_cast<const unsigned int*>(p))
+                               : (uint32_t)__ldcs(p) | ((uint32_t)__ldcs(p + 1) << 16);
             }
             uint32_t m2 = 0;
 #pragma unroll

@@ -49,13 +49,13 @@ constexpr uint64_t SG_WAIT_NS = 4000000000ull;             // an mbarrier wait g
 constexpr uint32_t SG_TS_Y = 1u, SG_TS_CODES = 2u, SG_TS_MASK = 4u;              // column-wise
 constexpr uint32_t SG_TS_YR = 8u, SG_TS_CODES_R = 16u, SG_TS_MASK_R = 32u;       // row-wise
 
-// Staged outputs of one tile. y tiles use the input's layout (four 4 KB
-// slabs of 64 columns with the 128-byte swizzle); codes are 32 rows of 128
-// bytes with the 128-byte swizzle; masks are 32 rows of 32 bytes; row-wise
-// scales are 32 rows of 8 bytes.
+// Staged outputs of one tile; two buffers alternate between consecutive
+// tiles. y tiles use the input's layout (four 4 KB slabs of 64 columns with
+// the 128-byte swizzle); codes are 32 rows of 128 bytes with the 128-byte
+// swizzle; masks are 32 rows of 32 bytes; row-wise scales are 32 rows of 8
+// bytes. Row-wise y is written over the tile's input stage instead.
 struct __align__(1024) StagedOut {
     uint8_t ycol[SG_TILE_BYTES];
-    uint8_t yrow[SG_TILE_BYTES];
     uint8_t ccol[SG_CODE_BYTES];
     uint8_t crow[SG_CODE_BYTES];
     uint32_t mcol[SG_MASK_WORDS];
@@ -64,21 +64,20 @@ struct __align__(1024) StagedOut {
 };
 
 struct __align__(1024) StagedSmem {
-    uint8_t tiles[SG_STAGES][SG_TILE_BYTES];  // input stages (1024-aligned swizzle atoms)
-    StagedOut out;                            // staged outputs of the tile in flight
+    uint8_t tiles[SG_STAGES][SG_TILE_BYTES];  // input stages (1024-aligned swizzle atoms); row-wise y in place
+    StagedOut out[2];                         // staged outputs of tiles j (j even) and j (j odd)
     uint32_t limw[8][16];                     // per warp and column pair: 0x8000 + limit bits of each column
     int4 info[SG_STAGES];                     // row0, nrows, col0, row block of each stage's tile
     uint32_t lut[64];
     unsigned long long full[SG_STAGES];       // mbarriers: stage loaded (TMA transaction count)
-    unsigned long long sfree_c;               // mbarrier: the previous tile's column-wise stores have read their staging
-    unsigned long long sfree_r;               // mbarrier: the same for the row-wise stores
+    unsigned long long sfree[2];              // mbarriers: the stores of staging buffer b's last tile have read it
     int err;
 };
 
 constexpr int SG_THREADS = NTHREADS;
-// Thread 0 issues the TMA loads; thread SG_STORER (lane 0 of warp 1) issues
-// the TMA stores and waits for them, and its warp copies the row-wise scales.
-constexpr int SG_STORER = 32;
+// Thread SG_ASYNC (lane 0 of warp 1) issues every TMA load and store of the
+// CTA and waits for the stores; its warp copies the row-wise scales.
+constexpr int SG_ASYNC = 32;
 
 // TMA descriptors: the input and the outputs (an output map is only read
 // when its SG_TS_* flag is set).
@@ -191,21 +190,6 @@ __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b)
     return r;
 }
 
-// E2M1 byte of one word of signed packed bf16 codes (low element in the low
-// nibble). The high element is converted from the whole word read as fp32:
-// the low element's bits sit below its last bf16 bit and cannot move it to
-// another E2M1 value (a code of zero gives a subnormal of the same sign).
-__device__ __forceinline__ uint32_t e2m1_byte(uint32_t P)
-{
-    uint32_t r;
-    asm("{\n\t.reg .b8 b;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
-        "cvt.u32.u8 %0, b;\n\t}"
-        : "=r"(r)
-        : "f"(__uint_as_float(P)), "f"(__uint_as_float(P << 16)));
-    return r;
-}
-
 // E2M1 nibbles of four words of signed packed bf16 codes (8 elements).
 __device__ __forceinline__ uint32_t e2m1_word(const uint32_t* P)
 {
@@ -243,31 +227,50 @@ __device__ __forceinline__ bool k_fast_bf(int k) { return (uint32_t)(k + 125) <=
 // bf16 bits of 2^k for a fast-path k.
 __device__ __forceinline__ uint32_t bf16_pow2(int k) { return (uint32_t)(k + 127) << 7; }
 
-// One word (two bf16 elements) of fast-path blocks. aw: |x| bits; sg: the
-// sign bits to keep (those of nonzero elements). inv_*: 2^-k of each
-// element's block; s2: packed bf16 2^k of each element's block.
+// A word with its -0 halves turned into +0 (x + 0 in bf16 arithmetic, which
+// changes nothing else: nonzero values, subnormals and infinities pass
+// unchanged, a NaN stays a NaN). After this the sign bit of a half is set
+// exactly when the codebook's sign rule keeps a sign: sign(y) of a nonzero x.
+__device__ __forceinline__ uint32_t clear_neg_zero(uint32_t w)
+{
+    uint32_t r;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0u));
+    return r;
+}
+
+// One word (two bf16 elements) of fast-path blocks; wc has no -0 halves
+// (clear_neg_zero). inv_*: 2^-k of each element's block; s2: packed bf16
+// 2^k of each element's block.
 // t = 2^21 + |x| * 2^-k rounded down (fp32 spacing on [2^21, 2^22) is 1/4),
 // so t's bits are 0x4A000000 + floor(4|y|); lutb16 = table base - 0x28000000
-// folds that offset into the address shift-add. The high element is indexed
-// from the whole word: the low element's magnitude lies below its last bf16
-// bit and cannot carry it across a quarter of 2^k. Returns the dequantised
-// packed bf16 pair; P receives the signed codes.
-__device__ __forceinline__ uint32_t qword(uint32_t aw, uint32_t sg, float inv_lo, float inv_hi, uint32_t s2,
-                                          uint32_t lutb16, uint32_t& P)
+// folds that offset into the address shift-add. |x| is the fma's absolute-
+// value operand. The high element is indexed from the whole word: the low
+// element's magnitude lies below its last bf16 bit and cannot carry it across
+// a quarter of 2^k. Returns the dequantised packed bf16 pair; P receives the
+// signed codes.
+__device__ __forceinline__ uint32_t qword(uint32_t wc, float inv_lo, float inv_hi, uint32_t s2, uint32_t lutb16,
+                                          uint32_t& P)
 {
-    const float tl = __fmaf_rd(__uint_as_float(aw << 16), inv_lo, 0x1p21f);
-    const float th = __fmaf_rd(__uint_as_float(aw), inv_hi, 0x1p21f);
+    const float tl = __fmaf_rd(fabsf(__uint_as_float(wc << 16)), inv_lo, 0x1p21f);
+    const float th = __fmaf_rd(fabsf(__uint_as_float(wc)), inv_hi, 0x1p21f);
     const uint32_t el = lut_load(lutb16 + (__float_as_uint(tl) << 2));
     const uint32_t eh = lut_load(lutb16 + (__float_as_uint(th) << 2));
-    P = __byte_perm(el, eh, 0x7632) | sg;
+    P = __byte_perm(el, eh, 0x7632) | (wc & 0x80008000u);
     return hmul2_bf16(P, s2);
 }
 
-// |x| bits of a word and the sign bits of its nonzero halves (-0 gives +0).
-__device__ __forceinline__ void prep_bf(uint32_t w, uint32_t& aw, uint32_t& sg)
+// The E2M1 byte of one word of signed packed bf16 codes (low element in the
+// low nibble), stored at a shared-memory address. The high element is
+// converted from the whole word read as fp32: the low element's bits sit
+// below its last bf16 bit and cannot move it to another E2M1 value (a code of
+// zero gives a subnormal of the same sign).
+__device__ __forceinline__ void e2m1_byte_store(uint32_t saddr, uint32_t P)
 {
-    aw = w & 0x7FFF7FFFu;
-    sg = w & (aw + 0x7FFF7FFFu) & 0x80008000u;
+    asm volatile("{\n\t.reg .b8 b;\n\t"
+                 "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+                 "st.shared.b8 [%0], b;\n\t}" ::"r"(saddr),
+                 "f"(__uint_as_float(P)), "f"(__uint_as_float(P << 16))
+                 : "memory");
 }
 
 // ---- E2M1 rounding by the hardware convert ---------------------------------
@@ -407,8 +410,8 @@ struct TileWalk {
 // Copy staged outputs of a tile to global memory with the threads of the CTA
 // (group tails, outputs TMA cannot address). The flags select the outputs;
 // rows at or past nrows and columns at or past cols are skipped.
-__device__ __forceinline__ void copy_outputs(const KArgs& a, const StagedOut& o, int row0, int nrows, int col0,
-                                             uint32_t which)
+__device__ __forceinline__ void copy_outputs(const KArgs& a, const StagedOut& o, const uint8_t* yrow, int row0,
+                                             int nrows, int col0, uint32_t which)
 {
     const int tid = threadIdx.x;
     const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8;
@@ -427,7 +430,7 @@ __device__ __forceinline__ void copy_outputs(const KArgs& a, const StagedOut& o,
         if (which & SG_TS_Y)
             st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * 2, sm_ld128(o.ycol, yoff));
         if (which & SG_TS_YR)
-            st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * 2, sm_ld128(o.yrow, yoff));
+            st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * 2, sm_ld128(yrow, yoff));
         if (which & SG_TS_CODES)
             *reinterpret_cast<uint32_t*>(a.codes_col + row * cstride + col / 2) = sm_ld32(o.ccol, coff);
         if (which & SG_TS_CODES_R)
@@ -498,20 +501,20 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
     // slabs are placed on a 1024-byte boundary (1 KB of slack is requested)
     uint8_t* s_base = s_dyn + ((1024u - (smem_addr(s_dyn) & 1023u)) & 1023u);
     StagedSmem& sm = *reinterpret_cast<StagedSmem*>(s_base);
-    StagedOut& out = sm.out;
     int32_t* s_plan = reinterpret_cast<int32_t*>(s_base + sizeof(StagedSmem));
     int32_t* s_bpre = s_plan;
     int32_t* s_rst = s_plan + (GROUPS ? a.num_groups + 1 : 0);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool async_thread = tid == SG_ASYNC;
     if (tid < 64)
         sm.lut[tid] = lut_entry(tid);
     if (tid == 0) {
         sm.err = 0;
         for (int s = 0; s < SG_STAGES; ++s)
             mbar_init(smem_addr(&sm.full[s]), 1);
-        mbar_init(smem_addr(&sm.sfree_c), 1);
-        mbar_init(smem_addr(&sm.sfree_r), 1);
+        mbar_init(smem_addr(&sm.sfree[0]), 1);
+        mbar_init(smem_addr(&sm.sfree[1]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     uint32_t S;
@@ -538,7 +541,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
     const uint32_t row_out = (ROW && a.y_row ? SG_TS_YR : 0u) | (ROW && a.codes_row ? SG_TS_CODES_R : 0u) |
                              (ROW && a.mask_row ? SG_TS_MASK_R : 0u);
 
-    // producer state (thread 0): the next tile to load
+    // producer state (the async thread): the next tile to load
     TileWalk<GROUPS> pw;
     uint32_t t_issue = t_begin;
     auto issue = [&](int s) {
@@ -552,7 +555,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         ++t_issue;
         pw.next(a, s_bpre);
     };
-    if (tid == 0 && t_begin < t_end) {
+    if (async_thread && t_begin < t_end) {
         pw.start(a, s_bpre, t_begin);
         for (int s = 0; s < SG_STAGES && t_issue < t_end; ++s)
             issue(s);
@@ -586,13 +589,15 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
 
     int s = 0;
     uint32_t phase = 0;
-    for (uint32_t t = t_begin, j = 0; t < t_end; ++t, ++j) {
+    uint32_t t = t_begin;
+    for (uint32_t j = 0; t < t_end; ++t, ++j) {
         int row0 = 0, nrows = 0, col0 = 0;
         // the warp decides together, so that its shuffles and votes below
         // always see all 32 lanes
         const bool ok = __all_sync(FULL, mbar_wait(smem_addr(&sm.full[s]), phase));
-        const uint8_t* tile = sm.tiles[s];
-        uint32_t cw[16];  // the column pass's raw words
+        uint8_t* tile = sm.tiles[s];
+        StagedOut& out = sm.out[j & 1];
+        uint32_t cw[16];  // the column pass's words, -0 cleared
         int k_lo = 0, k_hi = 0;
         uint32_t A_lo = 0, A_hi = 0;
         bool fast = true;
@@ -609,8 +614,12 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             // ---- column pass, part 1: amax and parameters of the column pair
             if constexpr (COL) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                cw[i] = sm_ld32(tile, yo[i & 3] + (i >> 2) * 1024);
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t off = yo[i & 3] + (i >> 2) * 1024;
+                cw[i] = clear_neg_zero(sm_ld32(tile, off));
+                // written back: this warp's row pass reads these words cleaned
+                *reinterpret_cast<uint32_t*>(tile + off) = cw[i];
+            }
             if (!rows_full) {
                 // rows past a group tail belong to the next group: neither
                 // their values nor their amax take part
@@ -644,20 +653,19 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             }
             }  // COL
         }
-        // The staging buffers are free once the previous tile's stores have
-        // read them: the storer waits for that and signals; no CTA barrier.
-        // The column-wise stores go first (their own bulk group), so the
-        // row-wise ones have the column pass's time to finish reading.
-        if (tid == SG_STORER && j > 0) {
-            bulk_wait_read_but1();
-            mbar_arrive(smem_addr(&sm.sfree_c));
-        }
-        const bool go_c = ok && (j == 0 || __all_sync(FULL, mbar_wait(smem_addr(&sm.sfree_c), (j - 1) & 1u)));
-        __syncwarp();  // limw of this warp
+        // Staging buffer j & 1 was last filled by tile j - 2; the async
+        // thread arrived on sfree[j & 1] at the end of tile j - 1, once the
+        // stores of tile j - 2 had read it (the k-th arrival on a buffer's
+        // barrier completes its phase k - 1).
+        const bool go = ok && (j < 2 || __all_sync(FULL, mbar_wait(smem_addr(&sm.sfree[j & 1]), ((j >> 1) + 1) & 1u)));
+        if (!go)
+            sm.err = 1;
+        __syncwarp();  // limw and the cleaned words of this warp
 
         // ---- column pass, part 2: y and codes of the column pair
         uint32_t gsat = 0;  // saturation bits of a general-path column pair (bits 2i, 2i+1: word i)
-        if (COL && go_c) {
+        if (COL && go) {
+            const uint32_t cqs = smem_addr(out.ccol);
             uint32_t* yq[4];
             uint8_t* cq[4];
 #pragma unroll
@@ -671,10 +679,9 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                 const uint32_t s2 = bf16_pow2(k_lo) | (bf16_pow2(k_hi) << 16);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    uint32_t aw, sg, P;
-                    prep_bf(cw[i], aw, sg);
-                    yq[i & 3][(i >> 2) * 256] = qword(aw, sg, inv_lo, inv_hi, s2, lutb16, P);
-                    cq[i & 3][(i >> 2) * 1024] = (uint8_t)e2m1_byte(P);
+                    uint32_t P;
+                    yq[i & 3][(i >> 2) * 256] = qword(cw[i], inv_lo, inv_hi, s2, lutb16, P);
+                    e2m1_byte_store(cqs + co[i & 3] + (i >> 2) * 1024, P);
                 }
             };
             if (__all_sync(FULL, fast)) {
@@ -699,19 +706,14 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             }
         }
 
-        if (tid == SG_STORER && j > 0) {
-            bulk_wait_read_all();
-            mbar_arrive(smem_addr(&sm.sfree_r));
-        }
-        const bool go = go_c && (j == 0 || __all_sync(FULL, mbar_wait(smem_addr(&sm.sfree_r), (j - 1) & 1u)));
-        if (!go)
-            sm.err = 1;
 
         // ---- row pass: the lane's row-wise block (tile row rr, columns
-        // 32w..32w+31): row-wise outputs, and the column-wise saturation word
-        // of the same 32 elements
+        // 32w..32w+31): row-wise outputs (y over the block's own input words:
+        // the column pass of this warp, the only other reader of these
+        // columns, is done), and the column-wise saturation word of the same
+        // 32 elements
         if (go) {
-            uint32_t rw16[16];  // raw words of the lane's block
+            uint32_t rw16[16];  // the lane's block, -0 cleared by the column pass
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 const uint4 c = sm_ld128(tile, ro[jj]);
@@ -719,6 +721,11 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                 rw16[4 * jj + 1] = c.y;
                 rw16[4 * jj + 2] = c.z;
                 rw16[4 * jj + 3] = c.w;
+            }
+            if constexpr (!COL) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    rw16[i] = clear_neg_zero(rw16[i]);  // no column pass cleaned them
             }
             if (COL && a.mask_col) {
                 // rows past a group tail are not copied out; their word is don't-care
@@ -755,11 +762,10 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                         uint32_t P[4], o[4], a4w[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            uint32_t sg;
-                            prep_bf(rw16[4 * jj + u], a4w[u], sg);
-                            o[u] = qword(a4w[u], sg, inv, inv, s2, lutb16, P[u]);
+                            a4w[u] = rw16[4 * jj + u] & 0x7FFF7FFFu;
+                            o[u] = qword(rw16[4 * jj + u], inv, inv, s2, lutb16, P[u]);
                         }
-                        *reinterpret_cast<uint4*>(out.yrow + ro[jj]) = make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4*>(tile + ro[jj]) = make_uint4(o[0], o[1], o[2], o[3]);
                         nib[jj] = e2m1_word(P);
                         sats |= sat8(a4w, limx) << (8 * jj);
                     }
@@ -773,7 +779,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                     for (int jj = 0; jj < 4; ++jj) {
                         const uint4 dv = make_uint4(rw16[4 * jj], rw16[4 * jj + 1], rw16[4 * jj + 2], rw16[4 * jj + 3]);
                         const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
-                        *reinterpret_cast<uint4*>(out.yrow + ro[jj]) = gch.packed;
+                        *reinterpret_cast<uint4*>(tile + ro[jj]) = gch.packed;
                         nib[jj] = gch.nibs;
                         sats |= gch.sats << (8 * jj);
                     }
@@ -787,7 +793,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         // column pairs of the general path add their exact saturation bits
         if (COL && go && __any_sync(FULL, gsat != 0u))
             col_sat_store(out.mcol, gsat, h, p, warp);
-        fence_async_smem();  // staged outputs -> visible to the TMA stores
+        fence_async_smem();  // staged outputs and the stage's y -> visible to the TMA stores and loads
         __syncthreads();     // stage s consumed; staged outputs complete; errors visible
         if (sm.err)
             break;
@@ -799,11 +805,9 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         // rows and columns outside the tensor.
         const uint32_t tma = (nrows == SG_ROWS ? col_out : 0u) | row_out;
         const uint32_t copy = (col_out | row_out) & ~(tma & a.ts_flags);
-        if (tid == 0 && t_issue < t_end)
-            issue(s);  // refill the consumed stage
-        if (tid == SG_STORER) {
+        if (async_thread) {
             const uint32_t st = tma & a.ts_flags;
-            const uint32_t ybase_c = smem_addr(out.ycol), ybase_r = smem_addr(out.yrow);
+            const uint32_t ybase_c = smem_addr(out.ycol), ybase_r = smem_addr(tile);
 #pragma unroll
             for (int sl = 0; sl < 4; ++sl)
                 if ((st & SG_TS_Y) && col0 + sl * SG_SLAB_COLS < a.cols)
@@ -812,7 +816,6 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                 tma_store_box(&maps.codes, smem_addr(out.ccol), col0 / 2, row0);
             if (st & SG_TS_MASK)
                 tma_store_box(&maps.mask, smem_addr(out.mcol), col0 / 8, row0);
-            bulk_commit();  // column-wise group
 #pragma unroll
             for (int sl = 0; sl < 4; ++sl)
                 if ((st & SG_TS_YR) && col0 + sl * SG_SLAB_COLS < a.cols)
@@ -821,30 +824,48 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                 tma_store_box(&maps.codes_r, smem_addr(out.crow), col0 / 2, row0);
             if (st & SG_TS_MASK_R)
                 tma_store_box(&maps.mask_r, smem_addr(out.mrow), col0 / 8, row0);
-            bulk_commit();  // row-wise group
+            bulk_commit();  // this tile's group
+            if (j > 0) {
+                // tile j - 1's stores have read its staging buffer and its
+                // stage (they had this tile's time to do so): release the
+                // buffer to tile j + 1 and load tile j + 2 into the stage
+                bulk_wait_read_but1();
+                mbar_arrive(smem_addr(&sm.sfree[(j - 1) & 1]));
+                if (t_issue < t_end)
+                    issue(s == 0 ? SG_STAGES - 1 : s - 1);
+            }
         }
-        if (ROW && a.scales_row && warp == SG_STORER / 32)
+        if (ROW && a.scales_row && warp == SG_ASYNC / 32)
             copy_row_scales<SMMA>(a, out, row0, nrows, col0, lane);
-        if (copy) {
-            copy_outputs(a, out, row0, nrows, col0, copy);
-            __syncthreads();  // no warp writes the staging buffers before every copy is done
-        }
+        // (tile j + 1 writes the other staging buffer and stage: no barrier
+        // is needed before the next tile)
+        if (copy)
+            copy_outputs(a, out, tile, row0, nrows, col0, copy);
         if (++s == SG_STAGES) {
             s = 0;
             phase ^= 1u;
         }
     }
 
-    if (tid == 0 && sm.err) {
-        if (a.status)
-            *a.status = MXFP4_ECUDA;
-        // loads still in flight land in shared memory: wait for them
-        // (bounded) before the CTA releases it
-        for (int st = 0; st < SG_STAGES; ++st)
-            (void)mbar_wait(smem_addr(&sm.full[st]), phase ^ (st < s ? 1u : 0u));
-    }
-    if (tid == SG_STORER)
+    if (async_thread) {
+        if (sm.err) {
+            if (a.status)
+                *a.status = MXFP4_ECUDA;
+            // loads still in flight land in shared memory: wait for them
+            // (bounded) before the CTA releases it. They are the tiles from
+            // the one this loop stopped at (index t) up to t_issue, in stages
+            // s, s + 1, ... with the phase of their turn.
+            uint32_t ss = (uint32_t)s, ph = phase;
+            for (uint32_t k = t; k < t_issue; ++k) {
+                (void)mbar_wait(smem_addr(&sm.full[ss]), ph);
+                if (++ss == SG_STAGES) {
+                    ss = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
         bulk_wait_all();
+    }
 }
 
 // ---------------------------------------------------------------------------
