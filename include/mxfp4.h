@@ -297,6 +297,70 @@ int64_t mxfp4_colwise_operand_k_bound(int64_t rows, int64_t num_groups);
  * (k_alloc / 128); -1 for invalid arguments. */
 int64_t mxfp4_colwise_operand_scale_bytes(int64_t cols, int64_t k_alloc);
 
+/*
+ * Grouped block-scaled GEMM on the tensor cores, the consumer of the
+ * operands above (MindSpore hyper-parallel fake_w4a8_gmm_func.py,
+ * FakeW4A8GroupedLinear.grouped_matmul over the operands _select_operands
+ * picks for the layouts "NN", "NT" and "TN"):
+ *   D = A B^T, D[m][n] = sum_k decode(A[m][k]) 2^(sA[m][k/32] - 127)
+ *                              decode(B[n][k]) 2^(sB[n][k/32] - 127),
+ * accumulated in fp32, stored as fp32 or bf16 (round to nearest even).
+ *   elem_format   MXFP4_ELEM_E2M1 (codes_row / MXFP4_COLS_MMA codes: two per
+ *                 byte, first element in the low nibble) or MXFP4_ELEM_E4M3
+ *                 (one byte per element); both operands alike.
+ *   a, lda        A [m][k] codes, K-major, row stride lda bytes (a multiple
+ *                 of 16; a 16-byte aligned). k is a multiple of 128.
+ *   a_scales      E8M0 scales of A in the MXFP4_SCALES_MMA layout of the
+ *                 [m][k/32] scale matrix (mxfp4_scales_row_bytes(m, k, 32,
+ *                 MXFP4_SCALES_MMA) bytes).
+ *   b, ldb, b_scales  likewise for B.
+ *   group_mode    MXFP4_GMM_GROUP_M ("NN" forward, "NT" input gradient): the
+ *                 group list partitions the m rows of A and D; group g uses
+ *                 B_g = rows [g n, g n + n) of b (b holds num_groups stacked
+ *                 [n][k] matrices with row stride ldb) and its scale matrix
+ *                 at b_scales + g * mxfp4_scales_row_bytes(n, k, 32,
+ *                 MXFP4_SCALES_MMA).
+ *                 MXFP4_GMM_GROUP_K ("TN" weight gradient): A [m][k] and B
+ *                 [n][k] are column-wise operands in the MXFP4_COLS_MMA
+ *                 layout with k = k_alloc; the group list partitions k_rows
+ *                 rows (tokens) and group g contracts over its K slots
+ *                 [K0_g, K0_g + 128 ceil(n_g / 128)); D holds num_groups
+ *                 matrices [m][n], D_g at d + g * m * ldd; an empty group's
+ *                 D_g is zero.
+ *   d, ldd, d_dtype  output, row stride ldd elements (ldd * element size a
+ *                 multiple of 16, d 16-byte aligned), MXFP4_F32 or
+ *                 MXFP4_BF16.
+ *   status        optional device int32: the group list check (MXFP4_EINVAL:
+ *                 not a partition, or GROUP_K groups that need more than k
+ *                 slots; nothing is written then) or MXFP4_ECUDA.
+ * Argument errors are returned before any launch. Operand values are read
+ * as is: NaN scales (0xFF) and the E4M3 NaN code give NaN results.
+ */
+#define MXFP4_GMM_GROUP_M 0
+#define MXFP4_GMM_GROUP_K 1
+
+typedef struct mxfp4_gmm_args {
+    int32_t elem_format;
+    int32_t group_mode;
+    int64_t m, n, k;
+    const uint8_t* a;
+    int64_t lda;
+    const uint8_t* a_scales;
+    const uint8_t* b;
+    int64_t ldb;
+    const uint8_t* b_scales;
+    const int64_t* group_list;
+    int64_t num_groups;
+    int32_t group_list_type;
+    int32_t d_dtype;
+    int64_t k_rows;
+    void* d;
+    int64_t ldd;
+    int32_t* status;
+} mxfp4_gmm_args;
+
+mxfp4_status mxfp4_grouped_gemm(const mxfp4_gmm_args* args, mxfp4_stream_t stream);
+
 /* Static English text of a status; never NULL. */
 const char* mxfp4_status_string(mxfp4_status status);
 

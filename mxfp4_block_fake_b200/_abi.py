@@ -34,6 +34,7 @@ EXPORTS = (
     "mxfp4_colwise_operand_k",
     "mxfp4_colwise_operand_k_bound",
     "mxfp4_colwise_operand_scale_bytes",
+    "mxfp4_grouped_gemm",
     "mxfp4_status_string",
     "mxfp4_abi_version",
 )
@@ -67,6 +68,33 @@ class QdqArgs(ctypes.Structure):
         ("elem_format", ctypes.c_int32),
         ("col_layout", ctypes.c_int32),
         ("k_alloc", ctypes.c_int64),
+    ]
+
+
+GMM_GROUP_M, GMM_GROUP_K = 0, 1
+
+
+class GmmArgs(ctypes.Structure):
+    _fields_ = [
+        ("elem_format", ctypes.c_int32),
+        ("group_mode", ctypes.c_int32),
+        ("m", ctypes.c_int64),
+        ("n", ctypes.c_int64),
+        ("k", ctypes.c_int64),
+        ("a", ctypes.c_void_p),
+        ("lda", ctypes.c_int64),
+        ("a_scales", ctypes.c_void_p),
+        ("b", ctypes.c_void_p),
+        ("ldb", ctypes.c_int64),
+        ("b_scales", ctypes.c_void_p),
+        ("group_list", ctypes.c_void_p),
+        ("num_groups", ctypes.c_int64),
+        ("group_list_type", ctypes.c_int32),
+        ("d_dtype", ctypes.c_int32),
+        ("k_rows", ctypes.c_int64),
+        ("d", ctypes.c_void_p),
+        ("ldd", ctypes.c_int64),
+        ("status", ctypes.c_void_p),
     ]
 
 
@@ -115,6 +143,8 @@ def lib() -> ctypes.CDLL:
     L.mxfp4_colwise_operand_k_bound.restype = i64
     L.mxfp4_colwise_operand_scale_bytes.argtypes = [i64, i64]
     L.mxfp4_colwise_operand_scale_bytes.restype = i64
+    L.mxfp4_grouped_gemm.argtypes = [ctypes.POINTER(GmmArgs), P]
+    L.mxfp4_grouped_gemm.restype = i32
     L.mxfp4_status_string.argtypes = [i32]
     L.mxfp4_status_string.restype = ctypes.c_char_p
     L.mxfp4_abi_version.argtypes = []
@@ -173,3 +203,7 @@ def mxfp4_colwise_operand_k(host_group_list, group_list_type: int, rows: int) ->
     n = len(host_group_list)
     arr = (ctypes.c_int64 * n)(*[int(v) for v in host_group_list])
     return lib().mxfp4_colwise_operand_k(arr, n, group_list_type, rows)
+
+
+def mxfp4_grouped_gemm(args: GmmArgs, stream: int) -> int:
+    return lib().mxfp4_grouped_gemm(ctypes.byref(args), stream)

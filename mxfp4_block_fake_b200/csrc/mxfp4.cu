@@ -1166,6 +1166,7 @@ __global__ void __launch_bounds__(NTHREADS)
 
 #include "mxfp4_staged.cuh"
 #include "mxfp4_operand.cuh"
+#include "mxfp4_gemm.cuh"
 
 namespace mxfp4 {
 
@@ -1900,6 +1901,106 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     return st;
 }
 
+// ---- grouped block-scaled GEMM (mxfp4_grouped_gemm) -----------------------
+
+template <int FMT, bool GK, bool F32>
+static mxfp4_status launch_gmm_t(const GmMaps& maps, const GmArgs& g, int64_t tile_bound, cudaStream_t s)
+{
+    const void* fn = (const void*)gmm_kernel<FMT, GK, F32>;
+    const size_t smem = sizeof(GmSmem<FMT>) + 1024 + (size_t)(2 * (g.num_groups + 1)) * sizeof(int32_t);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MXFP4_ECUDA;
+    const int sms = device_sms();
+    if (sms <= 0)
+        return MXFP4_ECUDA;
+    int64_t grid = sms;
+    if (tile_bound < grid)
+        grid = tile_bound < 1 ? 1 : tile_bound;
+    GmMaps m = maps;
+    GmArgs a = g;
+    void* args[] = {&m, &a};
+    return cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(GM_THREADS), args, smem, s) == cudaSuccess ? MXFP4_OK
+                                                                                                    : MXFP4_ECUDA;
+}
+
+static mxfp4_status run_gmm(const mxfp4_gmm_args* A, cudaStream_t s)
+{
+    if (!A)
+        return MXFP4_EINVAL;
+    if (A->elem_format != MXFP4_ELEM_E2M1 && A->elem_format != MXFP4_ELEM_E4M3)
+        return MXFP4_EINVAL;
+    if (A->group_mode != MXFP4_GMM_GROUP_M && A->group_mode != MXFP4_GMM_GROUP_K)
+        return MXFP4_EINVAL;
+    if (A->d_dtype != MXFP4_F32 && A->d_dtype != MXFP4_BF16)
+        return MXFP4_EINVAL;
+    if (A->m < 0 || A->n < 0 || A->k < 0 || A->k % GM_BK != 0)
+        return MXFP4_EINVAL;
+    if (A->m > INT32_MAX || A->n > INT32_MAX || A->k > INT32_MAX)
+        return MXFP4_EUNSUPPORTED;
+    if (!A->group_list || A->num_groups < 1 || (A->group_list_type != 0 && A->group_list_type != 1) ||
+        !aligned(A->group_list, 8))
+        return MXFP4_EINVAL;
+    if (A->num_groups > MXFP4_MAX_GROUPS)
+        return MXFP4_EUNSUPPORTED;
+    const bool gk = A->group_mode == MXFP4_GMM_GROUP_K;
+    if (gk && A->k_rows < 0)
+        return MXFP4_EINVAL;
+    if (A->m == 0 || A->n == 0) {
+        if (A->status && cudaMemsetAsync(A->status, 0, sizeof(int32_t), s) != cudaSuccess)
+            return MXFP4_ECUDA;
+        return MXFP4_OK;
+    }
+    const int64_t kb = A->elem_format == MXFP4_ELEM_E2M1 ? A->k / 2 : A->k;  // bytes of a K row
+    const int esz = A->d_dtype == MXFP4_F32 ? 4 : 2;
+    if (!A->a || !A->b || !A->a_scales || !A->b_scales || !A->d)
+        return MXFP4_EINVAL;
+    if (A->lda < kb || A->ldb < kb || A->lda % 16 != 0 || A->ldb % 16 != 0 || !aligned(A->a, 16) || !aligned(A->b, 16))
+        return MXFP4_EINVAL;
+    if (!aligned(A->a_scales, 4) || !aligned(A->b_scales, 4) || A->ldd < A->n || !aligned(A->d, 16) ||
+        (A->ldd * esz) % 16 != 0)
+        return MXFP4_EINVAL;
+    const bool e2 = A->elem_format == MXFP4_ELEM_E2M1;
+    const int row_bytes = e2 ? GmFmt<MXFP4_ELEM_E2M1>::ROW_BYTES : GmFmt<MXFP4_ELEM_E4M3>::ROW_BYTES;
+    const CUtensorMapSwizzle sw = e2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    GmMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    const int64_t b_rows = gk ? A->n : A->n * A->num_groups;
+    if (!encode_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<uint8_t*>(A->a), (uint64_t)kb, (uint64_t)A->m,
+                   (uint64_t)A->lda, (uint32_t)row_bytes, GM_BM, sw) ||
+        !encode_2d(&maps.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<uint8_t*>(A->b), (uint64_t)kb, (uint64_t)b_rows,
+                   (uint64_t)A->ldb, (uint32_t)row_bytes, GM_BN, sw))
+        return MXFP4_ECUDA;
+    GmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.sfa = A->a_scales;
+    g.sfb = A->b_scales;
+    g.d = A->d;
+    g.group_list = A->group_list;
+    g.status = A->status;
+    g.a_rows = A->m;
+    g.n = A->n;
+    g.k = A->k;
+    g.ldd = A->ldd;
+    g.sfb_group_bytes = 512 * ((A->n + 127) / 128) * ((A->k / 32 + 3) / 4);
+    g.k_rows = A->k_rows;
+    g.num_groups = (int32_t)A->num_groups;
+    g.gl_type = A->group_list_type;
+    g.d_f32 = A->d_dtype == MXFP4_F32;
+    g.group_k = gk;
+    const int64_t n_nt = (A->n + GM_BN - 1) / GM_BN;
+    const int64_t bound = gk ? A->num_groups * ((A->m + GM_BM - 1) / GM_BM) * n_nt : (A->m / GM_BM + A->num_groups) * n_nt;
+    const bool f32 = A->d_dtype == MXFP4_F32;
+    if (e2)
+        return gk ? (f32 ? launch_gmm_t<MXFP4_ELEM_E2M1, true, true>(maps, g, bound, s)
+                         : launch_gmm_t<MXFP4_ELEM_E2M1, true, false>(maps, g, bound, s))
+                  : (f32 ? launch_gmm_t<MXFP4_ELEM_E2M1, false, true>(maps, g, bound, s)
+                         : launch_gmm_t<MXFP4_ELEM_E2M1, false, false>(maps, g, bound, s));
+    return gk ? (f32 ? launch_gmm_t<MXFP4_ELEM_E4M3, true, true>(maps, g, bound, s)
+                     : launch_gmm_t<MXFP4_ELEM_E4M3, true, false>(maps, g, bound, s))
+              : (f32 ? launch_gmm_t<MXFP4_ELEM_E4M3, false, true>(maps, g, bound, s)
+                     : launch_gmm_t<MXFP4_ELEM_E4M3, false, false>(maps, g, bound, s));
+}
+
 }  // namespace mxfp4
 
 using namespace mxfp4;
@@ -2098,6 +2199,11 @@ int64_t mxfp4_colwise_operand_scale_bytes(int64_t cols, int64_t k_alloc)
     if (cols < 0 || k_alloc < 0 || k_alloc % OP_KPAD != 0)
         return -1;
     return 512 * ((cols + 127) / 128) * (k_alloc / OP_KPAD);
+}
+
+mxfp4_status mxfp4_grouped_gemm(const mxfp4_gmm_args* args, mxfp4_stream_t stream)
+{
+    return run_gmm(args, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int32_t mxfp4_abi_version(void) { return MXFP4_ABI_VERSION; }

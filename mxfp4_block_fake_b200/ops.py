@@ -460,3 +460,77 @@ def mxfp4_colwise_mma_operand(x: torch.Tensor, *, group_list=None, group_list_ty
                       colwise=True, group_list=group_list, group_list_type=group_list_type, emit_values=False,
                       emit_codes=True, col_layout="mma", k_alloc=k_alloc, check=check)
     return r.codes_col.view(torch.float4_e2m1fn_x2), r.scales_col.view(torch.float8_e8m0fnu), r.k_alloc
+
+
+_GMM_MODES = {"m": _abi.GMM_GROUP_M, "k": _abi.GMM_GROUP_K}
+
+
+def mxfp4_grouped_gemm(a: torch.Tensor, a_scales: torch.Tensor, b: torch.Tensor, b_scales: torch.Tensor,
+                       group_list, *, k: int, group_mode: str = "m", elem_format: str = "e2m1",
+                       group_list_type: int = 0, k_rows: int | None = None, out_dtype=torch.float32,
+                       check: bool | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Grouped block-scaled GEMM D = A B^T on the tensor cores (include/mxfp4.h,
+    mxfp4_grouped_gemm), on operands as this library emits them.
+
+    a: [m, k/2] (E2M1) or [m, k] (E4M3) uint8 codes, K-major; a_scales: the
+    MMA-layout E8M0 scales of A. group_mode "m": the group list splits the
+    m rows; b is [G, n, row bytes] or [G * n, row bytes], b_scales G
+    consecutive MMA-layout scale buffers; D is [m, n]. group_mode "k": A and
+    B are column-wise operands (col_layout "mma", k = their k_alloc), the
+    group list splits k_rows rows; D is [G, m, n]. check (the default)
+    synchronises and raises for an invalid group list."""
+    fmt = _elem_format(elem_format)
+    if group_mode not in _GMM_MODES:
+        raise ValueError(f"group_mode must be 'm' or 'k', got {group_mode!r}")
+    for t, name in ((a, "a"), (a_scales, "a_scales"), (b, "b"), (b_scales, "b_scales")):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype not in (torch.uint8, torch.float4_e2m1fn_x2,
+                                                                                 torch.float8_e4m3fn, torch.float8_e8m0fnu):
+            raise ValueError(f"{name} must be a CUDA uint8 (or fp4 / fp8 / e8m0) tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    a8, b8 = a.view(torch.uint8), b.view(torch.uint8)
+    kb = k // 2 if fmt == _abi.ELEM_E2M1 else k
+    if k <= 0 or k % 128:
+        raise ValueError("k must be a positive multiple of 128")
+    a8 = a8.reshape(-1, a8.shape[-1])
+    b8 = b8.reshape(-1, b8.shape[-1])
+    if a8.shape[1] < kb or b8.shape[1] < kb:
+        raise ValueError("operand rows are shorter than k")
+    gl, ng = _group_args(group_list, group_list_type, a.device)
+    if gl is None:
+        raise ValueError("a group_list is required (one group: [rows])")
+    m = a8.shape[0]
+    gk = group_mode == "k"
+    if gk:
+        n = b8.shape[0]
+        if k_rows is None:
+            raise ValueError("group_mode 'k' needs k_rows (the rows the group list partitions)")
+        shape = (ng, m, n)
+    else:
+        if b8.shape[0] % ng:
+            raise ValueError("b must stack num_groups matrices of n rows")
+        n = b8.shape[0] // ng
+        shape = (m, n)
+    if check is None:
+        check = True
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    d = out if out is not None else torch.empty(shape, dtype=out_dtype, device=a.device)
+    if tuple(d.shape) != shape or d.dtype != out_dtype or not d.is_contiguous():
+        raise ValueError(f"out must be a contiguous {out_dtype} tensor of shape {list(shape)}")
+    st = torch.empty((1,), dtype=torch.int32, device=a.device)
+    g = _abi.GmmArgs()
+    g.elem_format = fmt
+    g.group_mode = _GMM_MODES[group_mode]
+    g.m, g.n, g.k = m, n, int(k)
+    g.a, g.lda, g.a_scales = a8.data_ptr(), a8.stride(0), a_scales.data_ptr()
+    g.b, g.ldb, g.b_scales = b8.data_ptr(), b8.stride(0), b_scales.data_ptr()
+    g.group_list, g.num_groups, g.group_list_type = gl.data_ptr(), ng, int(group_list_type)
+    g.d_dtype = _DTYPES[out_dtype]
+    g.k_rows = int(k_rows) if gk else 0
+    g.d, g.ldd = d.data_ptr(), n
+    g.status = st.data_ptr()
+    _abi.check(_abi.mxfp4_grouped_gemm(g, _stream(a.device)), "mxfp4_grouped_gemm")
+    if check:
+        _check_status(st, "mxfp4_grouped_gemm")
+    return d

@@ -51,13 +51,15 @@ def test_library_exports_every_declared_symbol(abi):
         assert hasattr(abi.lib(), name)
 
 
-def test_struct_layout_matches_c(abi, tmp_path):
-    fields = [f for f, _ in abi.QdqArgs._fields_]
+@pytest.mark.parametrize("cname,pyname", [("mxfp4_qdq_args", "QdqArgs"), ("mxfp4_gmm_args", "GmmArgs")])
+def test_struct_layout_matches_c(abi, tmp_path, cname, pyname):
+    cls = getattr(abi, pyname)
+    fields = [f for f, _ in cls._fields_]
     src = tmp_path / "layout.c"
-    body = "\n".join(f'  printf("{f} %zu\\n", offsetof(mxfp4_qdq_args, {f}));' for f in fields)
+    body = "\n".join(f'  printf("{f} %zu\\n", offsetof({cname}, {f}));' for f in fields)
     src.write_text(
         "#include <stdio.h>\n#include <stddef.h>\n#include \"mxfp4.h\"\n"
-        "int main(void) {\n" + body + '\n  printf("sizeof %zu\\n", sizeof(mxfp4_qdq_args));\n  return 0;\n}\n'
+        "int main(void) {\n" + body + f'\n  printf("sizeof %zu\\n", sizeof({cname}));\n  return 0;\n}}\n'
     )
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), "-o", str(exe), str(src)], check=True)
@@ -65,8 +67,33 @@ def test_struct_layout_matches_c(abi, tmp_path):
                                                       check=True).stdout.splitlines())
     import ctypes
     for f in fields:
-        assert int(got[f]) == getattr(abi.QdqArgs, f).offset, f
-    assert int(got["sizeof"]) == ctypes.sizeof(abi.QdqArgs)
+        assert int(got[f]) == getattr(cls, f).offset, f
+    assert int(got["sizeof"]) == ctypes.sizeof(cls)
+
+
+def _gmm(abi, **kw):
+    g = abi.GmmArgs()
+    g.elem_format, g.group_mode, g.m, g.n, g.k = abi.ELEM_E2M1, abi.GMM_GROUP_M, 256, 128, 256
+    g.a, g.lda, g.a_scales = 4096, 128, 8192
+    g.b, g.ldb, g.b_scales = 16384, 128, 32768
+    g.group_list, g.num_groups, g.group_list_type = 65536, 1, 0
+    g.d_dtype, g.d, g.ldd = abi.F32, 131072, 128
+    for k, v in kw.items():
+        setattr(g, k, v)
+    return g
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(elem_format=7), 1), (dict(group_mode=2), 1), (dict(d_dtype=5), 1), (dict(k=200), 1), (dict(k=-128), 1),
+    (dict(m=-1), 1), (dict(m=2 ** 31), 2), (dict(group_list=None), 1), (dict(num_groups=0), 1),
+    (dict(num_groups=5000), 2), (dict(group_list_type=3), 1), (dict(group_list=65540), 1),
+    (dict(group_mode=1, k_rows=-1), 1), (dict(a=None), 1), (dict(lda=64), 1), (dict(lda=136), 1),
+    (dict(a=4100), 1), (dict(ldb=100), 1), (dict(d=131076), 1), (dict(ldd=100), 1), (dict(ldd=130), 1),
+    (dict(a_scales=8194), 1),
+])
+def test_grouped_gemm_rejects_bad_arguments_on_host(abi, kw, expected):
+    assert abi.mxfp4_grouped_gemm(_gmm(abi, **kw), None) == expected
+    assert abi.lib().mxfp4_grouped_gemm(None, None) == abi.EINVAL
 
 
 def test_header_compiles_as_c_and_cpp(tmp_path):
