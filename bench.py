@@ -186,8 +186,9 @@ def measured_peaks():
 def kernel_source_sha() -> str:
     """sha256 over the CUDA sources of the library (the forward kernels)."""
     h = hashlib.sha256()
-    for name in ("mxfp4.cu", "mxfp4_staged.cuh"):
-        with open(os.path.join(ROOT, "mxfp4_block_fake_b200", "csrc", name), "rb") as f:
+    csrc = os.path.join(ROOT, "mxfp4_block_fake_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
@@ -424,6 +425,17 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
         call(_abi.mxfp4_qdq_fwd(fo_args, sp), "mxfp4_qdq_fwd")
         call(_abi.mxfp4_ste_bwd(bo_args, g_ptr, gi_ptr, a.cols, m_ptr, 1, sp), "mxfp4_ste_bwd")
 
+    # the column-wise GEMM operand over the groups (codes + scales, K-major)
+    k_op = ops.colwise_operand_k(gl, 0, a.rows)
+    opr = ops.alloc_outputs(xd, block=32, rowwise=False, colwise=True, num_groups=a.groups, emit_values=False,
+                            emit_codes=True, with_status=True, col_layout="mma", k_alloc=k_op)
+    op_args = ops.make_args(xd, block=32, scale_factor=6.0, scale_mode=a.scale_mode, dirs=_abi.COLWISE,
+                            group_list=gl, group_list_type=0, status=opr.status)
+    ops._fill_outputs(op_args, opr)
+
+    def col_operand():
+        call(_abi.mxfp4_qdq_fwd(op_args, sp), "mxfp4_qdq_fwd")
+
     def mxfp8_row():
         call(_abi.mxfp4_qdq_fwd(row8, sp), "mxfp4_qdq_fwd")
 
@@ -435,6 +447,7 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
     for name, fn, bpe in (("rowwise_fwd_all_outputs_ste_mask", row_step, 4 + 0.5 + 1 / 32 + 0.125 + 4.125),
                           ("training_step_rowwise_fwd_ste_recompute", train_step, 4 + 6),
                           ("mxfp4_mma_operand_rowwise_codes_scales", mma_operand, 2 + 0.5 + 1 / 32),
+                          ("mxfp4_mma_operand_colwise_grouped_codes_scales", col_operand, 2 + 0.5 + 1 / 32),
                           ("dual_block128_all_outputs", dual128, 2 + 4 + 1 + 2 / 128 + 0.25),
                           ("mxfp8_rowwise_all_outputs", mxfp8_row, 2 + 2 + 1 + 1 / 32 + 0.125),
                           ("mxfp8_dual_grouped_all_outputs", mxfp8_dual, 2 + 4 + 2 + 2 / 32 + 0.25),
@@ -452,7 +465,76 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
         gbs = n * bpe / (ms / 1e3) / 1e9
         out[name] = {"ms_per_step": round(ms, 4), "bytes_per_element": round(bpe, 4), "GB/s": round(gbs, 1),
                      "frac_of_measured_peak": round(gbs / peak, 4)}
+    del opr, r8, r128, mma_scales
+    torch.cuda.empty_cache()
+    out.update(time_gemm(a, xd, res, gl, stream, steps))
     return out
+
+
+def bf16_tflops_peak():
+    """Dense bf16 tensor-core peak: the measured burst figure, else the
+    fallback of this pool (TFLOP/s, kind)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), "measured"
+    except Exception:  # noqa: BLE001
+        return 1590.0, "fallback"
+
+
+def time_gemm(a, xd, res, gl, stream, steps: int = 20, n_expert: int = 2048):
+    """The grouped block-scaled GEMM that consumes the real-quantisation
+    operands: the MoE experts' forward on the bench tokens, D[rows of g] =
+    Q(x_g) Q(W_g)^T with one [n_expert, cols] weight per group (seeded
+    N(0, 0.02^2) on the device), MXFP4 (kind::mxf4) operands, bf16 output.
+    TFLOP/s against the dense bf16 peak times 4 (the nominal FP4 / bf16
+    ratio, 9 / 2.25 PFLOP/s)."""
+    import torch
+
+    from mxfp4_block_fake_b200 import _abi, ops
+
+    G, K = a.groups, a.cols
+    ca, sa = ops.mxfp4_mma_operand(xd)
+    sbytes = ops.scales_row_bytes(n_expert, K, 32, "mma")
+    wc = torch.empty((G * n_expert, K // 2), dtype=torch.uint8, device=xd.device)
+    ws = torch.zeros((G, sbytes), dtype=torch.uint8, device=xd.device)
+    gen = torch.Generator(device=xd.device).manual_seed(7)
+    for g in range(G):
+        w = (torch.randn(n_expert, K, generator=gen, device=xd.device) * 0.02).to(torch.bfloat16)
+        ops.mxfp4_qdq_fwd(w, block=32, rowwise=True, emit_values=False, emit_codes=True, scales_layout="mma",
+                          out=ops.QDQResult(codes_row=wc[g * n_expert:(g + 1) * n_expert], scales_row=ws[g],
+                                            scales_layout="mma"))
+    d = torch.empty((a.rows, n_expert), dtype=torch.bfloat16, device=xd.device)
+    st = torch.empty((1,), dtype=torch.int32, device=xd.device)
+    ga = _abi.GmmArgs()
+    ga.elem_format, ga.group_mode = _abi.ELEM_E2M1, _abi.GMM_GROUP_M
+    ga.m, ga.n, ga.k = a.rows, n_expert, K
+    ga.a, ga.lda, ga.a_scales = ca.data_ptr(), K // 2, sa.data_ptr()
+    ga.b, ga.ldb, ga.b_scales = wc.data_ptr(), K // 2, ws.data_ptr()
+    ga.group_list, ga.num_groups, ga.group_list_type = gl.data_ptr(), G, 0
+    ga.d_dtype, ga.d, ga.ldd, ga.status = _abi.BF16, d.data_ptr(), n_expert, st.data_ptr()
+    sp = stream.cuda_stream
+
+    def gemm():
+        _abi.check(_abi.mxfp4_grouped_gemm(ga, sp), "mxfp4_grouped_gemm")
+
+    for _ in range(3):
+        gemm()
+    torch.cuda.synchronize()
+    _abi.check(int(st.item()), "mxfp4_grouped_gemm (group_list)")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        gemm()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    flops = 2.0 * a.rows * n_expert * K
+    tf = flops / (ms / 1e3) / 1e12
+    peak, kind = bf16_tflops_peak()
+    return {f"grouped_gemm_mxfp4_moe_fwd_{a.rows}x{n_expert}x{K}_{G}experts": {
+        "ms_per_step": round(ms, 4), "TFLOP/s": round(tf, 1), "peak_TFLOP/s": round(4 * peak, 1),
+        "peak_kind": f"{kind} bf16 x 4 (nominal fp4/bf16 ratio)", "frac_of_peak": round(tf / (4 * peak), 4)}}
 
 
 def cpu_baseline(a, x_h, g_h, offsets, rows: int):

@@ -70,6 +70,11 @@ struct KArgs {
     int32_t srow_mma;   // scales_row in the MMA scale-factor layout (MXFP4_SCALES_MMA)
     int32_t fmt;        // MXFP4_ELEM_E2M1 or MXFP4_ELEM_E4M3
     int64_t k_alloc;    // column-wise operand layout: K slots per codes row (MXFP4_COLS_MMA)
+    // 4 and 65536, set by the host: the staged kernel scales table indices and
+    // moves halves with integer multiply-adds by these run-time values, which
+    // the compiler cannot turn back into shifts, so that this work runs on the
+    // multiply-add pipe beside the logic ops on the ALU pipe
+    uint32_t mul4, mul16;
 };
 
 // Byte offset of row-wise scale (row, b) of a [rows][nblk] scale matrix:
@@ -1748,6 +1753,8 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     k.sf = A->scale_factor;
     k.mode = A->scale_mode;
     k.grad_dir = grad ? (int32_t)grad_dir : 0;
+    k.mul4 = 4;
+    k.mul16 = 65536;
     if (row) {
         k.y_row = A->y_row;
         k.codes_row = A->codes_row;

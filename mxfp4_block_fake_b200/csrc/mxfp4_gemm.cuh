@@ -30,9 +30,10 @@
 //     scaled MMAs (tcgen05.mma kind::mxf4 K = 64, or kind::mxf8f6f4 K = 32),
 //     releasing the stage with tcgen05.commit; two accumulators of 128 fp32
 //     columns alternate between tiles.
-//   warps 2-5: epilogue (warps 6-7 only help build the group plan). Each warp reads its 32 lanes (rows) of the finished
-//     accumulator (tcgen05.ld 32x32b), converts and stores the valid rows
-//     and columns of the tile, and hands the accumulator back.
+//   warps 2-5: epilogue. Each warp reads its 32 lanes (rows) of the
+//     finished accumulator (tcgen05.ld 32x32b), converts and stores the
+//     valid rows and columns of the tile, and hands the accumulator back.
+//   warps 6-7 only help build the group plan.
 // Every wait on an mbarrier gives up after 4 s of global time; the CTA then
 // records MXFP4_ECUDA, waits (bounded) for its loads and MMAs in flight,
 // frees the tensor memory and exits.
@@ -386,8 +387,9 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
             (void)mbar_wait(smem_addr(&sm.done), 0);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 6) {
         // ---- epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31
+        // (exactly four warps: acc_empty counts four arrivals per tile)
         const int quad = warp & 3;
         const int r = 32 * quad + lane;  // tile row of this thread
         int acc = 0;

@@ -240,7 +240,7 @@ __device__ __forceinline__ uint32_t clear_neg_zero(uint32_t w)
 
 // One word (two bf16 elements) of fast-path blocks; wc has no -0 halves
 // (clear_neg_zero). inv_*: 2^-k of each element's block; s2: packed bf16
-// 2^k of each element's block.
+// 2^k of each element's block; mul4, mul16: 4 and 65536 (KArgs).
 // t = 2^21 + |x| * 2^-k rounded down (fp32 spacing on [2^21, 2^22) is 1/4),
 // so t's bits are 0x4A000000 + floor(4|y|); lutb16 = table base - 0x28000000
 // folds that offset into the address shift-add. |x| is the fma's absolute-
@@ -249,12 +249,12 @@ __device__ __forceinline__ uint32_t clear_neg_zero(uint32_t w)
 // a quarter of 2^k. Returns the dequantised packed bf16 pair; P receives the
 // signed codes.
 __device__ __forceinline__ uint32_t qword(uint32_t wc, float inv_lo, float inv_hi, uint32_t s2, uint32_t lutb16,
-                                          uint32_t& P)
+                                          uint32_t mul4, uint32_t mul16, uint32_t& P)
 {
-    const float tl = __fmaf_rd(fabsf(__uint_as_float(wc << 16)), inv_lo, 0x1p21f);
+    const float tl = __fmaf_rd(fabsf(__uint_as_float(wc * mul16)), inv_lo, 0x1p21f);
     const float th = __fmaf_rd(fabsf(__uint_as_float(wc)), inv_hi, 0x1p21f);
-    const uint32_t el = lut_load(lutb16 + (__float_as_uint(tl) << 2));
-    const uint32_t eh = lut_load(lutb16 + (__float_as_uint(th) << 2));
+    const uint32_t el = lut_load(__float_as_uint(tl) * mul4 + lutb16);
+    const uint32_t eh = lut_load(__float_as_uint(th) * mul4 + lutb16);
     P = __byte_perm(el, eh, 0x7632) | (wc & 0x80008000u);
     return hmul2_bf16(P, s2);
 }
@@ -680,7 +680,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     uint32_t P;
-                    yq[i & 3][(i >> 2) * 256] = qword(cw[i], inv_lo, inv_hi, s2, lutb16, P);
+                    yq[i & 3][(i >> 2) * 256] = qword(cw[i], inv_lo, inv_hi, s2, lutb16, a.mul4, a.mul16, P);
                     e2m1_byte_store(cqs + co[i & 3] + (i >> 2) * 1024, P);
                 }
             };
@@ -763,7 +763,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             a4w[u] = rw16[4 * jj + u] & 0x7FFF7FFFu;
-                            o[u] = qword(rw16[4 * jj + u], inv, inv, s2, lutb16, P[u]);
+                            o[u] = qword(rw16[4 * jj + u], inv, inv, s2, lutb16, a.mul4, a.mul16, P[u]);
                         }
                         *reinterpret_cast<uint4*>(tile + ro[jj]) = make_uint4(o[0], o[1], o[2], o[3]);
                         nib[jj] = e2m1_word(P);

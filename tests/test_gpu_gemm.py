@@ -130,3 +130,47 @@ def test_invalid_group_lists_are_reported():
     with pytest.raises(MXFP4ArgumentError):  # groups need more K slots than k_alloc
         ops.mxfp4_grouped_gemm(a, s_a, a, s_a, torch.tensor([1, 1, 198], dtype=torch.int64, device="cuda"),
                                k=ka, group_mode="k", group_list_type=1, k_rows=200)
+
+
+@pytest.mark.parametrize("mode", ["m", "k"])
+def test_many_tiles_per_cta(mode):
+    """Enough output tiles that every CTA of the persistent grid takes
+    several in turn (the stage ring and both accumulators wrap many times),
+    against the oracle on every output."""
+    if mode == "m":
+        counts = [5000, 0, 3000, 8384]
+        M, N, K = sum(counts), 1024, 512
+        x = rand_bf16(M, K, 21)
+        ws = [rand_bf16(N, K, 30 + g, 0.05) for g in range(len(counts))]
+        ca, sa = ops.mxfp4_mma_operand(x.cuda())
+        parts = [ops.mxfp4_mma_operand(w.cuda()) for w in ws]
+        cb = torch.cat([p[0].view(torch.uint8) for p in parts])
+        sb = torch.cat([p[1].view(torch.uint8) for p in parts])
+        gl = torch.tensor(counts, dtype=torch.int64, device="cuda")
+        d = ops.mxfp4_grouped_gemm(ca, sa, cb, sb, gl, k=K, group_list_type=1)
+        qx = deq(O.qdq_rowwise(u16(x), 32, 6.0, O.SCALE_PAGE)["y"])
+        r0 = 0
+        for g, n in enumerate(counts):
+            qw = deq(O.qdq_rowwise(u16(ws[g]), 32, 6.0, O.SCALE_PAGE)["y"])
+            ref = qx[r0:r0 + n] @ qw.T
+            mag = np.abs(qx[r0:r0 + n]) @ np.abs(qw).T
+            check(d[r0:r0 + n], ref, mag, K, False)
+            r0 += n
+    else:
+        counts = [300, 450, 0, 250]
+        T, cx, cy = sum(counts), 2048, 1536
+        x = rand_bf16(T, cx, 22)
+        dy = rand_bf16(T, cy, 23, 1e-3)
+        a, sa, ka = ops.mxfp4_colwise_mma_operand(x.cuda(), group_list=counts, group_list_type=1)
+        b, sb, _ = ops.mxfp4_colwise_mma_operand(dy.cuda(), group_list=counts, group_list_type=1)
+        gl = torch.tensor(counts, dtype=torch.int64, device="cuda")
+        d = ops.mxfp4_grouped_gemm(a, sa, b, sb, gl, k=ka, group_mode="k", group_list_type=1, k_rows=T)
+        ends = np.cumsum(counts)
+        qx = deq(O.qdq_colwise(u16(x), 32, 6.0, O.SCALE_PAGE, ends=ends)["y"])
+        qy = deq(O.qdq_colwise(u16(dy), 32, 6.0, O.SCALE_PAGE, ends=ends)["y"])
+        r0 = 0
+        for g, n in enumerate(counts):
+            ref = qx[r0:r0 + n].T @ qy[r0:r0 + n]
+            mag = np.abs(qx[r0:r0 + n]).T @ np.abs(qy[r0:r0 + n])
+            check(d[g], ref, mag, max(n, 1), False)
+            r0 += n
