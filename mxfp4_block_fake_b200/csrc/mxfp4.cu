@@ -1170,6 +1170,7 @@ __global__ void __launch_bounds__(NTHREADS)
 }  // namespace mxfp4
 
 #include "mxfp4_staged.cuh"
+#include "mxfp4_staged8.cuh"
 #include "mxfp4_operand.cuh"
 #include "mxfp4_gemm.cuh"
 
@@ -1553,6 +1554,67 @@ static mxfp4_status launch_staged(bool row, bool col, bool groups, const StagedM
     return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
 }
 
+// Maps of the MXFP8 staged kernel: x as for the block-32 staged kernel;
+// row-wise y (64 x 32 boxes, 128-byte swizzle; pitch ld_y * 2), row-wise
+// E4M3 codes [rows, cols] bytes in 128 x 32 boxes with the 128-byte swizzle,
+// masks [rows, cols/8] bytes in 32 x 32 boxes, each only where TMA can
+// address it and the tensor holds a full tile (ts_flags). Returns false when
+// the input map cannot be built.
+static bool make_staged8_maps(StagedMaps* m, const KArgs& k, uint32_t* ts_flags)
+{
+    memset(m, 0, sizeof(*m));
+    *ts_flags = 0;
+    if (!encode_2d(&m->x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(k.x), (uint64_t)k.cols,
+                   (uint64_t)k.rows, (uint64_t)k.ld * 2, SG_SLAB_COLS, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        return false;
+    if (k.cols < SG_COLS || k.rows < SG_ROWS)
+        return true;
+    if (k.y_row && aligned(k.y_row, 16) && (k.ld_y * 2) % 16 == 0 &&
+        encode_2d(&m->yr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.y_row, (uint64_t)k.cols, (uint64_t)k.rows,
+                  (uint64_t)k.ld_y * 2, SG_SLAB_COLS, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        *ts_flags |= SG_TS_YR;
+    if (k.codes_row && aligned(k.codes_row, 16) && k.cols % 16 == 0 &&
+        encode_2d(&m->codes_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.codes_row, (uint64_t)k.cols, (uint64_t)k.rows,
+                  (uint64_t)k.cols, 128, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        *ts_flags |= SG_TS_CODES_R;
+    if (k.mask_row && aligned(k.mask_row, 16) && (k.cols / 8) % 16 == 0 &&
+        encode_2d(&m->mask_r, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.mask_row, (uint64_t)k.cols / 8, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 8, SG_COLS / 8, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+        *ts_flags |= SG_TS_MASK_R;
+    if (k.mask_col && aligned(k.mask_col, 16) && (k.cols / 8) % 16 == 0 &&
+        encode_2d(&m->mask, CU_TENSOR_MAP_DATA_TYPE_UINT8, k.mask_col, (uint64_t)k.cols / 8, (uint64_t)k.rows,
+                  (uint64_t)k.cols / 8, SG_COLS / 8, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+        *ts_flags |= SG_TS_MASK;
+    return true;
+}
+
+template <bool ROW, bool GROUPS>
+static StagedFn pick_staged8(bool smma)
+{
+    return smma ? qdq_staged8_kernel<ROW, GROUPS, true> : qdq_staged8_kernel<ROW, GROUPS, false>;
+}
+
+// MXFP8 staged kernel (both directions or column-wise alone).
+static mxfp4_status launch_staged8(bool row, bool groups, const StagedMaps& maps, const KArgs& k, int64_t tiles,
+                                   size_t plan_smem, cudaStream_t s)
+{
+    const bool sm = k.srow_mma && k.scales_row;
+    StagedFn fn = row ? (groups ? pick_staged8<true, true>(sm) : pick_staged8<true, false>(sm))
+                      : (groups ? pick_staged8<false, true>(sm) : pick_staged8<false, false>(sm));
+    const size_t smem = sizeof(Staged8Smem) + 1024 + plan_smem;
+    if (cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MXFP4_ECUDA;
+    const int sms = device_sms();
+    const int occ = occupancy((const void*)fn, smem, S8_THREADS);
+    if (sms <= 0 || occ <= 0)
+        return MXFP4_ECUDA;
+    int64_t grid = (int64_t)sms * occ;
+    if (tiles < grid)
+        grid = tiles < 1 ? 1 : tiles;
+    fn<<<(unsigned)grid, S8_THREADS, smem, s>>>(maps, k);
+    return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
+}
+
 template <bool SMMA, bool VALS>
 static const void* pick_row_stream(int mode)
 {
@@ -1806,6 +1868,23 @@ static mxfp4_status run_qdq(const mxfp4_qdq_args* A, const void* g_out, void* g_
     const size_t plan_smem = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
     const int64_t s_bound = groups ? A->rows / bs + A->num_groups : (A->rows + bs - 1) / bs;
 
+    if (k.fmt == MXFP4_ELEM_E4M3 && esz == 2 && !grad && col && A->cols % 32 == 0 && A->ld % 8 == 0 &&
+        aligned(A->x, 16) && (!(k.y_row || k.y_col) || A->ld_y % 8 == 0) && (!k.y_row || aligned(k.y_row, 16)) &&
+        (!k.y_col || aligned(k.y_col, 16)) && (!k.codes_row || aligned(k.codes_row, 16)) &&
+        (!k.codes_col || aligned(k.codes_col, 2)) && (!k.scales_col || aligned(k.scales_col, 2)) &&
+        (!k.mask_row || aligned(k.mask_row, 4)) && (!k.mask_col || aligned(k.mask_col, 4)) &&
+        A->rows <= INT32_MAX - 2 * SG_ROWS && A->cols <= INT32_MAX - 2 * SG_COLS) {
+        // MXFP8 column-wise (and row-wise), bf16: the staged kernel, one read
+        // of each tile for both directions
+        StagedMaps maps;
+        if (make_staged8_maps(&maps, k, &k.ts_flags)) {
+            const int64_t n_ct = (A->cols + SG_COLS - 1) / SG_COLS;
+            if (s_bound * n_ct >= (int64_t)INT32_MAX)
+                return MXFP4_EUNSUPPORTED;
+            k.n_ct = (uint32_t)n_ct;
+            return launch_staged8(row, groups, maps, k, s_bound * n_ct, plan_smem, s);
+        }
+    }
     if (k.fmt == MXFP4_ELEM_E4M3 && esz == 2 && !grad) {
         // MXFP8, bf16: the row-wise part on the streaming kernel, the
         // column-wise part on the column-pair kernel, where their layout

@@ -2,8 +2,8 @@
 // column-wise or both directions (included by mxfp4.cu; shares its helpers).
 //
 // A tile is one column-wise block of 32 rows (shorter at a group tail) by 256
-// columns. Each CTA walks a contiguous range of tiles (row block major, so
-// consecutive tiles are neighbours along the row). TMA (cp.async.bulk.tensor,
+// columns. CTA b takes every G-th tile from tile b in row-block-major order
+// (TileWalk), so the grid sweeps the tensor a run of whole rows at a time. TMA (cp.async.bulk.tensor,
 // 2-D, no multicast) brings each tile into shared memory as four 64-column
 // slabs with the 128-byte swizzle, SG_STAGES tiles ahead of the computation.
 // Thread 0 also writes the tile's coordinates next to the stage, so the other
@@ -353,17 +353,24 @@ __device__ __forceinline__ uint32_t qword4_cvt(const uint32_t* w, float invn, fl
     return nibs;
 }
 
-// Tile sequence of one CTA: row block rb and column tile ct, advanced in
-// order; g tracks the group that holds rb (largest g with s_bpre[g] <= rb,
-// which skips empty groups). Tiles are TR rows (one column-wise block) by TC
-// columns.
+// Tile sequence of one CTA. Tiles are TR rows (one column-wise block) by TC
+// columns, numbered row block major (tile t is column tile t mod n_ct of row
+// block t / n_ct). CTA b takes tiles b, b + G, b + 2G, ... (G CTAs), so the
+// tiles in flight at any moment are a contiguous run of the numbering: whole
+// rows of the tensor are read and written at about the same time, and the
+// rows a group-tail tile reads past its group's end (the next row block's)
+// are read again by another CTA while they are still in L2. g tracks the
+// group that holds rb (largest g with s_bpre[g] <= rb, which skips empty
+// groups).
 template <bool GROUPS, int TR = SG_ROWS, int TC = SG_COLS>
 struct TileWalk {
-    uint32_t rb, ct;
+    uint32_t t, stride, rb, ct;
     int g;
 
-    __device__ void start(const KArgs& a, const int32_t* s_bpre, uint32_t t)
+    __device__ void start(const KArgs& a, const int32_t* s_bpre, uint32_t t0, uint32_t step)
     {
+        t = t0;
+        stride = step;
         rb = t / a.n_ct;
         ct = t - rb * a.n_ct;
         g = 0;
@@ -382,13 +389,12 @@ struct TileWalk {
 
     __device__ void next(const KArgs& a, const int32_t* s_bpre)
     {
-        if (++ct == a.n_ct) {
-            ct = 0;
-            ++rb;
-            if constexpr (GROUPS) {
-                while (g + 1 < a.num_groups && (uint32_t)s_bpre[g + 1] <= rb)
-                    ++g;
-            }
+        t += stride;
+        rb = t / a.n_ct;
+        ct = t - rb * a.n_ct;
+        if constexpr (GROUPS) {
+            while (g + 1 < a.num_groups && (uint32_t)s_bpre[g + 1] <= rb)
+                ++g;
         }
     }
 
@@ -530,8 +536,9 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         S = (uint32_t)((a.rows + SG_ROWS - 1) / SG_ROWS);
     }
     const uint32_t ntiles = S * a.n_ct;
-    const uint32_t t_begin = (uint32_t)(((uint64_t)blockIdx.x * ntiles) / gridDim.x);
-    const uint32_t t_end = (uint32_t)(((uint64_t)(blockIdx.x + 1) * ntiles) / gridDim.x);
+    // this CTA's tiles in sequence order 0..t_end-1 (TileWalk maps them)
+    const uint32_t t_begin = 0;
+    const uint32_t t_end = blockIdx.x < ntiles ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0u;
     const uint32_t lutb = smem_addr(sm.lut) - 0x2C000000u;
     const uint32_t lutb16 = lutb + 0x04000000u;
     // outputs present, as SG_TS_* bits; those TMA cannot address are copied
@@ -556,7 +563,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         pw.next(a, s_bpre);
     };
     if (async_thread && t_begin < t_end) {
-        pw.start(a, s_bpre, t_begin);
+        pw.start(a, s_bpre, blockIdx.x, gridDim.x);
         for (int s = 0; s < SG_STAGES && t_issue < t_end; ++s)
             issue(s);
     }
@@ -981,8 +988,9 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
         S = (uint32_t)((a.rows + SB_ROWS - 1) / SB_ROWS);
     }
     const uint32_t ntiles = S * a.n_ct;
-    const uint32_t t_begin = (uint32_t)(((uint64_t)blockIdx.x * ntiles) / gridDim.x);
-    const uint32_t t_end = (uint32_t)(((uint64_t)(blockIdx.x + 1) * ntiles) / gridDim.x);
+    // this CTA's tiles in sequence order 0..t_end-1 (TileWalk maps them)
+    const uint32_t t_begin = 0;
+    const uint32_t t_end = blockIdx.x < ntiles ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0u;
     const uint32_t lutb = smem_addr(sm.lut) - 0x2C000000u;
     const uint32_t col_out = COL ? (a.y_col ? SG_TS_Y : 0u) | (a.codes_col ? SG_TS_CODES : 0u) |
                                        (a.mask_col ? SG_TS_MASK : 0u)
@@ -1004,7 +1012,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
         pw.next(a, s_bpre);
     };
     if (tid == 0 && t_begin < t_end) {
-        pw.start(a, s_bpre, t_begin);
+        pw.start(a, s_bpre, blockIdx.x, gridDim.x);
         for (int s = 0; s < SB_STAGES && t_issue < t_end; ++s)
             issue(s);
     }

@@ -127,6 +127,52 @@ def test_mxfp8_every_bf16_value(cols):
     check(res, ora["row"], "row", f"sweep {cols}")
 
 
+# bf16 inputs with cols % 32 == 0 run the staged kernel in the column-wise
+# and dual calls: partial column tiles (warps past the last column), ragged
+# and group-tail row blocks, many tiles per CTA (the stage ring wraps)
+@pytest.mark.parametrize("shape,counts", [((96, 288), None), ((1000, 800), None), ((33, 32), None),
+                                          ((700, 1312), [0, 45, 320, 0, 1, 300, 34]),
+                                          ((16384, 2048), "moe")])
+def test_mxfp8_staged_shapes(shape, counts):
+    rows, cols = shape
+    if counts == "moe":
+        counts = W.moe_group_counts(rows, groups=64, seed=8).tolist()
+    x = W.mixed(rows, cols, seed=500 + cols)
+    res, ora = run(x, rowwise=True, colwise=True, counts=counts)
+    check(res, ora["row"], "row", f"dual {shape}")
+    check(res, ora["col"], "col", f"dual {shape}")
+    res, ora = run(x, rowwise=False, colwise=True, counts=counts)
+    check(res, ora["col"], "col", f"col {shape}")
+
+
+@pytest.mark.parametrize("counts", [None, [17, 47]])
+def test_mxfp8_every_bf16_value_along_columns(counts):
+    """The sweep of test_mxfp8_every_bf16_value laid along columns (each
+    32-element block is one column of 32 rows), through the staged kernel's
+    column pass, in both directions; with groups the blocks are cut at 17
+    rows."""
+    allv = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    blocks = []
+    for shift in (0, 2):
+        blk = np.zeros((65536, 32), np.uint16)
+        blk[:, 0] = allv
+        blk[:, 1] = np.where((allv & 0x7F80) >= (shift << 7), allv - (shift << 7), allv)
+        blk[:, 2] = allv ^ 0x8000
+        blocks.append(blk)
+    for mx in (0x43E0, 0x4380, 0x3F80, 0x0010, 0x7F7F, 0x0C00):
+        blk = np.zeros((65536, 32), np.uint16)
+        blk[:, 0] = mx
+        blk[:, 7] = allv
+        blocks.append(blk)
+    xb = np.concatenate(blocks)  # (524288, 32): one block per row
+    half = xb.shape[0] // 2
+    xb = np.concatenate([xb[:half].T, xb[half:].T])  # (64, 262144): one block per column
+    x = torch.from_numpy(np.ascontiguousarray(xb).view(np.int16)).view(torch.bfloat16)
+    res, ora = run(x, rowwise=True, colwise=True, counts=counts)
+    check(res, ora["col"], "col", "column sweep")
+    check(res, ora["row"], "row", "column sweep")
+
+
 @pytest.mark.parametrize("direction", ["rowwise", "colwise"])
 def test_mxfp8_ste(direction):
     x = W.mixed(96, 512, seed=17)
