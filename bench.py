@@ -59,6 +59,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-modes", action="store_true",
                    help="skip the extra single-GPU timings of the row-wise and training-step modes")
+    p.add_argument("--only-mode", default=None,
+                   help="time only this one of the extra modes (its name in the JSON line's modes)")
     return p.parse_args()
 
 
@@ -442,7 +444,7 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
     def mxfp8_dual():
         call(_abi.mxfp4_qdq_fwd(dual8, sp), "mxfp4_qdq_fwd")
 
-    peak, _ = measured_peaks()
+    peak, peak_kind = measured_peaks()
     out = {}
     for name, fn, bpe in (("rowwise_fwd_all_outputs_ste_mask", row_step, 4 + 0.5 + 1 / 32 + 0.125 + 4.125),
                           ("training_step_rowwise_fwd_ste_recompute", train_step, 4 + 6),
@@ -452,6 +454,8 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
                           ("mxfp8_rowwise_all_outputs", mxfp8_row, 2 + 2 + 1 + 1 / 32 + 0.125),
                           ("mxfp8_dual_grouped_all_outputs", mxfp8_dual, 2 + 4 + 2 + 2 / 32 + 0.25),
                           (f"bench_step_{other}_scale", step_other_mode, step_bytes(a.rows, a.cols, s_col)["step"] / n)):
+        if a.only_mode and name != a.only_mode:
+            continue
         for _ in range(3):
             fn()
         torch.cuda.synchronize()
@@ -464,10 +468,11 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
         ms = e0.elapsed_time(e1) / steps
         gbs = n * bpe / (ms / 1e3) / 1e9
         out[name] = {"ms_per_step": round(ms, 4), "bytes_per_element": round(bpe, 4), "GB/s": round(gbs, 1),
-                     "frac_of_measured_peak": round(gbs / peak, 4)}
+                     "frac_of_peak": round(gbs / peak, 4), "peak_kind": peak_kind}
     del opr, r8, r128, mma_scales
     torch.cuda.empty_cache()
-    out.update(time_gemm(a, xd, res, gl, stream, steps))
+    if not a.only_mode or a.only_mode.startswith("grouped_gemm"):
+        out.update(time_gemm(a, xd, res, gl, stream, steps))
     return out
 
 
@@ -679,7 +684,7 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded N(0,1) bf16, multinomial groups)",
                 "config": workload_desc(a, r["s_col"]),
-                "pct_of_peak": {"measured_copy_6458": round(100 * value / world / peak, 1),
+                "pct_of_peak": {f"{peak_kind}_copy_{int(peak)}": round(100 * value / world / peak, 1),
                                 "spec_8000": round(100 * value / world / SPEC_PEAK_GBS, 1)},
                 "elements_per_s": round(a.rows * a.cols * world * a.steps / (r["ms"] / 1e3), 1),
                 "parts_ms": {"qdq_fwd_dual": round(r["fwd_ms"], 4),

@@ -876,9 +876,10 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
 }
 
 // ---------------------------------------------------------------------------
-// Block 128 (bf16): the same staged scheme on tiles of 128 rows (one
-// column-wise block) by 128 columns (one row-wise block), 512 threads, one CTA
-// per SM. Per tile every thread owns 32 elements of each pass:
+// Block 128 (bf16): the staged scheme on tiles of 128 rows (one column-wise
+// block) by 128 columns (one row-wise block), 16 compute warps and one
+// producer warp, one CTA per SM. Per tile every compute thread owns 32
+// elements of each pass:
 //   * column pass: warp w owns tile columns 8w..8w+7; lane = column pair p
 //     (lane & 3) x row group g (lane >> 2) over rows 8i + g, i = 0..15, so
 //     the eight row groups of a 16-byte chunk hit eight different swizzle
@@ -886,10 +887,17 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
 //   * row pass: warp w owns tile rows 8w..8w+7; lanes 0-15 take the first
 //     half of each row's block (slab 0), lanes 16-31 the second (slab 1),
 //     32 elements per lane; the row amax takes two shuffles (xor 1, 16).
-// Inputs arrive as two 64 x 128 TMA boxes per tile (128-byte swizzle); all
-// outputs are staged and leave by TMA stores (codes with the 64-byte swizzle,
-// masks as 16-byte rows); row-wise scales (one byte per row) and group-tail
-// column-wise outputs are copied by the threads. Two CTA barriers per tile.
+// Inputs arrive as two 64 x 128 TMA boxes per tile (128-byte swizzle).
+// Row-wise y is written over the tile's own stage; the other outputs go to
+// one of two staging buffers (codes with the 64-byte swizzle, masks as
+// 16-byte rows) and leave by TMA stores, issued by the producer warp once the
+// compute warps have released the tile (one arrival each on its stage's
+// "empty" mbarrier); the producer warp also copies the row-wise scales and
+// the group-tail column-wise outputs, and once the stores of the tile before
+// have read their sources, releases that staging buffer ("sfree") and
+// refills its stage. One barrier among the compute warps per tile (named
+// barrier 1): every column pass has read its words from the stage (which
+// the row pass then overwrites with y) and published its column limits.
 // ---------------------------------------------------------------------------
 
 constexpr int SB_ROWS = 128, SB_COLS = 128;
@@ -898,40 +906,45 @@ constexpr int SB_TILE_BYTES = 2 * SB_SLAB_BYTES;           // 32768
 constexpr int SB_CODE_BYTES = SB_ROWS * SB_COLS / 2;       // 8192: 64-byte rows
 constexpr int SB_MASK_WORDS = SB_ROWS * SB_COLS / 32;      // 512: 16-byte rows
 constexpr int SB_STAGES = 3;
-constexpr int SB_THREADS = 512;
+constexpr int SB_COMPUTE_WARPS = 16;
+constexpr int SB_COMPUTE = 32 * SB_COMPUTE_WARPS;      // 512
+constexpr int SB_THREADS = SB_COMPUTE + 32;           // + the producer warp
+constexpr int SB_PRODUCER = SB_COMPUTE_WARPS;
 
 struct __align__(1024) StagedOut128 {
     uint8_t ycol[SB_TILE_BYTES];
-    uint8_t yrow[SB_TILE_BYTES];
     uint8_t ccol[SB_CODE_BYTES];
     uint8_t crow[SB_CODE_BYTES];
     uint32_t mcol[SB_MASK_WORDS];
     uint32_t mrow[SB_MASK_WORDS];
+    uint8_t srow[SB_ROWS];  // row-wise scale byte of each tile row
 };
 
 struct __align__(1024) Staged128Smem {
-    uint8_t tiles[SB_STAGES][SB_TILE_BYTES];
-    StagedOut128 out;
-    uint32_t limw[SB_COLS / 2];  // per column pair: 0x8000 + limit bits of each column (0xFFFF: never)
-    uint8_t srow[SB_ROWS];       // row-wise scale byte of each tile row
-    uint32_t gm[SB_MASK_WORDS];  // column-wise saturation bits of general-path column pairs (kept zero otherwise)
+    uint8_t tiles[SB_STAGES][SB_TILE_BYTES];  // input stages; row-wise y in place
+    StagedOut128 out[2];
+    uint32_t limw[2][SB_COLS / 2];  // per tile parity and column pair: 0x8000 + limit bits of each column (0xFFFF: never)
+    uint32_t gm[2][SB_MASK_WORDS];  // per tile parity: column-wise saturation bits of general-path column pairs
     int4 info[SB_STAGES];
     uint32_t lut[64];
     unsigned long long full[SB_STAGES];
+    unsigned long long empty[SB_STAGES];
+    unsigned long long sfree[2];
     int err;
 };
 
-// Thread copies of a block-128 tile's outputs (group tails, layouts TMA
-// cannot address): rows at or past nrows and columns at or past cols skipped.
-__device__ __forceinline__ void copy_outputs128(const KArgs& a, const StagedOut128& o, int row0, int nrows, int col0,
-                                                uint32_t which)
+// Copies of a block-128 tile's staged outputs by the producer warp (group
+// tails, layouts TMA cannot address): rows at or past nrows and columns at
+// or past cols skipped. yrow: the tile's stage (row-wise y).
+__device__ __forceinline__ void copy_outputs128(const KArgs& a, const StagedOut128& o, const uint8_t* yrow, int row0,
+                                                int nrows, int col0, uint32_t which, int lane)
 {
     const int64_t cstride = a.cols / 2, mstride = (a.cols + 7) / 8;
 #pragma unroll 1
-    for (int q = threadIdx.x; q < SB_ROWS * 16; q += SB_THREADS) {
+    for (int q = lane; q < SB_ROWS * 16; q += 32) {
         const int r = q >> 4, u = q & 15;  // row r, 8-column unit u
         if (r >= nrows)
-            continue;
+            break;
         const int col = col0 + 8 * u;
         if (col >= a.cols)
             continue;
@@ -941,7 +954,7 @@ __device__ __forceinline__ void copy_outputs128(const KArgs& a, const StagedOut1
         if (which & SG_TS_Y)
             st_stream(static_cast<char*>(a.y_col) + (row * a.ld_y + col) * 2, sm_ld128(o.ycol, yoff));
         if (which & SG_TS_YR)
-            st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * 2, sm_ld128(o.yrow, yoff));
+            st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * 2, sm_ld128(yrow, yoff));
         if (which & SG_TS_CODES)
             *reinterpret_cast<uint32_t*>(a.codes_col + row * cstride + col / 2) = sm_ld32(o.ccol, coff);
         if (which & SG_TS_CODES_R)
@@ -953,6 +966,22 @@ __device__ __forceinline__ void copy_outputs128(const KArgs& a, const StagedOut1
     }
 }
 
+// Barrier 1 among the compute warps; returns whether any of their threads
+// passed true (the same answer in every thread, so they leave together).
+__device__ __forceinline__ bool compute_bar_any(bool p)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, 1, %2, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)p), "n"(SB_COMPUTE)
+        : "memory");
+    return r != 0;
+}
+
 template <bool ROW, bool COL, bool GROUPS, int MODE>
 __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __grid_constant__ StagedMaps maps,
                                                                        const KArgs a)
@@ -960,19 +989,24 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
     extern __shared__ __align__(1024) uint8_t s_dyn[];
     uint8_t* s_base = s_dyn + ((1024u - (smem_addr(s_dyn) & 1023u)) & 1023u);
     Staged128Smem& sm = *reinterpret_cast<Staged128Smem*>(s_base);
-    StagedOut128& out = sm.out;
     int32_t* s_plan = reinterpret_cast<int32_t*>(s_base + sizeof(Staged128Smem));
     int32_t* s_bpre = s_plan;
     int32_t* s_rst = s_plan + (GROUPS ? a.num_groups + 1 : 0);
+    volatile int* err = &sm.err;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid < 64)
         sm.lut[tid] = lut_entry(tid);
-    sm.gm[tid] = 0u;  // SB_THREADS == SB_MASK_WORDS
+    for (int i = tid; i < 2 * SB_MASK_WORDS; i += SB_THREADS)
+        (&sm.gm[0][0])[i] = 0u;
     if (tid == 0) {
         sm.err = 0;
-        for (int s = 0; s < SB_STAGES; ++s)
+        for (int s = 0; s < SB_STAGES; ++s) {
             mbar_init(smem_addr(&sm.full[s]), 1);
+            mbar_init(smem_addr(&sm.empty[s]), SB_COMPUTE_WARPS);
+        }
+        mbar_init(smem_addr(&sm.sfree[0]), 1);
+        mbar_init(smem_addr(&sm.sfree[1]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     uint32_t S;
@@ -988,273 +1022,309 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
         S = (uint32_t)((a.rows + SB_ROWS - 1) / SB_ROWS);
     }
     const uint32_t ntiles = S * a.n_ct;
-    // this CTA's tiles in sequence order 0..t_end-1 (TileWalk maps them)
-    const uint32_t t_begin = 0;
-    const uint32_t t_end = blockIdx.x < ntiles ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0u;
-    const uint32_t lutb = smem_addr(sm.lut) - 0x2C000000u;
+    // this CTA's tiles: blockIdx.x, + gridDim.x, ... (TileWalk)
+    const uint32_t n = blockIdx.x < ntiles ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0u;
     const uint32_t col_out = COL ? (a.y_col ? SG_TS_Y : 0u) | (a.codes_col ? SG_TS_CODES : 0u) |
                                        (a.mask_col ? SG_TS_MASK : 0u)
                                  : 0u;
     const uint32_t row_out = (ROW && a.y_row ? SG_TS_YR : 0u) | (ROW && a.codes_row ? SG_TS_CODES_R : 0u) |
                              (ROW && a.mask_row ? SG_TS_MASK_R : 0u);
+    uint32_t issued = 0;  // producer lane 0: tiles whose load was issued
 
-    TileWalk<GROUPS, SB_ROWS, SB_COLS> pw;
-    uint32_t t_issue = t_begin;
-    auto issue = [&](int s) {
-        const int4 inf = pw.info(a, s_bpre, s_rst);
-        sm.info[s] = inf;
-        const uint32_t bar = smem_addr(&sm.full[s]);
-        mbar_expect_tx(bar, SB_TILE_BYTES);
+    if (warp == SB_PRODUCER) {
+        TileWalk<GROUPS, SB_ROWS, SB_COLS> pw;
+        auto load = [&](uint32_t j) {  // lane 0: tile j (in order) into stage j mod SB_STAGES
+            const int s = (int)(j % SB_STAGES);
+            const int4 inf = pw.info(a, s_bpre, s_rst);
+            sm.info[s] = inf;
+            const uint32_t bar = smem_addr(&sm.full[s]);
+            mbar_expect_tx(bar, SB_TILE_BYTES);
 #pragma unroll
-        for (int sl = 0; sl < 2; ++sl)
-            tma_load_slab(smem_addr(sm.tiles[s] + sl * SB_SLAB_BYTES), &maps.x, inf.z + sl * SG_SLAB_COLS, inf.x, bar);
-        ++t_issue;
-        pw.next(a, s_bpre);
-    };
-    if (tid == 0 && t_begin < t_end) {
-        pw.start(a, s_bpre, blockIdx.x, gridDim.x);
-        for (int s = 0; s < SB_STAGES && t_issue < t_end; ++s)
-            issue(s);
-    }
-
-    // column pass: warp w -> tile columns 8w..8w+7 (slab w/8, chunk w%8);
-    // lane -> pair p, row group g (rows 8i + g)
-    const int p = lane & 3, g = lane >> 2;
-    const int cpair = 8 * warp + 2 * p;
-    const uint32_t yo = (uint32_t)(warp >> 3) * SB_SLAB_BYTES + g * 128 + ((uint32_t)((warp & 7) ^ g) << 4) + 4 * p;
-    const uint32_t co = g * 64 + ((((uint32_t)warp >> 2) ^ (uint32_t)((g >> 1) & 3)) << 4) + ((4 * warp + p) & 15);
-    // row pass: warp w -> tile rows 8w..8w+7; lanes 0-15 the block's first
-    // 64 columns (q = lane & 1 picks 32 of them), lanes 16-31 the last 64
-    const int hq = lane >> 4, q = 2 * hq + (lane & 1);
-    const int rr = 8 * warp + ((lane & 15) >> 1);
-    uint32_t ro[4];
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj)
-        ro[jj] = (uint32_t)hq * SB_SLAB_BYTES + rr * 128 + ((uint32_t)((4 * (q & 1) + jj) ^ (rr & 7)) << 4);
-    const uint32_t rco = rr * 64 + (((uint32_t)q ^ (uint32_t)((rr >> 1) & 3)) << 4);
-    const int rw = rr * 4 + q;  // mask word of (row rr, columns 32q..32q+31)
-
-    int s = 0;
-    uint32_t phase = 0;
-    for (uint32_t t = t_begin; t < t_end; ++t) {
-        int row0 = 0, nrows = 0, col0 = 0;
-        const bool ok = __all_sync(FULL, mbar_wait(smem_addr(&sm.full[s]), phase));
-        const uint8_t* tile = sm.tiles[s];
-        uint32_t cw[16];
-        int k_lo = 0, k_hi = 0;
-        uint32_t A_lo = 0, A_hi = 0;
-        bool fast = true;
-        if (!ok) {
-            sm.err = 1;
-        } else {
+            for (int sl = 0; sl < 2; ++sl)
+                tma_load_slab(smem_addr(sm.tiles[s] + sl * SB_SLAB_BYTES), &maps.x, inf.z + sl * SG_SLAB_COLS, inf.x,
+                              bar);
+            ++issued;
+            pw.next(a, s_bpre);
+        };
+        if (lane == 0 && n > 0) {
+            pw.start(a, s_bpre, blockIdx.x, gridDim.x);
+            for (uint32_t j = 0; j < n && j < (uint32_t)SB_STAGES; ++j)
+                load(j);
+        }
+        for (uint32_t j = 0; j < n; ++j) {
+            const int s = (int)(j % SB_STAGES);
+            const bool ok = __all_sync(FULL, mbar_wait(smem_addr(&sm.empty[s]), (j / SB_STAGES) & 1u));
+            if (!ok || *err) {
+                if (lane == 0)
+                    *err = 1;
+                break;
+            }
             const int4 inf = sm.info[s];
-            row0 = inf.x;
-            nrows = inf.y;
-            col0 = inf.z;
-            const uint32_t rb = (uint32_t)inf.w;
-            if constexpr (COL) {
+            const int row0 = inf.x, nrows = inf.y, col0 = inf.z;
+            const StagedOut128& o = sm.out[j & 1];
+            // column-wise outputs of a group tail are copied; row-wise ones
+            // leave by TMA, the rows past a group tail included (they equal
+            // what the tile owning those rows writes)
+            const uint32_t st = ((nrows == SB_ROWS ? col_out : 0u) | row_out) & a.ts_flags;
+            if (lane == 0) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    cw[i] = sm_ld32(tile, yo + i * 1024);
-                if (nrows < SB_ROWS) {
+                for (int sl = 0; sl < 2; ++sl) {
+                    if ((st & SG_TS_Y) && col0 + sl * SG_SLAB_COLS < a.cols)
+                        tma_store_box(&maps.y, smem_addr(o.ycol) + sl * SB_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
+                    if ((st & SG_TS_YR) && col0 + sl * SG_SLAB_COLS < a.cols)
+                        tma_store_box(&maps.yr, smem_addr(sm.tiles[s]) + sl * SB_SLAB_BYTES, col0 + sl * SG_SLAB_COLS,
+                                      row0);
+                }
+                if (st & SG_TS_CODES)
+                    tma_store_box(&maps.codes, smem_addr(o.ccol), col0 / 2, row0);
+                if (st & SG_TS_CODES_R)
+                    tma_store_box(&maps.codes_r, smem_addr(o.crow), col0 / 2, row0);
+                if (st & SG_TS_MASK)
+                    tma_store_box(&maps.mask, smem_addr(o.mcol), col0 / 8, row0);
+                if (st & SG_TS_MASK_R)
+                    tma_store_box(&maps.mask_r, smem_addr(o.mrow), col0 / 8, row0);
+                bulk_commit();  // this tile's group
+            }
+            const uint32_t copy = (col_out | row_out) & ~st;
+            if (copy)
+                copy_outputs128(a, o, sm.tiles[s], row0, nrows, col0, copy, lane);
+            if (ROW && a.scales_row) {
+                const int64_t nblk = (a.cols + 127) / 128;
+                for (int r = lane; r < nrows; r += 32)
+                    a.scales_row[srow_off(a, (int64_t)row0 + r, col0 / 128, nblk)] = o.srow[r];
+            }
+            __syncwarp();
+            if (lane == 0 && j > 0) {
+                // tile j - 1's stores have read its staging buffer and its
+                // stage: release the buffer to tile j + 1 and refill the stage
+                bulk_wait_read_but1();
+                mbar_arrive(smem_addr(&sm.sfree[(j - 1) & 1]));
+                if (j - 1 + SB_STAGES < n)
+                    load(j - 1 + SB_STAGES);
+            }
+            __syncwarp();
+        }
+    } else {
+        const uint32_t lutb = smem_addr(sm.lut) - 0x2C000000u;
+        // column pass: warp w -> tile columns 8w..8w+7 (slab w/8, chunk w%8);
+        // lane -> pair p, row group g (rows 8i + g)
+        const int p = lane & 3, g = lane >> 2;
+        const int cpair = 8 * warp + 2 * p;
+        const uint32_t yo = (uint32_t)(warp >> 3) * SB_SLAB_BYTES + g * 128 + ((uint32_t)((warp & 7) ^ g) << 4) + 4 * p;
+        const uint32_t co =
+            g * 64 + ((((uint32_t)warp >> 2) ^ (uint32_t)((g >> 1) & 3)) << 4) + ((4 * warp + p) & 15);
+        // row pass: warp w -> tile rows 8w..8w+7; lanes 0-15 the block's first
+        // 64 columns (q = lane & 1 picks 32 of them), lanes 16-31 the last 64
+        const int hq = lane >> 4, q = 2 * hq + (lane & 1);
+        const int rr = 8 * warp + ((lane & 15) >> 1);
+        uint32_t ro[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+            ro[jj] = (uint32_t)hq * SB_SLAB_BYTES + rr * 128 + ((uint32_t)((4 * (q & 1) + jj) ^ (rr & 7)) << 4);
+        const uint32_t rco = rr * 64 + (((uint32_t)q ^ (uint32_t)((rr >> 1) & 3)) << 4);
+        const int rw = rr * 4 + q;  // mask word of (row rr, columns 32q..32q+31)
+
+        for (uint32_t j = 0; j < n; ++j) {
+            const int s = (int)(j % SB_STAGES);
+            const int par = (int)(j & 1);
+            int row0 = 0, nrows = 0, col0 = 0;
+            uint32_t rb = 0;
+            uint8_t* tile = sm.tiles[s];
+            StagedOut128& out = sm.out[par];
+            uint32_t* limw = sm.limw[par];
+            uint32_t* gm = sm.gm[par];
+            uint32_t cw[16];
+            int k_lo = 0, k_hi = 0;
+            uint32_t A_lo = 0, A_hi = 0;
+            bool fast = true;
+            // waits never break out before the barrier below: a warp that
+            // gives up records the error, and all compute warps leave together
+            bool ok = __all_sync(FULL, mbar_wait(smem_addr(&sm.full[s]), (j / SB_STAGES) & 1u));
+            if (ok) {
+                const int4 inf = sm.info[s];
+                row0 = inf.x;
+                nrows = inf.y;
+                col0 = inf.z;
+                rb = (uint32_t)inf.w;
+                if constexpr (COL) {
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        if (8 * i + g >= nrows)
-                            cw[i] = 0u;
-                }
-                uint32_t m2 = 0;
+                        cw[i] = sm_ld32(tile, yo + i * 1024);
+                    if (nrows < SB_ROWS) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    m2 = vmax2(m2, cw[i] & 0x7FFF7FFFu);
-                m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 4));
-                m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 8));
-                m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 16));
-                A_lo = m2 << 16;
-                A_hi = m2 & 0xFFFF0000u;
-                k_lo = block_kt<MODE>(A_lo, a.thr);
-                k_hi = block_kt<MODE>(A_hi, a.thr);
-                fast = k_fast_bf(k_lo) && k_fast_bf(k_hi);
-                if (!fast && a.mask_col) {
-                    // general-path column pair (rare): its exact saturation bits go to
-                    // gm before the barrier; the row pass ORs them into its words.
-                    // Word i of lane (p, g) is row 8i + g, columns 8w + 2p, +1.
-                    const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
+                        for (int i = 0; i < 16; ++i)
+                            if (8 * i + g >= nrows)
+                                cw[i] = 0u;
+                    }
+                    uint32_t m2 = 0;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        m2 = vmax2(m2, cw[i] & 0x7FFF7FFFu);
+                    m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 4));
+                    m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 8));
+                    m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 16));
+                    A_lo = m2 << 16;
+                    A_hi = m2 & 0xFFFF0000u;
+                    k_lo = block_kt<MODE>(A_lo, a.thr);
+                    k_hi = block_kt<MODE>(A_hi, a.thr);
+                    fast = k_fast_bf(k_lo) && k_fast_bf(k_hi);
+                    if (!fast && a.mask_col) {
+                        // general-path column pair (rare): its exact saturation
+                        // bits go to gm before the barrier; the row pass ORs
+                        // them into its words. Word i of lane (p, g) is row
+                        // 8i + g, columns 8w + 2p, +1.
+                        const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
 #pragma unroll 1
-                    for (int i0 = 0; i0 < 16; i0 += 4) {
-                        const ChunkOut gch = general_chunk<8, true>(
-                            make_uint4(cw[i0], cw[i0 + 1], cw[i0 + 2], cw[i0 + 3]), Ac, a.mode, a.thr, lutb);
-                        for (int u = 0; u < 4; ++u) {
-                            const uint32_t two = (gch.sats >> (2 * u)) & 3u;
-                            if (two)
-                                atomicOr(&sm.gm[(8 * (i0 + u) + g) * 4 + (warp >> 2)], two << ((8 * warp + 2 * p) & 31));
+                        for (int i0 = 0; i0 < 16; i0 += 4) {
+                            const ChunkOut gch = general_chunk<8, true>(
+                                make_uint4(cw[i0], cw[i0 + 1], cw[i0 + 2], cw[i0 + 3]), Ac, a.mode, a.thr, lutb);
+                            for (int u = 0; u < 4; ++u) {
+                                const uint32_t two = (gch.sats >> (2 * u)) & 3u;
+                                if (two)
+                                    atomicOr(&gm[(8 * (i0 + u) + g) * 4 + (warp >> 2)],
+                                             two << ((8 * warp + 2 * p) & 31));
+                            }
+                        }
+                    }
+                    if (g == 0) {
+                        limw[4 * warp + p] =
+                            fast ? (0x8000u + lim16_of_k(k_lo)) | ((0x8000u + lim16_of_k(k_hi)) << 16) : 0xFFFFFFFFu;
+                        if (a.scales_col && col0 + cpair < a.cols) {
+                            const uint32_t e8p = fast ? (uint32_t)(k_lo + 127) | ((uint32_t)(k_hi + 127) << 8)
+                                                      : e8_of(A_lo, k_lo) | (e8_of(A_hi, k_hi) << 8);
+                            *reinterpret_cast<uint16_t*>(a.scales_col + (int64_t)rb * a.cols + col0 + cpair) =
+                                (uint16_t)e8p;
                         }
                     }
                 }
-                if (g == 0) {
-                    sm.limw[4 * warp + p] =
-                        fast ? (0x8000u + lim16_of_k(k_lo)) | ((0x8000u + lim16_of_k(k_hi)) << 16) : 0xFFFFFFFFu;
-                    if (a.scales_col && col0 + cpair < a.cols) {
-                        const uint32_t e8p = fast ? (uint32_t)(k_lo + 127) | ((uint32_t)(k_hi + 127) << 8)
-                                                  : e8_of(A_lo, k_lo) | (e8_of(A_hi, k_hi) << 8);
-                        *reinterpret_cast<uint16_t*>(a.scales_col + (int64_t)rb * a.cols + col0 + cpair) =
-                            (uint16_t)e8p;
-                    }
-                }
+                // staging buffer par was last filled by tile j - 2, whose
+                // stores the producer saw read at tile j - 1
+                ok = __all_sync(FULL, j < 2 || mbar_wait(smem_addr(&sm.sfree[par]), ((j >> 1) + 1) & 1u));
             }
-        }
-        if (tid == 0)
-            bulk_wait_read_all();  // the previous tile's stores have read the staging buffers
-        __syncthreads();           // staging free; limw complete; errors visible
-        if (sm.err)
-            break;
+            if (!ok && lane == 0)
+                *err = 1;
+            // column words read, limits published, staging free (or an error)
+            if (compute_bar_any(!ok))
+                break;
 
-        if constexpr (COL) {
-            auto col_fast = [&]() {
-                const float invn_lo = inv_nudged(k_lo), invn_hi = inv_nudged(k_hi);
-                const float sc_lo = pow2f_k(k_lo), sc_hi = pow2f_k(k_hi);
+            if constexpr (COL) {
+                auto col_fast = [&]() {
+                    const float invn_lo = inv_nudged(k_lo), invn_hi = inv_nudged(k_hi);
+                    const float sc_lo = pow2f_k(k_lo), sc_hi = pow2f_k(k_hi);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    uint32_t byte;
-                    *reinterpret_cast<uint32_t*>(out.ycol + yo + i * 1024) =
-                        qword_cvt(cw[i], invn_lo, invn_hi, sc_lo, sc_hi, byte);
-                    out.ccol[co + i * 512] = (uint8_t)byte;
-                }
-            };
-            if (__all_sync(FULL, fast)) {
-                col_fast();
-            } else if (fast) {
-                col_fast();
-            } else {
-                const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
-#pragma unroll
-                for (int i0 = 0; i0 < 16; i0 += 4) {
-                    const uint4 dv = make_uint4(cw[i0], cw[i0 + 1], cw[i0 + 2], cw[i0 + 3]);
-                    const ChunkOut gch = general_chunk<8, true>(dv, Ac, a.mode, a.thr, lutb);
-                    const uint32_t ov[4] = {gch.packed.x, gch.packed.y, gch.packed.z, gch.packed.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        *reinterpret_cast<uint32_t*>(out.ycol + yo + (i0 + u) * 1024) = ov[u];
-                        out.ccol[co + (i0 + u) * 512] = (uint8_t)(gch.nibs >> (8 * u));
-                    }
-                }
-            }
-        }
-
-        // ---- row pass: the lane's 32 elements of row rr's block (q-th
-        // quarter), the block amax over its four lanes
-        {
-            uint32_t rw16[16];
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const uint4 c = sm_ld128(tile, ro[jj]);
-                rw16[4 * jj + 0] = c.x;
-                rw16[4 * jj + 1] = c.y;
-                rw16[4 * jj + 2] = c.z;
-                rw16[4 * jj + 3] = c.w;
-            }
-            if (COL && a.mask_col) {
-                uint32_t cm = 0;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint4 L = *reinterpret_cast<const uint4*>(&sm.limw[16 * q + 4 * jj]);
-                    const uint32_t lx[4] = {L.x, L.y, L.z, L.w};
-                    const uint32_t a4w[4] = {rw16[4 * jj] & 0x7FFF7FFFu, rw16[4 * jj + 1] & 0x7FFF7FFFu,
-                                             rw16[4 * jj + 2] & 0x7FFF7FFFu, rw16[4 * jj + 3] & 0x7FFF7FFFu};
-                    cm |= sat8(a4w, lx) << (8 * jj);
-                }
-                out.mcol[rw] = cm | sm.gm[rw];
-                sm.gm[rw] = 0u;  // this thread alone reads the word: clear it for the next tile
-            }
-            if constexpr (ROW) {
-                uint32_t m2 = 0;
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    m2 = vmax2(m2, rw16[i] & 0x7FFF7FFFu);
-                m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 1));
-                m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 16));
-                const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
-                const uint32_t A = am << 16;
-                const int k = block_kt<MODE>(A, a.thr);
-                const bool rfast = k_fast_bf(k);
-                uint32_t nib[4], sats = 0;
-                auto row_fast = [&]() {
-                    const float invn = inv_nudged(k), sc = pow2f_k(k);
-                    const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
-                    const uint32_t limx[4] = {lx, lx, lx, lx};
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        uint32_t o[4];
-                        nib[jj] = qword4_cvt(rw16 + 4 * jj, invn, sc, o);
-                        *reinterpret_cast<uint4*>(out.yrow + ro[jj]) = make_uint4(o[0], o[1], o[2], o[3]);
-                        const uint32_t a4w[4] = {rw16[4 * jj] & 0x7FFF7FFFu, rw16[4 * jj + 1] & 0x7FFF7FFFu,
-                                                 rw16[4 * jj + 2] & 0x7FFF7FFFu, rw16[4 * jj + 3] & 0x7FFF7FFFu};
-                        sats |= sat8(a4w, limx) << (8 * jj);
+                    for (int i = 0; i < 16; ++i) {
+                        uint32_t byte;
+                        *reinterpret_cast<uint32_t*>(out.ycol + yo + i * 1024) =
+                            qword_cvt(cw[i], invn_lo, invn_hi, sc_lo, sc_hi, byte);
+                        out.ccol[co + i * 512] = (uint8_t)byte;
                     }
                 };
-                if (__all_sync(FULL, rfast)) {
-                    row_fast();
-                } else if (rfast) {
-                    row_fast();
+                if (__all_sync(FULL, fast)) {
+                    col_fast();
+                } else if (fast) {
+                    col_fast();
                 } else {
+                    const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const uint4 dv = make_uint4(rw16[4 * jj], rw16[4 * jj + 1], rw16[4 * jj + 2], rw16[4 * jj + 3]);
-                        const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
-                        *reinterpret_cast<uint4*>(out.yrow + ro[jj]) = gch.packed;
-                        nib[jj] = gch.nibs;
-                        sats |= gch.sats << (8 * jj);
+                    for (int i0 = 0; i0 < 16; i0 += 4) {
+                        const uint4 dv = make_uint4(cw[i0], cw[i0 + 1], cw[i0 + 2], cw[i0 + 3]);
+                        const ChunkOut gch = general_chunk<8, true>(dv, Ac, a.mode, a.thr, lutb);
+                        const uint32_t ov[4] = {gch.packed.x, gch.packed.y, gch.packed.z, gch.packed.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            *reinterpret_cast<uint32_t*>(out.ycol + yo + (i0 + u) * 1024) = ov[u];
+                            out.ccol[co + (i0 + u) * 512] = (uint8_t)(gch.nibs >> (8 * u));
+                        }
                     }
                 }
-                *reinterpret_cast<uint4*>(out.crow + rco) = make_uint4(nib[0], nib[1], nib[2], nib[3]);
-                out.mrow[rw] = sats;
-                if (q == 0)
-                    sm.srow[rr] = (uint8_t)(rfast ? (uint32_t)(k + 127) : e8_of(A, k));
             }
-        }
-        fence_async_smem();
-        __syncthreads();  // stage s consumed; staged outputs complete
 
-        const uint32_t tma = (nrows == SB_ROWS ? col_out : 0u) | row_out;
-        const uint32_t copy = (col_out | row_out) & ~(tma & a.ts_flags);
-        if (tid == 0) {
-            const uint32_t st = tma & a.ts_flags;
+            // ---- row pass: the lane's 32 elements of row rr's block (q-th
+            // quarter), the block amax over its four lanes; y over the stage
+            {
+                uint32_t rw16[16];
 #pragma unroll
-            for (int sl = 0; sl < 2; ++sl) {
-                if ((st & SG_TS_Y) && col0 + sl * SG_SLAB_COLS < a.cols)
-                    tma_store_box(&maps.y, smem_addr(out.ycol) + sl * SB_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
-                if ((st & SG_TS_YR) && col0 + sl * SG_SLAB_COLS < a.cols)
-                    tma_store_box(&maps.yr, smem_addr(out.yrow) + sl * SB_SLAB_BYTES, col0 + sl * SG_SLAB_COLS, row0);
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint4 c = sm_ld128(tile, ro[jj]);
+                    rw16[4 * jj + 0] = c.x;
+                    rw16[4 * jj + 1] = c.y;
+                    rw16[4 * jj + 2] = c.z;
+                    rw16[4 * jj + 3] = c.w;
+                }
+                if (COL && a.mask_col) {
+                    uint32_t cm = 0;
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const uint4 L = *reinterpret_cast<const uint4*>(&limw[16 * q + 4 * jj]);
+                        const uint32_t lx[4] = {L.x, L.y, L.z, L.w};
+                        const uint32_t a4w[4] = {rw16[4 * jj] & 0x7FFF7FFFu, rw16[4 * jj + 1] & 0x7FFF7FFFu,
+                                                 rw16[4 * jj + 2] & 0x7FFF7FFFu, rw16[4 * jj + 3] & 0x7FFF7FFFu};
+                        cm |= sat8(a4w, lx) << (8 * jj);
+                    }
+                    out.mcol[rw] = cm | gm[rw];
+                    gm[rw] = 0u;  // this thread alone reads the word: clear it for tile j + 2
+                }
+                if constexpr (ROW) {
+                    uint32_t m2 = 0;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        m2 = vmax2(m2, rw16[i] & 0x7FFF7FFFu);
+                    m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 1));
+                    m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 16));
+                    const uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
+                    const uint32_t A = am << 16;
+                    const int k = block_kt<MODE>(A, a.thr);
+                    const bool rfast = k_fast_bf(k);
+                    uint32_t nib[4], sats = 0;
+                    auto row_fast = [&]() {
+                        const float invn = inv_nudged(k), sc = pow2f_k(k);
+                        const uint32_t lx = (0x8000u + lim16_of_k(k)) * 0x10001u;
+                        const uint32_t limx[4] = {lx, lx, lx, lx};
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            uint32_t o[4];
+                            nib[jj] = qword4_cvt(rw16 + 4 * jj, invn, sc, o);
+                            *reinterpret_cast<uint4*>(tile + ro[jj]) = make_uint4(o[0], o[1], o[2], o[3]);
+                            const uint32_t a4w[4] = {rw16[4 * jj] & 0x7FFF7FFFu, rw16[4 * jj + 1] & 0x7FFF7FFFu,
+                                                     rw16[4 * jj + 2] & 0x7FFF7FFFu, rw16[4 * jj + 3] & 0x7FFF7FFFu};
+                            sats |= sat8(a4w, limx) << (8 * jj);
+                        }
+                    };
+                    if (__all_sync(FULL, rfast)) {
+                        row_fast();
+                    } else if (rfast) {
+                        row_fast();
+                    } else {
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const uint4 dv =
+                                make_uint4(rw16[4 * jj], rw16[4 * jj + 1], rw16[4 * jj + 2], rw16[4 * jj + 3]);
+                            const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
+                            *reinterpret_cast<uint4*>(tile + ro[jj]) = gch.packed;
+                            nib[jj] = gch.nibs;
+                            sats |= gch.sats << (8 * jj);
+                        }
+                    }
+                    *reinterpret_cast<uint4*>(out.crow + rco) = make_uint4(nib[0], nib[1], nib[2], nib[3]);
+                    out.mrow[rw] = sats;
+                    if (q == 0)
+                        out.srow[rr] = (uint8_t)(rfast ? (uint32_t)(k + 127) : e8_of(A, k));
+                }
             }
-            if (st & SG_TS_CODES)
-                tma_store_box(&maps.codes, smem_addr(out.ccol), col0 / 2, row0);
-            if (st & SG_TS_CODES_R)
-                tma_store_box(&maps.codes_r, smem_addr(out.crow), col0 / 2, row0);
-            if (st & SG_TS_MASK)
-                tma_store_box(&maps.mask, smem_addr(out.mcol), col0 / 8, row0);
-            if (st & SG_TS_MASK_R)
-                tma_store_box(&maps.mask_r, smem_addr(out.mrow), col0 / 8, row0);
-            bulk_commit();
-            if (t_issue < t_end)
-                issue(s);
-        }
-        if (copy)
-            copy_outputs128(a, out, row0, nrows, col0, copy);
-        if (ROW && a.scales_row && tid < SB_ROWS && tid < nrows) {
-            const int64_t nblk = (a.cols + 127) / 128;
-            a.scales_row[srow_off(a, (int64_t)row0 + tid, col0 / 128, nblk)] = sm.srow[tid];
-        }
-        if (++s == SB_STAGES) {
-            s = 0;
-            phase ^= 1u;
+            fence_async_smem();  // staged outputs and the stage's y -> visible to the TMA stores
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&sm.empty[s]));  // this warp is done with tile j
         }
     }
 
-    if (tid == 0) {
-        if (sm.err) {
+    __syncthreads();
+    if (warp == SB_PRODUCER && lane == 0) {
+        if (*err) {
             if (a.status)
                 *a.status = MXFP4_ECUDA;
-            for (int st = 0; st < SB_STAGES; ++st)
-                (void)mbar_wait(smem_addr(&sm.full[st]), phase ^ (st < s ? 1u : 0u));
+            for (uint32_t i = issued > (uint32_t)SB_STAGES ? issued - SB_STAGES : 0u; i < issued; ++i)
+                (void)mbar_wait(smem_addr(&sm.full[i % SB_STAGES]), (i / SB_STAGES) & 1u);
         }
         bulk_wait_all();
     }

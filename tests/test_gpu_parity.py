@@ -372,6 +372,20 @@ def test_rowwise_codes_without_values(mode, layout, shape):
     assert np.array_equal(np_bits(res.scales_row).reshape(exp_s.shape), exp_s), "scales"
 
 
+@pytest.mark.parametrize("grouped", [False, True])
+def test_block128_many_tiles_per_cta(grouped):
+    """Blocks of 128 in both directions on 9000 x 2048 (ragged last row block)
+    and with 64 multinomial groups: every CTA of the persistent grid takes
+    several tiles in turn, so the stage ring, both staging buffers and the
+    per-parity column limits wrap many times."""
+    rows, cols = 9000, 2048
+    counts = W.moe_group_counts(rows, groups=64, seed=12).tolist() if grouped else None
+    x = W.mixed(rows, cols, seed=77)
+    res, ora = run_both(x, block=128, mode="page", rowwise=True, colwise=True, counts=counts)
+    check_dir(res, ora["row"], "row", cols, label="b128 many tiles")
+    check_dir(res, ora["col"], "col", cols, label="b128 many tiles")
+
+
 @pytest.mark.parametrize("mode", ["page", "floor"])
 def test_every_bf16_value_block128_both_directions(mode):
     """Every finite bf16 value, in the low and the high half of a 32-bit word
