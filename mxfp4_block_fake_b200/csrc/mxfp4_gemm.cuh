@@ -24,7 +24,10 @@
 //   warp 0: producer. Lane 0 loads the A and B tiles of one K stage (128 K
 //     elements) with TMA into swizzled shared memory; the warp gathers the
 //     128 rows' scale bytes of A and of B for the stage into one 512-byte
-//     atom each (A's rows of a group need not start on a multiple of 128).
+//     atom each (A's rows of a group need not start on a multiple of 128)
+//     with asynchronous 4-byte copies (cp.async, zero-filled past the last
+//     row), whose completion each lane signals on the stage's barrier, so
+//     the producer never waits for them.
 //   warp 1: allocates the tensor memory; lane 0 copies a stage's scale atoms
 //     into tensor memory (tcgen05.cp 32x128b.warpx4) and issues the block-
 //     scaled MMAs (tcgen05.mma kind::mxf4 K = 64, or kind::mxf8f6f4 K = 32),
@@ -242,7 +245,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
     if (tid == 0) {
         sm.err = 0;
         for (int s = 0; s < S; ++s) {
-            mbar_init(smem_addr(&sm.full[s]), 1);
+            mbar_init(smem_addr(&sm.full[s]), 1 + 32);  // the TMA transaction + each producer lane's copies
             mbar_init(smem_addr(&sm.empty[s]), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -288,30 +291,41 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
             const GmTile tl = gm_tile(a, s_tpre, s_rst, t, n_nt, n_mt);
             const int64_t brow0 = GROUP_K ? tl.n0 : (int64_t)tl.g * a.n + tl.n0;
             const uint8_t* sfb = a.sfb + (GROUP_K ? 0 : (int64_t)tl.g * a.sfb_group_bytes);
+            // this lane's rows r = lane + 32q of the tile: the address of
+            // their four scale bytes in atom column 0 (MMA layout), or a
+            // zero-filled copy past the last row
+            const uint8_t* pa[4];
+            const uint8_t* pb[4];
+            uint32_t na = 0, nb = 0;  // bit q: row of A / B inside the matrix
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = lane + 32 * q;
+                const int64_t ra = tl.a_row0 + r, rb = tl.n0 + r;
+                pa[q] = a.sfa + (ra < a.a_rows ? srow_off_mma(ra, 0, kblocks) : 0);
+                pb[q] = sfb + (rb < a.n ? srow_off_mma(rb, 0, kblocks) : 0);
+                na |= (ra < a.a_rows ? 1u : 0u) << q;
+                nb |= (rb < a.n ? 1u : 0u) << q;
+            }
             for (int ks = 0; ks < tl.nk; ++ks) {
                 if (!__all_sync(FULL, mbar_wait(smem_addr(&sm.empty[s]), ph ^ 1u))) {
                     sm.err = 1;
                     break;
                 }
                 const int64_t kel = tl.k0 + (int64_t)ks * GM_BK;  // first K element of the stage
-                const int64_t j = kel / 128;                        // atom column of the stage
-                // scale atoms: tile row r's four bytes at 16 (r % 32) + 4 (r / 32)
+                const int64_t jo = (kel / 128) * 512;               // atom column of the stage, in bytes
+                // tile row r's four bytes at 16 (r % 32) + 4 (r / 32) of the stage's atom
+                const uint32_t da = smem_addr(sm.sfa[s]) + 16 * lane, db = smem_addr(sm.sfb[s]) + 16 * lane;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int r = lane + 32 * q;
-                    const int64_t ra = tl.a_row0 + r;
-                    uint32_t va = 0x7F7F7F7Fu;  // rows past A: codes 0 (TMA fill), scale 2^0
-                    if (ra < a.a_rows)
-                        va = *reinterpret_cast<const uint32_t*>(a.sfa + srow_off_mma(ra, 4 * j, kblocks));
-                    const int64_t rb = tl.n0 + r;
-                    uint32_t vb = 0x7F7F7F7Fu;
-                    if (rb < a.n)
-                        vb = *reinterpret_cast<const uint32_t*>(sfb + srow_off_mma(rb, 4 * j, kblocks));
-                    *reinterpret_cast<uint32_t*>(sm.sfa[s] + 16 * (r & 31) + 4 * (r >> 5)) = va;
-                    *reinterpret_cast<uint32_t*>(sm.sfb[s] + 16 * (r & 31) + 4 * (r >> 5)) = vb;
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(da + 4 * q),
+                                 "l"(pa[q] + ((na >> q) & 1u ? jo : 0)), "r"((na >> q) & 1u ? 4u : 0u)
+                                 : "memory");
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(db + 4 * q),
+                                 "l"(pb[q] + ((nb >> q) & 1u ? jo : 0)), "r"((nb >> q) & 1u ? 4u : 0u)
+                                 : "memory");
                 }
-                fence_async_smem();
-                __syncwarp();
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(&sm.full[s]))
+                             : "memory");
                 if (lane == 0) {
                     const uint32_t bar = smem_addr(&sm.full[s]);
                     mbar_expect_tx(bar, 2 * TB);
@@ -353,6 +367,9 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
                         break;
                     }
                     gm_fence_after();
+                    // the scale atoms were written by the producer's copies
+                    // (generic proxy); tcgen05.cp reads them in the async proxy
+                    fence_async_smem();
                     const uint32_t sf_col = tmem + GM_SF_COL0 + 8u * (uint32_t)s;
                     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sf_col),
                                  "l"(gm_sf_desc(smem_addr(sm.sfa[s])))
