@@ -2019,7 +2019,7 @@ static mxfp4_status run_gmm(const mxfp4_gmm_args* A, cudaStream_t s)
         return MXFP4_EINVAL;
     if (A->d_dtype != MXFP4_F32 && A->d_dtype != MXFP4_BF16)
         return MXFP4_EINVAL;
-    if (A->m < 0 || A->n < 0 || A->k < 0 || A->k % GM_BK != 0)
+    if (A->m < 0 || A->n < 0 || A->k < 0 || A->k % GM_KU != 0)
         return MXFP4_EINVAL;
     if (A->m > INT32_MAX || A->n > INT32_MAX || A->k > INT32_MAX)
         return MXFP4_EUNSUPPORTED;
@@ -2046,8 +2046,8 @@ static mxfp4_status run_gmm(const mxfp4_gmm_args* A, cudaStream_t s)
         (A->ldd * esz) % 16 != 0)
         return MXFP4_EINVAL;
     const bool e2 = A->elem_format == MXFP4_ELEM_E2M1;
-    const int row_bytes = e2 ? GmFmt<MXFP4_ELEM_E2M1>::ROW_BYTES : GmFmt<MXFP4_ELEM_E4M3>::ROW_BYTES;
-    const CUtensorMapSwizzle sw = e2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    const int row_bytes = GM_ROW_BYTES;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
     GmMaps maps;
     memset(&maps, 0, sizeof(maps));
     const int64_t b_rows = gk ? A->n : A->n * A->num_groups;

@@ -21,16 +21,18 @@
 //     writes D_g [M][N] (D + g * M * ldd); an empty group writes zeros.
 //
 // Design (one CTA per SM, persistent over output tiles of 128 x 128):
-//   warp 0: producer. Lane 0 loads the A and B tiles of one K stage (128 K
-//     elements) with TMA into swizzled shared memory; the warp gathers the
-//     128 rows' scale bytes of A and of B for the stage into one 512-byte
-//     atom each (A's rows of a group need not start on a multiple of 128)
+//   warp 0: producer. Lane 0 loads the A and B tiles of one K stage (128-byte
+//     rows: 256 E2M1 or 128 E4M3 K elements) with TMA into shared memory
+//     with the 128-byte swizzle; the warp gathers the 128 rows' scale bytes
+//     of A and of B for the stage into 512-byte atoms (one per 128 K; A's
+//     rows of a group need not start on a multiple of 128)
 //     with asynchronous 4-byte copies (cp.async, zero-filled past the last
 //     row), whose completion each lane signals on the stage's barrier, so
 //     the producer never waits for them.
 //   warp 1: allocates the tensor memory; lane 0 copies a stage's scale atoms
 //     into tensor memory (tcgen05.cp 32x128b.warpx4) and issues the block-
-//     scaled MMAs (tcgen05.mma kind::mxf4 K = 64, or kind::mxf8f6f4 K = 32),
+//     scaled MMAs (tcgen05.mma kind::mxf4 K = 64, or kind::mxf8f6f4 K = 32;
+//     a group's K range that ends halfway through a stage takes half of them),
 //     releasing the stage with tcgen05.commit; two accumulators of 128 fp32
 //     columns alternate between tiles.
 //   warps 2-5: epilogue. Each warp reads its 32 lanes (rows) of the
@@ -43,7 +45,8 @@
 
 namespace mxfp4 {
 
-constexpr int GM_BM = 128, GM_BN = 128, GM_BK = 128;  // tile rows, tile columns, K elements per stage
+constexpr int GM_BM = 128, GM_BN = 128;  // tile rows, tile columns
+constexpr int GM_KU = 128;               // K elements per scale atom column (4 blocks of 32): the unit of K ranges
 constexpr int GM_THREADS = 256;  // 8 warps: producer, MMA, 4 epilogue, 2 that only build the group plan
 constexpr uint32_t GM_TMEM_COLS = 512;  // 2 accumulators x 128 + scale atoms of every stage
 constexpr uint32_t GM_SF_COL0 = 256;    // first tensor-memory column of the scale atoms
@@ -52,30 +55,29 @@ template <int FMT>
 struct GmFmt;
 template <>
 struct GmFmt<MXFP4_ELEM_E2M1> {
-    static constexpr int ROW_BYTES = 64;   // 128 codes per row per stage
-    static constexpr int STAGES = 8;
-    static constexpr int MMAS = 2;         // kind::mxf4, K = 64 (32 bytes) per MMA
-    static constexpr uint64_t LAYOUT = 4;  // 64-byte swizzle
-    static constexpr uint32_t SBO = 512;   // 8 rows x 64 bytes
+    static constexpr int BK = 256;         // K elements per stage (128-byte rows)
+    static constexpr int STAGES = 6;
+    static constexpr int MMA_K = 64;       // kind::mxf4: K = 64 (32 bytes) per MMA
     static constexpr uint32_t AB_FMT = 1;  // E2M1 in the kind::mxf4 encoding
 };
 template <>
 struct GmFmt<MXFP4_ELEM_E4M3> {
-    static constexpr int ROW_BYTES = 128;  // 128 codes per row per stage
+    static constexpr int BK = 128;
     static constexpr int STAGES = 5;
-    static constexpr int MMAS = 4;         // kind::mxf8f6f4, K = 32 (32 bytes) per MMA
-    static constexpr uint64_t LAYOUT = 2;  // 128-byte swizzle
-    static constexpr uint32_t SBO = 1024;  // 8 rows x 128 bytes
+    static constexpr int MMA_K = 32;       // kind::mxf8f6f4: K = 32 (32 bytes) per MMA
     static constexpr uint32_t AB_FMT = 0;  // E4M3
 };
+constexpr int GM_ROW_BYTES = 128;       // bytes of a tile row per stage, both formats
+constexpr uint64_t GM_LAYOUT = 2;       // 128-byte swizzle (smem descriptor layout type)
+constexpr uint32_t GM_SBO = 1024;       // 8 rows x 128 bytes
 
 template <int FMT>
 struct __align__(1024) GmSmem {
-    static constexpr int S = GmFmt<FMT>::STAGES, TB = GM_BM * GmFmt<FMT>::ROW_BYTES;
-    uint8_t a[S][TB];      // swizzled A tiles (1024-aligned)
-    uint8_t b[S][TB];      // swizzled B tiles
-    uint8_t sfa[S][512];   // A's scale atom of each stage
-    uint8_t sfb[S][512];   // B's scale atom of each stage
+    static constexpr int S = GmFmt<FMT>::STAGES, TB = GM_BM * GM_ROW_BYTES, ATOMS = GmFmt<FMT>::BK / GM_KU;
+    uint8_t a[S][TB];             // swizzled A tiles (1024-aligned)
+    uint8_t b[S][TB];             // swizzled B tiles
+    uint8_t sfa[S][512 * ATOMS];  // A's scale atoms of each stage
+    uint8_t sfb[S][512 * ATOMS];  // B's scale atoms of each stage
     unsigned long long full[S], empty[S], acc_full[2], acc_empty[2], done;
     uint32_t tmem_base;
     int err;
@@ -171,8 +173,8 @@ __device__ __forceinline__ void gm_ld32(uint32_t taddr, uint32_t (&v)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// 2-D TMA load of a byte tile (box of ROW_BYTES x 128 rows) with the
-// operand map's swizzle; the inner coordinate is a multiple of 64 bytes.
+// 2-D TMA load of a byte tile (box of 128 bytes x 128 rows, 128-byte
+// swizzle); the inner coordinate is a multiple of 64 bytes.
 __device__ __forceinline__ void gm_tma_load(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar)
 {
     asm volatile(
@@ -190,7 +192,7 @@ struct GmTile {
     int rows;         // valid rows (<= 128)
     int64_t n0;
     int64_t k0;       // first K element of the group's range
-    int nk;           // K stages
+    int ku;           // K units (GM_KU elements) of the range
 };
 
 // The plan (GROUP_M): s_tpre[g] = sum_{j<g} ceil(m_j / 128) row tiles,
@@ -208,8 +210,8 @@ __device__ __forceinline__ GmTile gm_tile(const GmArgs& a, const int32_t* s_tpre
         r.a_row0 = mi * GM_BM;
         r.d_row0 = mi * GM_BM;
         r.rows = (int)min((int64_t)GM_BM, a.a_rows - r.a_row0);
-        r.k0 = (int64_t)s_tpre[g] * GM_BK;
-        r.nk = s_tpre[g + 1] - s_tpre[g];
+        r.k0 = (int64_t)s_tpre[g] * GM_KU;
+        r.ku = s_tpre[g + 1] - s_tpre[g];
     } else {
         int lo = 0, hi = a.num_groups - 1;  // largest g with s_tpre[g] <= mt (skips empty groups)
         while (lo < hi) {
@@ -224,7 +226,7 @@ __device__ __forceinline__ GmTile gm_tile(const GmArgs& a, const int32_t* s_tpre
         r.d_row0 = r.a_row0;
         r.rows = (int)min((int64_t)GM_BM, (int64_t)s_rst[lo + 1] - r.a_row0);
         r.k0 = 0;
-        r.nk = (int)(a.k / GM_BK);
+        r.ku = (int)(a.k / GM_KU);
     }
     return r;
 }
@@ -234,7 +236,9 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
 {
     using F = GmFmt<FMT>;
     constexpr int S = F::STAGES;
-    constexpr uint32_t TB = GM_BM * F::ROW_BYTES;
+    constexpr int ATOMS = F::BK / GM_KU;               // scale atom columns per stage
+    constexpr int MMA_PER_UNIT = GM_KU / F::MMA_K;     // MMAs per K unit
+    constexpr uint32_t TB = GM_BM * GM_ROW_BYTES;
     extern __shared__ __align__(1024) uint8_t gm_dyn[];
     uint8_t* base = gm_dyn + ((1024u - (smem_addr(gm_dyn) & 1023u)) & 1023u);
     GmSmem<FMT>& sm = *reinterpret_cast<GmSmem<FMT>*>(base);
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
     gm_fence_after();
     const uint32_t tmem = sm.tmem_base;
     // GROUP_K: the groups' padded K slots must fit in k
-    const bool ok = units >= 0 && (!GROUP_K || units * GM_BK <= a.k);
+    const bool ok = units >= 0 && (!GROUP_K || units * GM_KU <= a.k);
     if (blockIdx.x == 0 && tid == 0 && a.status)
         *a.status = ok ? MXFP4_OK : MXFP4_EINVAL;
 
@@ -306,30 +310,38 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
                 na |= (ra < a.a_rows ? 1u : 0u) << q;
                 nb |= (rb < a.n ? 1u : 0u) << q;
             }
-            for (int ks = 0; ks < tl.nk; ++ks) {
+            const int nst = (tl.ku + ATOMS - 1) / ATOMS;  // stages of the tile
+            for (int ks = 0; ks < nst; ++ks) {
                 if (!__all_sync(FULL, mbar_wait(smem_addr(&sm.empty[s]), ph ^ 1u))) {
                     sm.err = 1;
                     break;
                 }
-                const int64_t kel = tl.k0 + (int64_t)ks * GM_BK;  // first K element of the stage
-                const int64_t jo = (kel / 128) * 512;               // atom column of the stage, in bytes
-                // tile row r's four bytes at 16 (r % 32) + 4 (r / 32) of the stage's atom
-                const uint32_t da = smem_addr(sm.sfa[s]) + 16 * lane, db = smem_addr(sm.sfb[s]) + 16 * lane;
+                const int64_t kel = tl.k0 + (int64_t)ks * F::BK;  // first K element of the stage
+                const int nu = min(ATOMS, tl.ku - ks * ATOMS);     // K units of the stage
+                // tile row r's four bytes at 16 (r % 32) + 4 (r / 32) of each of
+                // the stage's atoms (atom column kel / 128 + i, 512 bytes apart)
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(da + 4 * q),
-                                 "l"(pa[q] + ((na >> q) & 1u ? jo : 0)), "r"((na >> q) & 1u ? 4u : 0u)
-                                 : "memory");
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(db + 4 * q),
-                                 "l"(pb[q] + ((nb >> q) & 1u ? jo : 0)), "r"((nb >> q) & 1u ? 4u : 0u)
-                                 : "memory");
+                for (int i = 0; i < ATOMS; ++i) {
+                    const int64_t jo = (kel / GM_KU + i) * 512;
+                    const uint32_t da = smem_addr(sm.sfa[s]) + 512 * i + 16 * lane;
+                    const uint32_t db = smem_addr(sm.sfb[s]) + 512 * i + 16 * lane;
+                    const uint32_t ua = i < nu ? na : 0u, ub = i < nu ? nb : 0u;  // a unit past the range: zeros
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(da + 4 * q),
+                                     "l"(pa[q] + ((ua >> q) & 1u ? jo : 0)), "r"((ua >> q) & 1u ? 4u : 0u)
+                                     : "memory");
+                        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(db + 4 * q),
+                                     "l"(pb[q] + ((ub >> q) & 1u ? jo : 0)), "r"((ub >> q) & 1u ? 4u : 0u)
+                                     : "memory");
+                    }
                 }
                 asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(&sm.full[s]))
                              : "memory");
                 if (lane == 0) {
                     const uint32_t bar = smem_addr(&sm.full[s]);
                     mbar_expect_tx(bar, 2 * TB);
-                    const int kx = (int)(kel * F::ROW_BYTES / GM_BK);
+                    const int kx = (int)(kel * GM_ROW_BYTES / F::BK);
                     gm_tma_load(smem_addr(sm.a[s]), &maps.a, kx, (int)tl.a_row0, bar);
                     gm_tma_load(smem_addr(sm.b[s]), &maps.b, kx, (int)brow0, bar);
                 }
@@ -361,7 +373,8 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
                 }
                 gm_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * GM_BN);
-                for (int ks = 0; ks < tl.nk; ++ks) {
+                const int nst = (tl.ku + ATOMS - 1) / ATOMS;
+                for (int ks = 0; ks < nst; ++ks) {
                     if (!mbar_wait(smem_addr(&sm.full[s]), ph)) {
                         sm.err = 1;
                         break;
@@ -370,22 +383,27 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
                     // the scale atoms were written by the producer's copies
                     // (generic proxy); tcgen05.cp reads them in the async proxy
                     fence_async_smem();
-                    const uint32_t sf_col = tmem + GM_SF_COL0 + 8u * (uint32_t)s;
-                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sf_col),
-                                 "l"(gm_sf_desc(smem_addr(sm.sfa[s])))
-                                 : "memory");
-                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sf_col + 4u),
-                                 "l"(gm_sf_desc(smem_addr(sm.sfb[s])))
-                                 : "memory");
-                    const uint64_t ad = gm_smem_desc(smem_addr(sm.a[s]), F::LAYOUT, F::SBO);
-                    const uint64_t bd = gm_smem_desc(smem_addr(sm.b[s]), F::LAYOUT, F::SBO);
+                    const uint32_t sf_col = tmem + GM_SF_COL0 + (uint32_t)(8 * ATOMS * s);
 #pragma unroll
-                    for (int kk = 0; kk < F::MMAS; ++kk) {
-                        // 32 bytes of K per MMA: the start address moves by 2 units of 16 bytes;
-                        // kind::mxf4 uses scale bytes 2kk, 2kk+1, kind::mxf8f6f4 byte kk
-                        const uint32_t sf_id = FMT == MXFP4_ELEM_E2M1 ? 2u * kk : (uint32_t)kk;
-                        gm_mma<FMT>(d_tmem, ad + 2u * kk, bd + 2u * kk, gm_idesc(F::AB_FMT, sf_id), sf_col, sf_col + 4u,
-                                    (ks > 0 || kk > 0) ? 1u : 0u);
+                    for (int i = 0; i < ATOMS; ++i) {
+                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sf_col + 4u * i),
+                                     "l"(gm_sf_desc(smem_addr(sm.sfa[s]) + 512 * i))
+                                     : "memory");
+                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sf_col + 4u * (ATOMS + i)),
+                                     "l"(gm_sf_desc(smem_addr(sm.sfb[s]) + 512 * i))
+                                     : "memory");
+                    }
+                    const uint64_t ad = gm_smem_desc(smem_addr(sm.a[s]), GM_LAYOUT, GM_SBO);
+                    const uint64_t bd = gm_smem_desc(smem_addr(sm.b[s]), GM_LAYOUT, GM_SBO);
+                    const int nmma = min(ATOMS, tl.ku - ks * ATOMS) * MMA_PER_UNIT;
+                    for (int kk = 0; kk < nmma; ++kk) {
+                        // 32 bytes of K per MMA: the start address moves by 2 units of 16
+                        // bytes; its first scale block kk * MMA_K / 32 is byte (block % 4)
+                        // of atom (block / 4)
+                        const int blk = kk * (F::MMA_K / 32);
+                        const uint32_t ai = (uint32_t)(blk >> 2);
+                        gm_mma<FMT>(d_tmem, ad + 2u * kk, bd + 2u * kk, gm_idesc(F::AB_FMT, (uint32_t)(blk & 3)),
+                                    sf_col + 4u * ai, sf_col + 4u * (ATOMS + ai), (ks > 0 || kk > 0) ? 1u : 0u);
                     }
                     gm_commit(smem_addr(&sm.empty[s]));  // the stage is free once these MMAs have read it
                     if (++s == S) {
@@ -393,7 +411,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
                         ph ^= 1u;
                     }
                 }
-                gm_commit(smem_addr(&sm.acc_full[acc]));  // nk == 0: completes at once, D of the tile is zero
+                gm_commit(smem_addr(&sm.acc_full[acc]));  // ku == 0: completes at once, D of the tile is zero
                 if (++acc == 2) {
                     acc = 0;
                     aph ^= 1u;
@@ -418,7 +436,7 @@ __global__ void __launch_bounds__(GM_THREADS, 1) gmm_kernel(const __grid_constan
                 break;
             }
             gm_fence_after();
-            const bool zero = tl.nk == 0;
+            const bool zero = tl.ku == 0;
             const bool row_ok = r < tl.rows;
             const int64_t drow = (GROUP_K ? (int64_t)tl.g * a.a_rows : 0) + tl.d_row0 + r;
 #pragma unroll 1
