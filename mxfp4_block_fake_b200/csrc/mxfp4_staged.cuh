@@ -1,36 +1,39 @@
 // mxfp4_staged.cuh -- the shared-memory-staged forward for bf16, block 32,
-// column-wise or both directions (included by mxfp4.cu; shares its helpers).
+// column-wise or both directions (included by mxfp4.cu; shares its helpers),
+// and the other kernels of the bf16 fast paths.
 //
 // A tile is one column-wise block of 32 rows (shorter at a group tail) by 256
 // columns. CTA b takes every G-th tile from tile b in row-block-major order
-// (TileWalk), so the grid sweeps the tensor a run of whole rows at a time. TMA (cp.async.bulk.tensor,
-// 2-D, no multicast) brings each tile into shared memory as four 64-column
-// slabs with the 128-byte swizzle, SG_STAGES tiles ahead of the computation.
-// Thread 0 also writes the tile's coordinates next to the stage, so the other
-// threads never search the group plan.
+// (TileWalk), so the grid sweeps the tensor a run of whole rows at a time.
+// TMA (cp.async.bulk.tensor, 2-D, no multicast) brings each tile into shared
+// memory as four 64-column slabs with the 128-byte swizzle, SG_STAGES tiles
+// ahead of the computation. The thread that issues the loads also writes the
+// tile's coordinates next to the stage, so the other threads never search the
+// group plan.
 //
-// Per tile every one of the 256 threads owns
-//   * one row-wise block (32 elements of one row), stored straight to global
-//     memory with 32- and 16-byte stores; and
-//   * one column pair over 16 of the 32 rows of the column-wise pass: lanes
-//     l and l ^ 16 of a warp share the pair (rows with bit 2 clear / set), so
-//     the column amax takes one shuffle and each thread derives the two
-//     columns' parameters itself. Its column-wise outputs go to a staging
-//     tile in shared memory (same swizzled layout as the input), which TMA
-//     stores (cp.async.bulk.tensor ... bulk_group) write to global memory
-//     once the tile is complete. Group-tail and ragged tiles, and outputs
-//     whose layout TMA cannot address, are copied out by the threads instead.
-// Shared-memory accesses are conflict-free by construction: the two
-// half-warps of the column pass read and write rows whose swizzle phases
-// differ by 4, i.e. disjoint 64-byte halves of the bank space.
+// Per tile warp w owns tile columns 32w..32w+31 in both passes:
+//   * column pass: lanes l and l ^ 16 share one column pair over 16 rows each
+//     (rows with bit 2 clear / set), so the column amax takes one shuffle and
+//     each thread derives the two columns' parameters itself. Element core:
+//     the nudged hardware convert (qword_cvt). Its y and codes go to a
+//     staging tile in shared memory, which TMA stores write to global memory
+//     once the tile is complete;
+//   * row pass: one row-wise block per lane (32 elements of one row).
+//     Element core: the floor(4|y|) code table (qword). Its y is written over
+//     the tile's own input words; codes, masks and scales are staged.
+// The two cores load different pipes (the converter and the table's integer
+// work), which is why the passes use different ones. Group-tail and ragged
+// tiles, and outputs whose layout TMA cannot address, are copied out by the
+// threads instead. Shared-memory accesses of the passes are conflict-free by
+// construction: the two half-warps of the column pass read rows whose
+// swizzle phases differ by 4, i.e. disjoint 64-byte halves of the bank space.
 //
-// One CTA barrier per tile. Before it, thread 0 waits until the previous
-// tile's TMA stores have read their staging buffer (double-buffered), so the
-// next tile may write it; after it, thread 0 issues this tile's stores and
-// refills the freed input stage. Every wait on an mbarrier is bounded; on
-// expiry the CTA records MXFP4_ECUDA in the caller's status word (when
-// given), waits (bounded) for its own loads still in flight and for its
-// stores, and returns.
+// One CTA barrier per tile (tile done). Staging buffers alternate between
+// tiles; a buffer and the tile's stage are released once the tile's TMA
+// stores have read them (an mbarrier per buffer), and the freed stage is
+// refilled. Every wait on an mbarrier is bounded; on expiry the CTA records
+// MXFP4_ECUDA in the caller's status word (when given), waits (bounded) for
+// its own loads still in flight and for its stores, and returns.
 
 namespace mxfp4 {
 
@@ -243,34 +246,23 @@ __device__ __forceinline__ uint32_t clear_neg_zero(uint32_t w)
 // 2^k of each element's block; mul4, mul16: 4 and 65536 (KArgs).
 // t = 2^21 + |x| * 2^-k rounded down (fp32 spacing on [2^21, 2^22) is 1/4),
 // so t's bits are 0x4A000000 + floor(4|y|); lutb16 = table base - 0x28000000
-// folds that offset into the address shift-add. |x| is the fma's absolute-
-// value operand. The high element is indexed from the whole word: the low
-// element's magnitude lies below its last bf16 bit and cannot carry it across
-// a quarter of 2^k. Returns the dequantised packed bf16 pair; P receives the
-// signed codes.
+// folds that offset into the address multiply-add. Both halves take one
+// packed fma (fma.rm.f32x2) on (|low| as fp32, |word| as fp32): the high
+// element is indexed from the whole word, since the low element's magnitude
+// lies below its last bf16 bit and cannot carry it across a quarter of 2^k.
+// Returns the dequantised packed bf16 pair; P receives the signed codes.
 __device__ __forceinline__ uint32_t qword(uint32_t wc, float inv_lo, float inv_hi, uint32_t s2, uint32_t lutb16,
                                           uint32_t mul4, uint32_t mul16, uint32_t& P)
 {
-    const float tl = __fmaf_rd(fabsf(__uint_as_float(wc * mul16)), inv_lo, 0x1p21f);
-    const float th = __fmaf_rd(fabsf(__uint_as_float(wc)), inv_hi, 0x1p21f);
-    const uint32_t el = lut_load(__float_as_uint(tl) * mul4 + lutb16);
-    const uint32_t eh = lut_load(__float_as_uint(th) * mul4 + lutb16);
+    const uint32_t aw = wc & 0x7FFF7FFFu;
+    unsigned long long t;
+    const unsigned long long src = ((unsigned long long)aw << 32) | (unsigned long long)(aw * mul16);
+    const unsigned long long inv2 = ((unsigned long long)__float_as_uint(inv_hi) << 32) | __float_as_uint(inv_lo);
+    asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(t) : "l"(src), "l"(inv2), "l"(0x4A0000004A000000ull));
+    const uint32_t el = lut_load((uint32_t)t * mul4 + lutb16);
+    const uint32_t eh = lut_load((uint32_t)(t >> 32) * mul4 + lutb16);
     P = __byte_perm(el, eh, 0x7632) | (wc & 0x80008000u);
     return hmul2_bf16(P, s2);
-}
-
-// The E2M1 byte of one word of signed packed bf16 codes (low element in the
-// low nibble), stored at a shared-memory address. The high element is
-// converted from the whole word read as fp32: the low element's bits sit
-// below its last bf16 bit and cannot move it to another E2M1 value (a code of
-// zero gives a subnormal of the same sign).
-__device__ __forceinline__ void e2m1_byte_store(uint32_t saddr, uint32_t P)
-{
-    asm volatile("{\n\t.reg .b8 b;\n\t"
-                 "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
-                 "st.shared.b8 [%0], b;\n\t}" ::"r"(saddr),
-                 "f"(__uint_as_float(P)), "f"(__uint_as_float(P << 16))
-                 : "memory");
 }
 
 // ---- E2M1 rounding by the hardware convert ---------------------------------
@@ -604,7 +596,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         const bool ok = __all_sync(FULL, mbar_wait(smem_addr(&sm.full[s]), phase));
         uint8_t* tile = sm.tiles[s];
         StagedOut& out = sm.out[j & 1];
-        uint32_t cw[16];  // the column pass's words, -0 cleared
+        uint32_t cw[16];  // the column pass's words
         int k_lo = 0, k_hi = 0;
         uint32_t A_lo = 0, A_hi = 0;
         bool fast = true;
@@ -622,10 +614,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             if constexpr (COL) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const uint32_t off = yo[i & 3] + (i >> 2) * 1024;
-                cw[i] = clear_neg_zero(sm_ld32(tile, off));
-                // written back: this warp's row pass reads these words cleaned
-                *reinterpret_cast<uint32_t*>(tile + off) = cw[i];
+                cw[i] = sm_ld32(tile, yo[i & 3] + (i >> 2) * 1024);
             }
             if (!rows_full) {
                 // rows past a group tail belong to the next group: neither
@@ -667,12 +656,11 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         const bool go = ok && (j < 2 || __all_sync(FULL, mbar_wait(smem_addr(&sm.sfree[j & 1]), ((j >> 1) + 1) & 1u)));
         if (!go)
             sm.err = 1;
-        __syncwarp();  // limw and the cleaned words of this warp
+        __syncwarp();  // limw of this warp
 
         // ---- column pass, part 2: y and codes of the column pair
         uint32_t gsat = 0;  // saturation bits of a general-path column pair (bits 2i, 2i+1: word i)
         if (COL && go) {
-            const uint32_t cqs = smem_addr(out.ccol);
             uint32_t* yq[4];
             uint8_t* cq[4];
 #pragma unroll
@@ -681,14 +669,13 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                 cq[q] = out.ccol + co[q];
             }
             auto col_fast = [&]() {
-                const float inv_lo = __uint_as_float(0x3F800000u - ((uint32_t)k_lo << 23));
-                const float inv_hi = __uint_as_float(0x3F800000u - ((uint32_t)k_hi << 23));
-                const uint32_t s2 = bf16_pow2(k_lo) | (bf16_pow2(k_hi) << 16);
+                const float invn_lo = inv_nudged(k_lo), invn_hi = inv_nudged(k_hi);
+                const float sc_lo = pow2f_k(k_lo), sc_hi = pow2f_k(k_hi);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    uint32_t P;
-                    yq[i & 3][(i >> 2) * 256] = qword(cw[i], inv_lo, inv_hi, s2, lutb16, a.mul4, a.mul16, P);
-                    e2m1_byte_store(cqs + co[i & 3] + (i >> 2) * 1024, P);
+                    uint32_t byte;
+                    yq[i & 3][(i >> 2) * 256] = qword_cvt(cw[i], invn_lo, invn_hi, sc_lo, sc_hi, byte);
+                    cq[i & 3][(i >> 2) * 1024] = (uint8_t)byte;
                 }
             };
             if (__all_sync(FULL, fast)) {
@@ -720,7 +707,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
         // columns, is done), and the column-wise saturation word of the same
         // 32 elements
         if (go) {
-            uint32_t rw16[16];  // the lane's block, -0 cleared by the column pass
+            uint32_t rw16[16];  // the lane's block, -0 cleared
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 const uint4 c = sm_ld128(tile, ro[jj]);
@@ -729,11 +716,9 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
                 rw16[4 * jj + 2] = c.z;
                 rw16[4 * jj + 3] = c.w;
             }
-            if constexpr (!COL) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    rw16[i] = clear_neg_zero(rw16[i]);  // no column pass cleaned them
-            }
+            for (int i = 0; i < 16; ++i)
+                rw16[i] = clear_neg_zero(rw16[i]);
             if (COL && a.mask_col) {
                 // rows past a group tail are not copied out; their word is don't-care
                 uint32_t cm = 0;
