@@ -148,8 +148,8 @@ __global__ void __launch_bounds__(NTHREADS) col_operand_kernel(const KArgs a)
                 for (int m = 0; m < 4; ++m) {
                     uint4 vlo, vhi;
                     split_pair_rows(w + 8 * m, vlo, vhi);
-                    q[0][4 * b + m] = general_chunk<8, false>(vlo, &A[0], a.mode, a.thr, glutb).nibs;
-                    q[1][4 * b + m] = general_chunk<8, false>(vhi, &A[1], a.mode, a.thr, glutb).nibs;
+                    q[0][4 * b + m] = general_chunk_one(vlo, A[0], a.mode, a.thr, glutb).nibs;
+                    q[1][4 * b + m] = general_chunk_one(vhi, A[1], a.mode, a.thr, glutb).nibs;
                 }
             }
         }

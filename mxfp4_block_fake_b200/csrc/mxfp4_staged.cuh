@@ -345,6 +345,22 @@ __device__ __forceinline__ uint32_t qword4_cvt(const uint32_t* w, float invn, fl
     return nibs;
 }
 
+// The general element path with block amaxes passed by value: a column pair
+// (lo, hi alternating over the eight elements of a chunk) or one block. The
+// array general_chunk reads lives in these functions' frames, so a kernel
+// keeps nothing in local memory on its fast path.
+__device__ __noinline__ ChunkOut general_chunk_pair(uint4 dv, uint32_t A_lo, uint32_t A_hi, int mode, uint32_t thr,
+                                                    uint32_t lutb)
+{
+    const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
+    return general_chunk<8, true>(dv, Ac, mode, thr, lutb);
+}
+
+__device__ __noinline__ ChunkOut general_chunk_one(uint4 dv, uint32_t A, int mode, uint32_t thr, uint32_t lutb)
+{
+    return general_chunk<8, false>(dv, &A, mode, thr, lutb);
+}
+
 // Tile sequence of one CTA. Tiles are TR rows (one column-wise block) by TC
 // columns, numbered row block major (tile t is column tile t mod n_ct of row
 // block t / n_ct). CTA b takes tiles b, b + G, b + 2G, ... (G CTAs), so the
@@ -683,11 +699,10 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
             } else if (fast) {
                 col_fast();
             } else {
-                const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
 #pragma unroll
                 for (int i0 = 0; i0 < 16; i0 += 4) {
                     const uint4 dv = make_uint4(cw[i0], cw[i0 + 1], cw[i0 + 2], cw[i0 + 3]);
-                    const ChunkOut gch = general_chunk<8, true>(dv, Ac, a.mode, a.thr, lutb);
+                    const ChunkOut gch = general_chunk_pair(dv, A_lo, A_hi, a.mode, a.thr, lutb);
                     gsat |= (gch.sats & 0xFFu) << (2 * i0);
                     const uint32_t ov[4] = {gch.packed.x, gch.packed.y, gch.packed.z, gch.packed.w};
 #pragma unroll
@@ -770,7 +785,7 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const uint4 dv = make_uint4(rw16[4 * jj], rw16[4 * jj + 1], rw16[4 * jj + 2], rw16[4 * jj + 3]);
-                        const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
+                        const ChunkOut gch = general_chunk_one(dv, A, a.mode, a.thr, lutb);
                         *reinterpret_cast<uint4*>(tile + ro[jj]) = gch.packed;
                         nib[jj] = gch.nibs;
                         sats |= gch.sats << (8 * jj);
@@ -1158,11 +1173,10 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
                         // bits go to gm before the barrier; the row pass ORs
                         // them into its words. Word i of lane (p, g) is row
                         // 8i + g, columns 8w + 2p, +1.
-                        const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
-#pragma unroll 1
+#pragma unroll
                         for (int i0 = 0; i0 < 16; i0 += 4) {
-                            const ChunkOut gch = general_chunk<8, true>(
-                                make_uint4(cw[i0], cw[i0 + 1], cw[i0 + 2], cw[i0 + 3]), Ac, a.mode, a.thr, lutb);
+                            const ChunkOut gch = general_chunk_pair(
+                                make_uint4(cw[i0], cw[i0 + 1], cw[i0 + 2], cw[i0 + 3]), A_lo, A_hi, a.mode, a.thr, lutb);
                             for (int u = 0; u < 4; ++u) {
                                 const uint32_t two = (gch.sats >> (2 * u)) & 3u;
                                 if (two)
@@ -1209,11 +1223,10 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
                 } else if (fast) {
                     col_fast();
                 } else {
-                    const uint32_t Ac[8] = {A_lo, A_hi, A_lo, A_hi, A_lo, A_hi, A_lo, A_hi};
 #pragma unroll
                     for (int i0 = 0; i0 < 16; i0 += 4) {
                         const uint4 dv = make_uint4(cw[i0], cw[i0 + 1], cw[i0 + 2], cw[i0 + 3]);
-                        const ChunkOut gch = general_chunk<8, true>(dv, Ac, a.mode, a.thr, lutb);
+                        const ChunkOut gch = general_chunk_pair(dv, A_lo, A_hi, a.mode, a.thr, lutb);
                         const uint32_t ov[4] = {gch.packed.x, gch.packed.y, gch.packed.z, gch.packed.w};
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
@@ -1284,7 +1297,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
                         for (int jj = 0; jj < 4; ++jj) {
                             const uint4 dv =
                                 make_uint4(rw16[4 * jj], rw16[4 * jj + 1], rw16[4 * jj + 2], rw16[4 * jj + 3]);
-                            const ChunkOut gch = general_chunk<8, false>(dv, &A, a.mode, a.thr, lutb);
+                            const ChunkOut gch = general_chunk_one(dv, A, a.mode, a.thr, lutb);
                             *reinterpret_cast<uint4*>(tile + ro[jj]) = gch.packed;
                             nib[jj] = gch.nibs;
                             sats |= gch.sats << (8 * jj);
@@ -1372,8 +1385,8 @@ __global__ void __launch_bounds__(NTHREADS) ste_row_kernel(const KArgs a)
         } else {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const ChunkOut gch = general_chunk<8, false>(
-                    make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]), &A, a.mode, a.thr, glutb);
+                const ChunkOut gch = general_chunk_one(
+                    make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]), A, a.mode, a.thr, glutb);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     keep[4 * c + j] = ((gch.sats >> (2 * j)) & 1u ? 0u : 0xFFFFu) |
@@ -1462,8 +1475,8 @@ __global__ void __launch_bounds__(NTHREADS) row_stream_kernel(const KArgs a)
         } else {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const ChunkOut gch = general_chunk<8, false>(
-                    make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]), &A, a.mode, a.thr, glutb);
+                const ChunkOut gch = general_chunk_one(
+                    make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]), A, a.mode, a.thr, glutb);
                 nib[c] = gch.nibs;
                 sats |= gch.sats << (8 * c);
                 if constexpr (VALS) {
