@@ -1732,6 +1732,39 @@ static mxfp4_status launch_col_operand(const mxfp4_qdq_args* A, cudaStream_t s)
         k.thr = page_threshold(A->scale_factor);
     if (A->status && !groups && cudaMemsetAsync(A->status, 0, sizeof(int32_t), s) != cudaSuccess)
         return MXFP4_ECUDA;
+    const size_t plan_bytes = groups ? (size_t)(2 * (A->num_groups + 1)) * sizeof(int32_t) : 0;
+    // TMA-staged kernel where x is addressable by TMA and the outputs take
+    // its 32-byte and 16-bit stores
+    if (A->cols % 32 == 0 && A->ld % 8 == 0 && aligned(A->x, 16) && (!k.codes_col || aligned(k.codes_col, 32)) &&
+        A->rows <= INT32_MAX - 128 && A->cols <= INT32_MAX - SG_COLS) {
+        StagedMaps maps;
+        memset(&maps, 0, sizeof(maps));
+        const int64_t n_ct = (A->cols + SG_COLS - 1) / SG_COLS;
+        const int64_t pairs = 2 * (A->k_alloc / OP_KPAD);
+        if (pairs * n_ct < (int64_t)INT32_MAX &&
+            encode_2d(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(k.x), (uint64_t)k.cols,
+                      (uint64_t)k.rows, (uint64_t)k.ld * 2, SG_SLAB_COLS, SG_ROWS, CU_TENSOR_MAP_SWIZZLE_128B)) {
+            k.n_ct = (uint32_t)n_ct;
+            StagedFn sfn = A->scale_mode == MXFP4_SCALE_FLOOR
+                               ? (groups ? col_operand_staged_kernel<MXFP4_SCALE_FLOOR, true>
+                                         : col_operand_staged_kernel<MXFP4_SCALE_FLOOR, false>)
+                               : (groups ? col_operand_staged_kernel<MXFP4_SCALE_PAGE, true>
+                                         : col_operand_staged_kernel<MXFP4_SCALE_PAGE, false>);
+            const size_t smem = sizeof(OpsSmem) + 1024 + plan_bytes;
+            if (cudaFuncSetAttribute((const void*)sfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+                cudaSuccess)
+                return MXFP4_ECUDA;
+            const int sms = device_sms();
+            const int occ = occupancy((const void*)sfn, smem, OPS_THREADS);
+            if (sms <= 0 || occ <= 0)
+                return MXFP4_ECUDA;
+            int64_t grid = (int64_t)sms * occ;
+            if (pairs * n_ct < grid)
+                grid = pairs * n_ct < 1 ? 1 : pairs * n_ct;
+            sfn<<<(unsigned)grid, OPS_THREADS, smem, s>>>(maps, k);
+            return cudaGetLastError() == cudaSuccess ? MXFP4_OK : MXFP4_ECUDA;
+        }
+    }
     const void* fn;
     if (A->scale_mode == MXFP4_SCALE_FLOOR)
         fn = groups ? (const void*)col_operand_kernel<MXFP4_SCALE_FLOOR, true>

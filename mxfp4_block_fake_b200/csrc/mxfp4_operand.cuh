@@ -169,4 +169,261 @@ __global__ void __launch_bounds__(NTHREADS) col_operand_kernel(const KArgs a)
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// The same operand from TMA-staged tiles (bf16, cols % 32 == 0, x addressable
+// by TMA): a tile is one pair of 32-row blocks of the padded K numbering (64
+// rows; fewer, or none, at a group's end) by 256 columns, CTA b taking tiles
+// b, b + G, ... . Warp OPS_PRODUCER's lane 0 loads each block of a tile as
+// four 64 x 32 boxes (128-byte swizzle) into a ring of OPS_STAGES stages;
+// the eight compute warps release a stage with one arrival each on its
+// "empty" mbarrier. Compute warp w owns tile columns 32w..32w+31: lane =
+// column pair p (lane & 15) x row half h (lane >> 4) over rows 8i + 4h + q
+// (i = 0..7, q = 0..3), the two blocks' amaxes by one shuffle each. Four
+// consecutive rows of one column give one 16-bit piece of the K-major codes
+// (nudged hardware convert); after one exchange of pieces between the two
+// half-warps, lane h writes column 2p + h's 32 bytes (both blocks, one
+// sector) with one 32-byte store and its two scale bytes with one 16-bit
+// store. Every wait is bounded (SG_WAIT_NS).
+// ---------------------------------------------------------------------------
+
+constexpr int OPS_STAGES = 3;
+constexpr int OPS_COMPUTE_WARPS = SG_COLS / 32;                 // 8
+constexpr int OPS_THREADS = 32 * (OPS_COMPUTE_WARPS + 1);      // + the producer warp
+constexpr int OPS_PRODUCER = OPS_COMPUTE_WARPS;
+constexpr int OPS_TILE_BYTES = 2 * SG_TILE_BYTES;              // two blocks of 32 rows x 256 columns
+
+struct __align__(1024) OpsSmem {
+    uint8_t tiles[OPS_STAGES][OPS_TILE_BYTES];  // [block][slab][32 rows][128 bytes], swizzled
+    int4 info[OPS_STAGES];                      // row0, rows (0..64), col0, block pair of each stage's tile
+    uint32_t lut[64];
+    unsigned long long full[OPS_STAGES];
+    unsigned long long empty[OPS_STAGES];
+    int err;
+};
+
+// 32-byte store (eight words) to global memory, streaming.
+__device__ __forceinline__ void st_cs_v8w(void* p, const uint32_t (&v)[8])
+{
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
+template <int MODE, bool GROUPS>
+__global__ void __launch_bounds__(OPS_THREADS, 2) col_operand_staged_kernel(const __grid_constant__ StagedMaps maps,
+                                                                            const KArgs a)
+{
+    extern __shared__ __align__(1024) uint8_t s_dyn[];
+    uint8_t* s_base = s_dyn + ((1024u - (smem_addr(s_dyn) & 1023u)) & 1023u);
+    OpsSmem& sm = *reinterpret_cast<OpsSmem*>(s_base);
+    int32_t* s_apre = reinterpret_cast<int32_t*>(s_base + sizeof(OpsSmem));  // group g's first atom column
+    int32_t* s_rst = s_apre + (GROUPS ? a.num_groups + 1 : 0);              // group g's first row
+    volatile int* err = &sm.err;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid < 64)
+        sm.lut[tid] = lut_entry(tid);
+    if (tid == 0) {
+        sm.err = 0;
+        for (int s = 0; s < OPS_STAGES; ++s) {
+            mbar_init(smem_addr(&sm.full[s]), 1);
+            mbar_init(smem_addr(&sm.empty[s]), OPS_COMPUTE_WARPS);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    int64_t natoms;
+    if constexpr (GROUPS) {
+        natoms = build_plan<OP_KPAD>(a, s_apre, s_rst);  // contains __syncthreads
+        const bool ok = natoms >= 0 && natoms * OP_KPAD <= a.k_alloc;
+        if (blockIdx.x == 0 && tid == 0 && a.status)
+            *a.status = ok ? MXFP4_OK : MXFP4_EINVAL;
+        if (!ok)
+            return;
+    } else {
+        __syncthreads();
+        natoms = (a.rows + OP_KPAD - 1) / OP_KPAD;
+    }
+    const uint32_t ntiles = (uint32_t)(2 * natoms) * a.n_ct;  // block pairs x column tiles
+    const uint32_t n = blockIdx.x < ntiles ? (ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0u;
+    uint32_t issued = 0;
+
+    if (warp == OPS_PRODUCER) {
+        // tile t -> (block pair, column tile) and its rows
+        auto locate = [&](uint32_t t) {
+            const uint32_t bp = t / a.n_ct, ct = t - bp * a.n_ct;
+            int64_t row0, gend;
+            if constexpr (GROUPS) {
+                const int32_t at = (int32_t)(bp >> 1);
+                int lo = 0, hi = a.num_groups - 1;  // largest g with s_apre[g] <= at (skips empty groups)
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (s_apre[mid] <= at)
+                        lo = mid;
+                    else
+                        hi = mid - 1;
+                }
+                row0 = (int64_t)s_rst[lo] + ((int64_t)bp - 2 * (int64_t)s_apre[lo]) * 64;
+                gend = s_rst[lo + 1];
+            } else {
+                row0 = (int64_t)bp * 64;
+                gend = a.rows;
+            }
+            const int rows = (int)max((int64_t)0, min((int64_t)64, gend - row0));
+            return make_int4((int)(rows > 0 ? row0 : 0), rows, (int)(ct * SG_COLS), (int)bp);
+        };
+        auto load = [&](uint32_t j) {  // lane 0: the CTA's j-th tile into stage j mod OPS_STAGES
+            const int s = (int)(j % OPS_STAGES);
+            const int4 inf = locate(blockIdx.x + j * gridDim.x);
+            sm.info[s] = inf;
+            const uint32_t bar = smem_addr(&sm.full[s]);
+            const int nb = (inf.y + 31) >> 5;  // blocks with rows: 0, 1 or 2
+            if (nb == 0) {
+                mbar_arrive(bar);  // a padding pair: nothing to load
+            } else {
+                mbar_expect_tx(bar, (uint32_t)(nb * SG_TILE_BYTES));
+                for (int b = 0; b < nb; ++b)
+                    for (int sl = 0; sl < 4; ++sl)
+                        tma_load_slab(smem_addr(sm.tiles[s] + b * SG_TILE_BYTES + sl * SG_SLAB_BYTES), &maps.x,
+                                      inf.z + sl * SG_SLAB_COLS, inf.x + 32 * b, bar);
+            }
+            ++issued;
+        };
+        if (lane == 0) {
+            for (uint32_t j = 0; j < n && j < (uint32_t)OPS_STAGES; ++j)
+                load(j);
+            for (uint32_t j = OPS_STAGES; j < n; ++j) {
+                // round r >= 1 of a stage waits for the release of round r - 1
+                if (*err || !mbar_wait(smem_addr(&sm.empty[j % OPS_STAGES]), ((j / OPS_STAGES) - 1) & 1u)) {
+                    *err = 1;
+                    break;
+                }
+                load(j);
+            }
+        }
+    } else {
+        const uint32_t glutb = smem_addr(sm.lut) - 0x2C000000u;
+        const int p = lane & 15, h = lane >> 4;
+        const int cpair = 32 * warp + 2 * p;
+        const uint32_t cchunk = 4 * (warp & 1) + (p >> 2);
+        uint32_t yo[4];  // per q: byte offset of row 4h + q of block 0 in a stage
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t rq = 4 * h + q;
+            yo[q] = (uint32_t)(warp >> 1) * SG_SLAB_BYTES + rq * 128 + ((cchunk ^ rq) << 4) + 4 * (p & 3);
+        }
+        const int64_t kbytes = a.k_alloc / 2, nsc = a.k_alloc / 32;
+        for (uint32_t j = 0; j < n; ++j) {
+            const int s = (int)(j % OPS_STAGES);
+            if (!__all_sync(FULL, mbar_wait(smem_addr(&sm.full[s]), (j / OPS_STAGES) & 1u))) {
+                if (lane == 0)
+                    *err = 1;
+                break;
+            }
+            const int4 inf = sm.info[s];
+            const int rows = inf.y, col0 = inf.z;
+            const int64_t bp = inf.w;
+            const uint8_t* tile = sm.tiles[s];
+            if (col0 + 32 * warp < a.cols) {
+                // the lane's 32 words: word 4i + q is row 8i + 4h + q of the pair
+                uint32_t w[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        w[4 * i + q] = 8 * i + 4 * h + q < rows
+                                           ? sm_ld32(tile, (uint32_t)((i >> 2) * SG_TILE_BYTES + (i & 3) * 1024) + yo[q])
+                                           : 0u;
+                uint32_t pc[2][2][4];  // [column lo/hi][block][i & 3]: 16-bit pieces (rows 8i + 4h .. + 3)
+                uint32_t e8[2][2];     // [column][block]
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    uint32_t m2 = 0;
+#pragma unroll
+                    for (int i = 16 * b; i < 16 * b + 16; ++i)
+                        m2 = vmax2(m2, w[i] & 0x7FFF7FFFu);
+                    m2 = vmax2(m2, __shfl_xor_sync(FULL, m2, 16));
+                    const uint32_t A_lo = m2 << 16, A_hi = m2 & 0xFFFF0000u;
+                    const int k_lo = block_kt<MODE>(A_lo, a.thr), k_hi = block_kt<MODE>(A_hi, a.thr);
+                    const bool blk = 32 * b < rows;  // a padding block: codes 0, scale 2^0
+                    const bool fast = k_fast_bf(k_lo) && k_fast_bf(k_hi);
+                    e8[0][b] = !blk ? 127u : fast ? (uint32_t)(k_lo + 127) : e8_of(A_lo, k_lo);
+                    e8[1][b] = !blk ? 127u : fast ? (uint32_t)(k_hi + 127) : e8_of(A_hi, k_hi);
+                    if (!blk) {
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            pc[0][b][m] = pc[1][b][m] = 0u;
+                    } else if (fast) {
+                        const float invn_lo = inv_nudged(k_lo), invn_hi = inv_nudged(k_hi);
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            float ylo[4], yhi[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                nudged_pair(w[16 * b + 4 * m + q], invn_lo, invn_hi, ylo[q], yhi[q]);
+                            pc[0][b][m] = e2m1x4(ylo);
+                            pc[1][b][m] = e2m1x4(yhi);
+                        }
+                    } else {
+#pragma unroll
+                        for (int m = 0; m < 4; m += 2) {
+                            uint4 vlo, vhi;
+                            split_pair_rows(w + 16 * b + 4 * m, vlo, vhi);
+                            const uint32_t nlo = general_chunk_one(vlo, A_lo, a.mode, a.thr, glutb).nibs;
+                            const uint32_t nhi = general_chunk_one(vhi, A_hi, a.mode, a.thr, glutb).nibs;
+                            pc[0][b][m] = nlo & 0xFFFFu;
+                            pc[0][b][m + 1] = nlo >> 16;
+                            pc[1][b][m] = nhi & 0xFFFFu;
+                            pc[1][b][m + 1] = nhi >> 16;
+                        }
+                    }
+                }
+                // lane h writes column cpair + h: it keeps its own pieces of
+                // that column and receives the partner's (the partner sends
+                // the pieces of the column it does not write)
+                uint32_t give[4], got[4];
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int m = 0; m < 4; m += 2) {
+                        const int o = h ^ 1;  // the column the partner writes
+                        give[2 * b + m / 2] = (o == 0 ? pc[0][b][m] : pc[1][b][m]) |
+                                              ((o == 0 ? pc[0][b][m + 1] : pc[1][b][m + 1]) << 16);
+                    }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    got[u] = __shfl_xor_sync(FULL, give[u], 16);
+                // word m of block b: bytes 4m .. 4m + 3 = rows 8m .. 8m + 7:
+                // the h = 0 half's piece then the h = 1 half's
+                uint32_t out[8];
+#pragma unroll
+                for (int b = 0; b < 2; ++b)
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const uint32_t mine = h == 0 ? pc[0][b][m] : pc[1][b][m];
+                        const uint32_t theirs = (got[2 * b + m / 2] >> (16 * (m & 1))) & 0xFFFFu;
+                        out[4 * b + m] = h == 0 ? (mine | (theirs << 16)) : (theirs | (mine << 16));
+                    }
+                const int64_t c = col0 + cpair + h;
+                if (a.codes_col)
+                    st_cs_v8w(a.codes_col + c * kbytes + 32 * bp, out);
+                if (a.scales_col)
+                    *reinterpret_cast<uint16_t*>(a.scales_col + srow_off_mma(c, 2 * bp, nsc)) =
+                        (uint16_t)(h == 0 ? (e8[0][0] | (e8[0][1] << 8)) : (e8[1][0] | (e8[1][1] << 8)));
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&sm.empty[s]));
+        }
+    }
+
+    __syncthreads();
+    if (warp == OPS_PRODUCER && lane == 0 && *err) {
+        if (a.status)
+            *a.status = MXFP4_ECUDA;
+        for (uint32_t i = issued > (uint32_t)OPS_STAGES ? issued - OPS_STAGES : 0u; i < issued; ++i)
+            (void)mbar_wait(smem_addr(&sm.full[i % OPS_STAGES]), (i / OPS_STAGES) & 1u);
+    }
+}
+
 }  // namespace mxfp4

@@ -59,6 +59,26 @@ def test_colwise_operand_bytes(mode, case):
         assert bad.size == 0, f"{bad.size} scale bytes differ, first {bad[:4].tolist()}"
 
 
+@pytest.mark.parametrize("grouped", [False, True])
+def test_colwise_operand_many_tiles(grouped):
+    """cols % 32 == 0 runs the TMA-staged producer: 9000 x 2048 with 64
+    multinomial groups (or none), several tiles per CTA, so its stage ring
+    wraps, tails and padding block pairs of every kind occur."""
+    rows, cols = 9000, 2048
+    counts = W.moe_group_counts(rows, groups=64, seed=13).tolist() if grouped else None
+    x = W.mixed(rows, cols, seed=31)
+    ends = np.array([rows]) if counts is None else np.cumsum(np.asarray(counts, np.int64))
+    ora = O.qdq_colwise(u16(x), 32, 6.0, O.SCALE_PAGE, ends=None if counts is None else ends)
+    codes, scales, ka = ops.mxfp4_colwise_mma_operand(x.cuda(), group_list=counts, group_list_type=1)
+    exp_c, exp_s = O.colwise_operand_layout(ora["codes"], ora["scales"], ends, cols, k_alloc=ka)
+    got_c = codes.view(torch.uint8).cpu().numpy()
+    got_s = scales.view(torch.uint8).cpu().numpy()
+    bad = np.argwhere(got_c != exp_c)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first {bad[:3].tolist()}"
+    bad = np.flatnonzero(got_s != exp_s)
+    assert bad.size == 0, f"{bad.size} scale bytes differ, first {bad[:4].tolist()}"
+
+
 def test_dual_call_with_operand_layout():
     """Row-wise outputs, column-wise values and masks, and the column-wise
     operand from one call: each equals the oracle."""
