@@ -204,6 +204,40 @@ def test_mxfp8_mma_scale_layout():
     assert np.array_equal(np_bits(res.codes_row), ora["codes"])
 
 
+@pytest.mark.parametrize("shape,counts", [((300, 1024), None), ((261, 288), [100, 0, 61, 100]),
+                                          ((4096, 2048), "moe")])
+def test_mxfp8_dual_mma_scale_layout(shape, counts):
+    """Both directions with the row-wise scales in the MMA layout (the staged
+    kernel's SMMA form): the scales equal the oracle's placed by its layout
+    helper, unaligned by one byte too, and every other output is unchanged."""
+    rows, cols = shape
+    if counts == "moe":
+        counts = W.moe_group_counts(rows, groups=32, seed=14).tolist()
+    x = W.mixed(rows, cols, seed=60 + rows)
+    xd = x.cuda()
+    xo = oracle_in(x)
+    ora = O.qdq8_rowwise(xo)
+    for soff in (0, 1):
+        r = ops.alloc_outputs(xd, block=32, rowwise=True, colwise=True,
+                              num_groups=0 if counts is None else len(counts), emit_codes=True, emit_mask=True,
+                              with_status=True, scales_layout="mma", elem_format="e4m3")
+        n = r.scales_row.numel()
+        r.scales_row = torch.zeros((n + soff,), dtype=torch.uint8, device=xd.device)[soff:]
+        gl = None if counts is None else torch.tensor(counts, dtype=torch.int64, device=xd.device)
+        ops.mxfp4_qdq_fwd(xd, block=32, scale_mode="floor", rowwise=True, colwise=True, group_list=gl,
+                          group_list_type=1, emit_codes=True, emit_mask=True, out=r, check=True,
+                          elem_format="e4m3")
+        torch.cuda.synchronize()
+        got = r.scales_row.cpu().numpy()
+        exp = O.mma_scale_layout(ora["scales"])
+        bad = np.flatnonzero(got != exp)
+        assert bad.size == 0, f"{bad.size} scale bytes differ, first at {bad[:4].tolist()}"
+        r.scales_row = None
+        check(r, ora, "row", f"mma {shape}")
+        ends = None if counts is None else np.cumsum(np.asarray(counts, np.int64))
+        check(r, O.qdq8_colwise(xo, ends), "col", f"mma {shape}")
+
+
 def test_mxfp8_argument_errors():
     x = torch.randn(64, 64, device="cuda").to(torch.bfloat16)
     with pytest.raises(MXFP4ArgumentError):
