@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_qdq8_rowwise.restype = i32
         L.oracle_qdq8_colwise.argtypes = [P, i32, i64, i64, i64, P, i64, P, P, P, P]
         L.oracle_qdq8_colwise.restype = i32
+        L.oracle_dual_level_rowwise.argtypes = [P, i64, i64, i64, i32, f32, i32, P, P, P, P, P]
+        L.oracle_dual_level_rowwise.restype = i32
         _lib = L
     return _lib
 
@@ -184,6 +186,27 @@ def qdq8_colwise(x: np.ndarray, ends=None):
     return dict(y=y, codes=codes, scales=scales, mask=mask)
 
 
+def dual_level_rowwise(x: np.ndarray, level0_block: int = 512, scale_factor: float = 6.0,
+                       mode: int = SCALE_PAGE):
+    """Dual-level MX quantisation of bf16 bits [rows, cols] along rows:
+    dict(y bf16 bits, codes [rows, ceil(cols/2)], scales0 fp32 [rows,
+    ceil(cols/level0_block)], scales1 E8M0 [rows, ceil(cols/32)], mask)."""
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("dual-level quantisation takes bf16 bits (uint16)")
+    rows, cols = x.shape
+    y = np.empty_like(x)
+    codes = np.zeros((rows, (cols + 1) // 2), np.uint8)
+    s0 = np.zeros((rows, -(-cols // level0_block)), np.float32)
+    s1 = np.zeros((rows, -(-cols // 32)), np.uint8)
+    mask = np.zeros((rows, (cols + 7) // 8), np.uint8)
+    rc = lib().oracle_dual_level_rowwise(_ptr(x), rows, cols, cols, level0_block, scale_factor, mode,
+                                         _ptr(y), _ptr(codes), _ptr(s0), _ptr(s1), _ptr(mask))
+    if rc != 0:
+        raise ValueError("oracle_dual_level_rowwise: level0_block must be a positive multiple of 32")
+    return dict(y=y, codes=codes, scales0=s0, scales1=s1, mask=mask)
+
+
 def e4m3_value(code: int) -> float:
     return float(lib().oracle_e4m3_value(code & 0x7F)) * (-1.0 if code & 0x80 else 1.0)
 
@@ -288,5 +311,5 @@ __all__ = [
     "F32", "BF16", "SCALE_PAGE", "SCALE_FLOOR", "lib", "build", "bf16_to_f32", "f32_to_bf16",
     "scale_page", "scale_floor", "qdq_block", "group_ends", "colwise_scale_rows", "qdq_rowwise",
     "qdq_colwise", "ste_bwd", "unpack_bits", "unpack_nibbles", "mma_scale_layout", "qdq8_rowwise",
-    "qdq8_colwise", "e4m3_value", "e4m3_encode", "colwise_operand_k", "colwise_operand_layout",
+    "qdq8_colwise", "dual_level_rowwise", "e4m3_value", "e4m3_encode", "colwise_operand_k", "colwise_operand_layout",
 ]

@@ -18,7 +18,8 @@
  *          FakeW4A8GroupedLinear.normalize_group_list / quantize_input --
  *          group_list types and row/column ("rowwise"/"colwise") quantisation.
  *   [NPU]  sglang mxfp4_npu.py, process_weights_after_loading comment:
- *          "float4_e2m1fn_x2 (2 FP4 packed/byte)".
+ *          "float4_e2m1fn_x2 (2 FP4 packed/byte)"; NPUMXFP4DiffusionLinearMethod
+ *          (npu_dynamic_dual_level_mx_quant: codes, level-0 and level-1 scales).
  *
  * Every floating-point step is done in fp32 because [QAT] casts the input to
  * float32 before any arithmetic (_block_view) and keeps all tensors in fp32.
@@ -50,7 +51,13 @@
  *   - MXFP8 (oracle_qdq8_*, oracle_e4m3_*): the pages give no MXFP8
  *     arithmetic, so parity against them is unpinned; the functions are
  *     pinned against the E4M3 / OCP definitions (bit-field value set,
- *     nearest-even search over every bf16 value, torch's float8_e4m3fn cast).
+ *     nearest-even search over every bf16 value, torch's float8_e4m3fn cast);
+ *   - dual-level MX quantisation (oracle_dual_level_rowwise): the page names
+ *     the operator and its three results only, so parity against it is
+ *     unpinned; the function is pinned against its stated reading: reduction
+ *     to the single-level QDQ when the level-0 scale is a power of two, a
+ *     brute-force restatement on small inputs, a hand-worked block
+ *     (tests/golden) and the special blocks.
  */
 #include <math.h>
 #include <stdint.h>
@@ -574,4 +581,88 @@ void oracle_ste_bwd(const void* grad_out, int dtype, int64_t rows, int64_t cols,
             }
         }
     }
+}
+
+/* ---- [NPU] dual-level MX quantisation -------------------------------------- */
+
+/*
+ * [NPU] NPUMXFP4DiffusionLinearMethod quantises weights and activations with
+ * npu_dynamic_dual_level_mx_quant, which returns E2M1 codes, a level-0 scale
+ * of shape [rows, cols / level0_block] and a level-1 scale; the page gives no
+ * formula for either. Reading taken here (parity against the page unpinned):
+ *   - the input is bf16 (the page's activation dtypes are bf16 and fp16, and
+ *     weights of other dtypes are cast to bf16);
+ *   - level 0: blocks of level0_block consecutive elements of a row (the
+ *     last one partial); s0 = fl32(amax0 / 6), the fp32 level-0 scale, taken
+ *     as 1 when that quotient is 0 (an all-zero block);
+ *   - level 1: y = fl32(x / s0); y is quantised exactly as one row of the
+ *     MXFP4 QDQ above (blocks of 32, the same scale rule, codes, E8M0 bytes
+ *     and saturation |y| > 6 * 2^k1);
+ *   - output fl32((code * 2^k1) * s0) (the first product is exact), cast to
+ *     bf16;
+ *   - a level-0 block holding a NaN or +-inf is non-finite: NaN outputs,
+ *     codes 0, E8M0 bytes 0xFF, no saturation bits, s0 = NaN.
+ * Layouts: y [rows][cols] (row stride cols), codes [rows][ceil(cols/2)],
+ * scales0 [rows][ceil(cols/level0_block)] fp32, scales1 [rows][ceil(cols/32)],
+ * mask [rows][ceil(cols/8)]; any output may be NULL. Returns -1 when
+ * level0_block is not a positive multiple of 32 or memory runs out.
+ */
+int oracle_dual_level_rowwise(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                              int level0_block, float scale_factor, int mode,
+                              uint16_t* y, uint8_t* codes, float* scales0, uint8_t* scales1,
+                              uint8_t* mask)
+{
+    if (level0_block <= 0 || level0_block % 32 != 0)
+        return -1;
+    float* v = (float*)malloc(sizeof(float) * (size_t)level0_block);
+    if (!v)
+        return -1;
+    float w[32], o[32];
+    uint8_t nb[32], st[32];
+    int64_t nb0 = (cols + level0_block - 1) / level0_block, nb1 = (cols + 31) / 32;
+    int64_t cstride = (cols + 1) / 2, mstride = (cols + 7) / 8;
+    if (codes)
+        memset(codes, 0, (size_t)(rows * cstride));
+    if (mask)
+        memset(mask, 0, (size_t)(rows * mstride));
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t j = 0; j < nb0; ++j) {
+            int64_t c0 = j * level0_block;
+            int n0 = (int)((cols - c0) < level0_block ? (cols - c0) : level0_block);
+            for (int i = 0; i < n0; ++i)
+                v[i] = oracle_bf16_to_f32(x[r * ld + c0 + i]);
+            float a0 = block_amax(v, n0);
+            int finite = isfinite(a0);
+            float s0 = canonical_nan();
+            if (finite) {
+                s0 = a0 / MXFP4_E2M1_MAX; /* fp32 IEEE division */
+                if (s0 == 0.0f)
+                    s0 = 1.0f;
+            }
+            for (int b = 0; b * 32 < n0; ++b) {
+                int n1 = n0 - 32 * b < 32 ? n0 - 32 * b : 32;
+                int64_t cb = c0 + 32 * b;
+                uint8_t e8 = 0xFF;
+                if (finite) {
+                    for (int i = 0; i < n1; ++i)
+                        w[i] = v[32 * b + i] / s0;
+                    oracle_qdq_block(w, n1, scale_factor, mode, o, nb, st, &e8);
+                }
+                for (int i = 0; i < n1; ++i) {
+                    if (y)
+                        y[r * cols + cb + i] = oracle_f32_to_bf16(finite ? o[i] * s0 : canonical_nan());
+                    if (codes)
+                        put_nibble(codes + r * cstride, cb + i, finite ? nb[i] : 0);
+                    if (mask)
+                        put_bit(mask + r * mstride, cb + i, finite ? st[i] : 0);
+                }
+                if (scales1)
+                    scales1[r * nb1 + cb / 32] = e8;
+            }
+            if (scales0)
+                scales0[r * nb0 + j] = s0;
+        }
+    }
+    free(v);
+    return 0;
 }
