@@ -360,7 +360,9 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
     block-scaled MMA layout, no dequantised values), blocks of 128 in both
     directions with every output (ungrouped), the MXFP8 element format
     (E4M3, the OCP scale rule) row-wise and in both directions with the
-    groups, and the bench step itself with the other scale rule."""
+    groups, dual-level MX quantisation (fp32 level-0 scales per 512 elements,
+    MXFP4 level 1; every output), and the bench step itself with the other
+    scale rule."""
     import torch
 
     from mxfp4_block_fake_b200 import _abi, ops
@@ -444,6 +446,18 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
     def mxfp8_dual():
         call(_abi.mxfp4_qdq_fwd(dual8, sp), "mxfp4_qdq_fwd")
 
+    # dual-level MX quantisation (fp32 level-0 scale per 512, MXFP4 level 1), every output
+    dl = ops.mxfp4_dual_level_qdq(xd, scale_mode=a.scale_mode, emit_mask=True)
+    dl_args = _abi.DualLevelArgs()
+    dl_args.x, dl_args.dtype, dl_args.level0_block = xd.data_ptr(), _abi.BF16, 512
+    dl_args.rows, dl_args.cols, dl_args.ld, dl_args.ld_y = a.rows, a.cols, a.cols, a.cols
+    dl_args.scale_factor, dl_args.scale_mode = 6.0, _abi.SCALE_PAGE if a.scale_mode == "page" else _abi.SCALE_FLOOR
+    dl_args.y, dl_args.codes, dl_args.mask = dl.y.data_ptr(), dl.codes.data_ptr(), dl.mask.data_ptr()
+    dl_args.scales0, dl_args.scales1 = dl.scales0.data_ptr(), dl.scales1.data_ptr()
+
+    def dual_level():
+        call(_abi.mxfp4_dual_level_qdq(dl_args, sp), "mxfp4_dual_level_qdq")
+
     peak, peak_kind = measured_peaks()
     out = {}
     for name, fn, bpe in (("rowwise_fwd_all_outputs_ste_mask", row_step, 4 + 0.5 + 1 / 32 + 0.125 + 4.125),
@@ -453,6 +467,7 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
                           ("dual_block128_all_outputs", dual128, 2 + 4 + 1 + 2 / 128 + 0.25),
                           ("mxfp8_rowwise_all_outputs", mxfp8_row, 2 + 2 + 1 + 1 / 32 + 0.125),
                           ("mxfp8_dual_grouped_all_outputs", mxfp8_dual, 2 + 4 + 2 + 2 / 32 + 0.25),
+                          ("dual_level_mx_all_outputs", dual_level, 2 + 2 + 0.5 + 1 / 32 + 4 / 512 + 0.125),
                           (f"bench_step_{other}_scale", step_other_mode, step_bytes(a.rows, a.cols, s_col)["step"] / n)):
         if a.only_mode and name != a.only_mode:
             continue
@@ -469,7 +484,7 @@ def time_modes(a, xd, gd, res, gi, stream, gl, s_col, steps: int = 20):
         gbs = n * bpe / (ms / 1e3) / 1e9
         out[name] = {"ms_per_step": round(ms, 4), "bytes_per_element": round(bpe, 4), "GB/s": round(gbs, 1),
                      "frac_of_peak": round(gbs / peak, 4), "peak_kind": peak_kind}
-    del opr, r8, r128, mma_scales
+    del opr, r8, r128, mma_scales, dl
     torch.cuda.empty_cache()
     if not a.only_mode or a.only_mode.startswith("grouped_gemm"):
         out.update(time_gemm(a, xd, res, gl, stream, steps))

@@ -168,7 +168,7 @@ typedef enum {
 #define MXFP4_COLS_ROWMAJOR 0
 #define MXFP4_COLS_MMA 1
 
-#define MXFP4_ABI_VERSION 4
+#define MXFP4_ABI_VERSION 5
 
 /*
  * Arguments of one QDQ call. Zero-initialise and fill what is used; every
@@ -360,6 +360,59 @@ typedef struct mxfp4_gmm_args {
 } mxfp4_gmm_args;
 
 mxfp4_status mxfp4_grouped_gemm(const mxfp4_gmm_args* args, mxfp4_stream_t stream);
+
+/*
+ * Dual-level MX quantisation (sglang mxfp4_npu.py, NPUMXFP4DiffusionLinearMethod:
+ * npu_dynamic_dual_level_mx_quant turns a bf16 [rows, cols] tensor into E2M1
+ * codes, a level-0 scale of shape [rows, cols / level0_block] and a level-1
+ * scale, which npu_dual_level_quant_matmul consumes; the page names the
+ * operators and their results only, so the arithmetic below is this
+ * library's reading of them):
+ *   level 0   blocks of level0_block consecutive elements of a row (the last
+ *             one partial): s0 = fl32(amax0 / 6), the fp32 level-0 scale
+ *             (1 when that quotient is 0, i.e. an all-zero block);
+ *   level 1   y = fl32(x / s0) (IEEE division), quantised like one row of
+ *             mxfp4_qdq_fwd with block 32: E8M0 scale 2^k1 by scale_mode /
+ *             scale_factor from the block's max |y|, E2M1 code of y / 2^k1,
+ *             saturation |y| > 6 * 2^k1;
+ *   output    fl32((code * 2^k1) * s0) rounded to bf16 (nearest even);
+ *   a level-0 block holding a NaN or +-inf writes the quiet NaN 0x7FC0 to
+ *   its outputs, code 0, E8M0 bytes 0xFF, no saturation bits and s0 =
+ *   0x7FC00000.
+ * Arguments (zero-initialise; NULL outputs are skipped):
+ *   x            bf16 [rows][cols], leading dimension ld (>= cols) elements.
+ *   dtype        MXFP4_BF16 (anything else: MXFP4_EUNSUPPORTED).
+ *   level0_block 512 (other positive multiples of 32: MXFP4_EUNSUPPORTED;
+ *                anything else MXFP4_EINVAL).
+ *   scale_factor, scale_mode  the level-1 scale rule, as for mxfp4_qdq_fwd.
+ *   y            bf16 [rows][cols], leading dimension ld_y (>= cols).
+ *   codes        [rows][ceil(cols/2)] bytes, E2M1 nibbles as codes_row.
+ *   scales0      fp32 [rows][ceil(cols/level0_block)], row-major.
+ *   scales1      [rows][ceil(cols/32)] E8M0 bytes, row-major.
+ *   mask         [rows][ceil(cols/8)] saturation bits as mask_row; the
+ *                clipped STE backward reads it through mxfp4_ste_bwd
+ *                (saved_mask) unchanged.
+ * Device pointers owned by the caller; no allocation; asynchronous on
+ * `stream`; argument errors are returned before any launch.
+ */
+typedef struct mxfp4_dual_level_args {
+    const void* x;
+    int32_t dtype;
+    int32_t level0_block;
+    int64_t rows;
+    int64_t cols;
+    int64_t ld;
+    float scale_factor;
+    int32_t scale_mode;
+    void* y;
+    int64_t ld_y;
+    uint8_t* codes;
+    float* scales0;
+    uint8_t* scales1;
+    uint8_t* mask;
+} mxfp4_dual_level_args;
+
+mxfp4_status mxfp4_dual_level_qdq(const mxfp4_dual_level_args* args, mxfp4_stream_t stream);
 
 /* Static English text of a status; never NULL. */
 const char* mxfp4_status_string(mxfp4_status status);

@@ -10,9 +10,11 @@ Layers:
 """
 from ._abi import MXFP4ArgumentError, MXFP4Error
 from .ops import (
+    DualLevelResult,
     QDQResult,
     colwise_scale_rows_bound,
     mxfp4_colwise_scale_rows,
+    mxfp4_dual_level_qdq,
     mxfp4_qdq_fwd,
     mxfp4_qdq_fwd_bwd,
     mxfp4_ste_bwd,
@@ -29,7 +31,7 @@ from .qat import (
 )
 
 __all__ = [
-    "MXFP4Error", "MXFP4ArgumentError", "QDQResult", "colwise_scale_rows_bound", "mxfp4_colwise_scale_rows",
+    "MXFP4Error", "MXFP4ArgumentError", "QDQResult", "DualLevelResult", "mxfp4_dual_level_qdq", "colwise_scale_rows_bound", "mxfp4_colwise_scale_rows",
     "mxfp4_qdq_fwd", "mxfp4_qdq_fwd_bwd", "mxfp4_ste_bwd", "MXFP4FakeQuantizer", "MXFP4QATConfig",
     "MXFP4QATLinear", "convert_to_mxfp4_qat", "mxfp4_fake_quant", "mxfp4_quant_dequant",
     "mxfp4_saturation_mask", "unpack_mask",

@@ -21,7 +21,7 @@ SCALES_ROWMAJOR, SCALES_MMA = 0, 1
 COLS_ROWMAJOR, COLS_MMA = 0, 1
 ELEM_E2M1, ELEM_E4M3 = 0, 1
 MAX_GROUPS = 4096
-ABI_VERSION = 4
+ABI_VERSION = 5
 
 # Every symbol include/mxfp4.h declares.
 EXPORTS = (
@@ -35,6 +35,7 @@ EXPORTS = (
     "mxfp4_colwise_operand_k_bound",
     "mxfp4_colwise_operand_scale_bytes",
     "mxfp4_grouped_gemm",
+    "mxfp4_dual_level_qdq",
     "mxfp4_status_string",
     "mxfp4_abi_version",
 )
@@ -98,6 +99,25 @@ class GmmArgs(ctypes.Structure):
     ]
 
 
+class DualLevelArgs(ctypes.Structure):
+    _fields_ = [
+        ("x", ctypes.c_void_p),
+        ("dtype", ctypes.c_int32),
+        ("level0_block", ctypes.c_int32),
+        ("rows", ctypes.c_int64),
+        ("cols", ctypes.c_int64),
+        ("ld", ctypes.c_int64),
+        ("scale_factor", ctypes.c_float),
+        ("scale_mode", ctypes.c_int32),
+        ("y", ctypes.c_void_p),
+        ("ld_y", ctypes.c_int64),
+        ("codes", ctypes.c_void_p),
+        ("scales0", ctypes.c_void_p),
+        ("scales1", ctypes.c_void_p),
+        ("mask", ctypes.c_void_p),
+    ]
+
+
 class MXFP4Error(RuntimeError):
     """A libmxfp4 call returned a non-OK status."""
 
@@ -145,6 +165,8 @@ def lib() -> ctypes.CDLL:
     L.mxfp4_colwise_operand_scale_bytes.restype = i64
     L.mxfp4_grouped_gemm.argtypes = [ctypes.POINTER(GmmArgs), P]
     L.mxfp4_grouped_gemm.restype = i32
+    L.mxfp4_dual_level_qdq.argtypes = [ctypes.POINTER(DualLevelArgs), P]
+    L.mxfp4_dual_level_qdq.restype = i32
     L.mxfp4_status_string.argtypes = [i32]
     L.mxfp4_status_string.restype = ctypes.c_char_p
     L.mxfp4_abi_version.argtypes = []
@@ -207,3 +229,7 @@ def mxfp4_colwise_operand_k(host_group_list, group_list_type: int, rows: int) ->
 
 def mxfp4_grouped_gemm(args: GmmArgs, stream: int) -> int:
     return lib().mxfp4_grouped_gemm(ctypes.byref(args), stream)
+
+
+def mxfp4_dual_level_qdq(args: DualLevelArgs, stream: int) -> int:
+    return lib().mxfp4_dual_level_qdq(ctypes.byref(args), stream)

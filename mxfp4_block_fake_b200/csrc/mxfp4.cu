@@ -2120,6 +2120,8 @@ static mxfp4_status run_gmm(const mxfp4_gmm_args* A, cudaStream_t s)
                      : launch_gmm_t<MXFP4_ELEM_E4M3, false, false>(maps, g, bound, s));
 }
 
+#include "mxfp4_dual.cuh"
+
 }  // namespace mxfp4
 
 using namespace mxfp4;
@@ -2318,6 +2320,11 @@ int64_t mxfp4_colwise_operand_scale_bytes(int64_t cols, int64_t k_alloc)
     if (cols < 0 || k_alloc < 0 || k_alloc % OP_KPAD != 0)
         return -1;
     return 512 * ((cols + 127) / 128) * (k_alloc / OP_KPAD);
+}
+
+mxfp4_status mxfp4_dual_level_qdq(const mxfp4_dual_level_args* args, mxfp4_stream_t stream)
+{
+    return run_dual_level(args, reinterpret_cast<cudaStream_t>(stream));
 }
 
 mxfp4_status mxfp4_grouped_gemm(const mxfp4_gmm_args* args, mxfp4_stream_t stream)

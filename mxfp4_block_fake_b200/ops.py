@@ -534,3 +534,52 @@ def mxfp4_grouped_gemm(a: torch.Tensor, a_scales: torch.Tensor, b: torch.Tensor,
     if check:
         _check_status(st, "mxfp4_grouped_gemm")
     return d
+
+
+@dataclasses.dataclass
+class DualLevelResult:
+    y: torch.Tensor | None = None
+    codes: torch.Tensor | None = None
+    scales0: torch.Tensor | None = None
+    scales1: torch.Tensor | None = None
+    mask: torch.Tensor | None = None
+
+
+def mxfp4_dual_level_qdq(x: torch.Tensor, *, level0_block: int = 512, scale_factor: float = 6.0,
+                         scale_mode: str = "page", emit_values: bool = True, emit_codes: bool = True,
+                         emit_mask: bool = False, out: DualLevelResult | None = None) -> DualLevelResult:
+    """Dual-level MX quantisation of a bf16 tensor along its last dimension
+    (include/mxfp4.h, mxfp4_dual_level_qdq): fp32 level-0 scales
+    [rows, ceil(cols/level0_block)], E8M0 level-1 scales [rows, ceil(cols/32)],
+    packed E2M1 codes, and on request the dequantised bf16 values and the
+    bit-packed saturation mask (which mxfp4_ste_bwd takes as saved_mask).
+    Asynchronous on the current stream."""
+    x = _as_2d(x)
+    if x.dtype != torch.bfloat16:
+        raise TypeError("dual-level quantisation takes bfloat16 input")
+    if scale_mode not in _MODES:
+        raise ValueError(f"scale_mode must be 'page' or 'floor', got {scale_mode!r}")
+    rows, cols = x.shape
+    dev = x.device
+    r = out if out is not None else DualLevelResult(
+        y=torch.empty((rows, cols), dtype=torch.bfloat16, device=dev) if emit_values else None,
+        codes=torch.empty((rows, (cols + 1) // 2), dtype=torch.uint8, device=dev) if emit_codes else None,
+        scales0=torch.empty((rows, -(-cols // max(level0_block, 1))), dtype=torch.float32, device=dev),
+        scales1=torch.empty((rows, -(-cols // 32)), dtype=torch.uint8, device=dev),
+        mask=torch.empty((rows, (cols + 7) // 8), dtype=torch.uint8, device=dev) if emit_mask else None)
+    if r.y is not None:
+        _need(r.y, "y", (rows, cols), torch.bfloat16, dev)
+    for t, name, shape, dt in ((r.codes, "codes", (rows, (cols + 1) // 2), torch.uint8),
+                               (r.scales0, "scales0", (rows, -(-cols // max(level0_block, 1))), torch.float32),
+                               (r.scales1, "scales1", (rows, -(-cols // 32)), torch.uint8),
+                               (r.mask, "mask", (rows, (cols + 7) // 8), torch.uint8)):
+        if t is not None:
+            _need(t, name, shape, dt, dev)
+    a = _abi.DualLevelArgs()
+    a.x, a.dtype, a.level0_block = x.data_ptr(), _abi.BF16, int(level0_block)
+    a.rows, a.cols, a.ld = rows, cols, _ld(x)
+    a.scale_factor, a.scale_mode = float(scale_factor), _MODES[scale_mode]
+    a.y, a.ld_y = _ptr(r.y), cols
+    a.codes, a.scales0, a.scales1, a.mask = _ptr(r.codes), _ptr(r.scales0), _ptr(r.scales1), _ptr(r.mask)
+    _abi.check(_abi.mxfp4_dual_level_qdq(a, _stream(dev)), "mxfp4_dual_level_qdq")
+    return r

@@ -123,3 +123,18 @@ def ste_bwd(grad_out: np.ndarray, mask: np.ndarray, clip_grad: bool = True) -> n
         for f in fs:
             f.result()
     return out
+
+
+def dual_level_rowwise(x: np.ndarray, level0_block: int = 512, scale_factor: float = 6.0,
+                       mode: int = O.SCALE_PAGE) -> dict:
+    """O.dual_level_rowwise of the whole array, row chunks in parallel."""
+    rows, cols = x.shape
+    out = dict(y=np.empty_like(x), codes=np.zeros((rows, (cols + 1) // 2), np.uint8),
+               scales0=np.zeros((rows, -(-cols // level0_block)), np.float32),
+               scales1=np.zeros((rows, -(-cols // 32)), np.uint8), mask=np.zeros((rows, (cols + 7) // 8), np.uint8))
+    with _pool() as p:
+        fs = [p.submit(_rowwise_into, O.dual_level_rowwise, x, out, r0, r1, level0_block, scale_factor, mode)
+              for r0, r1 in _row_chunks(rows, 4 * threads())]
+        for f in fs:
+            f.result()
+    return out

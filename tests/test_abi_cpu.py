@@ -51,7 +51,8 @@ def test_library_exports_every_declared_symbol(abi):
         assert hasattr(abi.lib(), name)
 
 
-@pytest.mark.parametrize("cname,pyname", [("mxfp4_qdq_args", "QdqArgs"), ("mxfp4_gmm_args", "GmmArgs")])
+@pytest.mark.parametrize("cname,pyname", [("mxfp4_qdq_args", "QdqArgs"), ("mxfp4_gmm_args", "GmmArgs"),
+                                          ("mxfp4_dual_level_args", "DualLevelArgs")])
 def test_struct_layout_matches_c(abi, tmp_path, cname, pyname):
     cls = getattr(abi, pyname)
     fields = [f for f, _ in cls._fields_]
@@ -205,6 +206,28 @@ def test_scales_row_bytes(abi, oracle_mod, rows, cols, block):
     assert L.mxfp4_scales_row_bytes(rows, cols, block, abi.SCALES_MMA) == mma
     assert L.mxfp4_scales_row_bytes(rows, cols, block, 7) == -1
     assert L.mxfp4_scales_row_bytes(-1, cols, block, abi.SCALES_ROWMAJOR) == -1
+
+
+def _dual(abi, **kw):
+    a = abi.DualLevelArgs()
+    a.x, a.dtype, a.level0_block, a.rows, a.cols, a.ld = 4096, abi.BF16, 512, 4, 1024, 1024
+    a.scale_factor, a.scale_mode, a.ld_y = 6.0, abi.SCALE_PAGE, 1024
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(rows=-1), 1), (dict(cols=-2), 1), (dict(dtype=3), 1), (dict(level0_block=0), 1),
+    (dict(level0_block=48), 1), (dict(level0_block=-512), 1), (dict(scale_factor=0.0), 1),
+    (dict(scale_factor=float("nan")), 1), (dict(scale_factor=float("inf")), 1), (dict(scale_mode=2), 1),
+    (dict(dtype=0), 2), (dict(level0_block=256), 2), (dict(level0_block=1024), 2),
+    (dict(x=None), 1), (dict(ld=1000), 1), (dict(y=8192, ld_y=1000), 1),
+    (dict(rows=0), 0), (dict(cols=0, x=None), 0),
+])
+def test_dual_level_rejects_bad_arguments_on_host(abi, kw, expected):
+    assert abi.mxfp4_dual_level_qdq(_dual(abi, **kw), None) == expected
+    assert abi.lib().mxfp4_dual_level_qdq(None, None) == abi.EINVAL
 
 
 def test_null_args_and_bad_bwd_arguments(abi):
