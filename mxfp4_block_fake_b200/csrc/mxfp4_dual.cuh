@@ -15,10 +15,24 @@
 // 16-byte loads (and the 16-byte stores of y) covers 512 contiguous bytes, and
 // a level-1 block of 32 is four neighbouring lanes of one half. Per unit:
 // level-0 amax by one warp reduction, s0 and its reciprocal, y = x / s0 by a
-// corrected reciprocal product (dl_div), the level-1 amax by two shuffles,
-// the scale and codes as in the single-level kernels, the output as one more
-// fp32 multiply. Grid-stride over units, consecutive warps on consecutive
-// units, so that the grid streams through memory in order.
+// corrected reciprocal product, the level-1 amax by two shuffles, then the
+// codes and outputs. Grid-stride over units, consecutive warps on
+// consecutive units, so that the grid streams through memory in order; a
+// warp copies its next units into shared memory while it works on the
+// current one.
+//
+// Two element paths. The fast path (full, aligned units whose level-1
+// scales are at most 1, which covers every block at the default scale
+// factor 6) works on element pairs with the packed fp32 instructions:
+// y = x / s0 (dl_div's steps), y1 = y * 2^-k1 (exact, as 2^-k1 >= 1),
+// floor(4 |y1|) by one fma rounding down into 2^23, the code magnitude from a
+// 64-entry shared table, the sign of y1 (never -0 here), the E2M1 nibbles by
+// the hardware convert of the exact signed codes, and the output
+// fl32(code * 2^k1 * s0) as one multiply by S = 2^k1 s0 when S is exact (a
+// normal number), else as two. It stores nothing before it has decided to
+// handle the unit. The general path (dual_unit) takes every other unit:
+// ragged or unaligned ones, non-finite or tiny level-0 blocks, level-1
+// scales above 1 (small PAGE scale factors).
 
 constexpr int DL_BLOCK0 = 512;
 
@@ -33,7 +47,12 @@ struct DualArgs {
     uint8_t* mask;
     float sf;
     int32_t mode;
-    int32_t vec;  // full units may use 16-byte loads / stores (host-checked alignment)
+    int32_t vec;   // full units may use 16-byte loads / stores (host-checked alignment)
+    int32_t fast;  // the fast path's scale rule is available (FLOOR, or PAGE with thr)
+    uint32_t thr;  // PAGE mode: fp32 bits of the qparams threshold T0
+    // 4 and 65536 (set by the host): multiply-adds by these run-time values
+    // stay on the multiply-add pipe instead of becoming shifts
+    uint32_t mul4, mul16;
     int64_t nb0, nb1, cstride, mstride, units;
 };
 
@@ -57,7 +76,7 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 template <bool VEC>
-__device__ __forceinline__ void dual_unit(const DualArgs& a, int64_t row, int64_t j, int lane)
+__device__ __noinline__ void dual_unit(const DualArgs& a, int64_t row, int64_t j, int lane)
 {
     const int64_t c0 = j * DL_BLOCK0;
     const uint16_t* xr = a.x + row * a.ld;
@@ -196,16 +215,288 @@ __device__ __forceinline__ void dual_unit(const DualArgs& a, int64_t row, int64_
         a.s0[row * a.nb0 + j] = s0;
 }
 
+typedef unsigned long long u64;
+
+__device__ __forceinline__ u64 pk2(float lo, float hi)
+{
+    u64 d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+
+__device__ __forceinline__ void upk2(u64 v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ u64 mul2(u64 a, u64 b)
+{
+    u64 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c)
+{
+    u64 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ u64 fma2_rm(u64 a, u64 b, u64 c)
+{
+    u64 d;
+    asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t vmin2(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// y = fl32(x / s0) of one value, r = fl32(1 / s0): the corrected reciprocal
+// product where |x| >= tf (dl_div's conditions hold), the IEEE quotient
+// otherwise.
+__device__ __forceinline__ float dl_quot(float x, float s0, float r, float tf)
+{
+    if (fabsf(x) >= tf) {
+        const float q = __fmul_rn(x, r);
+        return __fmaf_rn(__fmaf_rn(-q, s0, x), r, q);
+    }
+    return __fdiv_rn(x, s0) + 0.0f;
+}
+
+// Fast path of one full, aligned unit whose 16 bf16 pairs are w (w[0..3]:
+// elements 8 lane .. 8 lane + 7 of the first half, w[4..7] of the second).
+// Returns false, having stored nothing, when the unit needs dual_unit; the
+// decision is uniform across the warp.
+//
+// s0 = fl32(a0 / 6) and r = fl32(1 / s0) come from a table over the seven
+// significand bits of the bf16 amax a0 (entries for a0 in [1, 2)), shifted by
+// a0's exponent: both roundings commute with power-of-two scaling while the
+// results stay normal, which holds for every a0 >= 2^-65 taken here. The
+// quotients are formed from |x| (the sign is put back on the code), so
+// |y| = fl32(|x| / s0) feeds both the floor and the saturation test. The
+// level-1 amax is taken on x: fl32(|x| / s0) is a monotone function of |x|,
+// so max |y| over a block is the quotient of max |x|. floor(4 |y 2^-k1|)
+// comes from one packed fma rounding down into 2^21, where the fp32 spacing
+// is 1/4 (y 2^-k1 is exact: 2^-k1 >= 1 on this path, and |y 2^-k1| < 16);
+// the table entry at that index is the code magnitude. Elements whose y is
+// zero (x = +-0, or a quotient that underflows) get a +0 code, as sign(y) = 0
+// there.
+__device__ __forceinline__ bool dual_unit_fast(const DualArgs& a, int64_t row, int64_t j, int lane,
+                                               const uint32_t (&w)[8], uint32_t lutb, const float2* s0r)
+{
+    uint32_t aw[8], mh[2] = {0u, 0u}, mn = 0x7FFF7FFFu;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        aw[i] = w[i] & 0x7FFF7FFFu;
+        mh[i >> 2] = vmax2(mh[i >> 2], aw[i]);
+        mn = vmin2(mn, aw[i]);
+    }
+    // level-1 blocks are four lanes of a half: both halves' maxima in one word
+    uint32_t P = __byte_perm(max(mh[0] & 0xFFFFu, mh[0] >> 16), max(mh[1] & 0xFFFFu, mh[1] >> 16), 0x5410);
+    P = vmax2(P, __shfl_xor_sync(FULL, P, 1));
+    P = vmax2(P, __shfl_xor_sync(FULL, P, 2));
+    const uint32_t A0 = __reduce_max_sync(FULL, max(P & 0xFFFFu, P >> 16));
+    if (A0 >= 0x7F80u || A0 < 0x1F00u)  // non-finite, or a0 < 2^-65 (tiny or all-zero block)
+        return false;
+    const float2 t0 = s0r[A0 & 0x7Fu];
+    const int e0 = (int)(A0 >> 7) - 127;
+    const float s0 = __uint_as_float(__float_as_uint(t0.x) + ((uint32_t)e0 << 23));
+    const float r = __uint_as_float(__float_as_uint(t0.y) - ((uint32_t)e0 << 23));
+    // |x| >= tf meets both conditions under which the corrected reciprocal
+    // product is the IEEE quotient (|x| >= 2^-102, |x r| >= 2^-124); s0 2^-123
+    // is exact whenever it exceeds 2^-102. tb: tf rounded up to bf16 bits.
+    const float tf = fmaxf(0x1p-102f, s0 * 0x1p-123f);
+    const uint32_t tb = (__float_as_uint(tf) + 0xFFFFu) >> 16;
+    // a lane with an |x| below tf (zeros included) checks its elements one by one
+    const bool lane_slow = min(mn & 0xFFFFu, mn >> 16) < tb;
+
+    QP p[2];
+    bool big = false, exact = true;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float yamax = dl_quot(__uint_as_float(h ? P & 0xFFFF0000u : P << 16), s0, r, tf);
+        p[h] = qparams(__float_as_uint(yamax), a.mode, a.thr);
+        big = big || !(p[h].inv >= 1.0f);
+        exact = exact && p[h].scale * s0 >= 0x1p-126f;  // 2^k1 s0 normal, hence exact
+    }
+    if (__any_sync(FULL, big))  // a level-1 scale above 1: y * 2^-k1 may round
+        return false;
+    exact = __all_sync(FULL, exact);
+
+    const u64 R2 = pk2(r, r), NS2 = pk2(-s0, -s0);
+    u64 Y[8];
+    uint32_t sg[8];  // sign sources: x with -0 turned into +0
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const u64 X = pk2(__uint_as_float(aw[i] * a.mul16), __uint_as_float(aw[i] & 0xFFFF0000u));
+        const u64 Q = mul2(X, R2);
+        Y[i] = fma2(fma2(Q, NS2, X), R2, Q);
+        sg[i] = clear_neg_zero(w[i]);
+    }
+    if (lane_slow) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float ylo, yhi;
+            upk2(Y[i], ylo, yhi);
+            const uint32_t alo = aw[i] & 0xFFFFu, ahi = aw[i] >> 16;
+            if (alo - 1u < tb - 1u) {  // 0 < |x| < tf: the IEEE quotient; an underflow to 0 drops the sign
+                ylo = __fdiv_rn(__uint_as_float(alo << 16), s0);
+                if (ylo == 0.0f)
+                    sg[i] &= 0xFFFF7FFFu;
+            }
+            if (ahi - 1u < tb - 1u) {
+                yhi = __fdiv_rn(__uint_as_float(ahi << 16), s0);
+                if (yhi == 0.0f)
+                    sg[i] &= 0x7FFFFFFFu;
+            }
+            Y[i] = pk2(ylo, yhi);
+        }
+    }
+
+    const int64_t c0 = j * DL_BLOCK0;
+    const int64_t cl = c0 + 8 * lane;
+    uint16_t* yp = a.y + row * a.ld_y + cl;
+    uint8_t* cp = a.codes + row * a.cstride + cl / 2;
+    uint8_t* mp = a.mask + row * a.mstride + cl / 8;
+    uint8_t* s1p = a.s1 + row * a.nb1 + c0 / 32 + (lane >> 2);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const u64 INV2 = pk2(p[h].inv, p[h].inv);
+        const float S = p[h].scale * s0;
+        const u64 A2 = exact ? pk2(S, S) : pk2(p[h].scale, p[h].scale);
+        const u64 B2 = pk2(s0, s0);
+        const uint32_t lim = __float_as_uint(p[h].scale * 6.0f);  // exact: 2^k1 >= 2^-127
+        uint32_t ob[4], sats = 0;
+        float cv[8];
+#pragma unroll
+        for (int q = 3; q >= 0; --q) {
+            const int i = 4 * h + q;
+            float ylo, yhi;
+            upk2(Y[i], ylo, yhi);
+            float tlo, thi;
+            upk2(fma2_rm(Y[i], INV2, pk2(2097152.0f, 2097152.0f)), tlo, thi);
+            uint32_t elo, ehi;
+            asm("ld.shared.u32 %0, [%1];" : "=r"(elo) : "r"(__float_as_uint(tlo) * a.mul4 + lutb));
+            asm("ld.shared.u32 %0, [%1];" : "=r"(ehi) : "r"(__float_as_uint(thi) * a.mul4 + lutb));
+            cv[2 * q] = __uint_as_float(elo | ((sg[i] << 16) & 0x80000000u));
+            cv[2 * q + 1] = __uint_as_float(ehi | (sg[i] & 0x80000000u));
+            u64 O = mul2(pk2(cv[2 * q], cv[2 * q + 1]), A2);
+            if (!exact)
+                O = mul2(O, B2);
+            float olo, ohi;
+            upk2(O, olo, ohi);
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(ob[q]) : "f"(ohi), "f"(olo));
+            // saturation |y| > 6 * 2^k1: the sign of lim - |y|, element 2q + 1 first
+            sats = (sats << 1) | ((lim - __float_as_uint(yhi)) >> 31);
+            sats = (sats << 1) | ((lim - __float_as_uint(ylo)) >> 31);
+        }
+        if (a.y)
+            st_stream(yp + 256 * h, make_uint4(ob[0], ob[1], ob[2], ob[3]));
+        if (a.codes)
+            *reinterpret_cast<uint32_t*>(cp + 128 * h) = e2m1x8(cv);
+        if (a.mask)
+            mp[32 * h] = (uint8_t)sats;
+        if ((lane & 3) == 0 && a.s1)
+            s1p[8 * h] = (uint8_t)qp_e8(p[h]);
+    }
+    if (lane == 0 && a.s0)
+        a.s0[row * a.nb0 + j] = s0;
+    return true;
+}
+
+// Each warp streams its units through a private ring of DL_STAGES 1 KB
+// stages in shared memory: every lane copies its own two 16-byte pieces of a
+// unit with cp.async, DL_STAGES - 1 units ahead of the one it works on, and
+// later reads back only what it copied itself, so no barrier is needed (a
+// lane's wait_group makes its own copies visible to it). The copies in flight
+// per SM no longer depend on how many registers the element work needs.
+constexpr int DL_STAGES = 4;
+
+__device__ __forceinline__ void dl_cp16(uint32_t saddr, const void* g)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
+}
+
+__device__ __forceinline__ void dl_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+__device__ __forceinline__ void dl_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(DL_STAGES - 1) : "memory"); }
+
 __global__ void __launch_bounds__(NTHREADS) dual_level_kernel(const DualArgs a)
 {
-    const int lane = threadIdx.x & 31;
+    __shared__ uint32_t s_lut[64];
+    __shared__ float2 s_s0r[128];  // (fl32(a0 / 6), fl32(1 / that)) for a0 = 1 + i / 128
+    __shared__ __align__(16) uint4 s_ring[NTHREADS / 32][DL_STAGES][64];
+    if (threadIdx.x < 64)
+        s_lut[threadIdx.x] = lut_entry(threadIdx.x);
+    if (threadIdx.x < 128) {
+        const float s0 = __fdiv_rn(__uint_as_float((0x3F80u + threadIdx.x) << 16), 6.0f);
+        s_s0r[threadIdx.x] = make_float2(s0, __frcp_rn(s0));
+    }
+    __syncthreads();
+    // table address of t = 2^21 + floor(4|y|) / 4: base + 4 (bits(t) - 0x4A000000)
+    const uint32_t lutb = (uint32_t)__cvta_generic_to_shared(s_lut) - 0x28000000u;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(&s_ring[warp][0][lane]);
+    // units u = row * nb0 + j, warp w takes u = w, w + nwarps, ...; (row, j)
+    // advance by (drow, dj) with a carry, so no division runs per unit
     const int64_t nwarps = (int64_t)gridDim.x * (NTHREADS / 32);
-    for (int64_t u = (int64_t)blockIdx.x * (NTHREADS / 32) + (threadIdx.x >> 5); u < a.units; u += nwarps) {
-        const int64_t row = u / a.nb0, j = u - row * a.nb0;
-        if (a.vec && (j + 1) * DL_BLOCK0 <= a.cols)
-            dual_unit<true>(a, row, j, lane);
-        else
-            dual_unit<false>(a, row, j, lane);
+    const int64_t u0 = (int64_t)blockIdx.x * (NTHREADS / 32) + warp;
+    const int64_t drow = nwarps / a.nb0, dj = nwarps - drow * a.nb0;
+    // units j < j_full are full and aligned: they take the ring and the fast path
+    const int64_t j_full = a.fast && a.vec ? a.cols / DL_BLOCK0 : 0;
+    auto advance = [&](int64_t& rr, int64_t& jj) {
+        rr += drow;
+        jj += dj;
+        if (jj >= a.nb0) {
+            jj -= a.nb0;
+            rr += 1;
+        }
+    };
+    auto issue = [&](int64_t rr, int64_t jj, int st) {
+        if (rr < a.rows && jj < j_full) {
+            const uint16_t* g = a.x + rr * a.ld + jj * DL_BLOCK0 + 8 * lane;
+            const uint32_t sa = ring + (uint32_t)st * 1024u;
+            dl_cp16(sa, g);
+            dl_cp16(sa + 512u, g + 256);
+        }
+        dl_commit();  // one group per unit, empty or not, so that the counting stays uniform
+    };
+    int64_t row = u0 / a.nb0, j = u0 - row * a.nb0;  // the unit worked on
+    int64_t rp = row, jp = j;                         // the next unit to copy
+#pragma unroll
+    for (int st = 0; st < DL_STAGES - 1; ++st) {
+        issue(rp, jp, st);
+        advance(rp, jp);
+    }
+    for (int st = 0; row < a.rows; st = st + 1 == DL_STAGES ? 0 : st + 1) {
+        issue(rp, jp, st == 0 ? DL_STAGES - 1 : st - 1);  // the stage used one unit ago
+        advance(rp, jp);
+        dl_wait();
+        bool done = false;
+        if (j < j_full) {
+            const uint32_t sa = ring + (uint32_t)st * 1024u;
+            uint32_t w[8];
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                         : "r"(sa));
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                         : "r"(sa + 512u));
+            done = dual_unit_fast(a, row, j, lane, w, lutb, s_s0r);
+        }
+        if (!done) {
+            if (a.vec && (j + 1) * DL_BLOCK0 <= a.cols)
+                dual_unit<true>(a, row, j, lane);
+            else
+                dual_unit<false>(a, row, j, lane);
+        }
+        advance(row, j);
     }
 }
 
@@ -245,6 +536,10 @@ static mxfp4_status run_dual_level(const mxfp4_dual_level_args* A, cudaStream_t 
     k.cstride = (A->cols + 1) / 2;
     k.mstride = (A->cols + 7) / 8;
     k.units = A->rows * k.nb0;
+    k.mul4 = 4;
+    k.mul16 = 65536;
+    k.fast = A->scale_mode == MXFP4_SCALE_FLOOR || page_fast_ok(A->scale_factor);
+    k.thr = A->scale_mode == MXFP4_SCALE_PAGE && k.fast ? page_threshold(A->scale_factor) : 0u;
     k.vec = aligned(A->x, 16) && A->ld % 8 == 0 && A->cols % 8 == 0 &&
             (!A->y || (aligned(A->y, 16) && A->ld_y % 8 == 0)) && (!A->codes || aligned(A->codes, 4));
     const int sms = device_sms();
