@@ -7,6 +7,11 @@
  * is compared with the IEEE quotient fl32(x / s0) wherever the kernel uses it
  * (|x| >= 2^-102 and |q| >= 2^-124); zeros and the remaining elements take
  * other routes there (+0, IEEE division). Prints "pairs N fast F bad B".
+ *
+ * Also checks the kernel's table for s0 and r: for every bf16 a0 >= 2^-65
+ * (exponent field >= 62), fl32(a0 / 6) and fl32(1 / s0) equal the entries
+ * computed for a0's significand at exponent 0, shifted by a0's exponent.
+ * Prints "table T table_bad B".
  * Built with -ffp-contract=off so that every product and fma is the one
  * written.
  */
@@ -51,5 +56,23 @@ int main(void)
         }
     }
     printf("pairs %lld fast %lld bad %lld\n", pairs, fast, bad);
+
+    long long table = 0, table_bad = 0;
+    for (uint32_t ab = 62u << 7; ab < 0x7F80u; ++ab) {
+        const float a0 = f_of(ab << 16);
+        const float s0 = a0 / 6.0f, r = 1.0f / s0;
+        const float t_s0 = f_of((0x3F80u + (ab & 0x7Fu)) << 16) / 6.0f;
+        const float t_r = 1.0f / t_s0;
+        const int e = (int)(ab >> 7) - 127;
+        uint32_t us0, ur, uts0, utr;
+        memcpy(&us0, &s0, 4);
+        memcpy(&ur, &r, 4);
+        memcpy(&uts0, &t_s0, 4);
+        memcpy(&utr, &t_r, 4);
+        ++table;
+        if (us0 != uts0 + ((uint32_t)e << 23) || ur != utr - ((uint32_t)e << 23))
+            ++table_bad;
+    }
+    printf("table %lld table_bad %lld\n", table, table_bad);
     return 0;
 }

@@ -7,7 +7,9 @@ one fma correction where that is exact, and falls back to the IEEE division
 elsewhere. dual_level_division_check.c replays those steps in C for every
 pair of a bf16 level-0 amax and a bf16 element of a block it can head, with
 both signs, and counts the pairs where the corrected product differs from
-x / s0 in any bit; the count must be zero."""
+x / s0 in any bit; the count must be zero. It also checks the kernel's
+table for s0 = fl32(a0 / 6) and fl32(1 / s0): the entries for a0's
+significand at exponent 0, shifted by a0's exponent, for every a0 >= 2^-65."""
 from __future__ import annotations
 
 import os
@@ -27,3 +29,4 @@ def test_corrected_reciprocal_product_is_the_ieee_quotient(tmp_path):
     assert got["pairs"] == 2 * sum(range(1, 0x7F80)), got  # every (a0, x) pair with 0 < |x| <= a0
     assert got["fast"] > got["pairs"] // 2, got            # the corrected product covers most pairs
     assert got["bad"] == 0, got
+    assert got["table"] == 0x7F80 - (62 << 7) and got["table_bad"] == 0, got
