@@ -382,6 +382,7 @@ mxfp4_status mxfp4_grouped_gemm(const mxfp4_gmm_args* args, mxfp4_stream_t strea
  * Arguments (zero-initialise; NULL outputs are skipped):
  *   x            bf16 [rows][cols], leading dimension ld (>= cols) elements.
  *   dtype        MXFP4_BF16 (anything else: MXFP4_EUNSUPPORTED).
+ *   rows, cols   >= 0 and below 2^30 (else MXFP4_EUNSUPPORTED).
  *   level0_block 512 (other positive multiples of 32: MXFP4_EUNSUPPORTED;
  *                anything else MXFP4_EINVAL).
  *   scale_factor, scale_mode  the level-1 scale rule, as for mxfp4_qdq_fwd.

@@ -269,10 +269,11 @@ __device__ __forceinline__ float dl_quot(float x, float s0, float r, float tf)
     return __fdiv_rn(x, s0) + 0.0f;
 }
 
-// Fast path of one full, aligned unit whose 16 bf16 pairs are w (w[0..3]:
-// elements 8 lane .. 8 lane + 7 of the first half, w[4..7] of the second).
-// Returns false, having stored nothing, when the unit needs dual_unit; the
-// decision is uniform across the warp.
+// Fast path of one full, aligned unit. The lane holds w = elements
+// 16 lane .. 16 lane + 15 of the unit (8 bf16 pairs): half of one level-1
+// block, whose other half is the neighbouring lane. Returns false, having
+// stored nothing, when the unit needs dual_unit; the decision is uniform
+// across the warp.
 //
 // s0 = fl32(a0 / 6) and r = fl32(1 / s0) come from a table over the seven
 // significand bits of the bf16 amax a0 (entries for a0 in [1, 2)), shifted by
@@ -286,28 +287,27 @@ __device__ __forceinline__ float dl_quot(float x, float s0, float r, float tf)
 // is 1/4 (y 2^-k1 is exact: 2^-k1 >= 1 on this path, and |y 2^-k1| < 16);
 // the table entry at that index is the code magnitude. Elements whose y is
 // zero (x = +-0, or a quotient that underflows) get a +0 code, as sign(y) = 0
-// there.
-__device__ __forceinline__ bool dual_unit_fast(const DualArgs& a, int64_t row, int64_t j, int lane,
-                                               const uint32_t (&w)[8], uint32_t lutb, const float2* s0r)
+// there. The output is (code * A) * B with (A, B) = (2^k1 s0, 1) when that
+// product is a normal number (so exact), else (2^k1, s0).
+__device__ __forceinline__ bool dual_unit_fast(const DualArgs& a, int row, int j, int lane, const uint32_t (&w)[8],
+                                               uint32_t lutb, const float2* s0r)
 {
-    uint32_t aw[8], mh[2] = {0u, 0u}, mn = 0x7FFF7FFFu;
+    uint32_t aw[8], m = 0u, mn = 0x7FFF7FFFu;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         aw[i] = w[i] & 0x7FFF7FFFu;
-        mh[i >> 2] = vmax2(mh[i >> 2], aw[i]);
+        m = vmax2(m, aw[i]);
         mn = vmin2(mn, aw[i]);
     }
-    // level-1 blocks are four lanes of a half: both halves' maxima in one word
-    uint32_t P = __byte_perm(max(mh[0] & 0xFFFFu, mh[0] >> 16), max(mh[1] & 0xFFFFu, mh[1] >> 16), 0x5410);
-    P = vmax2(P, __shfl_xor_sync(FULL, P, 1));
-    P = vmax2(P, __shfl_xor_sync(FULL, P, 2));
-    const uint32_t A0 = __reduce_max_sync(FULL, max(P & 0xFFFFu, P >> 16));
+    uint32_t mb = max(m & 0xFFFFu, m >> 16);
+    mb = max(mb, __shfl_xor_sync(FULL, mb, 1));  // the level-1 block's max |x| (bf16 bits)
+    const uint32_t A0 = __reduce_max_sync(FULL, mb);
     if (A0 >= 0x7F80u || A0 < 0x1F00u)  // non-finite, or a0 < 2^-65 (tiny or all-zero block)
         return false;
     const float2 t0 = s0r[A0 & 0x7Fu];
-    const int e0 = (int)(A0 >> 7) - 127;
-    const float s0 = __uint_as_float(__float_as_uint(t0.x) + ((uint32_t)e0 << 23));
-    const float r = __uint_as_float(__float_as_uint(t0.y) - ((uint32_t)e0 << 23));
+    const uint32_t esh = ((A0 >> 7) - 127u) << 23;
+    const float s0 = __uint_as_float(__float_as_uint(t0.x) + esh);
+    const float r = __uint_as_float(__float_as_uint(t0.y) - esh);
     // |x| >= tf meets both conditions under which the corrected reciprocal
     // product is the IEEE quotient (|x| >= 2^-102, |x r| >= 2^-124); s0 2^-123
     // is exact whenever it exceeds 2^-102. tb: tf rounded up to bf16 bits.
@@ -316,18 +316,11 @@ __device__ __forceinline__ bool dual_unit_fast(const DualArgs& a, int64_t row, i
     // a lane with an |x| below tf (zeros included) checks its elements one by one
     const bool lane_slow = min(mn & 0xFFFFu, mn >> 16) < tb;
 
-    QP p[2];
-    bool big = false, exact = true;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const float yamax = dl_quot(__uint_as_float(h ? P & 0xFFFF0000u : P << 16), s0, r, tf);
-        p[h] = qparams(__float_as_uint(yamax), a.mode, a.thr);
-        big = big || !(p[h].inv >= 1.0f);
-        exact = exact && p[h].scale * s0 >= 0x1p-126f;  // 2^k1 s0 normal, hence exact
-    }
-    if (__any_sync(FULL, big))  // a level-1 scale above 1: y * 2^-k1 may round
+    const QP p = qparams(__float_as_uint(dl_quot(__uint_as_float(mb << 16), s0, r, tf)), a.mode, a.thr);
+    if (__any_sync(FULL, !(p.inv >= 1.0f)))  // a level-1 scale above 1: y * 2^-k1 may round
         return false;
-    exact = __all_sync(FULL, exact);
+    const float S = p.scale * s0;
+    const bool exact = S >= 0x1p-126f;  // 2^k1 s0 normal, hence exact
 
     const u64 R2 = pk2(r, r), NS2 = pk2(-s0, -s0);
     u64 Y[8];
@@ -359,63 +352,56 @@ __device__ __forceinline__ bool dual_unit_fast(const DualArgs& a, int64_t row, i
         }
     }
 
-    const int64_t c0 = j * DL_BLOCK0;
-    const int64_t cl = c0 + 8 * lane;
-    uint16_t* yp = a.y + row * a.ld_y + cl;
-    uint8_t* cp = a.codes + row * a.cstride + cl / 2;
-    uint8_t* mp = a.mask + row * a.mstride + cl / 8;
-    uint8_t* s1p = a.s1 + row * a.nb1 + c0 / 32 + (lane >> 2);
+    const u64 INV2 = pk2(p.inv, p.inv);
+    const u64 A2 = exact ? pk2(S, S) : pk2(p.scale, p.scale);
+    const u64 B2 = exact ? pk2(1.0f, 1.0f) : pk2(s0, s0);
+    const uint32_t lim = __float_as_uint(p.scale * 6.0f);  // exact: 2^k1 >= 2^-127
+    uint32_t ob[8], sats = 0;
+    float cv[16];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const u64 INV2 = pk2(p[h].inv, p[h].inv);
-        const float S = p[h].scale * s0;
-        const u64 A2 = exact ? pk2(S, S) : pk2(p[h].scale, p[h].scale);
-        const u64 B2 = pk2(s0, s0);
-        const uint32_t lim = __float_as_uint(p[h].scale * 6.0f);  // exact: 2^k1 >= 2^-127
-        uint32_t ob[4], sats = 0;
-        float cv[8];
-#pragma unroll
-        for (int q = 3; q >= 0; --q) {
-            const int i = 4 * h + q;
-            float ylo, yhi;
-            upk2(Y[i], ylo, yhi);
-            float tlo, thi;
-            upk2(fma2_rm(Y[i], INV2, pk2(2097152.0f, 2097152.0f)), tlo, thi);
-            uint32_t elo, ehi;
-            asm("ld.shared.u32 %0, [%1];" : "=r"(elo) : "r"(__float_as_uint(tlo) * a.mul4 + lutb));
-            asm("ld.shared.u32 %0, [%1];" : "=r"(ehi) : "r"(__float_as_uint(thi) * a.mul4 + lutb));
-            cv[2 * q] = __uint_as_float(elo | ((sg[i] << 16) & 0x80000000u));
-            cv[2 * q + 1] = __uint_as_float(ehi | (sg[i] & 0x80000000u));
-            u64 O = mul2(pk2(cv[2 * q], cv[2 * q + 1]), A2);
-            if (!exact)
-                O = mul2(O, B2);
-            float olo, ohi;
-            upk2(O, olo, ohi);
-            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(ob[q]) : "f"(ohi), "f"(olo));
-            // saturation |y| > 6 * 2^k1: the sign of lim - |y|, element 2q + 1 first
-            sats = (sats << 1) | ((lim - __float_as_uint(yhi)) >> 31);
-            sats = (sats << 1) | ((lim - __float_as_uint(ylo)) >> 31);
-        }
-        if (a.y)
-            st_stream(yp + 256 * h, make_uint4(ob[0], ob[1], ob[2], ob[3]));
-        if (a.codes)
-            *reinterpret_cast<uint32_t*>(cp + 128 * h) = e2m1x8(cv);
-        if (a.mask)
-            mp[32 * h] = (uint8_t)sats;
-        if ((lane & 3) == 0 && a.s1)
-            s1p[8 * h] = (uint8_t)qp_e8(p[h]);
+    for (int i = 7; i >= 0; --i) {
+        float ylo, yhi;
+        upk2(Y[i], ylo, yhi);
+        float tlo, thi;
+        upk2(fma2_rm(Y[i], INV2, pk2(2097152.0f, 2097152.0f)), tlo, thi);
+        uint32_t elo, ehi;
+        asm("ld.shared.u32 %0, [%1];" : "=r"(elo) : "r"(__float_as_uint(tlo) * a.mul4 + lutb));
+        asm("ld.shared.u32 %0, [%1];" : "=r"(ehi) : "r"(__float_as_uint(thi) * a.mul4 + lutb));
+        cv[2 * i] = __uint_as_float(elo | ((sg[i] * a.mul16) & 0x80000000u));
+        cv[2 * i + 1] = __uint_as_float(ehi | (sg[i] & 0x80000000u));
+        float olo, ohi;
+        upk2(mul2(mul2(pk2(cv[2 * i], cv[2 * i + 1]), A2), B2), olo, ohi);
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(ob[i]) : "f"(ohi), "f"(olo));
+        // saturation |y| > 6 * 2^k1: the sign of lim - |y|, element 2i + 1 first
+        sats = (sats << 1) | ((lim - __float_as_uint(yhi)) >> 31);
+        sats = (sats << 1) | ((lim - __float_as_uint(ylo)) >> 31);
     }
+    const int64_t c = (int64_t)j * DL_BLOCK0 + 16 * lane;
+    if (a.y) {
+        uint16_t* yp = a.y + (int64_t)row * a.ld_y + c;
+        st_stream(yp, make_uint4(ob[0], ob[1], ob[2], ob[3]));
+        st_stream(yp + 8, make_uint4(ob[4], ob[5], ob[6], ob[7]));
+    }
+    if (a.codes) {
+        const float (&c0)[8] = *reinterpret_cast<const float(*)[8]>(&cv[0]);
+        const float (&c1)[8] = *reinterpret_cast<const float(*)[8]>(&cv[8]);
+        *reinterpret_cast<uint2*>(a.codes + (int64_t)row * a.cstride + c / 2) = make_uint2(e2m1x8(c0), e2m1x8(c1));
+    }
+    if (a.mask)
+        *reinterpret_cast<uint16_t*>(a.mask + (int64_t)row * a.mstride + c / 8) = (uint16_t)sats;
+    if ((lane & 1) == 0 && a.s1)
+        a.s1[(int64_t)row * a.nb1 + c / 32] = (uint8_t)qp_e8(p);
     if (lane == 0 && a.s0)
-        a.s0[row * a.nb0 + j] = s0;
+        a.s0[(int64_t)row * a.nb0 + j] = s0;
     return true;
 }
 
 // Each warp streams its units through a private ring of DL_STAGES 1 KB
-// stages in shared memory: every lane copies its own two 16-byte pieces of a
-// unit with cp.async, DL_STAGES - 1 units ahead of the one it works on, and
-// later reads back only what it copied itself, so no barrier is needed (a
-// lane's wait_group makes its own copies visible to it). The copies in flight
-// per SM no longer depend on how many registers the element work needs.
+// stages in shared memory: every lane copies its own 32 bytes of a unit with
+// cp.async, DL_STAGES - 1 units ahead of the one it works on, and later reads
+// back only what it copied itself, so no barrier is needed (a lane's
+// wait_group makes its own copies visible to it). The copies in flight per SM
+// no longer depend on how many registers the element work needs.
 constexpr int DL_STAGES = 4;
 
 __device__ __forceinline__ void dl_cp16(uint32_t saddr, const void* g)
@@ -442,39 +428,42 @@ __global__ void __launch_bounds__(NTHREADS) dual_level_kernel(const DualArgs a)
     // table address of t = 2^21 + floor(4|y|) / 4: base + 4 (bits(t) - 0x4A000000)
     const uint32_t lutb = (uint32_t)__cvta_generic_to_shared(s_lut) - 0x28000000u;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(&s_ring[warp][0][lane]);
-    // units u = row * nb0 + j, warp w takes u = w, w + nwarps, ...; (row, j)
-    // advance by (drow, dj) with a carry, so no division runs per unit
+    const uint32_t ring = (uint32_t)__cvta_generic_to_shared(&s_ring[warp][0][2 * lane]);
+    // units u = row * nb0 + j (rows and nb0 below 2^30, host-checked); warp w
+    // takes u = w, w + nwarps, ...; (row, j) advance by (drow, dj) with a carry
+    const int nb0 = (int)a.nb0, rows = (int)a.rows;
     const int64_t nwarps = (int64_t)gridDim.x * (NTHREADS / 32);
     const int64_t u0 = (int64_t)blockIdx.x * (NTHREADS / 32) + warp;
-    const int64_t drow = nwarps / a.nb0, dj = nwarps - drow * a.nb0;
+    const int drow = (int)(nwarps / nb0), dj = (int)(nwarps % nb0);
     // units j < j_full are full and aligned: they take the ring and the fast path
-    const int64_t j_full = a.fast && a.vec ? a.cols / DL_BLOCK0 : 0;
-    auto advance = [&](int64_t& rr, int64_t& jj) {
+    const int j_full = a.fast && a.vec ? (int)(a.cols / DL_BLOCK0) : 0;
+    auto advance = [&](int& rr, int& jj) {
         rr += drow;
         jj += dj;
-        if (jj >= a.nb0) {
-            jj -= a.nb0;
+        if (jj >= nb0) {
+            jj -= nb0;
             rr += 1;
         }
     };
-    auto issue = [&](int64_t rr, int64_t jj, int st) {
-        if (rr < a.rows && jj < j_full) {
-            const uint16_t* g = a.x + rr * a.ld + jj * DL_BLOCK0 + 8 * lane;
+    auto issue = [&](int rr, int jj, int st) {
+        if (rr < rows && jj < j_full) {
+            const uint16_t* g = a.x + (int64_t)rr * a.ld + jj * DL_BLOCK0 + 16 * lane;
             const uint32_t sa = ring + (uint32_t)st * 1024u;
             dl_cp16(sa, g);
-            dl_cp16(sa + 512u, g + 256);
+            dl_cp16(sa + 16u, g + 8);
         }
         dl_commit();  // one group per unit, empty or not, so that the counting stays uniform
     };
-    int64_t row = u0 / a.nb0, j = u0 - row * a.nb0;  // the unit worked on
-    int64_t rp = row, jp = j;                         // the next unit to copy
+    int row = (int)(u0 / nb0), j = (int)(u0 % nb0);  // the unit worked on (u0 < rows * nb0 when row < rows)
+    int rp = row, jp = j;                            // the next unit to copy
+    if (u0 >= (int64_t)rows * nb0)
+        return;
 #pragma unroll
     for (int st = 0; st < DL_STAGES - 1; ++st) {
         issue(rp, jp, st);
         advance(rp, jp);
     }
-    for (int st = 0; row < a.rows; st = st + 1 == DL_STAGES ? 0 : st + 1) {
+    for (int st = 0; row < rows; st = st + 1 == DL_STAGES ? 0 : st + 1) {
         issue(rp, jp, st == 0 ? DL_STAGES - 1 : st - 1);  // the stage used one unit ago
         advance(rp, jp);
         dl_wait();
@@ -487,11 +476,11 @@ __global__ void __launch_bounds__(NTHREADS) dual_level_kernel(const DualArgs a)
                          : "r"(sa));
             asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-                         : "r"(sa + 512u));
+                         : "r"(sa + 16u));
             done = dual_unit_fast(a, row, j, lane, w, lutb, s_s0r);
         }
         if (!done) {
-            if (a.vec && (j + 1) * DL_BLOCK0 <= a.cols)
+            if (a.vec && (int64_t)(j + 1) * DL_BLOCK0 <= a.cols)
                 dual_unit<true>(a, row, j, lane);
             else
                 dual_unit<false>(a, row, j, lane);
@@ -512,7 +501,7 @@ static mxfp4_status run_dual_level(const mxfp4_dual_level_args* A, cudaStream_t 
         return MXFP4_EINVAL;
     if (A->scale_mode != MXFP4_SCALE_PAGE && A->scale_mode != MXFP4_SCALE_FLOOR)
         return MXFP4_EINVAL;
-    if (A->dtype != MXFP4_BF16 || A->level0_block != DL_BLOCK0)
+    if (A->dtype != MXFP4_BF16 || A->level0_block != DL_BLOCK0 || A->rows >= (1 << 30) || A->cols >= (1 << 30))
         return MXFP4_EUNSUPPORTED;
     if (A->rows == 0 || A->cols == 0)
         return MXFP4_OK;
@@ -540,8 +529,11 @@ static mxfp4_status run_dual_level(const mxfp4_dual_level_args* A, cudaStream_t 
     k.mul16 = 65536;
     k.fast = A->scale_mode == MXFP4_SCALE_FLOOR || page_fast_ok(A->scale_factor);
     k.thr = A->scale_mode == MXFP4_SCALE_PAGE && k.fast ? page_threshold(A->scale_factor) : 0u;
-    k.vec = aligned(A->x, 16) && A->ld % 8 == 0 && A->cols % 8 == 0 &&
-            (!A->y || (aligned(A->y, 16) && A->ld_y % 8 == 0)) && (!A->codes || aligned(A->codes, 4));
+    // full units take 16-byte loads and y stores, 8-byte code stores and
+    // 2-byte mask stores
+    k.vec = aligned(A->x, 16) && A->ld % 8 == 0 && A->cols % 16 == 0 &&
+            (!A->y || (aligned(A->y, 16) && A->ld_y % 8 == 0)) && (!A->codes || aligned(A->codes, 8)) &&
+            (!A->mask || aligned(A->mask, 2));
     const int sms = device_sms();
     const int occ = occupancy((const void*)dual_level_kernel, 0);
     if (sms <= 0 || occ <= 0)

@@ -223,7 +223,7 @@ def _dual(abi, **kw):
     (dict(scale_factor=float("nan")), 1), (dict(scale_factor=float("inf")), 1), (dict(scale_mode=2), 1),
     (dict(dtype=0), 2), (dict(level0_block=256), 2), (dict(level0_block=1024), 2),
     (dict(x=None), 1), (dict(ld=1000), 1), (dict(y=8192, ld_y=1000), 1),
-    (dict(rows=0), 0), (dict(cols=0, x=None), 0),
+    (dict(rows=0), 0), (dict(cols=0, x=None), 0), (dict(rows=2 ** 30), 2), (dict(cols=2 ** 30, ld=2 ** 30), 2),
 ])
 def test_dual_level_rejects_bad_arguments_on_host(abi, kw, expected):
     assert abi.mxfp4_dual_level_qdq(_dual(abi, **kw), None) == expected
