@@ -76,7 +76,7 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 template <bool VEC>
-__device__ __noinline__ void dual_unit(const DualArgs& a, int64_t row, int64_t j, int lane)
+__device__ __forceinline__ void dual_unit(const DualArgs& a, int64_t row, int64_t j, int lane)
 {
     const int64_t c0 = j * DL_BLOCK0;
     const uint16_t* xr = a.x + row * a.ld;
