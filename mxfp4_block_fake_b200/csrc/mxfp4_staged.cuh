@@ -1407,7 +1407,8 @@ __global__ void __launch_bounds__(NTHREADS) ste_row_kernel(const KArgs a)
 
 // ---------------------------------------------------------------------------
 // Row-wise bf16 block 32, one streaming pass: one thread per block, two
-// 32-byte loads, amax, k, the codes by the nudged hardware convert, then the
+// 32-byte loads (the next block's issued before this block is worked on),
+// amax, k, the codes by the nudged hardware convert, then the
 // outputs asked for: dequantised values (VALS: two 32-byte streaming
 // stores), one 16-byte code store, one 4-byte mask word and one scale byte
 // (SMMA: in the MMA layout). Without values this is the real-quantisation
@@ -1443,12 +1444,23 @@ __global__ void __launch_bounds__(NTHREADS) row_stream_kernel(const KArgs a)
         s_lut[threadIdx.x] = lut_entry(threadIdx.x);
     __syncthreads();
     const uint32_t glutb = smem_addr(s_lut) - 0x2C000000u;
-    for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < total; u += gridDim.x * blockDim.x) {
+    const uint32_t stride = gridDim.x * blockDim.x;
+    auto load = [&](uint32_t uu, uint32_t (&ww)[16]) {
+        const uint32_t rr = uu / nb, bb = uu - rr * nb;
+        const char* xp = static_cast<const char*>(a.x) + ((int64_t)rr * a.ld + 32 * bb) * 2;
+        ld_nc_v8(xp, ww);
+        ld_nc_v8(xp + 32, ww + 8);
+    };
+    uint32_t w[16];
+    uint32_t u = blockIdx.x * blockDim.x + threadIdx.x;
+    if (u < total)
+        load(u, w);
+    for (; u < total; u += stride) {
         const uint32_t row = u / nb, blk = u - row * nb;
-        const char* xp = static_cast<const char*>(a.x) + ((int64_t)row * a.ld + 32 * blk) * 2;
-        uint32_t w[16];
-        ld_nc_v8(xp, w);
-        ld_nc_v8(xp + 32, w + 8);
+        uint32_t wn[16];
+        const bool more = u + stride < total;
+        if (more)
+            load(u + stride, wn);  // the next block's loads are in flight while this one is worked on
         uint32_t m2 = 0;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -1499,12 +1511,18 @@ __global__ void __launch_bounds__(NTHREADS) row_stream_kernel(const KArgs a)
             *reinterpret_cast<uint32_t*>(a.mask_row + (int64_t)row * (a.cols / 8) + 4 * blk) = sats;
         if (a.scales_row)
             a.scales_row[SMMA ? srow_off_mma(row, blk, nb) : (int64_t)row * nb + blk] = (uint8_t)e8;
+        if (more) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                w[i] = wn[i];
+        }
     }
 }
 
 // ---------------------------------------------------------------------------
 // MXFP8 row-wise, bf16, block 32, one streaming pass: one thread per block,
-// two 32-byte loads, amax and k (floor(log2 amax) - 8, at least -127), per
+// two 32-byte loads (the next block's issued before this block is worked
+// on), amax and k (floor(log2 amax) - 8, at least -127), per
 // pair of elements one E4M3 convert (nearest even, saturating at 448) and one
 // back to exact f16 codes, widened and multiplied by 2^k (exact), then the
 // outputs asked for: two 32-byte stores of values, one 32-byte store of codes,
@@ -1517,12 +1535,23 @@ __global__ void __launch_bounds__(NTHREADS) row_stream8_kernel(const KArgs a)
 {
     const uint32_t nb = (uint32_t)(a.cols / 32);
     const uint32_t total = (uint32_t)a.rows * nb;
-    for (uint32_t u = blockIdx.x * blockDim.x + threadIdx.x; u < total; u += gridDim.x * blockDim.x) {
+    const uint32_t stride = gridDim.x * blockDim.x;
+    auto load = [&](uint32_t uu, uint32_t (&ww)[16]) {
+        const uint32_t rr = uu / nb, bb = uu - rr * nb;
+        const char* xp = static_cast<const char*>(a.x) + ((int64_t)rr * a.ld + 32 * bb) * 2;
+        ld_nc_v8(xp, ww);
+        ld_nc_v8(xp + 32, ww + 8);
+    };
+    uint32_t w[16];
+    uint32_t u = blockIdx.x * blockDim.x + threadIdx.x;
+    if (u < total)
+        load(u, w);
+    for (; u < total; u += stride) {
         const uint32_t row = u / nb, blk = u - row * nb;
-        const char* xp = static_cast<const char*>(a.x) + ((int64_t)row * a.ld + 32 * blk) * 2;
-        uint32_t w[16];
-        ld_nc_v8(xp, w);
-        ld_nc_v8(xp + 32, w + 8);
+        uint32_t wn[16];
+        const bool more = u + stride < total;
+        if (more)
+            load(u + stride, wn);  // the next block's loads are in flight while this one is worked on
         uint32_t m2 = 0;
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -1582,6 +1611,11 @@ __global__ void __launch_bounds__(NTHREADS) row_stream8_kernel(const KArgs a)
             *reinterpret_cast<uint32_t*>(a.mask_row + (int64_t)row * (a.cols / 8) + 4 * blk) = sats;
         if (a.scales_row)
             a.scales_row[SMMA ? srow_off_mma(row, blk, nb) : (int64_t)row * nb + blk] = (uint8_t)e8;
+        if (more) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                w[i] = wn[i];
+        }
     }
 }
 
