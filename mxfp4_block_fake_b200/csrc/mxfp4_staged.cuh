@@ -887,15 +887,17 @@ __global__ void __launch_bounds__(SG_THREADS, 2) qdq_staged_kernel(const __grid_
 //   * row pass: warp w owns tile rows 8w..8w+7; lanes 0-15 take the first
 //     half of each row's block (slab 0), lanes 16-31 the second (slab 1),
 //     32 elements per lane; the row amax takes two shuffles (xor 1, 16).
-// Inputs arrive as two 64 x 128 TMA boxes per tile (128-byte swizzle).
-// Row-wise y is written over the tile's own stage; the other outputs go to
-// one of two staging buffers (codes with the 64-byte swizzle, masks as
-// 16-byte rows) and leave by TMA stores, issued by the producer warp once the
-// compute warps have released the tile (one arrival each on its stage's
-// "empty" mbarrier); the producer warp also copies the row-wise scales and
-// the group-tail column-wise outputs, and once the stores of the tile before
-// have read their sources, releases that staging buffer ("sfree") and
-// refills its stage. One barrier among the compute warps per tile (named
+// Inputs arrive as two 64 x 128 TMA boxes per tile (128-byte swizzle), four
+// stages deep. Row-wise y is written over the tile's own stage; row-wise codes
+// go straight from registers to global memory (a lane's 32 elements are 16
+// contiguous code bytes of its row), which leaves room for the fourth stage;
+// the other outputs go to one of two staging buffers (column-wise codes with
+// the 64-byte swizzle, masks as 16-byte rows) and leave by TMA stores, issued
+// by the producer warp once the compute warps have released the tile (one
+// arrival each on its stage's "empty" mbarrier); the producer warp also
+// copies the row-wise scales and the group-tail column-wise outputs, and once
+// the stores of the tile before have read their sources, releases that
+// staging buffer ("sfree") and refills its stage. One barrier among the compute warps per tile (named
 // barrier 1): every column pass has read its words from the stage (which
 // the row pass then overwrites with y) and published its column limits.
 // ---------------------------------------------------------------------------
@@ -905,7 +907,7 @@ constexpr int SB_SLAB_BYTES = SG_SLAB_COLS * 2 * SB_ROWS;  // 16384
 constexpr int SB_TILE_BYTES = 2 * SB_SLAB_BYTES;           // 32768
 constexpr int SB_CODE_BYTES = SB_ROWS * SB_COLS / 2;       // 8192: 64-byte rows
 constexpr int SB_MASK_WORDS = SB_ROWS * SB_COLS / 32;      // 512: 16-byte rows
-constexpr int SB_STAGES = 3;
+constexpr int SB_STAGES = 4;
 constexpr int SB_COMPUTE_WARPS = 16;
 constexpr int SB_COMPUTE = 32 * SB_COMPUTE_WARPS;      // 512
 constexpr int SB_THREADS = SB_COMPUTE + 32;           // + the producer warp
@@ -914,7 +916,6 @@ constexpr int SB_PRODUCER = SB_COMPUTE_WARPS;
 struct __align__(1024) StagedOut128 {
     uint8_t ycol[SB_TILE_BYTES];
     uint8_t ccol[SB_CODE_BYTES];
-    uint8_t crow[SB_CODE_BYTES];
     uint32_t mcol[SB_MASK_WORDS];
     uint32_t mrow[SB_MASK_WORDS];
     uint8_t srow[SB_ROWS];  // row-wise scale byte of each tile row
@@ -957,8 +958,6 @@ __device__ __forceinline__ void copy_outputs128(const KArgs& a, const StagedOut1
             st_stream(static_cast<char*>(a.y_row) + (row * a.ld_y + col) * 2, sm_ld128(yrow, yoff));
         if (which & SG_TS_CODES)
             *reinterpret_cast<uint32_t*>(a.codes_col + row * cstride + col / 2) = sm_ld32(o.ccol, coff);
-        if (which & SG_TS_CODES_R)
-            *reinterpret_cast<uint32_t*>(a.codes_row + row * cstride + col / 2) = sm_ld32(o.crow, coff);
         if (which & SG_TS_MASK)
             a.mask_col[row * mstride + col / 8] = reinterpret_cast<const uint8_t*>(o.mcol)[r * 16 + u];
         if (which & SG_TS_MASK_R)
@@ -1027,7 +1026,7 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
     const uint32_t col_out = COL ? (a.y_col ? SG_TS_Y : 0u) | (a.codes_col ? SG_TS_CODES : 0u) |
                                        (a.mask_col ? SG_TS_MASK : 0u)
                                  : 0u;
-    const uint32_t row_out = (ROW && a.y_row ? SG_TS_YR : 0u) | (ROW && a.codes_row ? SG_TS_CODES_R : 0u) |
+    const uint32_t row_out = (ROW && a.y_row ? SG_TS_YR : 0u) |
                              (ROW && a.mask_row ? SG_TS_MASK_R : 0u);
     uint32_t issued = 0;  // producer lane 0: tiles whose load was issued
 
@@ -1077,8 +1076,6 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
                 }
                 if (st & SG_TS_CODES)
                     tma_store_box(&maps.codes, smem_addr(o.ccol), col0 / 2, row0);
-                if (st & SG_TS_CODES_R)
-                    tma_store_box(&maps.codes_r, smem_addr(o.crow), col0 / 2, row0);
                 if (st & SG_TS_MASK)
                     tma_store_box(&maps.mask, smem_addr(o.mcol), col0 / 8, row0);
                 if (st & SG_TS_MASK_R)
@@ -1121,7 +1118,6 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj)
             ro[jj] = (uint32_t)hq * SB_SLAB_BYTES + rr * 128 + ((uint32_t)((4 * (q & 1) + jj) ^ (rr & 7)) << 4);
-        const uint32_t rco = rr * 64 + (((uint32_t)q ^ (uint32_t)((rr >> 1) & 3)) << 4);
         const int rw = rr * 4 + q;  // mask word of (row rr, columns 32q..32q+31)
 
         for (uint32_t j = 0; j < n; ++j) {
@@ -1303,7 +1299,20 @@ __global__ void __launch_bounds__(SB_THREADS, 1) qdq_staged128_kernel(const __gr
                             sats |= gch.sats << (8 * jj);
                         }
                     }
-                    *reinterpret_cast<uint4*>(out.crow + rco) = make_uint4(nib[0], nib[1], nib[2], nib[3]);
+                    if (a.codes_row && (int64_t)row0 + rr < a.rows) {
+                        // row-wise codes straight from registers: the lane's 32
+                        // elements are 16 contiguous code bytes of its row
+                        const int gcol = col0 + 32 * q;
+                        uint8_t* cp = a.codes_row + ((int64_t)row0 + rr) * (a.cols / 2) + gcol / 2;
+                        if (gcol + 32 <= a.cols && (a.ts_flags & SG_TS_CODES_R)) {
+                            st_stream(cp, make_uint4(nib[0], nib[1], nib[2], nib[3]));
+                        } else {
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj)
+                                if (gcol + 8 * jj < a.cols)
+                                    *reinterpret_cast<uint32_t*>(cp + 4 * jj) = nib[jj];
+                        }
+                    }
                     out.mrow[rw] = sats;
                     if (q == 0)
                         out.srow[rr] = (uint8_t)(rfast ? (uint32_t)(k + 127) : e8_of(A, k));
