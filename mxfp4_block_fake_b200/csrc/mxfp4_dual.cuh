@@ -10,29 +10,28 @@
 // of 32; the output is fl32(code 2^k1 s0) in bf16. A level-0 block holding a
 // NaN or an infinity is written as NaN (code 0, E8M0 0xFF, s0 NaN).
 //
-// Work layout: a warp owns one level-0 block of a row (a "unit"). Lane l
-// holds elements 8l..8l+7 of each 256-element half, so each of the warp's two
-// 16-byte loads (and the 16-byte stores of y) covers 512 contiguous bytes, and
-// a level-1 block of 32 is four neighbouring lanes of one half. Per unit:
-// level-0 amax by one warp reduction, s0 and its reciprocal, y = x / s0 by a
-// corrected reciprocal product, the level-1 amax by two shuffles, then the
-// codes and outputs. Grid-stride over units, consecutive warps on
-// consecutive units, so that the grid streams through memory in order; a
-// warp copies its next units into shared memory while it works on the
+// Work layout: a warp owns one level-0 block of a row (a "unit", 1 KB of
+// bf16). Grid-stride over units, consecutive warps on consecutive units, so
+// that the grid streams through memory in order; each warp copies its next
+// units into a private shared-memory ring (cp.async) while it works on the
 // current one.
 //
-// Two element paths. The fast path (full, aligned units whose level-1
-// scales are at most 1, which covers every block at the default scale
-// factor 6) works on element pairs with the packed fp32 instructions:
-// y = x / s0 (dl_div's steps), y1 = y * 2^-k1 (exact, as 2^-k1 >= 1),
-// floor(4 |y1|) by one fma rounding down into 2^23, the code magnitude from a
-// 64-entry shared table, the sign of y1 (never -0 here), the E2M1 nibbles by
-// the hardware convert of the exact signed codes, and the output
-// fl32(code * 2^k1 * s0) as one multiply by S = 2^k1 s0 when S is exact (a
-// normal number), else as two. It stores nothing before it has decided to
-// handle the unit. The general path (dual_unit) takes every other unit:
-// ragged or unaligned ones, non-finite or tiny level-0 blocks, level-1
-// scales above 1 (small PAGE scale factors).
+// Two element paths. The fast path (dual_unit_fast: full, aligned units
+// whose level-1 scales are at most 1, which covers every block at the default
+// scale factor 6) gives lane l the 16 consecutive elements 16l..16l+15, half
+// of one level-1 block (the other half is lane l ^ 1): the level-0 amax is a
+// packed 16-bit max, one shuffle and one warp reduction; s0 and 1/s0 come
+// from a table; y = |x| / s0 is a corrected reciprocal product in packed
+// f32x2 arithmetic (dl_div's steps); the level-1 scale is computed once per
+// lane from the quotient of the block's max |x|; floor(4 |y| 2^-k1) indexes a
+// 64-entry code table; the E2M1 nibbles come from the hardware convert of
+// the exact signed codes and the output from one or two fp32 multiplies. It
+// stores nothing before it has decided to handle the unit. The general path
+// (dual_unit: lane l holds elements 8l..8l+7 of each 256-element half, a
+// level-1 block is four lanes) takes every other unit: ragged or unaligned
+// ones, non-finite or tiny level-0 blocks, level-1 scales above 1 (small
+// PAGE scale factors); it divides with dl_div or IEEE division and quantises
+// each element with the single-level element routine.
 
 constexpr int DL_BLOCK0 = 512;
 
@@ -60,8 +59,8 @@ struct DualArgs {
 // residual e = x - q s0 (exact, by one fma) and fl(q + e r). For bf16 x with
 // |x| >= 2^-102 and |q| >= 2^-124 this is the IEEE quotient for every bf16
 // level-0 amax (an exhaustive CPU replay of these steps checks every pair);
-// x = +-0 gives +0, which quantises exactly as -0 does; every other element
-// is flagged `slow` and takes the IEEE division instead.
+// x = +-0 gives +0, which quantises exactly as -0 does; an element outside
+// those bounds is flagged `slow` and takes the IEEE division instead.
 __device__ __forceinline__ float dl_div(float x, float s0, float r, bool& slow)
 {
     const float q = __fmul_rn(x, r);
@@ -401,7 +400,7 @@ __device__ __forceinline__ bool dual_unit_fast(const DualArgs& a, int row, int j
 // cp.async, DL_STAGES - 1 units ahead of the one it works on, and later reads
 // back only what it copied itself, so no barrier is needed (a lane's
 // wait_group makes its own copies visible to it). The copies in flight per SM
-// no longer depend on how many registers the element work needs.
+// do not depend on how many registers the element work needs.
 constexpr int DL_STAGES = 4;
 
 __device__ __forceinline__ void dl_cp16(uint32_t saddr, const void* g)
