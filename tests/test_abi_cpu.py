@@ -251,6 +251,9 @@ def test_product_path_has_no_cpu_fallback():
     from mxfp4_block_fake_b200 import mxfp4_quant_dequant
     with pytest.raises(ValueError, match="CUDA"):
         mxfp4_quant_dequant(torch.ones(4, 64))
+    from mxfp4_block_fake_b200 import mxfp4_dual_level_qdq
+    with pytest.raises(ValueError, match="CUDA"):
+        mxfp4_dual_level_qdq(torch.ones(4, 512, dtype=torch.bfloat16))
 
 
 def test_product_code_never_imports_the_oracle():

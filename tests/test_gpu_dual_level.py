@@ -164,3 +164,28 @@ def test_dual_level_full_size(mode):
     r = ops.mxfp4_dual_level_qdq(x.cuda(), scale_mode=mode, emit_mask=True)
     torch.cuda.synchronize()
     check_all(r, OP.dual_level_rowwise(u16(x), 512, 6.0, MODES[mode]), f"full size {mode}")
+
+
+def test_dual_level_into_caller_buffers():
+    """Outputs written into caller-provided tensors (the `out` argument); a
+    buffer of the wrong shape or dtype is rejected before any launch."""
+    x = W.mixed(20, 1024, seed=31, specials=False)
+    xd = x.cuda()
+    dev = xd.device
+    out = ops.DualLevelResult(y=torch.empty((20, 1024), dtype=torch.bfloat16, device=dev),
+                              codes=torch.empty((20, 512), dtype=torch.uint8, device=dev),
+                              scales0=torch.empty((20, 2), dtype=torch.float32, device=dev),
+                              scales1=torch.empty((20, 32), dtype=torch.uint8, device=dev),
+                              mask=torch.empty((20, 128), dtype=torch.uint8, device=dev))
+    r = ops.mxfp4_dual_level_qdq(xd, scale_mode="floor", out=out)
+    torch.cuda.synchronize()
+    assert r is out
+    check_all(r, O.dual_level_rowwise(u16(x), 512, 6.0, O.SCALE_FLOOR), "out buffers")
+    bad = ops.DualLevelResult(y=None, codes=None, scales0=torch.empty((20, 3), dtype=torch.float32, device=dev),
+                              scales1=torch.empty((20, 32), dtype=torch.uint8, device=dev))
+    with pytest.raises(ValueError):
+        ops.mxfp4_dual_level_qdq(xd, out=bad)
+    bad = ops.DualLevelResult(y=None, codes=None, scales0=torch.empty((20, 2), dtype=torch.float64, device=dev),
+                              scales1=torch.empty((20, 32), dtype=torch.uint8, device=dev))
+    with pytest.raises(TypeError):
+        ops.mxfp4_dual_level_qdq(xd, out=bad)
